@@ -1,0 +1,202 @@
+/*
+ * dc.h -- C ABI of the B200 multi-tenant mixed-precision delta library.
+ *
+ * What it computes.  Delta-CoMe keeps the delta between a fine-tuned linear layer and its
+ * backbone, Delta = W_ft - W_base, as SVD factors Delta ~= U diag(S) V^T whose singular vectors
+ * are quantised at 8, 3 or 2 bits by singular-value rank, with the smallest ranks dropped (0 bit):
+ *   - "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法" (paooo.com), section
+ *     "Delta-CoMe的技术原理": SVD of the delta; more bits for the singular vectors of larger
+ *     singular values; long-tail spectrum;
+ *   - "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language
+ *     Models" (atlas.scime.ai summary), section "Approach": 8/3/2-bit groups for successive
+ *     singular vectors, the smallest ones 0-bit, at the size of a 1-bit delta; sections
+ *     "Problem" and "Key results": many fine-tuned models served from one GPU.
+ * At serving time every token k of a batch carries a tenant id tau(k) and gets
+ *     y_k = W_base x_k + U_hat_tau (S_tau * (V_hat_tau^T x_k)),
+ * with tenant id -1 meaning "backbone only".  Quantisation is round-to-nearest in groups of 128
+ * consecutive elements of each singular vector with an fp16 scale and an fp16 zero point per
+ * group: v_hat = (code - zero) * scale.
+ *
+ * Conventions.
+ *   - Every entry point returns dc_status; DC_OK is 0.  No entry point aborts or traps.  The
+ *     text of the last error of the calling thread is returned by dc_last_error().
+ *   - The library never allocates device memory.  The caller allocates every device buffer
+ *     (packed stores, tenant tables, workspaces, outputs) and passes raw device pointers and a
+ *     cudaStream_t (as void*; NULL = legacy default stream).  Host pointers are borrowed for the
+ *     duration of the call only.
+ *   - Device entry points are asynchronous on the given stream unless stated otherwise.
+ *   - Device pointers must be 16-byte aligned (DC_ERR_ALIGN otherwise).
+ *   - d_out and d_in must be multiples of 128 (DC_ERR_SHAPE otherwise).
+ *   - Bit widths must be 0, 2, 3 or 8 (DC_ERR_BITS otherwise).
+ *   - Errors found by a kernel (a tenant id out of range) are written to a status word in the
+ *     workspace and read back with dc_read_device_status(); the kernel skips the bad token.
+ */
+#ifndef DC_H
+#define DC_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef int32_t dc_status;
+enum {
+  DC_OK = 0,
+  DC_ERR_INVALID_ARG = 1,  /* null pointer, negative size, non-finite factor, ...        */
+  DC_ERR_SHAPE = 2,        /* dimension not a multiple of 128, rank above min(d_out,d_in) */
+  DC_ERR_BITS = 3,         /* bit width not in {0, 2, 3, 8}                               */
+  DC_ERR_ALIGN = 4,        /* device pointer not 16-byte aligned                          */
+  DC_ERR_WORKSPACE = 5,    /* workspace or destination buffer too small                   */
+  DC_ERR_TENANT = 6,       /* tenant id out of range (host check or device status word)    */
+  DC_ERR_CUDA = 7,         /* a CUDA runtime call failed                                  */
+  DC_ERR_UNSUPPORTED = 8   /* a valid request this build does not serve (see message)     */
+};
+
+enum { DC_DTYPE_F32 = 0, DC_DTYPE_BF16 = 1 };
+
+/* flags of dc_delta_linear_segmented / dc_layer_forward */
+enum {
+  DC_BASE = 1,          /* add W_base x                                                  */
+  DC_DELTA = 2,         /* add U_hat (S * (V_hat^T x)) of the token's tenant             */
+  DC_REUSE_ROUTING = 4  /* skip dc_build_segments: the workspace already holds the routing
+                           of these tenant ids (e.g. every layer after the first)        */
+};
+
+#define DC_MAX_BANDS 4
+#define DC_GROUP 128
+
+/* Rank bands of one tenant's linear, in descending singular-value order: band j holds rank[j]
+ * consecutive ranks stored at bits[j] bits (8, 3, 2; 0 = dropped, stores nothing). */
+typedef struct {
+  int32_t d_out, d_in;
+  int32_t n_bands;
+  int32_t bits[DC_MAX_BANDS];
+  int32_t rank[DC_MAX_BANDS];
+} dc_factor_desc;
+
+/* Where one tenant's packed delta lives.  Plain data: copy it by value, or into a device-side
+ * tenant table (dc_tenant_table_upload).  dev_base == 0 means "this tenant has no delta for
+ * this linear" (its tokens get the backbone only). */
+typedef struct {
+  uint64_t dev_base;   /* device address of the packed blob (256-byte aligned) */
+  uint64_t bytes;      /* size of the blob                                      */
+  dc_factor_desc desc;
+  int32_t rank_total;  /* sum of the ranks of the non-zero bands                */
+  int32_t reserved;
+} dc_delta_handle;
+
+/* One linear of the backbone plus the deltas of every tenant for it. */
+typedef struct {
+  const void* W_base;        /* device, row-major [d_out, d_in], dtype w_dtype                */
+  int32_t w_dtype;           /* DC_DTYPE_BF16 (tensor-core path) or DC_DTYPE_F32              */
+  int32_t d_out, d_in;
+  int32_t n_tenants;         /* tenant ids run over 0..n_tenants-1                            */
+  int32_t max_rank;          /* upper bound of rank_total over the tenants (workspace sizing) */
+  const dc_delta_handle* tenants_dev;  /* device array [n_tenants] (dc_tenant_table_upload)   */
+} dc_linear;
+
+/* Text of the last error raised on the calling thread ("" if none). */
+const char* dc_last_error(void);
+
+/* Library version string. */
+const char* dc_version(void);
+
+/* Size in bytes of the packed blob of one tenant's linear.  Returns 0 for an invalid descriptor
+ * (and sets dc_last_error).  The blob holds: S as fp32 [r]; V_hat^T codes as bit planes in
+ * 16-rank tiles; U_hat codes as bit planes in 16-row tiles; fp16 scale and zero per group of
+ * 128 for every kept singular vector. */
+size_t dc_packed_size(const dc_factor_desc* desc);
+
+/* Host round-to-nearest quantiser (deterministic, fp64 arithmetic), one rule for every group
+ * of 128 elements of every kept singular vector:
+ *   lo = min(0, min g), hi = max(0, max g), qmax = 2^b - 1,
+ *   scale = fp16_rne((hi - lo) / qmax) (1 if it is 0), zero = clamp(rint(-lo / scale), 0, qmax),
+ *   code = clamp(rint(v / scale) + zero, 0, qmax), rint = round half to even.
+ * U:  fp32 column-major [d_out, r] (column i = u_i);  Vt: fp32 row-major [r, d_in] (row i = v_i)
+ * where r = sum of the ranks of the non-zero bands, bands in order.
+ * Outputs (host, caller-owned): codes_u uint8 [r, d_out] (row i = codes of u_i),
+ * codes_v uint8 [r, d_in], sz_u uint16 [r, d_out/128, 2] and sz_v uint16 [r, d_in/128, 2]
+ * holding the fp16 bit patterns of (scale, zero).  DC_ERR_INVALID_ARG on a non-finite input or
+ * a scale that overflows fp16. */
+dc_status dc_quantize_rtn(const dc_factor_desc* desc, const float* U, const float* Vt,
+                          uint8_t* codes_u, uint8_t* codes_v, uint16_t* sz_u, uint16_t* sz_v);
+
+/* Pack host codes into the serving layout and copy them to dev_dst (caller-owned, at least
+ * dc_packed_size bytes, 256-byte aligned).  S: host fp32 [r].  Synchronises the stream before
+ * returning so the host buffers may be freed.  Fills *out. */
+dc_status dc_pack_upload(const dc_factor_desc* desc, const uint8_t* codes_u, const uint8_t* codes_v,
+                         const uint16_t* sz_u, const uint16_t* sz_v, const float* S,
+                         void* dev_dst, size_t dev_bytes, void* stream, dc_delta_handle* out);
+
+/* Device quantiser + packer: the same rule as dc_quantize_rtn, run on the GPU from device fp32
+ * factors (U column-major [d_out, r], Vt row-major [r, d_in], S [r]) straight into the serving
+ * layout at dev_dst.  Produces bit-identical codes to dc_quantize_rtn.  Asynchronous.
+ * scratch: caller device buffer of dc_quantize_scratch_size(desc) bytes; its first int32 is a
+ * status word set to DC_ERR_INVALID_ARG if a group held a non-finite value or its fp16 scale
+ * overflowed (that group is stored with zero codes); read it with dc_read_device_status. */
+dc_status dc_quantize_pack_device(const dc_factor_desc* desc, const float* U_dev, const float* Vt_dev,
+                                  const float* S_dev, void* dev_dst, size_t dev_bytes, void* scratch,
+                                  size_t scratch_bytes, void* stream, dc_delta_handle* out);
+
+/* Copy n handles into a caller-owned device array (n * sizeof(dc_delta_handle) bytes).
+ * Asynchronous; the host array must stay alive until the stream reaches the copy. */
+dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int32_t n, void* dev_dst,
+                                 size_t dev_bytes, void* stream);
+
+/* Bytes of workspace needed by dc_delta_linear_segmented / dc_layer_forward for a batch of at
+ * most T tokens whose linears have ranks up to max_rank, inputs up to max_d_in columns and at
+ * most max_tenants tenants (n_linears = 1 or 7).  The workspace holds the routing result, the
+ * per-token activation limbs, the rank-reduction results and the device status word.  The same
+ * arguments must be passed to the calls that use the workspace (through dc_linear.max_rank and
+ * the batch size); a workspace smaller than this gives DC_ERR_WORKSPACE. */
+size_t dc_workspace_size(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_linears,
+                         int32_t max_tenants);
+
+/* Quantise on the device needs plain codes as scratch: bytes of scratch for one descriptor. */
+size_t dc_quantize_scratch_size(const dc_factor_desc* desc);
+
+/* Token routing: stable counting sort of tenant ids (device int32 [T], -1 = backbone only, -1
+ * first) into the workspace: permutation, inverse permutation and the segment list
+ * {tenant, start, length} in ascending tenant order.  Resets the device status word.  Ids out
+ * of range set DC_ERR_TENANT in the status word and are routed as -1. */
+dc_status dc_build_segments(const int32_t* tenant_ids_dev, int32_t T, int32_t n_tenants,
+                            void* ws, size_t ws_bytes, void* stream);
+
+/* Copy the routing result out of the workspace (debug/test helper; device -> caller device
+ * buffers): perm int32 [T], inv_perm int32 [T], segments int32 [T, 3] (first n_segments rows
+ * valid), n_segments int32 [1]. */
+dc_status dc_read_segments(const void* ws, int32_t T, int32_t* perm_dev, int32_t* inv_perm_dev,
+                           int32_t* segments_dev, int32_t* n_segments_dev, void* stream);
+
+/* y[T, d_out] = (flags & DC_BASE ? W_base x : 0) + (flags & DC_DELTA ? U_hat (S * V_hat^T x) : 0)
+ * for every token with its own tenant.  x: device [T, d_in] of dtype_in; y: device [T, d_out]
+ * of dtype_out (F32 or BF16).  Runs dc_build_segments itself.  T >= 0 (T = 0 is a no-op). */
+dc_status dc_delta_linear_segmented(const dc_linear* lin, const void* x, void* y,
+                                    const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
+                                    int32_t dtype_out, int32_t flags, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/* The seven projections of one Llama-style decoder layer in one call, sharing one routing:
+ * lin[0..6] = q, k, v, o, gate, up, down.  q, k, v, gate and up read x_h [T, hidden]; o reads
+ * x_o [T, hidden]; down reads x_f [T, ffn].  y[p] receives [T, lin[p].d_out]. */
+dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* x_o, const void* x_f,
+                           void* const y[7], const int32_t* tenant_ids_dev, int32_t T,
+                           int32_t dtype_in, int32_t dtype_out, int32_t flags, void* ws,
+                           size_t ws_bytes, void* stream);
+
+/* Decode the integer codes of one tenant's linear back out of the packed layout, with the same
+ * device decode functions the serving kernels use.  which = 0: U codes as uint8 [r, d_out]
+ * (row i = codes of u_i); which = 1: V codes as uint8 [r, d_in].  out_dev: caller device
+ * buffer. */
+dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t which, uint8_t* out_dev,
+                                void* stream);
+
+/* Read (and then clear) the device status word of a workspace; synchronises the stream. */
+dc_status dc_read_device_status(void* ws, void* stream, int32_t* host_status);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* DC_H */

@@ -1,0 +1,303 @@
+"""Python binding of the B200 multi-tenant mixed-precision delta library (include/dc.h).
+
+Argument marshalling only: every step of the serving path runs in the CUDA library
+``libdc.so`` built in this directory.  PyTorch is used by callers for device memory and streams;
+functions here take tensors (device pointers are read with ``data_ptr()``) or numpy arrays
+(host buffers) and return the C status as a raised ``DcError`` when it is not DC_OK.
+
+If the library has not been built, every entry point raises ``DcLibraryMissing``: there is no
+fallback implementation.
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libdc.so")
+SYNTH_LIB_PATH = os.path.join(_HERE, "libdc_synth.so")
+
+DC_OK, DC_ERR_INVALID_ARG, DC_ERR_SHAPE, DC_ERR_BITS, DC_ERR_ALIGN = 0, 1, 2, 3, 4
+DC_ERR_WORKSPACE, DC_ERR_TENANT, DC_ERR_CUDA, DC_ERR_UNSUPPORTED = 5, 6, 7, 8
+DC_DTYPE_F32, DC_DTYPE_BF16 = 0, 1
+DC_BASE, DC_DELTA, DC_REUSE_ROUTING = 1, 2, 4
+DC_MAX_BANDS = 4
+DC_GROUP = 128
+
+
+class DcError(RuntimeError):
+    def __init__(self, status: int, message: str):
+        super().__init__(f"dc status {status}: {message}")
+        self.status = status
+
+
+class DcLibraryMissing(RuntimeError):
+    pass
+
+
+class dc_factor_desc(C.Structure):
+    _fields_ = [("d_out", C.c_int32), ("d_in", C.c_int32), ("n_bands", C.c_int32),
+                ("bits", C.c_int32 * DC_MAX_BANDS), ("rank", C.c_int32 * DC_MAX_BANDS)]
+
+
+class dc_delta_handle(C.Structure):
+    _fields_ = [("dev_base", C.c_uint64), ("bytes", C.c_uint64), ("desc", dc_factor_desc),
+                ("rank_total", C.c_int32), ("reserved", C.c_int32)]
+
+
+class dc_linear(C.Structure):
+    _fields_ = [("W_base", C.c_void_p), ("w_dtype", C.c_int32), ("d_out", C.c_int32), ("d_in", C.c_int32),
+                ("n_tenants", C.c_int32), ("max_rank", C.c_int32), ("tenants_dev", C.c_void_p)]
+
+
+_lib = None
+
+
+def _load():
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise DcLibraryMissing(f"{LIB_PATH} is not built; run `python -m tenant_mixed_precision_b200.build`")
+    lib = C.CDLL(LIB_PATH)
+    P, I32, SZ, VP = C.POINTER, C.c_int32, C.c_size_t, C.c_void_p
+    sig = {
+        "dc_last_error": (C.c_char_p, []),
+        "dc_version": (C.c_char_p, []),
+        "dc_packed_size": (SZ, [P(dc_factor_desc)]),
+        "dc_quantize_rtn": (I32, [P(dc_factor_desc), VP, VP, VP, VP, VP, VP]),
+        "dc_pack_upload": (I32, [P(dc_factor_desc), VP, VP, VP, VP, VP, VP, SZ, VP, P(dc_delta_handle)]),
+        "dc_quantize_pack_device": (I32, [P(dc_factor_desc), VP, VP, VP, VP, SZ, VP, SZ, VP, P(dc_delta_handle)]),
+        "dc_quantize_scratch_size": (SZ, [P(dc_factor_desc)]),
+        "dc_tenant_table_upload": (I32, [P(dc_delta_handle), I32, VP, SZ, VP]),
+        "dc_workspace_size": (SZ, [I32, I32, I32, I32, I32]),
+        "dc_build_segments": (I32, [VP, I32, I32, VP, SZ, VP]),
+        "dc_read_segments": (I32, [VP, I32, VP, VP, VP, VP, VP]),
+        "dc_delta_linear_segmented": (I32, [P(dc_linear), VP, VP, VP, I32, I32, I32, I32, VP, SZ, VP]),
+        "dc_layer_forward": (I32, [P(dc_linear), VP, VP, VP, P(VP), VP, I32, I32, I32, I32, VP, SZ, VP]),
+        "dc_unpack_codes_debug": (I32, [P(dc_delta_handle), I32, VP, VP]),
+        "dc_read_device_status": (I32, [VP, VP, P(I32)]),
+    }
+    for name, (res, args) in sig.items():
+        f = getattr(lib, name)
+        f.restype = res
+        f.argtypes = args
+    _lib = lib
+    return lib
+
+
+def lib():
+    return _load()
+
+
+def exported_symbols() -> list[str]:
+    """Names of the C entry points this binding declares (all must be exported by libdc.so)."""
+    return ["dc_last_error", "dc_version", "dc_packed_size", "dc_quantize_rtn", "dc_pack_upload",
+            "dc_quantize_pack_device", "dc_quantize_scratch_size", "dc_tenant_table_upload",
+            "dc_workspace_size", "dc_build_segments", "dc_read_segments", "dc_delta_linear_segmented",
+            "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status"]
+
+
+def _check(st: int):
+    if st != DC_OK:
+        raise DcError(st, _load().dc_last_error().decode())
+
+
+def _stream(stream) -> int | None:
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except ImportError:
+            pass
+        return None
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t) -> int | None:
+    if t is None:
+        return None
+    if isinstance(t, np.ndarray):
+        return t.ctypes.data
+    if isinstance(t, int):
+        return t
+    return t.data_ptr()
+
+
+def _dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.float32:
+        return DC_DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DC_DTYPE_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+# ------------------------------------------------------------------------------------------
+# descriptors
+# ------------------------------------------------------------------------------------------
+def make_desc(d_out: int, d_in: int, plan) -> dc_factor_desc:
+    """plan: [(bits, rank), ...] in descending singular-value order (at most 4 bands)."""
+    plan = list(plan)
+    if len(plan) > DC_MAX_BANDS:
+        raise ValueError("at most 4 bands")
+    d = dc_factor_desc()
+    d.d_out, d.d_in, d.n_bands = d_out, d_in, len(plan)
+    for i, (b, r) in enumerate(plan):
+        d.bits[i], d.rank[i] = int(b), int(r)
+    return d
+
+
+def desc_rank(desc: dc_factor_desc) -> int:
+    return sum(desc.rank[i] for i in range(desc.n_bands) if desc.bits[i])
+
+
+# ------------------------------------------------------------------------------------------
+# entry points (same names as the C ABI)
+# ------------------------------------------------------------------------------------------
+def dc_version() -> str:
+    return _load().dc_version().decode()
+
+
+def dc_last_error() -> str:
+    return _load().dc_last_error().decode()
+
+
+def dc_packed_size(desc: dc_factor_desc) -> int:
+    n = _load().dc_packed_size(C.byref(desc))
+    if n == 0:
+        raise DcError(DC_ERR_INVALID_ARG, dc_last_error())
+    return n
+
+
+def dc_quantize_rtn(desc: dc_factor_desc, U: np.ndarray, Vt: np.ndarray):
+    """Host RTN.  U: float32 [d_out, r] (any order), Vt: float32 [r, d_in].
+    Returns (codes_u uint8 [r, d_out], codes_v uint8 [r, d_in], sz_u uint16 [r, d_out/128, 2],
+    sz_v uint16 [r, d_in/128, 2])."""
+    r = desc_rank(desc)
+    Uc = np.ascontiguousarray(np.asarray(U, dtype=np.float32).T)  # [r, d_out] = column-major U
+    Vc = np.ascontiguousarray(np.asarray(Vt, dtype=np.float32))
+    cu = np.zeros((r, desc.d_out), np.uint8)
+    cv = np.zeros((r, desc.d_in), np.uint8)
+    su = np.zeros((r, desc.d_out // DC_GROUP, 2), np.uint16)
+    sv = np.zeros((r, desc.d_in // DC_GROUP, 2), np.uint16)
+    _check(_load().dc_quantize_rtn(C.byref(desc), _ptr(Uc), _ptr(Vc), _ptr(cu), _ptr(cv), _ptr(su), _ptr(sv)))
+    return cu, cv, su, sv
+
+
+def dc_pack_upload(desc: dc_factor_desc, codes_u, codes_v, sz_u, sz_v, S, dev_dst, stream=None) -> dc_delta_handle:
+    h = dc_delta_handle()
+    arrs = [np.ascontiguousarray(a) for a in (codes_u, codes_v, sz_u, sz_v)]
+    S = np.ascontiguousarray(np.asarray(S, dtype=np.float32))
+    nbytes = dev_dst.numel() * dev_dst.element_size()
+    _check(_load().dc_pack_upload(C.byref(desc), *[_ptr(a) for a in arrs], _ptr(S), _ptr(dev_dst), nbytes,
+                                  _stream(stream), C.byref(h)))
+    return h
+
+
+def dc_quantize_scratch_size(desc: dc_factor_desc) -> int:
+    return _load().dc_quantize_scratch_size(C.byref(desc))
+
+
+def dc_quantize_pack_device(desc: dc_factor_desc, U_dev, Vt_dev, S_dev, dev_dst, scratch, stream=None,
+                            dst_offset: int = 0, dst_bytes: int | None = None) -> dc_delta_handle:
+    """U_dev: float32 device [r, d_out] contiguous (= column-major U), Vt_dev: [r, d_in], S_dev: [r]."""
+    h = dc_delta_handle()
+    nbytes = dst_bytes if dst_bytes is not None else dev_dst.numel() * dev_dst.element_size() - dst_offset
+    _check(_load().dc_quantize_pack_device(C.byref(desc), _ptr(U_dev), _ptr(Vt_dev), _ptr(S_dev),
+                                           _ptr(dev_dst) + dst_offset, nbytes, _ptr(scratch),
+                                           scratch.numel() * scratch.element_size(), _stream(stream), C.byref(h)))
+    return h
+
+
+def dc_tenant_table_upload(handles, dev_dst, stream=None):
+    n = len(handles)
+    arr = (dc_delta_handle * max(n, 1))(*handles)
+    _check(_load().dc_tenant_table_upload(arr, n, _ptr(dev_dst), dev_dst.numel() * dev_dst.element_size(),
+                                          _stream(stream)))
+    return arr  # keep alive until the stream reaches the copy
+
+
+def empty_handle() -> dc_delta_handle:
+    return dc_delta_handle()
+
+
+def dc_workspace_size(T: int, max_rank: int, max_d_in: int, n_linears: int, max_tenants: int) -> int:
+    return _load().dc_workspace_size(T, max_rank, max_d_in, n_linears, max_tenants)
+
+
+def dc_build_segments(tenant_ids, T: int, n_tenants: int, ws, stream=None):
+    _check(_load().dc_build_segments(_ptr(tenant_ids), T, n_tenants, _ptr(ws), ws.numel() * ws.element_size(),
+                                     _stream(stream)))
+
+
+def dc_read_segments(ws, T: int, perm, inv_perm, segments, n_segments, stream=None):
+    _check(_load().dc_read_segments(_ptr(ws), T, _ptr(perm), _ptr(inv_perm), _ptr(segments), _ptr(n_segments),
+                                    _stream(stream)))
+
+
+def make_linear(W_base, d_out: int, d_in: int, n_tenants: int, max_rank: int, tenants_dev,
+                w_dtype: int | None = None) -> dc_linear:
+    lin = dc_linear()
+    lin.W_base = _ptr(W_base)
+    lin.w_dtype = _dtype_code(W_base) if w_dtype is None and W_base is not None else (w_dtype or DC_DTYPE_BF16)
+    lin.d_out, lin.d_in, lin.n_tenants, lin.max_rank = d_out, d_in, n_tenants, max_rank
+    lin.tenants_dev = _ptr(tenants_dev)
+    return lin
+
+
+def dc_delta_linear_segmented(lin: dc_linear, x, y, tenant_ids, T: int, flags: int, ws, stream=None):
+    _check(_load().dc_delta_linear_segmented(C.byref(lin), _ptr(x), _ptr(y), _ptr(tenant_ids), T, _dtype_code(x),
+                                             _dtype_code(y), flags, _ptr(ws), ws.numel() * ws.element_size(),
+                                             _stream(stream)))
+
+
+def dc_layer_forward(lins, x_h, x_o, x_f, ys, tenant_ids, T: int, flags: int, ws, stream=None):
+    arr = (dc_linear * 7)(*lins)
+    yp = (C.c_void_p * 7)(*[_ptr(y) for y in ys])
+    _check(_load().dc_layer_forward(arr, _ptr(x_h), _ptr(x_o), _ptr(x_f), yp, _ptr(tenant_ids), T,
+                                    _dtype_code(x_h), _dtype_code(ys[0]), flags, _ptr(ws),
+                                    ws.numel() * ws.element_size(), _stream(stream)))
+
+
+def dc_unpack_codes_debug(handle: dc_delta_handle, which: int, out_dev, stream=None):
+    _check(_load().dc_unpack_codes_debug(C.byref(handle), which, _ptr(out_dev), _stream(stream)))
+
+
+def dc_read_device_status(ws, stream=None) -> int:
+    v = C.c_int32(0)
+    _check(_load().dc_read_device_status(_ptr(ws), _stream(stream), C.byref(v)))
+    return v.value
+
+
+# ------------------------------------------------------------------------------------------
+# device input generator (test/benchmark inputs; twin of synth.py's counter-based stream)
+# ------------------------------------------------------------------------------------------
+_synth_lib = None
+
+
+def _synth_loader():
+    global _synth_lib
+    if _synth_lib is None:
+        if not os.path.exists(SYNTH_LIB_PATH):
+            raise DcLibraryMissing(f"{SYNTH_LIB_PATH} is not built")
+        l = C.CDLL(SYNTH_LIB_PATH)
+        for n in ("dcs_normal_f32", "dcs_normal_bf16"):
+            f = getattr(l, n)
+            f.restype = C.c_int
+            f.argtypes = [C.c_uint64, C.c_uint64, C.c_uint64, C.c_uint64, C.c_float, C.c_void_p, C.c_void_p]
+        _synth_lib = l
+    return _synth_lib
+
+
+def synth_normal_device(out, seed: int, stream_id: int, start: int, c: float, stream=None):
+    """Fill a float32 or bf16 device tensor with the counter-based stream (see synth.py)."""
+    import torch
+    l = _synth_loader()
+    f = l.dcs_normal_f32 if out.dtype == torch.float32 else l.dcs_normal_bf16
+    rc = f(seed, stream_id, start, out.numel(), C.c_float(c), _ptr(out), _stream(stream))
+    if rc != 0:
+        raise RuntimeError(f"synth kernel launch failed: {rc}")

@@ -1,0 +1,196 @@
+// Packed serving layout of one tenant's delta (host packer and device kernels share it).
+//
+// A tenant's delta for one linear is Delta_hat = U_hat diag(S) V_hat^T with ranks split into
+// bands of equal bit width in descending singular-value order (the 8/3/2/0-bit groups of
+// "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language Models",
+// section "Approach").  Each kept vector is quantised in groups of 128 with an fp16 scale and
+// zero per group.  The blob is laid out for the two serving kernels:
+//
+//   [S fp32 r] [V codes, band by band] [V meta] [U codes, band by band] [U meta]
+//
+// V side (rank reduction t = S * (V_hat^T x)): the kernel's MMA tile is 16 ranks x 32 columns of
+// d_in (mma.m16n8k32, u8 codes).  Ranks of a band are cut into tiles of 16 (the last may be
+// partial); rows of a tile are in two halves (rows 0-7, rows 8-15); d_in is cut into blocks of
+// 4 groups (512 columns, the last block may hold fewer groups).  Within a block a lane
+// (g = lane/4, t = lane%4) of a half owns row g of the half, and within each group the 32
+// columns 32t .. 32t+31; the column of MMA step s (0..3), k-half hh (0/1) and byte b is
+// 32t + 8s + 4hh + b (the B operand uses the same permutation, so activations stay in natural
+// order).  Storage per (tile, block, half): one array per bit plane, lanes in order, only the
+// lanes of valid rows (4 per row) present:
+//   2-bit, full block : 8 words per lane; word 2s+hh, bits [8b+2p, 8b+2p+2) hold the code of
+//                       group p (p = 0..3) -- a register is extracted with one AND and carries
+//                       the weight 4^p, removed in the fp32 epilogue ("mask" layout);
+//   2-bit, tail block : 2 words per group; word s/2, bits [8b+2q, 8b+2q+2), q = 2(s%2)+hh
+//                       ("shift" layout);
+//   3-bit             : the 2-bit plane in the shift layout plus a 1-bit plane of one word per
+//                       group, bit 8b + 2s + hh = bit 2 of the code;
+//   8-bit             : 8 words per group, word 2s+hh byte b = the code.
+// V meta: per (tile, group, g, half) the fp16 pair (scale, zero) of row g + 8*half: 64 bytes per
+// (tile, group), rows past the band padded with zeros.
+//
+// U side (y += U_hat * B with B = scale * t): the MMA tile is 16 output rows x 32 ranks.  A band
+// of 2 or 3 bits is cut into steps of 32 ranks; lane (g, t) owns rows g and g+8 and, within a
+// step, ranks 8t .. 8t+7: register j (a0..a3) is row g + 8*(j&1), ranks 8t + 4*(j>>1) + b.
+//   2-bit, full quad of 4 steps : 4 words per lane; word j, bits [8b+2p, 8b+2p+2) = step p
+//                                 (mask layout, weight 4^p);
+//   other steps (2-bit leftovers, every 3-bit step): one word per lane (shift layout: register
+//                                 j = bits [8b+2j, 8b+2j+2)); for 3 bits also a 1-bit plane of
+//                                 2 bytes per lane, bit 4j+b = bit 2 of the code of register j
+//                                 byte b;
+//   the last step of a band may be partial: only lanes with 8t < valid ranks are stored
+//   (ranks inside a lane padded to 8 with code 0).
+// 8-bit bands of U are small (the top singular vectors) and are stored row-major [d_out][R8]
+// as bytes for a scalar path.
+// U meta: [d_out/128][r] fp16 pairs (scale, zero).
+#pragma once
+#include <stdint.h>
+
+#include "dc.h"
+
+#if defined(__CUDACC__)
+#define DC_HD __host__ __device__ __forceinline__
+#else
+#define DC_HD inline
+#endif
+
+struct DcBand {
+  int32_t bits;        // 2, 3 or 8
+  int32_t rank;        // ranks in the band
+  int32_t r0;          // first rank of the band (index into S, t and U meta)
+  int32_t bsm_off;     // offset of the band in the U-stage staging of B (multiple of 32)
+  int32_t v_tiles;     // ceil(rank / 16)
+  int32_t u_quads;     // U: full 4-step quads in the mask layout (2-bit only)
+  int32_t u_steps;     // U: steps in the shift layout after the quads (incl. a partial last one)
+  int32_t u_last;      // U: valid ranks of the last shift-layout step (32 if it is full)
+  int64_t v_off;       // V codes of the band
+  int64_t v_tile_bytes;// bytes of one full 16-row tile
+  int64_t v_meta_off;  // V meta of the band
+  int64_t u_off;       // U codes of the band
+  int64_t u_otile_bytes; // bytes per 16-row output tile (MMA bands); R8 for 8-bit bands
+};
+
+struct DcLayout {
+  int32_t d_out, d_in, n_bands, r;
+  int32_t groups_in;   // d_in / 128
+  int32_t groups_out;  // d_out / 128
+  int32_t nkb;         // ceil(groups_in / 4) blocks of 512 columns
+  int32_t tail_groups; // groups in the last block (1..4)
+  int32_t bsm_total;   // extent of the U-stage B staging (ranks, padded)
+  int32_t valid;       // 1 if the descriptor is valid
+  int64_t s_off, u_meta_off, bytes;
+  int64_t dev_base;    // device address of the blob (filled where a layout is bound to a blob)
+  DcBand band[DC_MAX_BANDS];
+};
+
+DC_HD int64_t dc_align(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+
+// bytes of one lane's codes for one group of one row (all planes)
+DC_HD int32_t dc_v_lane_group_bytes(int32_t bits) { return bits == 2 ? 8 : (bits == 3 ? 12 : 32); }
+// bytes of plane 0 (2-bit plane or the 8-bit plane) of one lane for ngrp groups
+DC_HD int32_t dc_v_plane0_bytes(int32_t bits, int32_t ngrp) { return (bits == 8 ? 32 : 8) * ngrp; }
+// bytes of one (tile, block): 4 lanes per valid row, all planes
+DC_HD int64_t dc_v_block_bytes(int32_t bits, int32_t rows, int32_t ngrp) {
+  return (int64_t)4 * rows * dc_v_lane_group_bytes(bits) * ngrp;
+}
+// byte offset of half h inside a (tile, block) region
+DC_HD int64_t dc_v_half_off(int32_t bits, int32_t rows, int32_t ngrp, int32_t h) {
+  int32_t n0 = rows < 8 ? rows : 8;
+  return h == 0 ? 0 : (int64_t)4 * n0 * dc_v_lane_group_bytes(bits) * ngrp;
+}
+// bytes of one U shift-layout step holding nl lanes (both planes, each padded to 16)
+DC_HD int64_t dc_u_step_bytes(int32_t bits, int32_t nl) {
+  return dc_align((int64_t)nl * 4, 16) + (bits == 3 ? dc_align((int64_t)nl * 2, 16) : 0);
+}
+DC_HD int32_t dc_u_step_lanes(int32_t valid_ranks) {  // lanes (of 32) stored for a step
+  int32_t nt = (valid_ranks + 7) / 8;
+  return 8 * nt;
+}
+
+DC_HD bool dc_bits_ok(int32_t b) { return b == 0 || b == 2 || b == 3 || b == 8; }
+
+// Compute the layout of a descriptor; layout.valid = 0 on an invalid descriptor.
+DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
+  DcLayout L;
+  L.valid = 0;
+  L.d_out = d.d_out;
+  L.d_in = d.d_in;
+  L.n_bands = 0;
+  L.r = 0;
+  L.bytes = 0;
+  L.s_off = 0;
+  L.dev_base = 0;
+  L.u_meta_off = 0;
+  L.bsm_total = 0;
+  L.groups_in = d.d_in / DC_GROUP;
+  L.groups_out = d.d_out / DC_GROUP;
+  L.nkb = (L.groups_in + 3) / 4;
+  L.tail_groups = L.groups_in - 4 * (L.nkb - 1);
+  if (d.d_out <= 0 || d.d_in <= 0 || d.d_out % DC_GROUP || d.d_in % DC_GROUP) return L;
+  if (d.n_bands < 0 || d.n_bands > DC_MAX_BANDS) return L;
+  int32_t r = 0;
+  for (int i = 0; i < d.n_bands; ++i) {
+    if (!dc_bits_ok(d.bits[i]) || d.rank[i] < 0) return L;
+    if (d.bits[i] == 0 || d.rank[i] == 0) continue;
+    DcBand& B = L.band[L.n_bands++];
+    B.bits = d.bits[i];
+    B.rank = d.rank[i];
+    B.r0 = r;
+    r += d.rank[i];
+  }
+  int32_t cap = d.d_out < d.d_in ? d.d_out : d.d_in;
+  if (r > cap) return L;
+  L.r = r;
+  int64_t off = dc_align((int64_t)r * 4, 256);  // S
+  // V codes
+  for (int i = 0; i < L.n_bands; ++i) {
+    DcBand& B = L.band[i];
+    B.v_tiles = (B.rank + 15) / 16;
+    B.v_off = off;
+    B.v_tile_bytes = (int64_t)64 * dc_v_lane_group_bytes(B.bits) * L.groups_in;
+    int32_t last_rows = B.rank - 16 * (B.v_tiles - 1);
+    int64_t sz = B.v_tile_bytes * (B.v_tiles - 1) +
+                 (int64_t)4 * last_rows * dc_v_lane_group_bytes(B.bits) * L.groups_in;
+    off = dc_align(off + sz, 256);
+  }
+  // V meta
+  for (int i = 0; i < L.n_bands; ++i) {
+    DcBand& B = L.band[i];
+    B.v_meta_off = off;
+    off = dc_align(off + (int64_t)B.v_tiles * L.groups_in * 64, 256);
+  }
+  // U codes
+  int32_t bsm = 0;
+  for (int i = 0; i < L.n_bands; ++i) {
+    DcBand& B = L.band[i];
+    B.u_off = off;
+    B.bsm_off = bsm;
+    if (B.bits == 8) {
+      B.u_quads = 0;
+      B.u_steps = 0;
+      B.u_last = 0;
+      B.u_otile_bytes = B.rank;
+      off = dc_align(off + (int64_t)d.d_out * B.rank, 256);
+      continue;
+    }
+    B.u_quads = B.bits == 2 ? B.rank / 128 : 0;
+    int32_t rest = B.rank - 128 * B.u_quads;
+    B.u_steps = (rest + 31) / 32;
+    B.u_last = rest - 32 * (B.u_steps - 1);
+    if (B.u_steps == 0) B.u_last = 32;
+    int64_t ot = (int64_t)B.u_quads * 512;
+    for (int s = 0; s < B.u_steps; ++s) {
+      int32_t valid = (s == B.u_steps - 1) ? B.u_last : 32;
+      ot += dc_u_step_bytes(B.bits, dc_u_step_lanes(valid));
+    }
+    B.u_otile_bytes = ot;
+    off = dc_align(off + ot * (d.d_out / 16), 256);
+    bsm += (int32_t)dc_align(B.rank, 32);
+  }
+  L.bsm_total = bsm;
+  // U meta
+  L.u_meta_off = off;
+  off = dc_align(off + (int64_t)L.groups_out * r * 4, 256);
+  L.bytes = off;
+  L.valid = 1;
+  return L;
+}
