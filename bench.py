@@ -1,0 +1,384 @@
+#!/usr/bin/env python
+"""Benchmark: 50-tenant 7B mixed-precision delta decode on B200.
+
+One step = one decode pass of a batch of 64 tokens (tenants drawn uniformly from 50 resident
+deltas) through the full 32-layer x 7-projection Llama-2-7B linear stack: token routing, then per
+layer the activation prep, the rank reduction t = S * (V_hat^T x) and the output kernel
+y = W_base x + U_hat t, all through the library's C ABI (dc_layer_forward), replayed as a CUDA
+graph.  Inputs are synthetic (seeded), generated on the GPU, and already resident in HBM when
+the timed region starts; every step reads ~46 GB, far more than the 126 MB L2, so no L2 flush is
+needed between steps.
+
+Prints one JSON line (rank 0).  --impl reference times the fp64 CPU oracle instead on a bounded
+sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "tokens/s and % of HBM roofline, 50-tenant 7B mixed-precision delta decode"
+WORKLOAD = dict(name="llama2-7b linear stack decode, 50 resident tenant deltas at 1/16",
+                hidden=4096, ffn=11008, layers=32, n_tenants=50, T=64, seed=20241, ids_seed=3)
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d.get("hbm_gbs", FALLBACK_HBM_GBS)), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def _ids(n_tenants: int, T: int, seed: int):
+    import numpy as np
+    from tenant_mixed_precision_b200 import synth
+    return synth.uniform_tenants(np.random.default_rng(seed), T, n_tenants)
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle sampling during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            out, _ = self.proc.communicate(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+            out, _ = self.proc.communicate()
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    with open(os.path.join(ROOT, "tenant_mixed_precision_b200", "csrc", "dc_kernels.cu"), "rb") as f:
+        h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def _ncu_traffic(kernel: str):
+    """Per-launch DRAM bytes of `kernel` from the committed ncu summary, if it matches this source."""
+    path = os.path.join(ROOT, "profiles", "traffic.txt")
+    if not os.path.exists(path):
+        return None
+    sha = _kernel_source_sha()
+    with open(path) as f:
+        for line in f:
+            kv = dict(p.split("=", 1) for p in line.split() if "=" in p)
+            if kv.get("kernel") == kernel and kv.get("source_sha") == sha:
+                return float(kv["dram_bytes_per_launch"])
+    return None
+
+
+# ------------------------------------------------------------------------------------------------
+# CPU oracle baseline (test infrastructure; the only oracle use in this file)
+# ------------------------------------------------------------------------------------------------
+class OracleSample:
+    """Layer 0, projection q (4096x4096) for the first `n_tok` tokens of the batch, through the fp64
+    oracle.  Extrapolated to the full step by the number of weight and factor elements the oracle
+    touches: backbone parameters plus, per (layer, projection), the factor elements of each
+    distinct tenant of the batch."""
+
+    def __init__(self, ids, n_tok: int):
+        import numpy as np
+
+        import oracle
+        from tenant_mixed_precision_b200 import plans, synth
+        from tenant_mixed_precision_b200.synth_stack import host_activations, host_factors
+        W = WORKLOAD
+        self.oracle = oracle
+        self.ids = np.asarray(ids[:n_tok], np.int32)
+        d = W["hidden"]
+        plan = plans.budget_plan(d, d, 1 / 16, plans.MIXED_1_16)
+        r = sum(x for _, x in plan)
+        self.arts = {}
+        for t in sorted(set(self.ids.tolist())):
+            f = host_factors(W["seed"], 0, 0, t, d, d, r)
+            self.arts[t] = oracle.compress_factors(f.U, f.S, f.Vt, plan)
+        _, wv = synth.stream_base_weight(W["seed"], 0, 0, d, d)
+        self.W = wv.astype(np.float64)
+        _, xv = host_activations(W["seed"], 0, 0, W["T"], d)
+        self.x = xv[:n_tok].astype(np.float64)
+        per_factor = {}
+        for (d_out, d_in) in synth.llama_proj_shapes(W["hidden"], W["ffn"]):
+            pl = plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+            per_factor[(d_out, d_in)] = sum(x for _, x in pl) * (d_out + d_in)
+        n_dist_full = len(set(int(t) for t in ids))
+        full = 0
+        for (d_out, d_in) in synth.llama_proj_shapes(W["hidden"], W["ffn"]):
+            full += d_out * d_in + n_dist_full * per_factor[(d_out, d_in)]
+        full *= W["layers"]
+        sample = d * d + len(self.arts) * per_factor[(d, d)]
+        self.scale = full / sample
+        self.desc = (f"layer 0 q-projection (4096x4096), {len(self.ids)} tokens / {len(self.arts)} tenants, "
+                     f"fp64 numpy oracle evaluation; extrapolated x{self.scale:.0f} by weight+factor elements to the "
+                     f"full 32-layer 64-token step")
+
+    def run_once(self) -> float:
+        t0 = time.perf_counter()
+        self.oracle.delta_linear(self.W, self.arts, self.x, self.ids)
+        return time.perf_counter() - t0
+
+    def tokens_per_s(self, seconds: float) -> float:
+        return WORKLOAD["T"] / (seconds * self.scale)
+
+
+def _cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except AttributeError:
+        return os.cpu_count() or 1
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    ids = _ids(WORKLOAD["n_tenants"], WORKLOAD["T"], WORKLOAD["ids_seed"])
+    s = OracleSample(ids, n_tok=8)
+    for _ in range(args.warmup):
+        s.run_once()
+    times = [s.run_once() for _ in range(args.steps)]
+    step_s = sum(times) / len(times)
+    v = s.tokens_per_s(step_s)
+    line = {"metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_s * s.scale * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD["name"], "T": WORKLOAD["T"], "layers": WORKLOAD["layers"],
+                       "tenants": WORKLOAD["n_tenants"]},
+            "impl": "reference",
+            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": _cores(), "kind": "oracle", "sample": s.desc},
+            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ------------------------------------------------------------------------------------------------
+# GPU arm
+# ------------------------------------------------------------------------------------------------
+def run_gpu(args):
+    import numpy as np
+    import torch
+
+    import tenant_mixed_precision_b200 as dc
+    from tenant_mixed_precision_b200 import plans
+    from tenant_mixed_precision_b200.stack import DeltaStack
+    from tenant_mixed_precision_b200.synth_stack import populate
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
+    W = WORKLOAD
+    T = W["T"]
+
+    def plan_fn(l, p, d_out, d_in, t):
+        return plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+
+    t_setup = time.time()
+    stack = DeltaStack(W["hidden"], W["ffn"], W["layers"], W["n_tenants"], T, plan_fn, out_dtype=torch.bfloat16)
+    populate(stack, W["seed"])
+    ids = _ids(W["n_tenants"], T, W["ids_seed"] + 1000 * rank)
+    ids_dev = torch.from_numpy(ids).cuda()
+    setup_s = time.time() - t_setup
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        stack.forward(ids_dev, T)  # eager warm-up (sets kernel attributes before capture)
+    stream.synchronize()
+    assert dc.dc_read_device_status(stack.ws, stream) == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        stack.forward(ids_dev, T)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+
+    # ---- device-resident timed region
+    clocks = ClockSampler(local)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    ck = clocks.stop()
+    if dist:
+        dist.barrier()
+    ms = ev0.elapsed_time(ev1)
+    ms_t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
+    ms_max = float(ms_t.item())
+    tokens = T * args.steps * world
+    value = tokens / (ms_max / 1e3)
+    ms_per_step = ms_max / args.steps
+    status = dc.dc_read_device_status(stack.ws, stream)
+
+    # ---- end to end: pinned host inputs in, graph, result out (every step)
+    h_ids = torch.from_numpy(ids).pin_memory()
+    h_x = [x[:T].cpu().pin_memory() for x in stack.x[0]]
+    h_y = [torch.empty(y.shape, dtype=y.dtype).pin_memory() for y in stack.y[-1]]
+    h2d = h_ids.numel() * 4 + sum(x.numel() * x.element_size() for x in h_x)
+    d2h = sum(y.numel() * y.element_size() for y in h_y)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        e0.record(stream)
+        for _ in range(args.steps):
+            ids_dev.copy_(h_ids, non_blocking=True)
+            for hx, dx in zip(h_x, stack.x[0]):
+                dx[:T].copy_(hx, non_blocking=True)
+            graph.replay()
+            for hy, dy in zip(h_y, stack.y[-1]):
+                hy.copy_(dy, non_blocking=True)
+        e1.record(stream)
+    e1.synchronize()
+    e2e_ms = e0.elapsed_time(e1)
+    e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
+    if dist:
+        dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
+    e2e_value = tokens / (float(e_t.item()) / 1e3)
+
+    # ---- per-kernel durations (eager calls with CUDA events around every launch on its stream)
+    n_prof = max(3, min(args.steps, 10))
+    cap = n_prof * (1 + 3 * W["layers"]) + 8
+    torch.cuda.synchronize()
+    dc.dc_profile_begin(cap)
+    with torch.cuda.stream(stream):
+        for _ in range(n_prof):
+            stack.forward(ids_dev, T)
+    rec = dc.dc_profile_end(cap)
+    per = {}
+    for kind, m in rec:
+        per.setdefault(kind, []).append(m)
+    tot = {k: sum(v) for k, v in per.items()}
+    dom = max(tot, key=tot.get)
+    dom_avg_ms = statistics.mean(per[dom])
+    ab = stack.algorithmic_bytes(ids)
+    per_launch_bytes = {
+        "output": (ab["backbone"] + ab["delta_u"] + ab["activations"]) / W["layers"],
+        "rank_reduction": ab["delta_v"] / W["layers"],
+    }
+    peak, peak_kind = _peaks()
+    achieved = per_launch_bytes.get(dom, 0.0) / (dom_avg_ms * 1e-3) / 1e9
+    kname = {"output": "k_ustage", "rank_reduction": "k_vstage", "prep": "k_prep", "routing": "k_segments"}[dom]
+    step_gbs = ab["total"] / (ms_per_step * 1e-3) / 1e9
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        s = OracleSample(ids, n_tok=8)
+        s.run_once()
+        times = []
+        t_end = time.time() + args.cpu_seconds
+        while time.time() < t_end or len(times) < 2:
+            times.append(s.run_once())
+        cpu = {"value": s.tokens_per_s(statistics.mean(times)), "unit": "tokens/s", "cores": _cores(),
+               "kind": "oracle", "sample": s.desc + f"; {len(times)} repetitions"}
+
+    if dist:
+        dist.barrier()
+        graph = None
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+    line = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "u8xs8->s32 delta, bf16xbf16->f32 backbone", "data": "synthetic",
+        "config": {"workload": W["name"], "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
+                   "tenants_resident": W["n_tenants"], "T": T, "distinct_tenants": ab["distinct_tenants"],
+                   "budget": "1/16: 8-bit x2, 3-bit x32, 2-bit remainder", "output_dtype": "bf16",
+                   "l2": "inputs larger than L2 (~46 GB read per step); no flush", "cuda_graph": True,
+                   "parallelism": f"replicas x{world}"},
+        "step_hbm": {"algorithmic_bytes": ab["total"], "achieved_gbs": step_gbs, "peak_gbs": peak,
+                     "frac": step_gbs / peak, "peak_source": peak_kind},
+        "roofline": {"bound": "hbm", "kernel": kname, "achieved": achieved, "peak": peak, "unit": "GB/s",
+                     "frac": achieved / peak, "peak_source": f"{peak_kind} hbm_gbs",
+                     "traffic": _ncu_traffic(kname), "algorithmic_bytes_per_launch": per_launch_bytes.get(dom),
+                     "avg_launch_ms": dom_avg_ms},
+        "kernel_ms_per_step": {k: v / n_prof for k, v in tot.items()},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "what": "per step: tenant ids and layer-0 activations in from pinned host memory, layer-31 outputs out"},
+        "gpu_launches": (1 + 3 * W["layers"]) * args.steps,
+        "cpu_baseline": cpu,
+        "clocks": ck,
+        "device_status": status,
+        "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="dc", choices=["dc", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_gpu(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -193,6 +193,16 @@ dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* 
 dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t which, uint8_t* out_dev,
                                 void* stream);
 
+/* Per-kernel timing: after dc_profile_begin(capacity) every kernel launched by the serving entry
+ * points on this thread is bracketed by two CUDA events recorded on its stream (at most
+ * `capacity` launches).  dc_profile_end synchronises those events, writes each launch's duration
+ * in milliseconds and its kernel kind (0 routing, 1 activation prep, 2 rank reduction, 3 output)
+ * to the caller's host arrays, destroys the events and returns the number of launches recorded
+ * (negative on error).  Events recorded during stream capture become graph nodes; profile eager
+ * calls only. */
+dc_status dc_profile_begin(int32_t capacity);
+int32_t dc_profile_end(float* ms_out, int32_t* kind_out, int32_t capacity);
+
 /* Read (and then clear) the device status word of a workspace; synchronises the stream. */
 dc_status dc_read_device_status(void* ws, void* stream, int32_t* host_status);
 

@@ -79,6 +79,8 @@ def _load():
         "dc_layer_forward": (I32, [P(dc_linear), VP, VP, VP, P(VP), VP, I32, I32, I32, I32, VP, SZ, VP]),
         "dc_unpack_codes_debug": (I32, [P(dc_delta_handle), I32, VP, VP]),
         "dc_read_device_status": (I32, [VP, VP, P(I32)]),
+        "dc_profile_begin": (I32, [I32]),
+        "dc_profile_end": (I32, [P(C.c_float), P(I32), I32]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -97,7 +99,8 @@ def exported_symbols() -> list[str]:
     return ["dc_last_error", "dc_version", "dc_packed_size", "dc_quantize_rtn", "dc_pack_upload",
             "dc_quantize_pack_device", "dc_quantize_scratch_size", "dc_tenant_table_upload",
             "dc_workspace_size", "dc_build_segments", "dc_read_segments", "dc_delta_linear_segmented",
-            "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status"]
+            "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status", "dc_profile_begin",
+            "dc_profile_end"]
 
 
 def _check(st: int):
@@ -271,6 +274,23 @@ def dc_read_device_status(ws, stream=None) -> int:
     v = C.c_int32(0)
     _check(_load().dc_read_device_status(_ptr(ws), _stream(stream), C.byref(v)))
     return v.value
+
+
+KERNEL_KINDS = ("routing", "prep", "rank_reduction", "output")
+
+
+def dc_profile_begin(capacity: int):
+    _check(_load().dc_profile_begin(capacity))
+
+
+def dc_profile_end(capacity: int):
+    """Returns a list of (kind name, milliseconds) per recorded launch."""
+    ms = (C.c_float * capacity)()
+    kinds = (C.c_int32 * capacity)()
+    n = _load().dc_profile_end(ms, kinds, capacity)
+    if n < 0:
+        raise DcError(DC_ERR_CUDA, "profiling failed: " + dc_last_error())
+    return [(KERNEL_KINDS[kinds[i]], float(ms[i])) for i in range(min(n, capacity))]
 
 
 # ------------------------------------------------------------------------------------------

@@ -705,15 +705,20 @@ __device__ void u_base_bf16(const DcFwd& F, const DcLinDev& lin, const int* perm
     }
     __syncthreads();
     const __nv_bfloat16* xb = xst + (kc & 1) * 64 * U_XROW;
+    // Each 128-column chunk is summed in a fresh MMA chain and added to the running sum with an
+    // IEEE fp32 add, so the tensor core's internal accumulation rounding spans 8 steps, not d_in/16.
 #pragma unroll
-    for (int k32 = 0; k32 < 4; ++k32) {
+    for (int nt = 0; nt < 8; ++nt) {
+      if (nt < ntv) {
+        float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        if (nt < ntv) {
+        for (int k32 = 0; k32 < 4; ++k32) {
           const uint4 xv = *reinterpret_cast<const uint4*>(xb + (8 * nt + g) * U_XROW + 32 * k32 + 8 * t);
-          mma_bf16(acc[nt], wa[k32].x, wb[k32].x, wa[k32].y, wb[k32].y, xv.x, xv.y);
-          mma_bf16(acc[nt], wa[k32].z, wb[k32].z, wa[k32].w, wb[k32].w, xv.z, xv.w);
+          mma_bf16(part, wa[k32].x, wb[k32].x, wa[k32].y, wb[k32].y, xv.x, xv.y);
+          mma_bf16(part, wa[k32].z, wb[k32].z, wa[k32].w, wb[k32].w, xv.z, xv.w);
         }
+#pragma unroll
+        for (int q = 0; q < 4; ++q) acc[nt][q] += part[q];
       }
     }
     __syncthreads();
@@ -1155,6 +1160,70 @@ __global__ void k_pack_words(DcLayout L, DcPlain Pl, uint32_t* dst) {
 // ---------------------------------------------------------------------------------------------
 static inline bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
 
+// ---- per-kernel timing hook (dc_profile_begin / dc_profile_end)
+struct ProfState {
+  cudaEvent_t* ev = nullptr;
+  int32_t* kind = nullptr;
+  int32_t cap = 0, n = 0;
+};
+static thread_local ProfState g_prof;
+
+static void prof_before(cudaStream_t s, int kind) {
+  if (!g_prof.ev || g_prof.n >= g_prof.cap) return;
+  cudaEventRecord(g_prof.ev[2 * g_prof.n], s);
+  g_prof.kind[g_prof.n] = kind;
+}
+static void prof_after(cudaStream_t s) {
+  if (!g_prof.ev || g_prof.n >= g_prof.cap) return;
+  cudaEventRecord(g_prof.ev[2 * g_prof.n + 1], s);
+  g_prof.n++;
+}
+
+extern "C" dc_status dc_profile_begin(int32_t capacity) {
+  dc_clear_error();
+  if (g_prof.ev) return dc_fail(DC_ERR_INVALID_ARG, "profiling already active");
+  if (capacity <= 0) return dc_fail(DC_ERR_INVALID_ARG, "capacity must be positive");
+  g_prof.ev = new cudaEvent_t[2 * (size_t)capacity];
+  g_prof.kind = new int32_t[capacity];
+  g_prof.cap = capacity;
+  g_prof.n = 0;
+  for (int i = 0; i < 2 * capacity; ++i) {
+    dc_status st = dc_cuda_check(cudaEventCreate(&g_prof.ev[i]), "event create");
+    if (st) {
+      for (int j = 0; j < i; ++j) cudaEventDestroy(g_prof.ev[j]);
+      delete[] g_prof.ev;
+      delete[] g_prof.kind;
+      g_prof = ProfState();
+      return st;
+    }
+  }
+  return DC_OK;
+}
+
+extern "C" int32_t dc_profile_end(float* ms_out, int32_t* kind_out, int32_t capacity) {
+  dc_clear_error();
+  if (!g_prof.ev) return -1;
+  int32_t n = g_prof.n;
+  int32_t rc = n;
+  for (int i = 0; i < n; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) {
+      rc = -1;
+      break;
+    }
+    float ms = 0.f;
+    cudaEventElapsedTime(&ms, g_prof.ev[2 * i], g_prof.ev[2 * i + 1]);
+    if (i < capacity) {
+      if (ms_out) ms_out[i] = ms;
+      if (kind_out) kind_out[i] = g_prof.kind[i];
+    }
+  }
+  for (int i = 0; i < 2 * g_prof.cap; ++i) cudaEventDestroy(g_prof.ev[i]);
+  delete[] g_prof.ev;
+  delete[] g_prof.kind;
+  g_prof = ProfState();
+  return rc;
+}
+
 extern "C" size_t dc_quantize_scratch_size(const dc_factor_desc* desc) {
   DcLayout L;
   if (dc_check_desc(desc, &L) != DC_OK) return 0;
@@ -1306,11 +1375,15 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (max_ten > DC_MAX_TENANTS) return dc_fail(DC_ERR_UNSUPPORTED, "too many tenants");
     const size_t smem = (size_t)2 * (max_ten + 1) * 4;
     if (smem > 48 * 1024) cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    prof_before(s, 0);
     k_segments<<<1, 256, smem, s>>>(ids, T, max_ten, (uint8_t*)ws, F.ws);
+    prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "routing kernel");
     if (st) return st;
   }
+  prof_before(s, 1);
   k_prep<<<dim3(T + 1, n_in), 256, 0, s>>>(F, (uint8_t*)ws);
+  prof_after(s);
   st = dc_cuda_check(cudaGetLastError(), "prep kernel");
   if (st) return st;
   if (flags & DC_DELTA) {
@@ -1321,7 +1394,9 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
       cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
       if (n_sm <= 0) n_sm = 148;
     }
+    prof_before(s, 2);
     k_vstage<<<n_sm * 4, 256, 0, s>>>(F, (uint8_t*)ws);
+    prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "rank-reduction kernel");
     if (st) return st;
   }
@@ -1333,7 +1408,9 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     usmem_set = usmem;
   }
   const dim3 ugrid(F.tile_prefix[n_lin], (T + DC_TOK_BLOCK - 1) / DC_TOK_BLOCK);
+  prof_before(s, 3);
   k_ustage<<<ugrid, 256, usmem, s>>>(F, (uint8_t*)ws);
+  prof_after(s);
   return dc_cuda_check(cudaGetLastError(), "output kernel");
 }
 
