@@ -214,7 +214,11 @@ def run_gpu(args):
 
         import torch.distributed as dist
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300))
-    W = WORKLOAD
+    W = dict(WORKLOAD)
+    if args.layers:
+        W["layers"] = args.layers
+    if args.tenants:
+        W["n_tenants"] = args.tenants
     T = W["T"]
 
     def plan_fn(l, p, d_out, d_in, t):
@@ -296,7 +300,7 @@ def run_gpu(args):
 
     # ---- per-kernel durations (eager calls with CUDA events around every launch on its stream)
     n_prof = max(3, min(args.steps, 10))
-    cap = n_prof * (1 + 3 * W["layers"]) + 8
+    cap = n_prof * (1 + 4 * W["layers"]) + 8
     torch.cuda.synchronize()
     dc.dc_profile_begin(cap)
     with torch.cuda.stream(stream):
@@ -311,16 +315,18 @@ def run_gpu(args):
     dom_avg_ms = statistics.mean(per[dom])
     ab = stack.algorithmic_bytes(ids)
     per_launch_bytes = {
-        "output": (ab["backbone"] + ab["delta_u"] + ab["activations"]) / W["layers"],
+        "backbone_output": (ab["backbone"] + ab["activations"]) / W["layers"],
+        "delta_output": ab["delta_u"] / W["layers"],
         "rank_reduction": ab["delta_v"] / W["layers"],
     }
     peak, peak_kind = _peaks()
     achieved = per_launch_bytes.get(dom, 0.0) / (dom_avg_ms * 1e-3) / 1e9
-    kname = {"output": "k_ustage", "rank_reduction": "k_vstage", "prep": "k_prep", "routing": "k_segments"}[dom]
+    kname = {"backbone_output": "k_base", "delta_output": "k_udelta", "rank_reduction": "k_vstage", "prep": "k_prep",
+             "routing": "k_segments"}[dom]
     step_gbs = ab["total"] / (ms_per_step * 1e-3) / 1e9
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.layers and not args.tenants:
         s = OracleSample(ids, n_tok=8)
         s.run_once()
         times = []
@@ -352,9 +358,10 @@ def run_gpu(args):
                      "traffic": _ncu_traffic(kname), "algorithmic_bytes_per_launch": per_launch_bytes.get(dom),
                      "avg_launch_ms": dom_avg_ms},
         "kernel_ms_per_step": {k: v / n_prof for k, v in tot.items()},
+        "kernel_gbs": {k: per_launch_bytes[k] / (statistics.mean(per[k]) * 1e-3) / 1e9 for k in per_launch_bytes if k in per},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "what": "per step: tenant ids and layer-0 activations in from pinned host memory, layer-31 outputs out"},
-        "gpu_launches": (1 + 3 * W["layers"]) * args.steps,
+        "gpu_launches": (1 + 4 * W["layers"]) * args.steps,
         "cpu_baseline": cpu,
         "clocks": ck,
         "device_status": status,
@@ -372,6 +379,8 @@ def main():
     ap.add_argument("--impl", default="dc", choices=["dc", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    ap.add_argument("--layers", type=int, default=0, help="smaller stack for profiling captures (default: 32)")
+    ap.add_argument("--tenants", type=int, default=0, help="fewer resident tenants (default: 50)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3

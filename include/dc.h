@@ -146,7 +146,7 @@ dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int32_t n, void
                                  size_t dev_bytes, void* stream);
 
 /* Bytes of workspace needed by dc_delta_linear_segmented / dc_layer_forward for a batch of at
- * most T tokens whose linears have ranks up to max_rank, inputs up to max_d_in columns and at
+ * most T tokens whose linears have ranks up to max_rank, d_in and d_out up to max_d_in and at
  * most max_tenants tenants (n_linears = 1 or 7).  The workspace holds the routing result, the
  * per-token activation limbs, the rank-reduction results and the device status word.  The same
  * arguments must be passed to the calls that use the workspace (through dc_linear.max_rank and
@@ -196,7 +196,8 @@ dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t which, uint8_t
 /* Per-kernel timing: after dc_profile_begin(capacity) every kernel launched by the serving entry
  * points on this thread is bracketed by two CUDA events recorded on its stream (at most
  * `capacity` launches).  dc_profile_end synchronises those events, writes each launch's duration
- * in milliseconds and its kernel kind (0 routing, 1 activation prep, 2 rank reduction, 3 output)
+ * in milliseconds and its kernel kind (0 routing, 1 activation prep, 2 rank reduction, 3 delta
+ * output, 4 backbone output)
  * to the caller's host arrays, destroys the events and returns the number of launches recorded
  * (negative on error).  Events recorded during stream capture become graph nodes; profile eager
  * calls only. */

@@ -276,7 +276,7 @@ def dc_read_device_status(ws, stream=None) -> int:
     return v.value
 
 
-KERNEL_KINDS = ("routing", "prep", "rank_reduction", "output")
+KERNEL_KINDS = ("routing", "prep", "rank_reduction", "delta_output", "backbone_output")
 
 
 def dc_profile_begin(capacity: int):

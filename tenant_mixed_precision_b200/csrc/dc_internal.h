@@ -19,22 +19,55 @@ double dc_f16_to_f64(uint16_t h);
 #define DC_TOK_BLOCK 64         // tokens per output block of the decode output kernel
 #define DC_V_NT 2               // 16-rank tiles per V work item
 #define DC_V_TOKS 4             // tokens per V/U pass (two pairs)
+#define DC_XBLK 1600            // per (token, 512-column block): 3 limb rows of 512 B + 4 x 4 fp32 limb sums
 
 // Status word slots at the start of the workspace.
-enum { DC_WS_STATUS = 0, DC_WS_VCOUNTER = 1, DC_WS_NITEMS = 2, DC_WS_NSEG = 3, DC_WS_SLOTS = 64 };
+enum {
+  DC_WS_STATUS = 0,
+  DC_WS_NSEG = 1,
+  DC_WS_VCOUNTER = 2,
+  DC_WS_NITEMS = 3,
+  DC_WS_UCOUNTER = 4,
+  DC_WS_BCOUNTER = 5,
+  DC_WS_SLOTS = 64
+};
 
-// One V work item: projection p, segment seg, token pass, band, first tile, tile count.
-struct DcVItem {
-  int16_t p, band;
-  int32_t seg;
-  int32_t tile0;
-  int16_t ntiles, pass;
+// One V work item, self-contained (written by the prep kernel, read with one 64-byte load):
+// a band's tiles tile0 .. tile0+ntiles-1 of one tenant's linear for one 4-token pass.
+// 16-byte aligned: it is moved with 16-byte vector loads and stores.
+struct alignas(16) DcVItem {
+  int64_t vbase;       // device address of the tile group's first block
+  int64_t sbase;       // device address of S[rank0]
+  int32_t f4;          // bytes of one full 512-column block of the group (distance between blocks)
+  int32_t bits;
+  int32_t rows_left;   // ranks of the band from tile0 on (rows of tile i = min(16, rows_left - 16 i))
+  int32_t ntiles;
+  int32_t nkb, tail_groups;
+  int32_t p, m;        // linear, input
+  int32_t tok0, ntok;  // sorted token positions of the pass
+  int32_t rank0;       // rank of row 0 of tile0
+  int32_t pad;
+};
+
+// One (linear, segment) record for the output kernel, self-contained.
+struct DcUBand {
+  int32_t bits, rank, r0, bsm_off;
+  int32_t quads, steps, last, region;  // region: bytes of the band for one 128-row output group
+  int64_t u_off;                       // band offset in the blob
+  int32_t otile;                       // bytes per 16-row tile (2/3-bit) or R8 (8-bit)
+  int32_t pad;
+};
+struct alignas(16) DcURec {  // moved with 16-byte vector loads and stores
+  int64_t blob;
+  int32_t valid, tenant, st, len, r, r4, n_bands, u_meta_off;
+  int32_t pad[2];
+  DcUBand band[DC_MAX_BANDS];
 };
 
 // Workspace layout (byte offsets from the workspace base).
 struct DcWs {
-  int32_t T, max_rank, max_d_in, n_lin, n_in, r_stride, max_items, max_tenants;
-  int64_t status, perm, inv, segs, items, layouts, xl, xs, xe, tws, total;
+  int32_t T, max_rank, max_d_in, n_lin, n_in, r_stride, max_items, max_tenants, nkb, pad;
+  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, total;
 };
 
 DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, int32_t max_tenants);

@@ -4,8 +4,8 @@
 //   k_segments  token routing: stable counting sort of tenant ids into segments.
 //   k_prep      per sorted token: the activation as a 24-bit fixed-point integer split into three
 //               signed 8-bit limbs (so u8 x s8 tensor-core MMAs reproduce x exactly to 2^-22 of
-//               the token's largest entry), limb sums per group of 128, and (one extra block)
-//               the per-(linear, tenant) layouts plus the V work list.
+//               the token's largest entry), limb sums per group of 128; extra blocks write one
+//               self-contained record per (linear, segment) and the V work list.
 //   k_vstage    rank reduction t = S * (V_hat^T x) per (linear, segment): 2/3/8-bit codes are
 //               unpacked in registers into u8 MMA operands (mma.m16n8k32), the zero point and
 //               the per-group fp16 scale are applied in an fp32 epilogue per group of 128.
@@ -19,6 +19,8 @@
 // Delta-Compression with Mixed-Precision for Large Language Models", "Approach".
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -28,6 +30,7 @@
 #include "dc_internal.h"
 #include "dc_layout.h"
 #include "dc_pack.h"
+#include "dc_tma.h"
 
 #define FULLMASK 0xffffffffu
 
@@ -121,11 +124,14 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.inv = take((int64_t)T * 4);
   W.segs = take((int64_t)T * 12);
   W.items = take((int64_t)W.max_items * sizeof(DcVItem));
-  W.layouts = take((int64_t)n_lin * max_tenants * sizeof(DcLayout));
-  W.xl = take((int64_t)W.n_in * 3 * T * W.max_d_in);
-  W.xs = take((int64_t)W.n_in * T * (W.max_d_in / 128) * 16);
+  W.urecs = take((int64_t)n_lin * (T > 0 ? T : 1) * sizeof(DcURec));
+  W.nkb = (W.max_d_in + 511) / 512;
+  W.xl = take((int64_t)W.n_in * T * W.nkb * DC_XBLK);
+  W.xsort = take((int64_t)W.n_in * T * W.max_d_in * 2);
   W.xe = take((int64_t)W.n_in * T * 4);
   W.tws = take((int64_t)n_lin * T * W.r_stride * 4);
+  W.yd = take((int64_t)n_lin * T * W.max_d_in * 4);
+  W.dflag = take((int64_t)n_lin * T);
   W.total = off;
   return W;
 }
@@ -144,6 +150,8 @@ struct DcLinDev {
 };
 
 struct DcFwd {
+  CUtensorMap wmap[7];     // backbone weights, box 64 columns x 128 rows, 128-byte swizzle
+  CUtensorMap xmap[3];     // tenant-sorted bf16 activations, box 64 columns x 64 tokens
   DcLinDev lin[7];
   const void* x[3];
   int32_t dx[3];
@@ -159,11 +167,13 @@ struct WsPtr {
   int* inv;
   int* segs;
   DcVItem* items;
-  DcLayout* layouts;
-  int8_t* xl;
-  int* xs;
+  DcURec* urecs;
+  uint8_t* xl;
+  uint8_t* xsort;
   int* xe;
   float* tws;
+  float* yd;
+  uint8_t* dflag;
 };
 __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   WsPtr p;
@@ -172,11 +182,13 @@ __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   p.inv = (int*)(ws + W.inv);
   p.segs = (int*)(ws + W.segs);
   p.items = (DcVItem*)(ws + W.items);
-  p.layouts = (DcLayout*)(ws + W.layouts);
-  p.xl = (int8_t*)(ws + W.xl);
-  p.xs = (int*)(ws + W.xs);
+  p.urecs = (DcURec*)(ws + W.urecs);
+  p.xl = ws + W.xl;
+  p.xsort = ws + W.xsort;
   p.xe = (int*)(ws + W.xe);
   p.tws = (float*)(ws + W.tws);
+  p.yd = (float*)(ws + W.yd);
+  p.dflag = ws + W.dflag;
   return p;
 }
 
@@ -248,99 +260,117 @@ __global__ void k_segments(const int32_t* __restrict__ ids, int T, int n, uint8_
 }
 
 // ---------------------------------------------------------------------------------------------
-// k_prep: activation limbs, limb sums, exponents; the last block builds layouts and V items.
+// k_prep: activation limbs, limb sums, exponents; extra blocks write the (linear, segment)
+// records and the V work list.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ int sext8(int v) { return (int)(int8_t)(v & 0xff); }
 
-__device__ void build_layouts_and_items(const DcFwd& F, const WsPtr& P) {
+__device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) {
   const DcWs& W = F.ws;
-  const int tid = threadIdx.x;
-  for (int idx = tid; idx < F.n_lin * W.max_tenants; idx += blockDim.x) {
-    const int p = idx / W.max_tenants, tau = idx % W.max_tenants;
-    DcLayout L;
-    L.valid = 0;
-    if (tau < F.lin[p].n_tenants) {
-      const dc_delta_handle* h = F.lin[p].tenants + tau;
-      if (h->dev_base != 0) {
-        L = dc_layout(h->desc);
-        if (L.valid && (L.d_out != F.lin[p].d_out || L.d_in != F.lin[p].d_in || L.r > W.r_stride ||
-                        L.bsm_total > F.bsm_max)) {
-          L.valid = 0;
-          set_status(P.st, DC_ERR_SHAPE);
-        }
-        if (!L.valid) set_status(P.st, DC_ERR_SHAPE);
-        L.dev_base = (int64_t)h->dev_base;
+  const int tau = P.segs[3 * s], st = P.segs[3 * s + 1], len = P.segs[3 * s + 2];
+  DcURec R;
+  R.blob = 0;
+  R.valid = 0;
+  R.tenant = tau;
+  R.st = st;
+  R.len = len;
+  R.r = R.r4 = R.n_bands = R.u_meta_off = 0;
+  R.pad[0] = R.pad[1] = 0;
+  DcLayout L;
+  L.valid = 0;
+  if (tau < F.lin[p].n_tenants) {
+    const dc_delta_handle* h = F.lin[p].tenants + tau;
+    if (h->dev_base != 0) {
+      L = dc_layout(h->desc);
+      if (!L.valid || L.d_out != F.lin[p].d_out || L.d_in != F.lin[p].d_in || L.r > W.r_stride ||
+          L.bsm_total > F.bsm_max) {
+        L.valid = 0;
+        set_status(P.st, DC_ERR_SHAPE);
       }
     }
-    P.layouts[idx] = L;
-  }
-  __syncthreads();
-  __shared__ int n_items;
-  if (tid == 0) n_items = 0;
-  __syncthreads();
-  const int nseg = P.st[DC_WS_NSEG];
-  if (F.flags & DC_DELTA) {
-    // projections in decreasing d_in so that long items are handed out first
-    int ord[7];
-    for (int i = 0; i < F.n_lin; ++i) ord[i] = i;
-    for (int i = 0; i < F.n_lin; ++i)
-      for (int j = i + 1; j < F.n_lin; ++j)
-        if (F.lin[ord[j]].d_in > F.lin[ord[i]].d_in) {
-          const int tmp = ord[i];
-          ord[i] = ord[j];
-          ord[j] = tmp;
-        }
-    for (int oi = 0; oi < F.n_lin; ++oi) {
-      const int p = ord[oi];
-      for (int s = tid; s < nseg; s += blockDim.x) {
-        const int tau = P.segs[3 * s], len = P.segs[3 * s + 2];
-        if (tau >= F.lin[p].n_tenants || tau >= W.max_tenants) continue;
-        const DcLayout& L = P.layouts[p * W.max_tenants + tau];
-        if (!L.valid) continue;
-        const int passes = (len + DC_V_TOKS - 1) / DC_V_TOKS;
-        int per_pass = 0;
-        for (int b = 0; b < L.n_bands; ++b) per_pass += (L.band[b].v_tiles + DC_V_NT - 1) / DC_V_NT;
-        const int count = passes * per_pass;
-        const int base = atomicAdd(&n_items, count);
-        if (base + count > W.max_items) {
-          set_status(P.st, DC_ERR_WORKSPACE);
+    if (L.valid) {
+      R.blob = (int64_t)h->dev_base;
+      R.valid = 1;
+      R.r = L.r;
+      R.r4 = L.r4;
+      R.n_bands = L.n_bands;
+      R.u_meta_off = (int32_t)L.u_meta_off;
+      for (int b = 0; b < DC_MAX_BANDS; ++b) {
+        DcUBand& U = R.band[b];
+        if (b >= L.n_bands) {
+          U.bits = U.rank = U.r0 = U.bsm_off = U.quads = U.steps = U.last = U.region = U.otile = U.pad = 0;
+          U.u_off = 0;
           continue;
         }
-        int k = base;
-        for (int ps = 0; ps < passes; ++ps)
-          for (int b = 0; b < L.n_bands; ++b)
-            for (int t0 = 0; t0 < L.band[b].v_tiles; t0 += DC_V_NT) {
-              DcVItem it;
-              it.p = (int16_t)p;
-              it.band = (int16_t)b;
-              it.seg = s;
-              it.tile0 = t0;
-              it.ntiles = (int16_t)min(DC_V_NT, L.band[b].v_tiles - t0);
-              it.pass = (int16_t)ps;
-              P.items[k++] = it;
-            }
+        const DcBand& B = L.band[b];
+        U.bits = B.bits;
+        U.rank = B.rank;
+        U.r0 = B.r0;
+        U.bsm_off = B.bsm_off;
+        U.quads = B.u_quads;
+        U.steps = B.u_steps;
+        U.last = B.u_last;
+        U.otile = (int32_t)B.u_otile_bytes;
+        U.region = B.bits == 8 ? 128 * B.rank : (int32_t)(8 * B.u_otile_bytes);
+        U.u_off = B.u_off;
+        U.pad = 0;
       }
-      __syncthreads();
     }
   }
-  __syncthreads();
-  if (tid == 0) {
-    P.st[DC_WS_NITEMS] = min(n_items, W.max_items);
-    P.st[DC_WS_VCOUNTER] = 0;
+  P.urecs[(int64_t)p * W.T + s] = R;
+  for (int k = 0; k < len; ++k) P.dflag[(int64_t)p * W.T + st + k] = (uint8_t)R.valid;
+  if (!R.valid || !(F.flags & DC_DELTA)) return;
+  const int passes = (len + DC_V_TOKS - 1) / DC_V_TOKS;
+  int per_pass = 0;
+  for (int b = 0; b < L.n_bands; ++b) per_pass += (L.band[b].v_tiles + L.band[b].v_group - 1) / L.band[b].v_group;
+  const int count = passes * per_pass;
+  const int base = atomicAdd(P.st + DC_WS_NITEMS, count);
+  if (base + count > W.max_items) {
+    set_status(P.st, DC_ERR_WORKSPACE);
+    return;
   }
+  int k = base;
+  for (int ps = 0; ps < passes; ++ps)
+    for (int b = 0; b < L.n_bands; ++b) {
+      const DcBand& B = L.band[b];
+      const int tpi = B.v_group;
+      for (int t0 = 0; t0 < B.v_tiles; t0 += tpi) {
+        DcVItem it;
+        it.vbase = R.blob + B.v_off + dc_v_group_block_off(B, L, t0 / tpi, 0);
+        it.sbase = R.blob + 4 * (int64_t)(B.r0 + 16 * t0);
+        it.f4 = (int32_t)dc_v_group_block_bytes(B, t0 / tpi, 4);
+        it.bits = B.bits;
+        it.rows_left = B.rank - 16 * t0;
+        it.ntiles = min(tpi, B.v_tiles - t0);
+        it.nkb = L.nkb;
+        it.tail_groups = L.tail_groups;
+        it.p = p;
+        it.m = F.lin[p].input;
+        it.tok0 = st + DC_V_TOKS * ps;
+        it.ntok = min(DC_V_TOKS, len - DC_V_TOKS * ps);
+        it.rank0 = B.r0 + 16 * t0;
+        it.pad = 0;
+        P.items[k++] = it;
+      }
+    }
 }
 
 __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, uint8_t* ws) {
   const DcWs& W = F.ws;
   WsPtr P = ws_ptr(W, ws);
-  if (blockIdx.x == (unsigned)W.T) {
-    if (blockIdx.y == 0) build_layouts_and_items(F, P);
+  if (blockIdx.x >= (unsigned)W.T) {
+    // record blocks: block (T + i, y) handles (linear y, segments i, i + #record blocks, ...)
+    const int nseg = P.st[DC_WS_NSEG];
+    const int p = blockIdx.y;
+    if (p >= F.n_lin) return;
+    for (int s = (blockIdx.x - W.T) * blockDim.x + threadIdx.x; s < nseg; s += (gridDim.x - W.T) * blockDim.x)
+      build_records_for(F, P, p, s);
     return;
   }
-  if (!(F.flags & DC_DELTA)) return;
+  if (blockIdx.y >= (unsigned)W.n_in) return;
   const int j = blockIdx.x, m = blockIdx.y;
   const int d = F.dx[m];
-  const int T = W.T, maxd = W.max_d_in, G = maxd / 128;
+  const int T = W.T, maxd = W.max_d_in;
   const int i = P.perm[j];
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   auto load4 = [&](int k, float (&v)[4]) {
@@ -374,9 +404,13 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
     frexpf(mx, &E);  // mx < 2^E
     e = 22 - E;      // |x| * 2^e < 2^22
   }
+  uint8_t* xrow = P.xl + (int64_t)(m * T + j) * W.nkb * DC_XBLK;
   for (int k = tid * 4; k < d; k += 1024) {
     float v[4];
     load4(k, v);
+    if (F.dtype_in == DC_DTYPE_BF16)  // tenant-sorted copy for the backbone tiles
+      *reinterpret_cast<uint2*>(P.xsort + ((int64_t)(m * T + j) * maxd + k) * 2) =
+          *reinterpret_cast<const uint2*>((const __nv_bfloat16*)F.x[m] + (int64_t)i * d + k);
     uint32_t w0 = 0, w1 = 0, w2 = 0;
     int s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
@@ -391,344 +425,781 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
       w2 |= (uint32_t)(l2 & 0xff) << (8 * q);
       s0 += l0, s1 += l1, s2 += l2;
     }
-    int8_t* base = P.xl + ((int64_t)(m * 3) * T + j) * maxd + k;
-    *reinterpret_cast<uint32_t*>(base) = w0;
-    *reinterpret_cast<uint32_t*>(base + (int64_t)T * maxd) = w1;
-    *reinterpret_cast<uint32_t*>(base + (int64_t)2 * T * maxd) = w2;
+    // [kb][limb 0 | limb 1 | limb 2 | limb sums of the block's 4 groups]
+    uint8_t* blk = xrow + (int64_t)(k >> 9) * DC_XBLK;
+    const int within = k & 511;
+    *reinterpret_cast<uint32_t*>(blk + within) = w0;
+    *reinterpret_cast<uint32_t*>(blk + 512 + within) = w1;
+    *reinterpret_cast<uint32_t*>(blk + 1024 + within) = w2;
 #pragma unroll
     for (int o = 16; o; o >>= 1) {
       s0 += __shfl_xor_sync(FULLMASK, s0, o);
       s1 += __shfl_xor_sync(FULLMASK, s1, o);
       s2 += __shfl_xor_sync(FULLMASK, s2, o);
     }
-    if (lane == 0) {
-      int* xs = P.xs + ((int64_t)(m * T + j) * G + k / 128) * 4;
-      xs[0] = s0, xs[1] = s1, xs[2] = s2, xs[3] = 0;
+    if (lane == 0) {  // limb sums of the group (|sum| <= 128 * 128: exact in fp32)
+      float* xs = reinterpret_cast<float*>(blk + 1536 + 16 * (within >> 7));
+      xs[0] = (float)s0, xs[1] = (float)s1, xs[2] = (float)s2, xs[3] = 0.f;
     }
   }
   if (tid == 0) P.xe[m * T + j] = e;
 }
 
 // ---------------------------------------------------------------------------------------------
-// k_vstage: t = S * (V_hat^T x) for every (linear, segment, token pass, band, 2 tiles)
+// k_vstage: t = S * (V_hat^T x).  Persistent CTAs of 8 consumer warps + 1 producer warp.  The
+// producer takes one work item at a time (prefetching the next item's record), and streams the
+// item's 512-column blocks -- codes and meta of every tile, the activation limbs and limb sums of
+// the pass's tokens -- into a ring of shared-memory stages with bulk copies; consumer warp w
+// decodes tile w from shared memory into u8 MMA operands.
 // ---------------------------------------------------------------------------------------------
-struct VCtx {
-  const uint8_t* blob;
-  const DcLayout* L;
-  int band;
-  int tile0, ntiles;
-  int tok0, ntok;  // sorted token positions of this pass
-  int m, p;
+#define V_STAGES 6
+#define V_A_BYTES 18432   // one block of the item's tiles: 8 x 2304 (2-bit), 5 x 3328 (3-bit), 2 x 8448 (8-bit)
+#define V_XTOK 1616       // one token's limb block (DC_XBLK bytes) in shared memory, padded against bank conflicts
+#define V_X_BYTES (4 * V_XTOK)
+#define V_STAGE_BYTES (V_A_BYTES + V_X_BYTES)
+#define V_CONSUMERS 8
+#define V_THREADS (32 * (V_CONSUMERS + 1))
+
+struct VDesc {
+  int kind;  // 0 block, 1 end
+  int bits, rows_left, ntiles, tok0, ntok, m, p, kb, ngrp, first, last, rank0, pad;
+  int64_t sbase;
 };
 
-// Epilogue of one group for one tile: acc += (s/w) * (C - w z XS) for the valid pairs.
-__device__ __forceinline__ void v_group_epilogue(float (&acc)[2][4], const int (&C)[2][4], uint2 meta, float w,
-                                                 const int (&xs)[2][2], int npair) {
-  const __half2 m0 = *reinterpret_cast<const __half2*>(&meta.x);  // (scale, zero) of row g
-  const __half2 m1 = *reinterpret_cast<const __half2*>(&meta.y);  // row g+8
-  const float inv = 1.f / w;
-  const float sA = __low2float(m0) * inv, zA = __high2float(m0) * w;
-  const float sB = __low2float(m1) * inv, zB = __high2float(m1) * w;
+struct VSmemTail {
+  VDesc desc[V_STAGES];
+  uint64_t full[V_STAGES];
+  uint64_t empty[V_STAGES];
+  DcVItem rec[2];  // producer: current and next item
+};
+
+// acc[q] += s_row * (C[q] - z_row * xs_tok) for the C fragment entries that hold a valid token.
+// C entries: q = 0 (row g, pair token 0), 1 (row g, token 1), 2 (row g+8, token 0), 3 (row g+8, token 1).
+template <bool TOK1>
+__device__ __forceinline__ void v_epi(float (&acc)[4], const int (&C)[4], float sA, float zA, float sB, float zB,
+                                      float x0, float x1) {
+  acc[0] = fmaf(sA, fmaf(-zA, x0, (float)C[0]), acc[0]);
+  acc[2] = fmaf(sB, fmaf(-zB, x0, (float)C[2]), acc[2]);
+  if (TOK1) {
+    acc[1] = fmaf(sA, fmaf(-zA, x1, (float)C[1]), acc[1]);
+    acc[3] = fmaf(sB, fmaf(-zB, x1, (float)C[3]), acc[3]);
+  }
+}
+
+// One 512-column block of one 16-rank tile, NTOK tokens (1..4), all loops unrolled.
+// FULL: the block holds 4 groups (2-bit codes then use the mask layout); otherwise ngrp < 4.
+template <int BITS, int NTOK, bool FULL>
+__device__ __forceinline__ void v_block(int rows, int ngrp_rt, const uint8_t* A, const uint8_t* X,
+                                        float (&acc)[2][4], int lane) {
+  constexpr int NPAIR = (NTOK + 1) / 2;
+  const int ngrp = FULL ? 4 : ngrp_rt;
+  const int g = lane >> 2, t = lane & 3;
+  const int nh0 = min(rows, 8), nh1 = max(0, rows - 8);
+  const bool ok0 = g < nh0, ok1 = g < nh1;
+  const uint8_t* meta = A + dc_v_block_code_bytes(BITS, rows, ngrp);
+  // B operand: lane g < 6 supplies limb g>>1 of pass token 2 pr + (g&1); limb sums of lane t's limb
+  const int limb = g >> 1;
+  const uint8_t* xrow[NPAIR];
+  bool xval[NPAIR];
 #pragma unroll
-  for (int pr = 0; pr < 2; ++pr) {
-    if (pr < npair) {
-      acc[pr][0] += sA * fmaf(-zA, (float)xs[pr][0], (float)C[pr][0]);
-      acc[pr][1] += sA * fmaf(-zA, (float)xs[pr][1], (float)C[pr][1]);
-      acc[pr][2] += sB * fmaf(-zB, (float)xs[pr][0], (float)C[pr][2]);
-      acc[pr][3] += sB * fmaf(-zB, (float)xs[pr][1], (float)C[pr][3]);
+  for (int pr = 0; pr < NPAIR; ++pr) {
+    const int tk = 2 * pr + (g & 1);
+    xval[pr] = (g < 6) && (tk < NTOK);
+    xrow[pr] = X + (xval[pr] ? tk * V_XTOK + 512 * limb : 0) + 32 * t;
+  }
+  const float* xsum = reinterpret_cast<const float*>(X + 1536 + 4 * (t < 3 ? t : 0));
+  uint4 wm0a = make_uint4(0, 0, 0, 0), wm0b = wm0a, wm1a = wm0a, wm1b = wm0a;
+  if (BITS == 2 && FULL) {
+    if (ok0) {
+      const uint8_t* pp = A + lane * 32;
+      wm0a = *reinterpret_cast<const uint4*>(pp);
+      wm0b = *reinterpret_cast<const uint4*>(pp + 16);
+    }
+    if (ok1) {
+      const uint8_t* pp = A + dc_v_half_off(2, rows, 4, 1) + lane * 32;
+      wm1a = *reinterpret_cast<const uint4*>(pp);
+      wm1b = *reinterpret_cast<const uint4*>(pp + 16);
     }
   }
+#pragma unroll
+  for (int grp = 0; grp < 4; ++grp) {
+    if (!FULL && grp >= ngrp) break;
+    // activation limbs of this group (B fragments of the 4 steps) and limb sums
+    uint32_t bw[NPAIR][8];
+#pragma unroll
+    for (int pr = 0; pr < NPAIR; ++pr) {
+      uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
+      if (xval[pr]) {
+        q0 = *reinterpret_cast<const uint4*>(xrow[pr] + grp * 128);
+        q1 = *reinterpret_cast<const uint4*>(xrow[pr] + grp * 128 + 16);
+      }
+      bw[pr][0] = q0.x, bw[pr][1] = q0.y, bw[pr][2] = q0.z, bw[pr][3] = q0.w;
+      bw[pr][4] = q1.x, bw[pr][5] = q1.y, bw[pr][6] = q1.z, bw[pr][7] = q1.w;
+    }
+    float xs[NTOK];
+#pragma unroll
+    for (int k = 0; k < NTOK; ++k) xs[k] = t < 3 ? xsum[k * (V_XTOK / 4) + grp * 4] : 0.f;
+    const uint2 mt = *reinterpret_cast<const uint2*>(meta + (grp * 8 + g) * 8);
+    uint32_t a[4][4];  // [step][reg]
+    if (BITS == 2 && FULL) {
+      const uint32_t msk = 0x03030303u << (2 * grp);
+      a[0][0] = wm0a.x & msk, a[0][1] = wm1a.x & msk, a[0][2] = wm0a.y & msk, a[0][3] = wm1a.y & msk;
+      a[1][0] = wm0a.z & msk, a[1][1] = wm1a.z & msk, a[1][2] = wm0a.w & msk, a[1][3] = wm1a.w & msk;
+      a[2][0] = wm0b.x & msk, a[2][1] = wm1b.x & msk, a[2][2] = wm0b.y & msk, a[2][3] = wm1b.y & msk;
+      a[3][0] = wm0b.z & msk, a[3][1] = wm1b.z & msk, a[3][2] = wm0b.w & msk, a[3][3] = wm1b.w & msk;
+    } else {
+      const int p0 = dc_v_plane0_bytes(BITS, ngrp);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const bool ok = h ? ok1 : ok0;
+        const int nh = h ? nh1 : nh0;
+        const uint8_t* hb = A + dc_v_half_off(BITS, rows, ngrp, h);
+        if (BITS == 8) {
+          uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
+          if (ok) {
+            q0 = *reinterpret_cast<const uint4*>(hb + lane * p0 + 32 * grp);
+            q1 = *reinterpret_cast<const uint4*>(hb + lane * p0 + 32 * grp + 16);
+          }
+          a[0][h] = q0.x, a[0][h + 2] = q0.y, a[1][h] = q0.z, a[1][h + 2] = q0.w;
+          a[2][h] = q1.x, a[2][h + 2] = q1.y, a[3][h] = q1.z, a[3][h + 2] = q1.w;
+        } else {
+          uint2 w2 = make_uint2(0, 0);
+          uint32_t w1 = 0;
+          if (ok) {
+            w2 = *reinterpret_cast<const uint2*>(hb + lane * p0 + 8 * grp);
+            if (BITS == 3) w1 = *reinterpret_cast<const uint32_t*>(hb + 4 * nh * p0 + lane * (4 * ngrp) + 4 * grp);
+          }
+#pragma unroll
+          for (int s = 0; s < 4; ++s)
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+              uint32_t r = reg_shift2((s >> 1) ? w2.y : w2.x, 2 * (s & 1) + hh);
+              if (BITS == 3) r |= v_reg_hi3(w1, s, hh);
+              a[s][h + 2 * hh] = r;
+            }
+        }
+      }
+    }
+    int C[NPAIR][4];
+#pragma unroll
+    for (int pr = 0; pr < NPAIR; ++pr) {
+      C[pr][0] = C[pr][1] = C[pr][2] = C[pr][3] = 0;
+#pragma unroll
+      for (int s = 0; s < 4; ++s) mma_u8s8(C[pr], a[s][0], a[s][1], a[s][2], a[s][3], bw[pr][2 * s], bw[pr][2 * s + 1]);
+    }
+    // per-group scale and zero of rows g and g+8; 2-bit full blocks carry the weight 4^grp
+    const float w = (BITS == 2 && FULL) ? (float)(1 << (2 * grp)) : 1.f;
+    const __half2 m0 = *reinterpret_cast<const __half2*>(&mt.x);
+    const __half2 m1 = *reinterpret_cast<const __half2*>(&mt.y);
+    const float sA = __low2float(m0) * (1.f / w), zA = __high2float(m0) * w;
+    const float sB = __low2float(m1) * (1.f / w), zB = __high2float(m1) * w;
+    v_epi<(NTOK > 1)>(acc[0], C[0], sA, zA, sB, zB, xs[0], NTOK > 1 ? xs[NTOK > 1 ? 1 : 0] : 0.f);
+    if (NPAIR > 1)
+      v_epi<(NTOK > 3)>(acc[1], C[NPAIR - 1], sA, zA, sB, zB, xs[NTOK > 2 ? 2 : 0], NTOK > 3 ? xs[NTOK > 3 ? 3 : 0] : 0.f);
+  }
+}
+
+template <int BITS, int NTOK>
+__device__ __forceinline__ void v_block_dispatch_ngrp(bool full, int rows, int ngrp, const uint8_t* A,
+                                                      const uint8_t* X, float (&acc)[2][4], int lane) {
+  if (full)
+    v_block<BITS, NTOK, true>(rows, 4, A, X, acc, lane);
+  else
+    v_block<BITS, NTOK, false>(rows, ngrp, A, X, acc, lane);
 }
 
 template <int BITS>
-__device__ void v_item(const DcFwd& F, const WsPtr& P, const VCtx& c, int lane) {
-  const DcLayout& L = *c.L;
-  const DcBand& B = L.band[c.band];
-  const int g = lane >> 2, t = lane & 3;
-  const int T = F.ws.T, maxd = F.ws.max_d_in, G = maxd / 128;
-  const int npair = (c.ntok + 1) >> 1;
-  // B operand: lane g < 6 supplies limb g>>1 of token (g&1) of each pair
-  const int limb = g >> 1;
-  const int8_t* xsrc[2];
-  bool xval[2];
-#pragma unroll
-  for (int pr = 0; pr < 2; ++pr) {
-    const int tk = 2 * pr + (g & 1);
-    xval[pr] = (g < 6) && (tk < c.ntok);
-    xsrc[pr] = P.xl + ((int64_t)(c.m * 3 + (g < 6 ? limb : 0)) * T + c.tok0 + (xval[pr] ? tk : 0)) * maxd + 32 * t;
+__device__ __forceinline__ void v_block_dispatch(int ntok, bool full, int rows, int ngrp, const uint8_t* A,
+                                                 const uint8_t* X, float (&acc)[2][4], int lane) {
+  switch (ntok) {
+    case 1: v_block_dispatch_ngrp<BITS, 1>(full, rows, ngrp, A, X, acc, lane); break;
+    case 2: v_block_dispatch_ngrp<BITS, 2>(full, rows, ngrp, A, X, acc, lane); break;
+    case 3: v_block_dispatch_ngrp<BITS, 3>(full, rows, ngrp, A, X, acc, lane); break;
+    default: v_block_dispatch_ngrp<BITS, 4>(full, rows, ngrp, A, X, acc, lane); break;
   }
-  const int* xsp[2][2];
-  bool xsv[2][2];
-#pragma unroll
-  for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const int tk = 2 * pr + q;
-      xsv[pr][q] = (t < 3) && (tk < c.ntok);
-      xsp[pr][q] = P.xs + ((int64_t)(c.m * T + c.tok0 + (xsv[pr][q] ? tk : 0)) * G) * 4 + (t < 3 ? t : 0);
-    }
-  float acc[DC_V_NT][2][4];
-#pragma unroll
-  for (int a = 0; a < DC_V_NT; ++a)
-#pragma unroll
-    for (int b = 0; b < 2; ++b)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) acc[a][b][q] = 0.f;
-  int rows[DC_V_NT], nh[DC_V_NT][2];
-  const uint8_t* tb[DC_V_NT];
-#pragma unroll
-  for (int ti = 0; ti < DC_V_NT; ++ti) {
-    const int tile = c.tile0 + ti;
-    rows[ti] = ti < c.ntiles ? min(16, B.rank - 16 * tile) : 0;
-    nh[ti][0] = min(rows[ti], 8);
-    nh[ti][1] = max(0, rows[ti] - 8);
-    tb[ti] = c.blob + B.v_off + (int64_t)tile * B.v_tile_bytes;
-  }
-  const uint8_t* vmeta = c.blob + B.v_meta_off;
-  for (int kb = 0; kb < L.nkb; ++kb) {
-    const int ngrp = (kb == L.nkb - 1) ? L.tail_groups : 4;
-    const bool mask_layout = (BITS == 2) && (ngrp == 4);
-    uint4 wm[DC_V_NT][2][2];  // 2-bit mask layout: 8 words per lane-row for the block
-    if (mask_layout) {
-#pragma unroll
-      for (int ti = 0; ti < DC_V_NT; ++ti)
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          if (g < nh[ti][h]) {
-            const uint8_t* pp = tb[ti] + (int64_t)kb * dc_v_block_bytes(2, rows[ti], 4) +
-                                dc_v_half_off(2, rows[ti], 4, h) + lane * 32;
-            wm[ti][h][0] = ldg128(pp);
-            wm[ti][h][1] = ldg128(pp + 16);
-          } else {
-            wm[ti][h][0] = make_uint4(0, 0, 0, 0);
-            wm[ti][h][1] = make_uint4(0, 0, 0, 0);
-          }
-        }
-    }
-    for (int grp = 0; grp < ngrp; ++grp) {
-      const int gi = 4 * kb + grp;
-      uint32_t bw[2][8];
-#pragma unroll
-      for (int pr = 0; pr < 2; ++pr) {
-        if (xval[pr]) {
-          const uint4 q0 = ldg128(xsrc[pr] + gi * 128), q1 = ldg128(xsrc[pr] + gi * 128 + 16);
-          bw[pr][0] = q0.x, bw[pr][1] = q0.y, bw[pr][2] = q0.z, bw[pr][3] = q0.w;
-          bw[pr][4] = q1.x, bw[pr][5] = q1.y, bw[pr][6] = q1.z, bw[pr][7] = q1.w;
-        } else {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) bw[pr][q] = 0u;
-        }
-      }
-      int xs[2][2];
-#pragma unroll
-      for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
-        for (int q = 0; q < 2; ++q) xs[pr][q] = xsv[pr][q] ? xsp[pr][q][gi * 4] : 0;
-#pragma unroll
-      for (int ti = 0; ti < DC_V_NT; ++ti) {
-        if (ti >= c.ntiles) continue;
-        const uint2 meta = ldg64(vmeta + (((int64_t)(c.tile0 + ti) * L.groups_in + gi) * 8 + g) * 8);
-        // the lane-row words for this group (shift layouts and 8-bit load per group)
-        uint32_t a[4][4];  // [step][reg]
-        if (mask_layout) {
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            a[s][0] = v_reg_mask2(wsel(wm[ti][0][s >> 1], 2 * (s & 1)), grp);
-            a[s][1] = v_reg_mask2(wsel(wm[ti][1][s >> 1], 2 * (s & 1)), grp);
-            a[s][2] = v_reg_mask2(wsel(wm[ti][0][s >> 1], 2 * (s & 1) + 1), grp);
-            a[s][3] = v_reg_mask2(wsel(wm[ti][1][s >> 1], 2 * (s & 1) + 1), grp);
-          }
-        } else {
-          const uint8_t* blk = tb[ti] + (int64_t)kb * dc_v_block_bytes(BITS, rows[ti], 4);
-          const int p0 = dc_v_plane0_bytes(BITS, ngrp);
-#pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            const bool ok = g < nh[ti][h];
-            const uint8_t* hb = blk + dc_v_half_off(BITS, rows[ti], ngrp, h);
-            if (BITS == 8) {
-              uint4 q0 = make_uint4(0, 0, 0, 0), q1 = q0;
-              if (ok) {
-                q0 = ldg128(hb + lane * p0 + 32 * grp);
-                q1 = ldg128(hb + lane * p0 + 32 * grp + 16);
-              }
-#pragma unroll
-              for (int s = 0; s < 4; ++s) {
-                const uint4& q = (s < 2) ? q0 : q1;
-                a[s][h] = wsel(q, 2 * (s & 1));
-                a[s][h + 2] = wsel(q, 2 * (s & 1) + 1);
-              }
-            } else {
-              uint2 w2 = make_uint2(0, 0);
-              uint32_t w1 = 0;
-              if (ok) {
-                w2 = ldg64(hb + lane * p0 + 8 * grp);
-                if (BITS == 3) w1 = ldg32(hb + (int64_t)4 * nh[ti][h] * p0 + lane * (4 * ngrp) + 4 * grp);
-              }
-#pragma unroll
-              for (int s = 0; s < 4; ++s)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                  const uint32_t w = (s >> 1) ? w2.y : w2.x;
-                  uint32_t r = reg_shift2(w, 2 * (s & 1) + hh);
-                  if (BITS == 3) r |= v_reg_hi3(w1, s, hh);
-                  a[s][h + 2 * hh] = r;
-                }
-            }
-          }
-        }
-        int C[2][4];
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
-          for (int q = 0; q < 4; ++q) C[pr][q] = 0;
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          mma_u8s8(C[0], a[s][0], a[s][1], a[s][2], a[s][3], bw[0][2 * s], bw[0][2 * s + 1]);
-          if (npair > 1) mma_u8s8(C[1], a[s][0], a[s][1], a[s][2], a[s][3], bw[1][2 * s], bw[1][2 * s + 1]);
-        }
-        const float w = mask_layout ? (float)(1 << (2 * grp)) : 1.f;
-        v_group_epilogue(acc[ti], C, meta, w, xs, npair);
-      }
-    }
-  }
-  // combine the three limbs (lane t holds limb t), scale by 2^-e and S, store t
-  const float lw = (float)(1 << (8 * min(t, 2)));
-  const float* S = reinterpret_cast<const float*>(c.blob);
-#pragma unroll
-  for (int ti = 0; ti < DC_V_NT; ++ti)
-#pragma unroll
-    for (int pr = 0; pr < 2; ++pr)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v = t < 3 ? acc[ti][pr][q] * lw : 0.f;
-        v += __shfl_xor_sync(FULLMASK, v, 1);
-        v += __shfl_xor_sync(FULLMASK, v, 2);
-        const int row = g + 8 * (q >> 1);
-        const int tk = 2 * pr + (q & 1);
-        const int rowb = 16 * (c.tile0 + ti) + row;
-        if (t == 0 && ti < c.ntiles && row < rows[ti] && tk < c.ntok) {
-          const int rank = B.r0 + rowb;
-          const int tok = c.tok0 + tk;
-          const int e = P.xe[c.m * T + tok];
-          P.tws[((int64_t)c.p * T + tok) * F.ws.r_stride + rank] = ldexpf(v, -e) * S[rank];
-        }
-      }
 }
 
-__global__ void __launch_bounds__(256) k_vstage(const __grid_constant__ DcFwd F, uint8_t* ws) {
+__device__ __forceinline__ uint4 ldg128_item(const DcVItem* it, int lane) {
+  return ldg128(reinterpret_cast<const uint8_t*>(it) + 16 * lane);
+}
+
+__global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  extern __shared__ __align__(128) uint8_t vsm[];
+  VSmemTail* tail = reinterpret_cast<VSmemTail*>(vsm + V_STAGES * V_STAGE_BYTES);
   WsPtr P = ws_ptr(F.ws, ws);
-  const int lane = threadIdx.x & 31;
-  const int nitems = P.st[DC_WS_NITEMS];
-  for (;;) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < V_STAGES; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], V_CONSUMERS);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  const int T = F.ws.T;
+  if (warp == V_CONSUMERS) {
+    // ---------------- producer warp
+    const int nitems = P.st[DC_WS_NITEMS];
+    uint32_t seq = 0;
     int it = 0;
     if (lane == 0) it = atomicAdd(P.st + DC_WS_VCOUNTER, 1);
     it = __shfl_sync(FULLMASK, it, 0);
-    if (it >= nitems) break;
-    const DcVItem I = P.items[it];
-    const int tau = P.segs[3 * I.seg], st = P.segs[3 * I.seg + 1], len = P.segs[3 * I.seg + 2];
-    const DcLayout* L = P.layouts + I.p * F.ws.max_tenants + tau;
-    VCtx c;
-    c.blob = reinterpret_cast<const uint8_t*>(L->dev_base);
-    c.L = L;
-    c.band = I.band;
-    c.tile0 = I.tile0;
-    c.ntiles = I.ntiles;
-    c.tok0 = st + DC_V_TOKS * I.pass;
-    c.ntok = min(DC_V_TOKS, len - DC_V_TOKS * I.pass);
-    c.m = F.lin[I.p].input;
-    c.p = I.p;
-    const int bits = L->band[I.band].bits;
-    if (bits == 2)
-      v_item<2>(F, P, c, lane);
-    else if (bits == 3)
-      v_item<3>(F, P, c, lane);
-    else
-      v_item<8>(F, P, c, lane);
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// k_ustage: y = W_base x + sum over segments of U_hat (scale * t), one CTA per (linear, 128-row
-// output tile, 64-token block); warp w owns rows 16w..16w+15 of the tile.
-// ---------------------------------------------------------------------------------------------
-#define U_KC 128
-#define U_XROW (U_KC + 8)  // padded bf16 row of the staged activations
-
-struct USmem {
-  int exps[DC_V_TOKS];
-  int zc[2][3][2];
-  float red[8][DC_V_TOKS];
-};
-
-__device__ __forceinline__ void cp_async16(void* smem, const void* gmem) {
-  const unsigned s = (unsigned)__cvta_generic_to_shared(smem);
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(s), "l"(gmem));
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;\n" ::); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-  asm volatile("cp.async.wait_group %0;\n" ::"n"(N));
-}
-
-__device__ void u_base_bf16(const DcFwd& F, const DcLinDev& lin, const int* perm, int ot, int tb, int Tb,
-                            __nv_bfloat16* xst, float (&acc)[8][4]) {
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
-  const int d_in = lin.d_in;
-  const __nv_bfloat16* X = (const __nv_bfloat16*)F.x[lin.input];
-  const __nv_bfloat16* Wm = (const __nv_bfloat16*)lin.W;
-  const int row = ot * 128 + 16 * w + g;
-  const __nv_bfloat16* wr0 = Wm + (int64_t)row * d_in + 8 * t;
-  const __nv_bfloat16* wr1 = wr0 + (int64_t)8 * d_in;
-  const int nkc = d_in / U_KC;
-  const int ntv = (Tb + 7) >> 3;
-  auto stage = [&](int kc, int buf) {
-    __nv_bfloat16* dst = xst + buf * 64 * U_XROW;
-    for (int idx = tid; idx < 64 * (U_KC / 8); idx += blockDim.x) {
-      const int tok = idx / (U_KC / 8), cc = idx % (U_KC / 8);
-      if (tok < Tb) cp_async16(dst + tok * U_XROW + 8 * cc, X + (int64_t)perm[tb + tok] * d_in + kc * U_KC + 8 * cc);
-    }
-    cp_async_commit();
-  };
-  stage(0, 0);
-  for (int kc = 0; kc < nkc; ++kc) {
-    uint4 wa[4], wb[4];
-#pragma unroll
-    for (int k32 = 0; k32 < 4; ++k32) {
-      wa[k32] = ldg128(wr0 + kc * U_KC + 32 * k32);
-      wb[k32] = ldg128(wr1 + kc * U_KC + 32 * k32);
-    }
-    if (kc + 1 < nkc) {
-      stage(kc + 1, (kc + 1) & 1);
-      cp_async_wait<1>();
-    } else {
-      cp_async_wait<0>();
-    }
-    __syncthreads();
-    const __nv_bfloat16* xb = xst + (kc & 1) * 64 * U_XROW;
-    // Each 128-column chunk is summed in a fresh MMA chain and added to the running sum with an
-    // IEEE fp32 add, so the tensor core's internal accumulation rounding spans 8 steps, not d_in/16.
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      if (nt < ntv) {
-        float part[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int k32 = 0; k32 < 4; ++k32) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(xb + (8 * nt + g) * U_XROW + 32 * k32 + 8 * t);
-          mma_bf16(part, wa[k32].x, wb[k32].x, wa[k32].y, wb[k32].y, xv.x, xv.y);
-          mma_bf16(part, wa[k32].z, wb[k32].z, wa[k32].w, wb[k32].w, xv.z, xv.w);
+    uint4 pf = make_uint4(0, 0, 0, 0);
+    if (it < nitems && lane < 4) pf = ldg128_item(P.items + it, lane);
+    for (;;) {
+      // current record <- prefetched one; start fetching the next
+      __syncwarp();
+      if (lane < 4) reinterpret_cast<uint4*>(&tail->rec[0])[lane] = pf;
+      __syncwarp();
+      const bool end = it >= nitems;
+      int nx = 0;
+      if (!end) {
+        if (lane == 0) nx = atomicAdd(P.st + DC_WS_VCOUNTER, 1);
+        nx = __shfl_sync(FULLMASK, nx, 0);
+        if (nx < nitems && lane < 4) pf = ldg128_item(P.items + nx, lane);
+      }
+      const DcVItem& I = tail->rec[0];
+      const int nkb = end ? 1 : I.nkb;
+      for (int kb = 0; kb < nkb; ++kb) {
+        const int s = seq % V_STAGES;
+        if (seq >= V_STAGES && !mbar_wait(&tail->empty[s], ((seq / V_STAGES) - 1) & 1)) {
+          set_status(P.st, DC_ERR_CUDA);
+          return;
         }
+        fence_proxy_async();
+        uint8_t* stage = vsm + (size_t)s * V_STAGE_BYTES;
+        if (end) {
+          if (lane == 0) {
+            tail->desc[s].kind = 1;
+            mbar_arrive(&tail->full[s]);
+          }
+          return;
+        }
+        const int ngrp = (kb == I.nkb - 1) ? I.tail_groups : 4;
+        const int last_rows = min(16, I.rows_left - 16 * (I.ntiles - 1));
+        const uint32_t code_bytes = (uint32_t)((I.ntiles - 1) * dc_v_block_bytes(I.bits, 16, ngrp) +
+                                               dc_v_block_bytes(I.bits, last_rows, ngrp));
+        const uint32_t total = code_bytes + (uint32_t)(I.ntok * DC_XBLK);
+        if (lane == 0) {
+          VDesc& d = tail->desc[s];
+          d.kind = 0;
+          d.bits = I.bits;
+          d.rows_left = I.rows_left;
+          d.ntiles = I.ntiles;
+          d.tok0 = I.tok0;
+          d.ntok = I.ntok;
+          d.m = I.m;
+          d.p = I.p;
+          d.kb = kb;
+          d.ngrp = ngrp;
+          d.first = kb == 0;
+          d.last = kb == I.nkb - 1;
+          d.rank0 = I.rank0;
+          d.sbase = I.sbase;
+          mbar_arrive_expect_tx(&tail->full[s], total);
+        }
+        __syncwarp();
+        if (lane == 0) {
+          bulk_g2s(stage, reinterpret_cast<const uint8_t*>(I.vbase) + (int64_t)kb * I.f4, code_bytes, &tail->full[s]);
+        } else if (lane <= I.ntok) {
+          const int k = lane - 1;
+          const uint8_t* src = P.xl + ((int64_t)(I.m * T + I.tok0 + k) * F.ws.nkb + kb) * DC_XBLK;
+          bulk_g2s(stage + V_A_BYTES + k * V_XTOK, src, DC_XBLK, &tail->full[s]);
+        }
+        ++seq;
+      }
+      it = nx;
+    }
+  }
+  // ---------------- consumer warps
+  uint32_t seq = 0;
+  float acc[2][4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) acc[nt][q] += part[q];
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
+  const int g = lane >> 2, t = lane & 3;
+  for (;;) {
+    const int s = seq % V_STAGES;
+    if (!mbar_wait(&tail->full[s], (seq / V_STAGES) & 1)) {
+      set_status(P.st, DC_ERR_CUDA);
+      return;
+    }
+    const VDesc d = tail->desc[s];
+    if (d.kind == 1) return;
+    const uint8_t* stage = vsm + (size_t)s * V_STAGE_BYTES;
+    if (warp < d.ntiles) {
+      if (d.first) {
+#pragma unroll
+        for (int a = 0; a < 2; ++a)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
+      }
+      const int rows = min(16, d.rows_left - 16 * warp);
+      const uint8_t* A = stage + warp * dc_v_block_bytes(d.bits, 16, d.ngrp);
+      const uint8_t* X = stage + V_A_BYTES;
+      const bool full = d.ngrp == 4;
+      if (d.bits == 2)
+        v_block_dispatch<2>(d.ntok, full, rows, d.ngrp, A, X, acc, lane);
+      else if (d.bits == 3)
+        v_block_dispatch<3>(d.ntok, full, rows, d.ngrp, A, X, acc, lane);
+      else
+        v_block_dispatch<8>(d.ntok, full, rows, d.ngrp, A, X, acc, lane);
+      if (d.last) {
+        // combine the three limbs (lane t holds limb t), scale by 2^-e and S, store t
+        const float lw = (float)(1 << (8 * min(t, 2)));
+        const float* S = reinterpret_cast<const float*>(d.sbase);
+#pragma unroll
+        for (int pr = 0; pr < 2; ++pr)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            float v = t < 3 ? acc[pr][q] * lw : 0.f;
+            v += __shfl_xor_sync(FULLMASK, v, 1);
+            v += __shfl_xor_sync(FULLMASK, v, 2);
+            const int row = g + 8 * (q >> 1);
+            const int tk = 2 * pr + (q & 1);
+            if (t == 0 && row < rows && tk < d.ntok) {
+              const int rl = 16 * warp + row;  // row within the item
+              const int tok = d.tok0 + tk;
+              const int e = P.xe[d.m * T + tok];
+              P.tws[((int64_t)d.p * T + tok) * F.ws.r_stride + d.rank0 + rl] = ldexpf(v, -e) * S[rl];
+            }
+          }
       }
     }
-    __syncthreads();
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tail->empty[s]);
+    ++seq;
   }
 }
 
-// fp32 backbone (small fp32 layers): plain FFMA in the same fragment layout.
-__device__ void u_base_f32(const DcFwd& F, const DcLinDev& lin, const int* perm, int ot, int tb, int Tb,
-                           float (&acc)[8][4]) {
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5, g = lane >> 2, t = lane & 3;
+// ---------------------------------------------------------------------------------------------
+// k_udelta: ydelta[token, row] = (U_hat (scale * t))[row] for every token of every segment with a
+// delta.  Persistent CTAs of 8 consumer warps + 1 producer warp over items (linear, segment,
+// 128-row output group); segments partition the tokens, so items write disjoint outputs.  Per
+// 4-token pass the producer streams the item's U_hat codes of every band, the U meta of its
+// 128-row group and the pass's t rows into a shared-memory stage; consumer warp w owns rows
+// 16w..16w+15 of the group.
+// ---------------------------------------------------------------------------------------------
+#define U_STAGES 2
+#define U_STAGE_BYTES (100 * 1024)
+#define U_CONSUMERS 8
+#define U_THREADS (32 * (U_CONSUMERS + 1))
+
+struct UBandD {
+  int bits, rank, r0, bsm_off, quads, steps, last, otile, off;
+};
+struct UDesc {
+  int kind;  // 1 delta pass, 2 end
+  int p, ot, tok0, ntok;
+  int n_bands, r, off_meta, off_t, tstride, error;
+  UBandD band[DC_MAX_BANDS];
+};
+
+struct USmemTail {
+  UDesc desc[U_STAGES];
+  uint64_t full[U_STAGES];
+  uint64_t empty[U_STAGES];
+  DcURec rec;  // producer: record of the current segment
+  int exps[DC_V_TOKS];
+  int zc[2][3][2];
+  float red[U_CONSUMERS][DC_V_TOKS];
+};
+
+// item u -> (linear p, segment sg, output group ot); linears in F.order, segment-major inside a linear
+__device__ __forceinline__ bool ud_item(const DcFwd& F, int nseg, int u, int& p, int& sg, int& ot) {
+  for (int i = 0; i < F.n_lin; ++i) {
+    const int q = F.order[i];
+    const int n_ot = F.lin[q].d_out / 128;
+    const int cnt = nseg * n_ot;
+    if (u < cnt) {
+      p = q;
+      sg = u / n_ot;
+      ot = u % n_ot;
+      return true;
+    }
+    u -= cnt;
+  }
+  return false;
+}
+
+template <int NTOK>
+__device__ __forceinline__ void ud_pass(const DcFwd& F, const WsPtr& P, const UDesc& d, const uint8_t* stage,
+                                        uint8_t* bsm, USmemTail* tail, int warp, int lane) {
+  constexpr int NPAIR = (NTOK + 1) / 2;
+  const int tid = threadIdx.x;  // 0..255
+  const int g = lane >> 2, t = lane & 3;
+  const uint8_t* umeta = stage + d.off_meta;
+  const float* tst = reinterpret_cast<const float*>(stage + d.off_t);
+  const int T = F.ws.T;
+  // ---- B = scale * t: per-token exponent from the largest |B| over the 2/3-bit bands
+  float mx[NTOK];
+#pragma unroll
+  for (int q = 0; q < NTOK; ++q) mx[q] = 0.f;
+  for (int b = 0; b < d.n_bands; ++b) {
+    const UBandD& Bd = d.band[b];
+    if (Bd.bits == 8) continue;
+    for (int i = tid; i < Bd.rank; i += 32 * U_CONSUMERS) {
+      const int r = Bd.r0 + i;
+      const float sc = __low2float(*reinterpret_cast<const __half2*>(umeta + 4 * r));
+#pragma unroll
+      for (int q = 0; q < NTOK; ++q) mx[q] = fmaxf(mx[q], fabsf(sc * tst[q * d.tstride + r]));
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < NTOK; ++q) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) mx[q] = fmaxf(mx[q], __shfl_xor_sync(FULLMASK, mx[q], o));
+    if (lane == 0) tail->red[warp][q] = mx[q];
+  }
+  if (tid < 12) (&tail->zc[0][0][0])[tid] = 0;
+  named_bar(1, 32 * U_CONSUMERS);
+  if (tid < NTOK) {
+    float m = 0.f;
+#pragma unroll
+    for (int ww = 0; ww < U_CONSUMERS; ++ww) m = fmaxf(m, tail->red[ww][tid]);
+    int e = 0;
+    if (m > 0.f) {
+      int E;
+      frexpf(m, &E);
+      e = 22 - E;
+    }
+    tail->exps[tid] = e;
+  }
+  named_bar(1, 32 * U_CONSUMERS);
+  // ---- limbs of B into the staging buffer, 4 consecutive ranks per thread (ranks past the band's
+  //      end up to its 32-rank padding are written as zeros); zero-point correction sums
+  int zc[NPAIR][3][2];
+#pragma unroll
+  for (int a = 0; a < NPAIR; ++a)
+#pragma unroll
+    for (int b = 0; b < 3; ++b) zc[a][b][0] = zc[a][b][1] = 0;
+  float pe[NTOK];
+#pragma unroll
+  for (int q = 0; q < NTOK; ++q) pe[q] = ldexpf(1.f, tail->exps[q]);
+  for (int b = 0; b < d.n_bands; ++b) {
+    const UBandD& Bd = d.band[b];
+    if (Bd.bits == 8) continue;
+    const int padded = (Bd.rank + 31) & ~31;
+    for (int i4 = 4 * tid; i4 < padded; i4 += 4 * 32 * U_CONSUMERS) {
+      float sc[4];
+      int z[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        const bool ok = i4 + c < Bd.rank;
+        const __half2 mz = *reinterpret_cast<const __half2*>(umeta + 4 * (Bd.r0 + (ok ? i4 + c : 0)));
+        sc[c] = ok ? __low2float(mz) : 0.f;
+        z[c] = ok ? (int)__high2float(mz) : 0;
+      }
+#pragma unroll
+      for (int q = 0; q < NTOK; ++q) {
+        uint32_t w0 = 0, w1 = 0, w2 = 0;
+        const int pr = q >> 1, tk = q & 1;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int rr = Bd.r0 + (i4 + c < Bd.rank ? i4 + c : 0);
+          const int bi = __float2int_rn(sc[c] * tst[q * d.tstride + rr] * pe[q]);
+          const int l0 = sext8(bi);
+          const int x1 = (bi - l0) >> 8;
+          const int l1 = sext8(x1);
+          const int l2 = (x1 - l1) >> 8;
+          w0 |= (uint32_t)(l0 & 0xff) << (8 * c);
+          w1 |= (uint32_t)(l1 & 0xff) << (8 * c);
+          w2 |= (uint32_t)(l2 & 0xff) << (8 * c);
+          zc[pr][0][tk] += z[c] * l0;
+          zc[pr][1][tk] += z[c] * l1;
+          zc[pr][2][tk] += z[c] * l2;
+        }
+        uint8_t* col = bsm + (int64_t)(pr * 6) * F.bsm_max + Bd.bsm_off + i4;
+        *reinterpret_cast<uint32_t*>(col + (0 * 2 + tk) * F.bsm_max) = w0;
+        *reinterpret_cast<uint32_t*>(col + (1 * 2 + tk) * F.bsm_max) = w1;
+        *reinterpret_cast<uint32_t*>(col + (2 * 2 + tk) * F.bsm_max) = w2;
+      }
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < NPAIR; ++a)
+#pragma unroll
+    for (int b = 0; b < 3; ++b)
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        if (2 * a + k >= NTOK) continue;
+        int v = zc[a][b][k];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
+        if (lane == 0 && v != 0) atomicAdd(&tail->zc[a][b][k], v);
+      }
+  named_bar(1, 32 * U_CONSUMERS);
+  // ---- MMA over the rank steps of every 2/3-bit band (codes of this warp's 16 rows)
+  int C[NPAIR][4][4];  // [pair][position][reg]
+#pragma unroll
+  for (int a = 0; a < NPAIR; ++a)
+#pragma unroll
+    for (int b = 0; b < 4; ++b)
+#pragma unroll
+      for (int q = 0; q < 4; ++q) C[a][b][q] = 0;
+  float s8v[NPAIR];  // 8-bit band contribution of lane t: (row g + 8*(t>>1), token t&1) per pair
+#pragma unroll
+  for (int a = 0; a < NPAIR; ++a) s8v[a] = 0.f;
+  const bool bl = g < 6;  // B columns 2*limb + token; columns 6 and 7 are zero
+  for (int b = 0; b < d.n_bands; ++b) {
+    const UBandD& Bd = d.band[b];
+    if (Bd.bits == 8) {
+      const int row = g + 8 * (t >> 1);
+      const uint8_t* ur = stage + Bd.off + (16 * warp + row) * Bd.rank;
+#pragma unroll
+      for (int pr = 0; pr < NPAIR; ++pr) {
+        const int q = 2 * pr + (t & 1);
+        if (q >= NTOK) continue;
+        float sum = 0.f;
+        for (int i = 0; i < Bd.rank; ++i) {
+          const __half2 mz = *reinterpret_cast<const __half2*>(umeta + 4 * (Bd.r0 + i));
+          sum = fmaf(((float)ur[i] - __high2float(mz)) * __low2float(mz), tst[q * d.tstride + Bd.r0 + i], sum);
+        }
+        s8v[pr] += sum;
+      }
+      continue;
+    }
+    const uint8_t* ub = stage + Bd.off + (int64_t)warp * Bd.otile;
+    const uint8_t* bcol = bsm + (int64_t)(bl ? g : 0) * F.bsm_max + Bd.bsm_off + 8 * t;
+#pragma unroll 2
+    for (int q = 0; q < Bd.quads; ++q) {
+      const uint4 wq = *reinterpret_cast<const uint4*>(ub + 512 * q + 16 * lane);
+#pragma unroll
+      for (int ps = 0; ps < 4; ++ps) {
+        const int step = 4 * q + ps;
+        const uint32_t msk = 0x03030303u << (2 * ps);
+        const uint32_t a0 = wq.x & msk, a1 = wq.y & msk, a2 = wq.z & msk, a3 = wq.w & msk;
+#pragma unroll
+        for (int pr = 0; pr < NPAIR; ++pr) {
+          const uint2 bb = bl ? *reinterpret_cast<const uint2*>(bcol + (int64_t)(6 * pr) * F.bsm_max + 32 * step)
+                              : make_uint2(0, 0);
+          mma_u8s8(C[pr][ps], a0, a1, a2, a3, bb.x, bb.y);
+        }
+      }
+    }
+    const uint8_t* sb = ub + (int64_t)512 * Bd.quads;
+    for (int sidx = 0; sidx < Bd.steps; ++sidx) {
+      const int valid = (sidx == Bd.steps - 1) ? Bd.last : 32;
+      const int nl = dc_u_step_lanes(valid);
+      const int ntv = nl / 8;
+      uint32_t wv = 0, hv = 0;
+      if (t < ntv) {
+        wv = *reinterpret_cast<const uint32_t*>(sb + 4 * (g * ntv + t));
+        if (Bd.bits == 3) hv = *reinterpret_cast<const uint16_t*>(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t));
+      }
+      uint32_t a[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        a[j] = reg_shift2(wv, j);
+        if (Bd.bits == 3) a[j] |= u_reg_hi3(hv, j);
+      }
+      const int step = 4 * Bd.quads + sidx;
+#pragma unroll
+      for (int pr = 0; pr < NPAIR; ++pr) {
+        const uint2 bb = bl ? *reinterpret_cast<const uint2*>(bcol + (int64_t)(6 * pr) * F.bsm_max + 32 * step)
+                            : make_uint2(0, 0);
+        mma_u8s8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
+      }
+      sb += dc_u_step_bytes(Bd.bits, nl);
+    }
+  }
+  // ---- combine positions and limbs (lane t holds limb t of pair tokens 0, 1); write ydelta
+  const float lw = (float)(1 << (8 * min(t, 2)));
+  float* yd = P.yd + (int64_t)d.p * T * F.ws.max_d_in;
+#pragma unroll
+  for (int pr = 0; pr < NPAIR; ++pr)
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int tk = q & 1;
+      const int qq = 2 * pr + tk;
+      if (qq >= NTOK) continue;
+      const int cl = C[pr][0][q] + (C[pr][1][q] >> 2) + (C[pr][2][q] >> 4) + (C[pr][3][q] >> 6);
+      float v = t < 3 ? (float)(cl - tail->zc[pr][t][tk]) * lw : 0.f;
+      v += __shfl_xor_sync(FULLMASK, v, 1);
+      v += __shfl_xor_sync(FULLMASK, v, 2);
+      v = ldexpf(v, -tail->exps[qq]);
+      v += __shfl_sync(FULLMASK, s8v[pr], (lane & ~3) | q);
+      if (t == 0) {
+        const int row = d.ot * 128 + 16 * warp + g + 8 * (q >> 1);
+        yd[(int64_t)(d.tok0 + qq) * F.ws.max_d_in + row] = v;
+      }
+    }
+  named_bar(1, 32 * U_CONSUMERS);  // the staging buffer is reused by the next pass
+}
+
+__global__ void __launch_bounds__(U_THREADS, 1) k_udelta(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  extern __shared__ __align__(128) uint8_t usm[];
+  uint8_t* bsm = usm + U_STAGES * U_STAGE_BYTES;
+  USmemTail* tail = reinterpret_cast<USmemTail*>(bsm + 12 * F.bsm_max);
+  WsPtr P = ws_ptr(F.ws, ws);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = F.ws.T;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < U_STAGES; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], U_CONSUMERS);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == U_CONSUMERS) {
+    // ---------------- producer warp
+    const int nseg = P.st[DC_WS_NSEG];
+    constexpr int REC_VEC = sizeof(DcURec) / 16;
+    uint32_t seq = 0;
+    int cur_p = -1, cur_sg = -1;
+    auto acquire = [&](int& s) -> bool {
+      s = seq % U_STAGES;
+      if (seq >= U_STAGES && !mbar_wait(&tail->empty[s], ((seq / U_STAGES) - 1) & 1)) {
+        set_status(P.st, DC_ERR_CUDA);
+        return false;
+      }
+      fence_proxy_async();
+      return true;
+    };
+    for (;;) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(P.st + DC_WS_UCOUNTER, 1);
+      u = __shfl_sync(FULLMASK, u, 0);
+      int p = 0, sg = 0, ot = 0;
+      if (nseg == 0 || !ud_item(F, nseg, u, p, sg, ot)) {
+        int s;
+        if (!acquire(s)) return;
+        if (lane == 0) {
+          tail->desc[s].kind = 2;
+          mbar_arrive(&tail->full[s]);
+        }
+        return;
+      }
+      if (p != cur_p || sg != cur_sg) {
+        const uint4 v = lane < REC_VEC ? ldg128(reinterpret_cast<const uint8_t*>(P.urecs + (int64_t)p * T + sg) + 16 * lane)
+                                       : make_uint4(0, 0, 0, 0);
+        __syncwarp();
+        if (lane < REC_VEC) reinterpret_cast<uint4*>(&tail->rec)[lane] = v;
+        __syncwarp();
+        cur_p = p, cur_sg = sg;
+      }
+      const DcURec& R = tail->rec;
+      if (!R.valid) continue;
+      const uint8_t* blob = reinterpret_cast<const uint8_t*>(R.blob);
+      for (int pt0 = R.st; pt0 < R.st + R.len; pt0 += DC_V_TOKS) {
+        const int ntok = min(DC_V_TOKS, R.st + R.len - pt0);
+        int s;
+        if (!acquire(s)) return;
+        uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
+        int off = 0;
+        int offb[DC_MAX_BANDS] = {0, 0, 0, 0};
+#pragma unroll
+        for (int b = 0; b < DC_MAX_BANDS; ++b)
+          if (b < R.n_bands) {
+            offb[b] = off;
+            off += R.band[b].region;  // a multiple of 16
+          }
+        const int off_meta = off;
+        off += R.r4 * 4;
+        const int off_t = off;
+        const int tstride = R.r4;
+        off += ntok * tstride * 4;
+        const bool fits = off <= U_STAGE_BYTES;
+        if (lane == 0) {
+          UDesc& d = tail->desc[s];
+          d.kind = 1;
+          d.p = p, d.ot = ot, d.tok0 = pt0, d.ntok = ntok;
+          d.n_bands = R.n_bands, d.r = R.r, d.off_meta = off_meta, d.off_t = off_t, d.tstride = tstride;
+          d.error = fits ? 0 : 1;
+          for (int b = 0; b < DC_MAX_BANDS; ++b) {
+            const DcUBand& B = R.band[b];
+            d.band[b] = UBandD{B.bits, B.rank, B.r0, B.bsm_off, B.quads, B.steps, B.last, B.otile, offb[b]};
+          }
+          if (!fits) set_status(P.st, DC_ERR_UNSUPPORTED);
+          // every region size is a multiple of 16, so `off` is exactly the number of bytes copied
+          if (fits)
+            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)off);
+          else
+            mbar_arrive(&tail->full[s]);
+        }
+        __syncwarp();
+        if (fits) {
+          if (lane < R.n_bands) {
+            const DcUBand& B = R.band[lane];
+            const int64_t src = B.bits == 8 ? B.u_off + (int64_t)ot * 128 * B.rank : B.u_off + (int64_t)ot * 8 * B.otile;
+            bulk_g2s(stage + offb[lane], blob + src, (uint32_t)B.region, &tail->full[s]);
+          } else if (lane == 4) {
+            bulk_g2s(stage + off_meta, blob + R.u_meta_off + (int64_t)ot * R.r4 * 4, (uint32_t)(R.r4 * 4), &tail->full[s]);
+          } else if (lane >= 8 && lane < 8 + ntok) {
+            const int k = lane - 8;
+            bulk_g2s(stage + off_t + k * tstride * 4, P.tws + ((int64_t)p * T + pt0 + k) * F.ws.r_stride,
+                     (uint32_t)(tstride * 4), &tail->full[s]);
+          }
+        }
+        ++seq;
+      }
+    }
+  }
+  // ---------------- consumer warps
+  uint32_t seq = 0;
+  for (;;) {
+    const int s = seq % U_STAGES;
+    if (!mbar_wait(&tail->full[s], (seq / U_STAGES) & 1)) {
+      set_status(P.st, DC_ERR_CUDA);
+      return;
+    }
+    const UDesc& d = tail->desc[s];
+    if (d.kind == 2) return;
+    const uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
+    if (!d.error) {
+      switch (d.ntok) {
+        case 1: ud_pass<1>(F, P, d, stage, bsm, tail, warp, lane); break;
+        case 2: ud_pass<2>(F, P, d, stage, bsm, tail, warp, lane); break;
+        case 3: ud_pass<3>(F, P, d, stage, bsm, tail, warp, lane); break;
+        default: ud_pass<4>(F, P, d, stage, bsm, tail, warp, lane); break;
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tail->empty[s]);
+    ++seq;
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_base: y = W_base x + ydelta, persistent CTAs of 8 consumer warps + 1 producer warp over units
+// (linear, 128-row output tile, 64-token block), largest linears first.  The producer streams
+// 128 x 128 tiles of W_base and 64 x 128 tiles of the tenant-sorted activations with 2-D tensor
+// copies (128-byte swizzle); consumer warp w owns rows 16w..16w+15 and writes the unit's outputs,
+// plus the delta of k_udelta, in the tokens' original order.
+// ---------------------------------------------------------------------------------------------
+#define B_STAGES 4
+#define B_STAGE_BYTES (48 * 1024)  // a multiple of 1024 (128-byte-swizzled tensor tiles)
+#define B_KC 128                   // backbone columns per stage: two 64-column boxes
+#define B_WBOX 16384               // 128 rows x 64 bf16
+#define B_XBOX 8192                // 64 tokens x 64 bf16
+
+struct BDesc {
+  int kind;  // 0 backbone chunk (bf16), 2 end, 3 backbone fp32 (read in place), 4 unit without backbone
+  int first, last;
+  int p, ot, tb, Tb;
+};
+
+struct BSmemTail {
+  BDesc desc[B_STAGES];
+  uint64_t full[B_STAGES];
+  uint64_t empty[B_STAGES];
+};
+
+__device__ __forceinline__ void b_unit_coords(const DcFwd& F, int u, int nTB, int& p, int& ot, int& tb) {
+  int slot = 0;
+  while (slot + 1 < F.n_lin && u >= F.tile_prefix[slot + 1] * nTB) ++slot;
+  p = F.order[slot];
+  const int local = u - F.tile_prefix[slot] * nTB;
+  ot = local / nTB;
+  tb = (local % nTB) * DC_TOK_BLOCK;
+}
+
+// fp32 backbone (small fp32 layers): plain FFMA from global memory in the MMA fragment layout.
+__device__ void b_base_f32(const DcFwd& F, const DcLinDev& lin, const int* perm, int ot, int tb, int Tb, int w,
+                           int lane, float (&acc)[8][4]) {
+  const int g = lane >> 2, t = lane & 3;
   const int d_in = lin.d_in;
   const float* Wm = (const float*)lin.W;
   const int r0 = ot * 128 + 16 * w + g;
@@ -756,256 +1227,169 @@ __device__ void u_base_f32(const DcFwd& F, const DcLinDev& lin, const int* perm,
           s1 = fmaf(w1[k], xv, s1);
         }
       }
-      acc[nt][q] = s0;
-      acc[nt][2 + q] = s1;
+      acc[nt][q] += s0;
+      acc[nt][2 + q] += s1;
     }
   }
 }
 
-__global__ void __launch_bounds__(256, 2) k_ustage(const __grid_constant__ DcFwd F, uint8_t* ws) {
-  extern __shared__ __align__(16) uint8_t usm[];
+__global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  extern __shared__ __align__(1024) uint8_t bsm_raw[];
+  uint8_t* sm = bsm_raw + ((1024 - (smem_u32(bsm_raw) & 1023)) & 1023);  // 1024-aligned for swizzled tiles
+  BSmemTail* tail = reinterpret_cast<BSmemTail*>(sm + B_STAGES * B_STAGE_BYTES);
   WsPtr P = ws_ptr(F.ws, ws);
-  int slot = 0;
-  while (slot + 1 < F.n_lin && (int)blockIdx.x >= F.tile_prefix[slot + 1]) ++slot;
-  const int p = F.order[slot];
-  const int ot = blockIdx.x - F.tile_prefix[slot];
-  const DcLinDev& lin = F.lin[p];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = F.ws.T;
-  const int tb = blockIdx.y * DC_TOK_BLOCK;
-  const int Tb = min(DC_TOK_BLOCK, T - tb);
-  if (Tb <= 0) return;
-  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5, g = lane >> 2, t = lane & 3;
-  // shared memory: [x staging 2 x 64 x U_XROW bf16 | B staging 2 x 8 x bsm_max | yd 8x16x64 f32 | USmem]
-  __nv_bfloat16* xst = reinterpret_cast<__nv_bfloat16*>(usm);
-  uint8_t* bsm = usm + 2 * 64 * U_XROW * 2;
-  float* yd = reinterpret_cast<float*>(bsm + 16 * F.bsm_max);
-  USmem* us = reinterpret_cast<USmem*>(yd + 8 * 16 * DC_TOK_BLOCK);
-  float* ydw = yd + w * 16 * DC_TOK_BLOCK;
-
+  const int nTB = (T + DC_TOK_BLOCK - 1) / DC_TOK_BLOCK;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < B_STAGES; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], U_CONSUMERS);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == U_CONSUMERS) {
+    // ---------------- producer warp
+    const int n_units = F.tile_prefix[F.n_lin] * nTB;
+    uint32_t seq = 0;
+    auto acquire = [&](int& s) -> bool {
+      s = seq % B_STAGES;
+      if (seq >= B_STAGES && !mbar_wait(&tail->empty[s], ((seq / B_STAGES) - 1) & 1)) {
+        set_status(P.st, DC_ERR_CUDA);
+        return false;
+      }
+      fence_proxy_async();
+      return true;
+    };
+    for (;;) {
+      int u = 0;
+      if (lane == 0) u = atomicAdd(P.st + DC_WS_BCOUNTER, 1);
+      u = __shfl_sync(FULLMASK, u, 0);
+      if (u >= n_units) {
+        int s;
+        if (!acquire(s)) return;
+        if (lane == 0) {
+          tail->desc[s].kind = 2;
+          mbar_arrive(&tail->full[s]);
+        }
+        return;
+      }
+      int p, ot, tb;
+      b_unit_coords(F, u, nTB, p, ot, tb);
+      const DcLinDev& lin = F.lin[p];
+      const int Tb = min(DC_TOK_BLOCK, T - tb);
+      const bool base = (F.flags & DC_BASE) != 0;
+      const bool bf16 = lin.w_dtype == DC_DTYPE_BF16;
+      const int nkc = base ? (bf16 ? lin.d_in / B_KC : 1) : 1;
+      for (int kc = 0; kc < nkc; ++kc) {
+        int s;
+        if (!acquire(s)) return;
+        uint8_t* stage = sm + (size_t)s * B_STAGE_BYTES;
+        if (lane == 0) {
+          BDesc& d = tail->desc[s];
+          d.kind = base ? (bf16 ? 0 : 3) : 4, d.first = kc == 0, d.last = kc == nkc - 1;
+          d.p = p, d.ot = ot, d.tb = tb, d.Tb = Tb;
+          if (base && bf16)
+            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)(2 * B_WBOX + 2 * 128 * min(64, T)));
+          else
+            mbar_arrive(&tail->full[s]);
+          if (base && bf16)
+            for (int bx = 0; bx < 2; ++bx) {
+              tma_load_2d(stage + bx * B_WBOX, &F.wmap[p], kc * B_KC + 64 * bx, ot * 128, &tail->full[s]);
+              tma_load_2d(stage + 2 * B_WBOX + bx * B_XBOX, &F.xmap[lin.input], kc * B_KC + 64 * bx, tb,
+                          &tail->full[s]);
+            }
+        }
+        __syncwarp();
+        ++seq;
+      }
+    }
+  }
+  // ---------------- consumer warps
+  const int g = lane >> 2, t = lane & 3;
   float acc[8][4];
 #pragma unroll
   for (int a = 0; a < 8; ++a)
 #pragma unroll
     for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
-  for (int i = tid; i < 8 * 16 * DC_TOK_BLOCK; i += blockDim.x) yd[i] = 0.f;
-  if (F.flags & DC_BASE) {
-    if (lin.w_dtype == DC_DTYPE_BF16)
-      u_base_bf16(F, lin, P.perm, ot, tb, Tb, xst, acc);
-    else
-      u_base_f32(F, lin, P.perm, ot, tb, Tb, acc);
-  }
-  __syncthreads();
-
-  if (F.flags & DC_DELTA) {
-    const int nseg = P.st[DC_WS_NSEG];
-    const int go = ot;  // 128-row output group = quantisation group of the U columns
-    const int orow = ot * 128 + 16 * w;  // first row of this warp
-    for (int s = 0; s < nseg; ++s) {
-      const int tau = P.segs[3 * s], st = P.segs[3 * s + 1], len = P.segs[3 * s + 2];
-      const int s0 = max(st, tb), s1 = min(st + len, tb + Tb);
-      if (s0 >= s1 || tau >= lin.n_tenants || tau >= F.ws.max_tenants) continue;
-      const DcLayout& L = P.layouts[p * F.ws.max_tenants + tau];
-      if (!L.valid) continue;
-      const uint8_t* blob = reinterpret_cast<const uint8_t*>(L.dev_base);
-      const uint8_t* umeta = blob + L.u_meta_off + (int64_t)go * L.r * 4;
-      for (int pt0 = s0; pt0 < s1; pt0 += DC_V_TOKS) {
-        const int ntok = min(DC_V_TOKS, s1 - pt0);
-        const int npair = (ntok + 1) >> 1;
-        const float* tw = P.tws + ((int64_t)p * T + pt0) * F.ws.r_stride;
-        // ---- B = scale * t: per-token exponent from the largest |B| (MMA bands only)
-        float mx[DC_V_TOKS] = {0.f, 0.f, 0.f, 0.f};
-        for (int b = 0; b < L.n_bands; ++b) {
-          const DcBand& Bd = L.band[b];
-          if (Bd.bits == 8) continue;
-          for (int i = tid; i < Bd.rank; i += blockDim.x) {
-            const int r = Bd.r0 + i;
-            const float sc = __low2float(*reinterpret_cast<const __half2*>(umeta + 4 * r));
-#pragma unroll
-            for (int q = 0; q < DC_V_TOKS; ++q)
-              if (q < ntok) mx[q] = fmaxf(mx[q], fabsf(sc * tw[(int64_t)q * F.ws.r_stride + r]));
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < DC_V_TOKS; ++q) {
-#pragma unroll
-          for (int o = 16; o; o >>= 1) mx[q] = fmaxf(mx[q], __shfl_xor_sync(FULLMASK, mx[q], o));
-          if (lane == 0) us->red[w][q] = mx[q];
-        }
-        for (int i = tid; i < 16 * F.bsm_max / 4; i += blockDim.x) reinterpret_cast<uint32_t*>(bsm)[i] = 0u;
-        if (tid < 12) (&us->zc[0][0][0])[tid] = 0;
-        __syncthreads();
-        if (tid < DC_V_TOKS) {
-          float m = 0.f;
-          for (int ww = 0; ww < 8; ++ww) m = fmaxf(m, us->red[ww][tid]);
-          int e = 0;
-          if (m > 0.f) {
-            int E;
-            frexpf(m, &E);
-            e = 22 - E;
-          }
-          us->exps[tid] = e;
-        }
-        __syncthreads();
-        // ---- limbs of B into the staging buffer; zero-point correction sums
-        int zc[2][3][2];
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-          for (int b = 0; b < 3; ++b) zc[a][b][0] = zc[a][b][1] = 0;
-        for (int b = 0; b < L.n_bands; ++b) {
-          const DcBand& Bd = L.band[b];
-          if (Bd.bits == 8) continue;
-          for (int i = tid; i < Bd.rank; i += blockDim.x) {
-            const int r = Bd.r0 + i;
-            const __half2 mz = *reinterpret_cast<const __half2*>(umeta + 4 * r);
-            const float sc = __low2float(mz);
-            const int z = (int)__high2float(mz);
-#pragma unroll
-            for (int q = 0; q < DC_V_TOKS; ++q) {
-              if (q >= ntok) continue;
-              const int bi = __float2int_rn(ldexpf(sc * tw[(int64_t)q * F.ws.r_stride + r], us->exps[q]));
-              const int l0 = sext8(bi);
-              const int x1 = (bi - l0) >> 8;
-              const int l1 = sext8(x1);
-              const int l2 = (x1 - l1) >> 8;
-              const int pr = q >> 1, tk = q & 1;
-              uint8_t* col = bsm + (int64_t)(pr * 8) * F.bsm_max + Bd.bsm_off + i;
-              col[(0 * 2 + tk) * F.bsm_max] = (uint8_t)(l0 & 0xff);
-              col[(1 * 2 + tk) * F.bsm_max] = (uint8_t)(l1 & 0xff);
-              col[(2 * 2 + tk) * F.bsm_max] = (uint8_t)(l2 & 0xff);
-              zc[pr][0][tk] += z * l0;
-              zc[pr][1][tk] += z * l1;
-              zc[pr][2][tk] += z * l2;
-            }
-          }
-        }
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-          for (int b = 0; b < 3; ++b)
-#pragma unroll
-            for (int k = 0; k < 2; ++k) {
-              int v = zc[a][b][k];
-#pragma unroll
-              for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
-              if (lane == 0 && v != 0) atomicAdd(&us->zc[a][b][k], v);
-            }
-        __syncthreads();
-        // ---- MMA over the rank steps of every 2/3-bit band
-        int C[2][4][4];  // [pair][position][reg]
-#pragma unroll
-        for (int a = 0; a < 2; ++a)
-#pragma unroll
-          for (int b = 0; b < 4; ++b)
-#pragma unroll
-            for (int q = 0; q < 4; ++q) C[a][b][q] = 0;
-        for (int b = 0; b < L.n_bands; ++b) {
-          const DcBand& Bd = L.band[b];
-          if (Bd.bits == 8) continue;
-          const uint8_t* ub = blob + Bd.u_off + (int64_t)(ot * 8 + w) * Bd.u_otile_bytes;
-          const uint8_t* bcol0 = bsm + (int64_t)g * F.bsm_max + Bd.bsm_off + 8 * t;
-          const uint8_t* bcol1 = bcol0 + (int64_t)8 * F.bsm_max;
-          for (int q = 0; q < Bd.u_quads; ++q) {
-            const uint4 wq = ldg128(ub + 512 * q + 16 * lane);
-#pragma unroll
-            for (int ps = 0; ps < 4; ++ps) {
-              const int step = 4 * q + ps;
-              const uint2 b0 = *reinterpret_cast<const uint2*>(bcol0 + 32 * step);
-              const uint32_t a0 = u_reg_mask2(wq.x, ps), a1 = u_reg_mask2(wq.y, ps);
-              const uint32_t a2 = u_reg_mask2(wq.z, ps), a3 = u_reg_mask2(wq.w, ps);
-              mma_u8s8(C[0][ps], a0, a1, a2, a3, b0.x, b0.y);
-              if (npair > 1) {
-                const uint2 b1 = *reinterpret_cast<const uint2*>(bcol1 + 32 * step);
-                mma_u8s8(C[1][ps], a0, a1, a2, a3, b1.x, b1.y);
-              }
-            }
-          }
-          const uint8_t* sb = ub + (int64_t)512 * Bd.u_quads;
-          for (int sidx = 0; sidx < Bd.u_steps; ++sidx) {
-            const int valid = (sidx == Bd.u_steps - 1) ? Bd.u_last : 32;
-            const int nl = dc_u_step_lanes(valid);
-            const int ntv = nl / 8;
-            uint32_t wv = 0, hv = 0;
-            if (t < ntv) {
-              wv = ldg32(sb + 4 * (g * ntv + t));
-              if (Bd.bits == 3) hv = ldg16(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t));
-            }
-            uint32_t a[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              a[j] = reg_shift2(wv, j);
-              if (Bd.bits == 3) a[j] |= u_reg_hi3(hv, j);
-            }
-            const int step = 4 * Bd.u_quads + sidx;
-            const uint2 b0 = *reinterpret_cast<const uint2*>(bcol0 + 32 * step);
-            mma_u8s8(C[0][0], a[0], a[1], a[2], a[3], b0.x, b0.y);
-            if (npair > 1) {
-              const uint2 b1 = *reinterpret_cast<const uint2*>(bcol1 + 32 * step);
-              mma_u8s8(C[1][0], a[0], a[1], a[2], a[3], b1.x, b1.y);
-            }
-            sb += dc_u_step_bytes(Bd.bits, nl);
-          }
-        }
-        // ---- combine positions and limbs; lane t holds limb t of columns (tok 0, tok 1) of a pair
-        const float lw = (float)(1 << (8 * min(t, 2)));
-#pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          if (pr >= npair) continue;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int tk = q & 1;
-            int cl = C[pr][0][q] + (C[pr][1][q] >> 2) + (C[pr][2][q] >> 4) + (C[pr][3][q] >> 6);
-            float v = 0.f;
-            if (t < 3) v = (float)(cl - us->zc[pr][t][tk]) * lw;
-            v += __shfl_xor_sync(FULLMASK, v, 1);
-            v += __shfl_xor_sync(FULLMASK, v, 2);
-            const int qq = 2 * pr + tk;
-            if (t == 0 && qq < ntok) {
-              const int row = g + 8 * (q >> 1);
-              ydw[row * DC_TOK_BLOCK + (pt0 - tb) + qq] += ldexpf(v, -us->exps[qq]);
-            }
-          }
-        }
-        __syncwarp();
-        // ---- 8-bit bands: scalar path, lane -> (row = lane & 15, token parity = lane >> 4)
-        for (int b = 0; b < L.n_bands; ++b) {
-          const DcBand& Bd = L.band[b];
-          if (Bd.bits != 8) continue;
-          const int row = lane & 15;
-          const uint8_t* ur = blob + Bd.u_off + (int64_t)(orow + row) * Bd.rank;
-          for (int q = lane >> 4; q < ntok; q += 2) {
-            float sum = 0.f;
-            for (int i = 0; i < Bd.rank; ++i) {
-              const int r = Bd.r0 + i;
-              const __half2 mz = *reinterpret_cast<const __half2*>(umeta + 4 * r);
-              const float code = (float)ur[i];
-              sum = fmaf((code - __high2float(mz)) * __low2float(mz), tw[(int64_t)q * F.ws.r_stride + r], sum);
-            }
-            ydw[row * DC_TOK_BLOCK + (pt0 - tb) + q] += sum;
-          }
-        }
-        __syncthreads();
-      }
+  uint32_t seq = 0;
+  for (;;) {
+    const int s = seq % B_STAGES;
+    if (!mbar_wait(&tail->full[s], (seq / B_STAGES) & 1)) {
+      set_status(P.st, DC_ERR_CUDA);
+      return;
     }
-  }
-  __syncwarp();
-  // ---- output in the tokens' original order
+    const BDesc d = tail->desc[s];
+    if (d.kind == 2) return;
+    const uint8_t* stage = sm + (size_t)s * B_STAGE_BYTES;
+    if (d.first) {
 #pragma unroll
-  for (int nt = 0; nt < 8; ++nt)
+      for (int a = 0; a < 8; ++a)
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int tok = 8 * nt + 2 * t + (q & 1);
-      const int row = g + 8 * (q >> 1);
-      if (tok < Tb) {
-        const float v = acc[nt][q] + ydw[row * DC_TOK_BLOCK + tok];
-        const int dst = P.perm[tb + tok];
-        const int64_t o = (int64_t)dst * lin.d_out + ot * 128 + 16 * w + row;
-        if (F.dtype_out == DC_DTYPE_F32)
-          reinterpret_cast<float*>(lin.y)[o] = v;
-        else
-          reinterpret_cast<__nv_bfloat16*>(lin.y)[o] = __float2bfloat16_rn(v);
-      }
+        for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
     }
+    if (d.kind == 0) {
+      // rows 16w.. of W and the block's tokens, 128 columns in two 64-column boxes stored with the
+      // 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r & 7))
+      const int ntv = (d.Tb + 7) >> 3;
+      const int r0 = 16 * warp + g, r1 = r0 + 8;
+      uint4 wa[4], wb[4];
+#pragma unroll
+      for (int k32 = 0; k32 < 4; ++k32) {
+        const uint8_t* box = stage + (k32 >> 1) * B_WBOX;
+        const int c = 4 * (k32 & 1) + t;
+        wa[k32] = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((c ^ (r0 & 7)) << 4));
+        wb[k32] = *reinterpret_cast<const uint4*>(box + r1 * 128 + ((c ^ (r1 & 7)) << 4));
+      }
+      // each 128-column chunk is summed in a fresh MMA chain, then added with an IEEE fp32 add
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) {
+        if (nt < ntv) {
+          const int xr = 8 * nt + g;
+          float part[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+          for (int k32 = 0; k32 < 4; ++k32) {
+            const uint8_t* box = stage + 2 * B_WBOX + (k32 >> 1) * B_XBOX;
+            const int c = 4 * (k32 & 1) + t;
+            const uint4 xv = *reinterpret_cast<const uint4*>(box + xr * 128 + ((c ^ (xr & 7)) << 4));
+            mma_bf16(part, wa[k32].x, wb[k32].x, wa[k32].y, wb[k32].y, xv.x, xv.y);
+            mma_bf16(part, wa[k32].z, wb[k32].z, wa[k32].w, wb[k32].w, xv.z, xv.w);
+          }
+#pragma unroll
+          for (int q = 0; q < 4; ++q) acc[nt][q] += part[q];
+        }
+      }
+    } else if (d.kind == 3) {
+      b_base_f32(F, F.lin[d.p], P.perm, d.ot, d.tb, d.Tb, warp, lane, acc);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&tail->empty[s]);
+    if (d.last) {
+      // ---- output (+ delta) in the tokens' original order
+      const DcLinDev& lin = F.lin[d.p];
+      const float* yd = P.yd + (int64_t)d.p * T * F.ws.max_d_in;
+      const uint8_t* hasd = P.dflag + (int64_t)d.p * T;
+      const bool delta = (F.flags & DC_DELTA) != 0;
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int tok = 8 * nt + 2 * t + (q & 1);
+          const int row = d.ot * 128 + 16 * warp + g + 8 * (q >> 1);
+          if (tok < d.Tb) {
+            float v = acc[nt][q];
+            if (delta && hasd[d.tb + tok]) v += yd[(int64_t)(d.tb + tok) * F.ws.max_d_in + row];
+            const int64_t o = (int64_t)P.perm[d.tb + tok] * lin.d_out + row;
+            if (F.dtype_out == DC_DTYPE_F32)
+              reinterpret_cast<float*>(lin.y)[o] = v;
+            else
+              reinterpret_cast<__nv_bfloat16*>(lin.y)[o] = __float2bfloat16_rn(v);
+          }
+        }
+    }
+    ++seq;
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1024,8 +1408,8 @@ __global__ void k_unpack_v(const uint8_t* blob, DcLayout L, int bi, uint8_t* out
   const int nh = h == 0 ? min(rows, 8) : max(0, rows - 8);
   if (g >= nh) return;
   const int ngrp = (kb == L.nkb - 1) ? L.tail_groups : 4;
-  const uint8_t* blk = blob + B.v_off + (int64_t)tile * B.v_tile_bytes + (int64_t)kb * dc_v_block_bytes(B.bits, rows, 4) +
-                       dc_v_half_off(B.bits, rows, ngrp, h);
+  const uint8_t* blk = blob + B.v_off + dc_v_group_block_off(B, L, tile / B.v_group, kb) +
+                       (int64_t)(tile % B.v_group) * dc_v_block_bytes(B.bits, 16, ngrp) + dc_v_half_off(B.bits, rows, ngrp, h);
   const int p0 = dc_v_plane0_bytes(B.bits, ngrp);
   const int rank = B.r0 + 16 * tile + 8 * h + g;
   for (int grp = 0; grp < ngrp; ++grp)
@@ -1302,6 +1686,36 @@ extern "C" dc_status dc_read_segments(const void* ws, int32_t T, int32_t* perm_d
   return st;
 }
 
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency).
+static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+  }
+  return fn;
+}
+
+// 2-D bf16 tensor map: `rows` x `cols` (row pitch `pitch` elements), box 64 columns x box_rows rows,
+// 128-byte swizzle.
+static dc_status encode_bf16_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t pitch,
+                                 int box_rows) {
+  auto enc = tensor_map_encoder();
+  if (!enc) return dc_fail(DC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)pitch * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return dc_fail(DC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return DC_OK;
+}
+
 // Shared driver of the single-linear and the 7-linear calls.
 static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const* xs, const int* dxs, void* const* ys,
                              const int32_t* ids, int32_t T, int32_t dtype_in, int32_t dtype_out, int32_t flags,
@@ -1346,7 +1760,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (l.max_rank < 0 || l.max_rank > std::min(l.d_out, l.d_in)) return dc_fail(DC_ERR_SHAPE, "linear %d: max_rank", p);
     max_rank = std::max(max_rank, l.max_rank);
     max_ten = std::max(max_ten, l.n_tenants);
-    bsm_max = std::max(bsm_max, (int)dc_align(l.max_rank, 32) + 32 * DC_MAX_BANDS);
+    max_d_in = std::max(max_d_in, l.d_out);  // the workspace's per-token rows also hold outputs
+    bsm_max = std::max(bsm_max, (int)dc_align(dc_align(l.max_rank, 32) + 32 * DC_MAX_BANDS, 128) + 32);
     F.lin[p].W = l.W_base;
     F.lin[p].tenants = l.tenants_dev;
     F.lin[p].y = ys[p];
@@ -1360,6 +1775,19 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   F.ws = dc_ws_layout(T, max_rank, max_d_in, n_lin, max_ten);
   if (ws_bytes < (size_t)F.ws.total)
     return dc_fail(DC_ERR_WORKSPACE, "workspace holds %zu bytes, need %lld", ws_bytes, (long long)F.ws.total);
+  if (flags & DC_BASE) {
+    for (int p = 0; p < n_lin; ++p)
+      if (lins[p].w_dtype == DC_DTYPE_BF16) {
+        dc_status st0 = encode_bf16_map(&F.wmap[p], lins[p].W_base, lins[p].d_in, lins[p].d_out, lins[p].d_in, 128);
+        if (st0) return st0;
+      }
+    if (dtype_in == DC_DTYPE_BF16)
+      for (int m = 0; m < n_in; ++m) {
+        const uint8_t* xb = (const uint8_t*)ws + F.ws.xsort + (int64_t)m * T * F.ws.max_d_in * 2;
+        dc_status st0 = encode_bf16_map(&F.xmap[m], xb, dxs[m], T, F.ws.max_d_in, std::min(64, T));
+        if (st0) return st0;
+      }
+  }
   // U-kernel order: largest output tiles first (d_in decides the bytes per tile)
   int ord[7];
   for (int p = 0; p < n_lin; ++p) ord[p] = p;
@@ -1382,34 +1810,63 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (st) return st;
   }
   prof_before(s, 1);
-  k_prep<<<dim3(T + 1, n_in), 256, 0, s>>>(F, (uint8_t*)ws);
+  // work counters (item count, work cursors) and per-token delta flags start from zero on every call
+  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * 4, s), "counter reset");
+  if (st) return st;
+  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.dflag, 0, (size_t)n_lin * T, s), "flag reset");
+  if (st) return st;
+  const int nb_items = (T + 255) / 256;
+  k_prep<<<dim3(T + nb_items, std::max(n_in, n_lin)), 256, 0, s>>>(F, (uint8_t*)ws);
   prof_after(s);
   st = dc_cuda_check(cudaGetLastError(), "prep kernel");
   if (st) return st;
+  static int n_sm = 0;
+  if (!n_sm) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
+    if (n_sm <= 0) n_sm = 148;
+  }
   if (flags & DC_DELTA) {
-    static int n_sm = 0;
-    if (!n_sm) {
-      int dev = 0;
-      cudaGetDevice(&dev);
-      cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-      if (n_sm <= 0) n_sm = 148;
+    const size_t vsmem = (size_t)V_STAGES * V_STAGE_BYTES + sizeof(VSmemTail);
+    static bool vset = false;
+    if (!vset) {
+      st = dc_cuda_check(cudaFuncSetAttribute(k_vstage, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vsmem), "smem attr");
+      if (st) return st;
+      vset = true;
     }
     prof_before(s, 2);
-    k_vstage<<<n_sm * 4, 256, 0, s>>>(F, (uint8_t*)ws);
+    k_vstage<<<n_sm, V_THREADS, vsmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "rank-reduction kernel");
     if (st) return st;
   }
-  const size_t usmem = (size_t)2 * 64 * U_XROW * 2 + (size_t)16 * bsm_max + (size_t)8 * 16 * DC_TOK_BLOCK * 4 + sizeof(USmem);
-  static size_t usmem_set = 0;
-  if (usmem > usmem_set) {
-    st = dc_cuda_check(cudaFuncSetAttribute(k_ustage, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usmem), "smem attr");
+  if (flags & DC_DELTA) {
+    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + (size_t)12 * bsm_max + sizeof(USmemTail);
+    if (usmem > 227 * 1024)
+      return dc_fail(DC_ERR_UNSUPPORTED, "max_rank %d needs %zu bytes of shared memory", max_rank, usmem);
+    static size_t usmem_set = 0;
+    if (usmem > usmem_set) {
+      st = dc_cuda_check(cudaFuncSetAttribute(k_udelta, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usmem), "smem attr");
+      if (st) return st;
+      usmem_set = usmem;
+    }
+    prof_before(s, 3);
+    k_udelta<<<n_sm, U_THREADS, usmem, s>>>(F, (uint8_t*)ws);
+    prof_after(s);
+    st = dc_cuda_check(cudaGetLastError(), "delta output kernel");
     if (st) return st;
-    usmem_set = usmem;
   }
-  const dim3 ugrid(F.tile_prefix[n_lin], (T + DC_TOK_BLOCK - 1) / DC_TOK_BLOCK);
-  prof_before(s, 3);
-  k_ustage<<<ugrid, 256, usmem, s>>>(F, (uint8_t*)ws);
+  const size_t bsmem = 1024 + (size_t)B_STAGES * B_STAGE_BYTES + sizeof(BSmemTail);
+  static bool bset = false;
+  if (!bset) {
+    st = dc_cuda_check(cudaFuncSetAttribute(k_base, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem), "smem attr");
+    if (st) return st;
+    bset = true;
+  }
+  const int n_units = F.tile_prefix[n_lin] * ((T + DC_TOK_BLOCK - 1) / DC_TOK_BLOCK);
+  prof_before(s, 4);
+  k_base<<<std::min(n_sm, n_units), U_THREADS, bsmem, s>>>(F, (uint8_t*)ws);
   prof_after(s);
   return dc_cuda_check(cudaGetLastError(), "output kernel");
 }

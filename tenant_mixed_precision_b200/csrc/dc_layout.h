@@ -4,9 +4,11 @@
 // bands of equal bit width in descending singular-value order (the 8/3/2/0-bit groups of
 // "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language Models",
 // section "Approach").  Each kept vector is quantised in groups of 128 with an fp16 scale and
-// zero per group.  The blob is laid out for the two serving kernels:
+// zero per group.  The blob is laid out for the two serving kernels, which stream it through
+// shared memory with 1-D bulk copies (every region below starts on 16 bytes and is a multiple of
+// 16 bytes long):
 //
-//   [S fp32 r] [V codes, band by band] [V meta] [U codes, band by band] [U meta]
+//   [S fp32 r] [V codes + V meta, band by band] [U codes, band by band] [U meta]
 //
 // V side (rank reduction t = S * (V_hat^T x)): the kernel's MMA tile is 16 ranks x 32 columns of
 // d_in (mma.m16n8k32, u8 codes).  Ranks of a band are cut into tiles of 16 (the last may be
@@ -15,8 +17,12 @@
 // (g = lane/4, t = lane%4) of a half owns row g of the half, and within each group the 32
 // columns 32t .. 32t+31; the column of MMA step s (0..3), k-half hh (0/1) and byte b is
 // 32t + 8s + 4hh + b (the B operand uses the same permutation, so activations stay in natural
-// order).  Storage per (tile, block, half): one array per bit plane, lanes in order, only the
-// lanes of valid rows (4 per row) present:
+// order).  A (tile, block) region is [half 0 planes][half 1 planes][meta of the block's groups].
+// Tiles are gathered in groups of 8 (2-bit), 5 (3-bit) or 2 (8-bit) tiles -- one serving work
+// item -- stored block-major: [group][block][tile][(tile, block) region], so that one block of
+// every tile of a group is one contiguous run of bytes.
+// Storage per (tile, block, half): one array per bit plane, lanes in order, only the lanes of
+// valid rows (4 per row) present:
 //   2-bit, full block : 8 words per lane; word 2s+hh, bits [8b+2p, 8b+2p+2) hold the code of
 //                       group p (p = 0..3) -- a register is extracted with one AND and carries
 //                       the weight 4^p, removed in the fp32 epilogue ("mask" layout);
@@ -25,8 +31,8 @@
 //   3-bit             : the 2-bit plane in the shift layout plus a 1-bit plane of one word per
 //                       group, bit 8b + 2s + hh = bit 2 of the code;
 //   8-bit             : 8 words per group, word 2s+hh byte b = the code.
-// V meta: per (tile, group, g, half) the fp16 pair (scale, zero) of row g + 8*half: 64 bytes per
-// (tile, group), rows past the band padded with zeros.
+// V meta (inside the block, after the codes): per (group, g, half) the fp16 pair (scale, zero) of
+// row g + 8*half: 64 bytes per group, rows past the band padded with zeros.
 //
 // U side (y += U_hat * B with B = scale * t): the MMA tile is 16 output rows x 32 ranks.  A band
 // of 2 or 3 bits is cut into steps of 32 ranks; lane (g, t) owns rows g and g+8 and, within a
@@ -41,7 +47,7 @@
 //   (ranks inside a lane padded to 8 with code 0).
 // 8-bit bands of U are small (the top singular vectors) and are stored row-major [d_out][R8]
 // as bytes for a scalar path.
-// U meta: [d_out/128][r] fp16 pairs (scale, zero).
+// U meta: [d_out/128][r4] fp16 pairs (scale, zero), r4 = r rounded up to a multiple of 4.
 #pragma once
 #include <stdint.h>
 
@@ -59,12 +65,12 @@ struct DcBand {
   int32_t r0;          // first rank of the band (index into S, t and U meta)
   int32_t bsm_off;     // offset of the band in the U-stage staging of B (multiple of 32)
   int32_t v_tiles;     // ceil(rank / 16)
+  int32_t v_group;     // tiles per group (8, 5 or 2)
   int32_t u_quads;     // U: full 4-step quads in the mask layout (2-bit only)
   int32_t u_steps;     // U: steps in the shift layout after the quads (incl. a partial last one)
   int32_t u_last;      // U: valid ranks of the last shift-layout step (32 if it is full)
   int64_t v_off;       // V codes of the band
-  int64_t v_tile_bytes;// bytes of one full 16-row tile
-  int64_t v_meta_off;  // V meta of the band
+  int64_t v_tile_bytes;// bytes of one full 16-row tile (codes and meta of every block)
   int64_t u_off;       // U codes of the band
   int64_t u_otile_bytes; // bytes per 16-row output tile (MMA bands); R8 for 8-bit bands
 };
@@ -77,20 +83,26 @@ struct DcLayout {
   int32_t tail_groups; // groups in the last block (1..4)
   int32_t bsm_total;   // extent of the U-stage B staging (ranks, padded)
   int32_t valid;       // 1 if the descriptor is valid
+  int32_t r4;          // U meta row stride (entries)
   int64_t s_off, u_meta_off, bytes;
   int64_t dev_base;    // device address of the blob (filled where a layout is bound to a blob)
   DcBand band[DC_MAX_BANDS];
 };
 
 DC_HD int64_t dc_align(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
+DC_HD int32_t dc_min(int32_t a, int32_t b) { return a < b ? a : b; }
 
 // bytes of one lane's codes for one group of one row (all planes)
 DC_HD int32_t dc_v_lane_group_bytes(int32_t bits) { return bits == 2 ? 8 : (bits == 3 ? 12 : 32); }
 // bytes of plane 0 (2-bit plane or the 8-bit plane) of one lane for ngrp groups
 DC_HD int32_t dc_v_plane0_bytes(int32_t bits, int32_t ngrp) { return (bits == 8 ? 32 : 8) * ngrp; }
-// bytes of one (tile, block): 4 lanes per valid row, all planes
-DC_HD int64_t dc_v_block_bytes(int32_t bits, int32_t rows, int32_t ngrp) {
+// code bytes of one (tile, block): 4 lanes per valid row, all planes
+DC_HD int64_t dc_v_block_code_bytes(int32_t bits, int32_t rows, int32_t ngrp) {
   return (int64_t)4 * rows * dc_v_lane_group_bytes(bits) * ngrp;
+}
+// bytes of one (tile, block): codes, then 64 bytes of meta per group
+DC_HD int64_t dc_v_block_bytes(int32_t bits, int32_t rows, int32_t ngrp) {
+  return dc_v_block_code_bytes(bits, rows, ngrp) + (int64_t)64 * ngrp;
 }
 // byte offset of half h inside a (tile, block) region
 DC_HD int64_t dc_v_half_off(int32_t bits, int32_t rows, int32_t ngrp, int32_t h) {
@@ -108,6 +120,9 @@ DC_HD int32_t dc_u_step_lanes(int32_t valid_ranks) {  // lanes (of 32) stored fo
 
 DC_HD bool dc_bits_ok(int32_t b) { return b == 0 || b == 2 || b == 3 || b == 8; }
 
+// tiles of 16 ranks per group (= per serving work item) for a bit width
+DC_HD int32_t dc_v_group_tiles(int32_t bits) { return bits == 2 ? 8 : (bits == 3 ? 5 : 2); }
+
 // Compute the layout of a descriptor; layout.valid = 0 on an invalid descriptor.
 DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   DcLayout L;
@@ -121,6 +136,7 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   L.dev_base = 0;
   L.u_meta_off = 0;
   L.bsm_total = 0;
+  L.r4 = 0;
   L.groups_in = d.d_in / DC_GROUP;
   L.groups_out = d.d_out / DC_GROUP;
   L.nkb = (L.groups_in + 3) / 4;
@@ -141,22 +157,16 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   if (r > cap) return L;
   L.r = r;
   int64_t off = dc_align((int64_t)r * 4, 256);  // S
-  // V codes
+  // V codes with inline meta
   for (int i = 0; i < L.n_bands; ++i) {
     DcBand& B = L.band[i];
     B.v_tiles = (B.rank + 15) / 16;
+    B.v_group = dc_v_group_tiles(B.bits);
     B.v_off = off;
-    B.v_tile_bytes = (int64_t)64 * dc_v_lane_group_bytes(B.bits) * L.groups_in;
+    B.v_tile_bytes = dc_v_block_bytes(B.bits, 16, L.groups_in);
     int32_t last_rows = B.rank - 16 * (B.v_tiles - 1);
-    int64_t sz = B.v_tile_bytes * (B.v_tiles - 1) +
-                 (int64_t)4 * last_rows * dc_v_lane_group_bytes(B.bits) * L.groups_in;
+    int64_t sz = B.v_tile_bytes * (B.v_tiles - 1) + dc_v_block_bytes(B.bits, last_rows, L.groups_in);
     off = dc_align(off + sz, 256);
-  }
-  // V meta
-  for (int i = 0; i < L.n_bands; ++i) {
-    DcBand& B = L.band[i];
-    B.v_meta_off = off;
-    off = dc_align(off + (int64_t)B.v_tiles * L.groups_in * 64, 256);
   }
   // U codes
   int32_t bsm = 0;
@@ -188,9 +198,24 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   }
   L.bsm_total = bsm;
   // U meta
+  L.r4 = (int32_t)dc_align(r, 4);
   L.u_meta_off = off;
-  off = dc_align(off + (int64_t)L.groups_out * r * 4, 256);
+  off = dc_align(off + (int64_t)L.groups_out * L.r4 * 4, 256);
   L.bytes = off;
   L.valid = 1;
   return L;
+}
+
+// ---- V group geometry (groups of v_group tiles, block-major inside a group)
+DC_HD int32_t dc_v_tile_rows(const DcBand& B, int32_t tile) { return dc_min(16, B.rank - 16 * tile); }
+DC_HD int32_t dc_v_group_ntiles(const DcBand& B, int32_t grp) { return dc_min(B.v_group, B.v_tiles - grp * B.v_group); }
+// bytes of one block (ngrp groups of 128 columns) of every tile of group `grp`
+DC_HD int64_t dc_v_group_block_bytes(const DcBand& B, int32_t grp, int32_t ngrp) {
+  const int32_t n = dc_v_group_ntiles(B, grp);
+  const int32_t last_rows = dc_v_tile_rows(B, grp * B.v_group + n - 1);
+  return (int64_t)(n - 1) * dc_v_block_bytes(B.bits, 16, ngrp) + dc_v_block_bytes(B.bits, last_rows, ngrp);
+}
+// offset (inside the band) of group `grp`'s block `kb`; tile ti of it starts ti * dc_v_block_bytes(bits, 16, ngrp) later
+DC_HD int64_t dc_v_group_block_off(const DcBand& B, const DcLayout& L, int32_t grp, int32_t kb) {
+  return (int64_t)grp * B.v_group * B.v_tile_bytes + (int64_t)kb * dc_v_group_block_bytes(B, grp, 4);
 }

@@ -16,10 +16,7 @@ struct DcPlain {
 
 DC_HD int64_t dc_v_band_bytes(const DcLayout& L, const DcBand& B) {
   int32_t last_rows = B.rank - 16 * (B.v_tiles - 1);
-  return B.v_tile_bytes * (B.v_tiles - 1) + (int64_t)4 * last_rows * dc_v_lane_group_bytes(B.bits) * L.groups_in;
-}
-DC_HD int64_t dc_v_meta_bytes(const DcLayout& L, const DcBand& B) {
-  return (int64_t)B.v_tiles * L.groups_in * 64;
+  return B.v_tile_bytes * (B.v_tiles - 1) + dc_v_block_bytes(B.bits, last_rows, L.groups_in);
 }
 DC_HD int64_t dc_u_band_bytes(const DcLayout& L, const DcBand& B) {
   return B.bits == 8 ? (int64_t)L.d_out * B.rank : B.u_otile_bytes * (L.d_out / 16);
@@ -35,15 +32,32 @@ DC_HD uint32_t dc_cu(const DcLayout& L, const DcPlain& P, int32_t rank, int32_t 
 // Word at byte offset `off` (a multiple of 4) inside the V codes of band B.
 DC_HD uint32_t dc_pack_v_word(const DcLayout& L, const DcBand& B, int64_t off, const DcPlain& P) {
   const int32_t bits = B.bits;
-  int32_t j = (int32_t)(off / B.v_tile_bytes);
-  if (j > B.v_tiles - 1) j = B.v_tiles - 1;
-  const int64_t in_tile = off - (int64_t)j * B.v_tile_bytes;
-  const int32_t rows = (B.rank - 16 * j) < 16 ? (B.rank - 16 * j) : 16;
-  const int64_t fbb = dc_v_block_bytes(bits, rows, 4);
-  int32_t kb = (int32_t)(in_tile / fbb);
+  const int64_t gbytes = (int64_t)B.v_group * B.v_tile_bytes;  // a full group
+  const int32_t ngroups = (B.v_tiles + B.v_group - 1) / B.v_group;
+  int32_t grp = (int32_t)(off / gbytes);
+  if (grp > ngroups - 1) grp = ngroups - 1;
+  const int64_t in_g = off - (int64_t)grp * gbytes;
+  const int64_t f4 = dc_v_group_block_bytes(B, grp, 4);
+  int32_t kb = (int32_t)(in_g / f4);
   if (kb > L.nkb - 1) kb = L.nkb - 1;
-  const int64_t in_blk = in_tile - (int64_t)kb * fbb;
+  const int64_t in_kb = in_g - (int64_t)kb * f4;
   const int32_t ngrp = (kb == L.nkb - 1) ? L.tail_groups : 4;
+  const int64_t tb16 = dc_v_block_bytes(bits, 16, ngrp);
+  int32_t ti = (int32_t)(in_kb / tb16);
+  const int32_t nt = dc_v_group_ntiles(B, grp);
+  if (ti > nt - 1) ti = nt - 1;
+  const int64_t in_blk = in_kb - (int64_t)ti * tb16;
+  const int32_t j = grp * B.v_group + ti;
+  const int32_t rows = dc_v_tile_rows(B, j);
+  const int64_t cb = dc_v_block_code_bytes(bits, rows, ngrp);
+  if (in_blk >= cb) {  // inline meta: entry (group, g, half)
+    const int64_t e = (in_blk - cb) / 4;
+    const int32_t h = (int32_t)(e & 1), g = (int32_t)((e >> 1) & 7), cg = (int32_t)(e >> 4);
+    const int32_t row = 16 * j + 8 * h + g;
+    if (row >= B.rank || cg >= ngrp) return 0u;
+    const uint16_t* sz = P.szv + ((int64_t)(B.r0 + row) * L.groups_in + 4 * kb + cg) * 2;
+    return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
+  }
   const int64_t h1 = dc_v_half_off(bits, rows, ngrp, 1);
   const int32_t h = (rows > 8 && in_blk >= h1) ? 1 : 0;
   const int64_t in_half = in_blk - (h ? h1 : 0);
@@ -93,18 +107,6 @@ DC_HD uint32_t dc_pack_v_word(const DcLayout& L, const DcBand& B, int64_t off, c
                << (8 * b + 2 * s + hh);
   }
   return w;
-}
-
-// Word at byte offset `off` inside the V meta of band B.
-DC_HD uint32_t dc_pack_vmeta_word(const DcLayout& L, const DcBand& B, int64_t off, const DcPlain& P) {
-  const int64_t e = off / 4;
-  const int32_t h = (int32_t)(e & 1), g = (int32_t)((e >> 1) & 7);
-  const int64_t tg = e >> 4;  // tile * groups_in + group
-  const int32_t gi = (int32_t)(tg % L.groups_in), j = (int32_t)(tg / L.groups_in);
-  const int32_t row = 16 * j + 8 * h + g;
-  if (row >= B.rank) return 0u;
-  const uint16_t* sz = P.szv + ((int64_t)(B.r0 + row) * L.groups_in + gi) * 2;
-  return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
 }
 
 // Word at byte offset `off` inside the U codes of band B.
@@ -191,13 +193,12 @@ DC_HD uint32_t dc_pack_word(const DcLayout& L, int64_t off, const DcPlain& P) {
   for (int i = 0; i < L.n_bands; ++i) {
     const DcBand& B = L.band[i];
     if (off >= B.v_off && off < B.v_off + dc_v_band_bytes(L, B)) return dc_pack_v_word(L, B, off - B.v_off, P);
-    if (off >= B.v_meta_off && off < B.v_meta_off + dc_v_meta_bytes(L, B))
-      return dc_pack_vmeta_word(L, B, off - B.v_meta_off, P);
     if (off >= B.u_off && off < B.u_off + dc_u_band_bytes(L, B)) return dc_pack_u_word(L, B, off - B.u_off, P);
   }
-  if (off >= L.u_meta_off && off < L.u_meta_off + (int64_t)L.groups_out * L.r * 4) {
+  if (off >= L.u_meta_off && off < L.u_meta_off + (int64_t)L.groups_out * L.r4 * 4) {
     const int64_t e = (off - L.u_meta_off) / 4;
-    const int32_t go = (int32_t)(e / L.r), i = (int32_t)(e % L.r);
+    const int32_t go = (int32_t)(e / L.r4), i = (int32_t)(e % L.r4);
+    if (i >= L.r) return 0u;
     const uint16_t* sz = P.szu + ((int64_t)i * L.groups_out + go) * 2;
     return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
   }

@@ -101,7 +101,8 @@ def _run_linear(td, W, x, ids, flags, out_dtype=None):
     T = x.shape[0]
     n_ten = len(td.handles)
     y = torch.empty((T, td.d_out), dtype=out_dtype or torch.float32, device="cuda")
-    ws = torch.zeros(dc.dc_workspace_size(T, td.max_rank, td.d_in, 1, n_ten), dtype=torch.uint8, device="cuda")
+    ws = torch.zeros(dc.dc_workspace_size(T, td.max_rank, max(td.d_in, td.d_out), 1, n_ten), dtype=torch.uint8,
+                     device="cuda")
     lin = td.linear(W)
     ids_d = torch.from_numpy(np.asarray(ids, np.int32)).cuda()
     dc.dc_delta_linear_segmented(lin, x, y, ids_d, T, flags, ws)
