@@ -19,7 +19,7 @@ double dc_f16_to_f64(uint16_t h);
 #define DC_TOK_BLOCK 64         // tokens per output block of the decode output kernel
 #define DC_V_NT 2               // 16-rank tiles per V work item
 #define DC_V_TOKS 4             // tokens per V/U pass (two pairs)
-#define DC_XBLK 1600            // per (token, 512-column block): 3 limb rows of 512 B + 4 x 4 fp32 limb sums
+#define DC_XBLK 1616            // per (token, 512-column block): 3 limb rows of 512 B, 4 x 4 fp32 limb sums, pad
 
 // Status word slots at the start of the workspace.
 enum {
@@ -52,15 +52,15 @@ struct alignas(16) DcVItem {
 // One (linear, segment) record for the output kernel, self-contained.
 struct DcUBand {
   int32_t bits, rank, r0, bsm_off;
-  int32_t quads, steps, last, region;  // region: bytes of the band for one 128-row output group
-  int64_t u_off;                       // band offset in the blob
+  int32_t quads, steps, last, region;  // region: bytes of the band inside one 128-row group's run
+  int64_t boff;                        // offset of the band inside a run
   int32_t otile;                       // bytes per 16-row tile (2/3-bit) or R8 (8-bit)
   int32_t pad;
 };
 struct alignas(16) DcURec {  // moved with 16-byte vector loads and stores
   int64_t blob;
-  int32_t valid, tenant, st, len, r, r4, n_bands, u_meta_off;
-  int32_t pad[2];
+  int64_t u_off;  // start of the 128-row group runs (blob-relative)
+  int32_t valid, tenant, st, len, r, r4, n_bands, u_unit, u_meta_in, pad[3];
   DcUBand band[DC_MAX_BANDS];
 };
 

@@ -274,8 +274,9 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
   R.tenant = tau;
   R.st = st;
   R.len = len;
-  R.r = R.r4 = R.n_bands = R.u_meta_off = 0;
-  R.pad[0] = R.pad[1] = 0;
+  R.r = R.r4 = R.n_bands = R.u_unit = R.u_meta_in = 0;
+  R.u_off = 0;
+  R.pad[0] = R.pad[1] = R.pad[2] = 0;
   DcLayout L;
   L.valid = 0;
   if (tau < F.lin[p].n_tenants) {
@@ -294,12 +295,14 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
       R.r = L.r;
       R.r4 = L.r4;
       R.n_bands = L.n_bands;
-      R.u_meta_off = (int32_t)L.u_meta_off;
+      R.u_off = L.u_off;
+      R.u_unit = (int32_t)L.u_unit;
+      R.u_meta_in = (int32_t)L.u_meta_in;
       for (int b = 0; b < DC_MAX_BANDS; ++b) {
         DcUBand& U = R.band[b];
         if (b >= L.n_bands) {
           U.bits = U.rank = U.r0 = U.bsm_off = U.quads = U.steps = U.last = U.region = U.otile = U.pad = 0;
-          U.u_off = 0;
+          U.boff = 0;
           continue;
         }
         const DcBand& B = L.band[b];
@@ -311,8 +314,8 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
         U.steps = B.u_steps;
         U.last = B.u_last;
         U.otile = (int32_t)B.u_otile_bytes;
-        U.region = B.bits == 8 ? 128 * B.rank : (int32_t)(8 * B.u_otile_bytes);
-        U.u_off = B.u_off;
+        U.region = (int32_t)B.u_region;
+        U.boff = B.u_boff;
         U.pad = 0;
       }
     }
@@ -404,7 +407,7 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
     frexpf(mx, &E);  // mx < 2^E
     e = 22 - E;      // |x| * 2^e < 2^22
   }
-  uint8_t* xrow = P.xl + (int64_t)(m * T + j) * W.nkb * DC_XBLK;
+  uint8_t* xcol = P.xl + ((int64_t)m * W.nkb * T + j) * DC_XBLK;  // block kb at + kb * T * DC_XBLK
   for (int k = tid * 4; k < d; k += 1024) {
     float v[4];
     load4(k, v);
@@ -426,7 +429,7 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
       s0 += l0, s1 += l1, s2 += l2;
     }
     // [kb][limb 0 | limb 1 | limb 2 | limb sums of the block's 4 groups]
-    uint8_t* blk = xrow + (int64_t)(k >> 9) * DC_XBLK;
+    uint8_t* blk = xcol + (int64_t)(k >> 9) * T * DC_XBLK;
     const int within = k & 511;
     *reinterpret_cast<uint32_t*>(blk + within) = w0;
     *reinterpret_cast<uint32_t*>(blk + 512 + within) = w1;
@@ -452,9 +455,9 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
 // the pass's tokens -- into a ring of shared-memory stages with bulk copies; consumer warp w
 // decodes tile w from shared memory into u8 MMA operands.
 // ---------------------------------------------------------------------------------------------
-#define V_STAGES 6
+#define V_STAGES 8
 #define V_A_BYTES 18432   // one block of the item's tiles: 8 x 2304 (2-bit), 5 x 3328 (3-bit), 2 x 8448 (8-bit)
-#define V_XTOK 1616       // one token's limb block (DC_XBLK bytes) in shared memory, padded against bank conflicts
+#define V_XTOK DC_XBLK    // one token's limb block in shared memory (1616: offsets tokens by 20 banks)
 #define V_X_BYTES (4 * V_XTOK)
 #define V_STAGE_BYTES (V_A_BYTES + V_X_BYTES)
 #define V_CONSUMERS 8
@@ -701,10 +704,9 @@ __global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__
         __syncwarp();
         if (lane == 0) {
           bulk_g2s(stage, reinterpret_cast<const uint8_t*>(I.vbase) + (int64_t)kb * I.f4, code_bytes, &tail->full[s]);
-        } else if (lane <= I.ntok) {
-          const int k = lane - 1;
-          const uint8_t* src = P.xl + ((int64_t)(I.m * T + I.tok0 + k) * F.ws.nkb + kb) * DC_XBLK;
-          bulk_g2s(stage + V_A_BYTES + k * V_XTOK, src, DC_XBLK, &tail->full[s]);
+        } else if (lane == 1) {
+          const uint8_t* src = P.xl + (((int64_t)I.m * F.ws.nkb + kb) * T + I.tok0) * DC_XBLK;
+          bulk_g2s(stage + V_A_BYTES, src, (uint32_t)(I.ntok * DC_XBLK), &tail->full[s]);
         }
         ++seq;
       }
@@ -1088,51 +1090,31 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_udelta(const __grid_constant__
         int s;
         if (!acquire(s)) return;
         uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
-        int off = 0;
-        int offb[DC_MAX_BANDS] = {0, 0, 0, 0};
-#pragma unroll
-        for (int b = 0; b < DC_MAX_BANDS; ++b)
-          if (b < R.n_bands) {
-            offb[b] = off;
-            off += R.band[b].region;  // a multiple of 16
-          }
-        const int off_meta = off;
-        off += R.r4 * 4;
-        const int off_t = off;
-        const int tstride = R.r4;
-        off += ntok * tstride * 4;
-        const bool fits = off <= U_STAGE_BYTES;
+        const int off_t = R.u_unit;  // a multiple of 16
+        const int tstride = F.ws.r_stride;
+        const int total = off_t + ntok * tstride * 4;
+        const bool fits = total <= U_STAGE_BYTES;
         if (lane == 0) {
           UDesc& d = tail->desc[s];
           d.kind = 1;
           d.p = p, d.ot = ot, d.tok0 = pt0, d.ntok = ntok;
-          d.n_bands = R.n_bands, d.r = R.r, d.off_meta = off_meta, d.off_t = off_t, d.tstride = tstride;
+          d.n_bands = R.n_bands, d.r = R.r, d.off_meta = R.u_meta_in, d.off_t = off_t, d.tstride = tstride;
           d.error = fits ? 0 : 1;
           for (int b = 0; b < DC_MAX_BANDS; ++b) {
             const DcUBand& B = R.band[b];
-            d.band[b] = UBandD{B.bits, B.rank, B.r0, B.bsm_off, B.quads, B.steps, B.last, B.otile, offb[b]};
+            d.band[b] = UBandD{B.bits, B.rank, B.r0, B.bsm_off, B.quads, B.steps, B.last, B.otile, (int)B.boff};
           }
           if (!fits) set_status(P.st, DC_ERR_UNSUPPORTED);
-          // every region size is a multiple of 16, so `off` is exactly the number of bytes copied
-          if (fits)
-            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)off);
-          else
+          if (fits) {
+            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)total);
+            bulk_g2s(stage, blob + R.u_off + (int64_t)ot * R.u_unit, (uint32_t)R.u_unit, &tail->full[s]);
+            bulk_g2s(stage + off_t, P.tws + ((int64_t)p * T + pt0) * tstride, (uint32_t)(ntok * tstride * 4),
+                     &tail->full[s]);
+          } else {
             mbar_arrive(&tail->full[s]);
-        }
-        __syncwarp();
-        if (fits) {
-          if (lane < R.n_bands) {
-            const DcUBand& B = R.band[lane];
-            const int64_t src = B.bits == 8 ? B.u_off + (int64_t)ot * 128 * B.rank : B.u_off + (int64_t)ot * 8 * B.otile;
-            bulk_g2s(stage + offb[lane], blob + src, (uint32_t)B.region, &tail->full[s]);
-          } else if (lane == 4) {
-            bulk_g2s(stage + off_meta, blob + R.u_meta_off + (int64_t)ot * R.r4 * 4, (uint32_t)(R.r4 * 4), &tail->full[s]);
-          } else if (lane >= 8 && lane < 8 + ntok) {
-            const int k = lane - 8;
-            bulk_g2s(stage + off_t + k * tstride * 4, P.tws + ((int64_t)p * T + pt0 + k) * F.ws.r_stride,
-                     (uint32_t)(tstride * 4), &tail->full[s]);
           }
         }
+        __syncwarp();
         ++seq;
       }
     }
@@ -1169,9 +1151,9 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_udelta(const __grid_constant__
 // copies (128-byte swizzle); consumer warp w owns rows 16w..16w+15 and writes the unit's outputs,
 // plus the delta of k_udelta, in the tokens' original order.
 // ---------------------------------------------------------------------------------------------
-#define B_STAGES 4
-#define B_STAGE_BYTES (48 * 1024)  // a multiple of 1024 (128-byte-swizzled tensor tiles)
-#define B_KC 128                   // backbone columns per stage: two 64-column boxes
+#define B_STAGES 8
+#define B_STAGE_BYTES (24 * 1024)  // a multiple of 1024 (128-byte-swizzled tensor tiles)
+#define B_KC 64                    // backbone columns per stage: one 64-column box
 #define B_WBOX 16384               // 128 rows x 64 bf16
 #define B_XBOX 8192                // 64 tokens x 64 bf16
 
@@ -1291,15 +1273,13 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ D
           d.kind = base ? (bf16 ? 0 : 3) : 4, d.first = kc == 0, d.last = kc == nkc - 1;
           d.p = p, d.ot = ot, d.tb = tb, d.Tb = Tb;
           if (base && bf16)
-            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)(2 * B_WBOX + 2 * 128 * min(64, T)));
+            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)(B_WBOX + 128 * min(64, T)));
           else
             mbar_arrive(&tail->full[s]);
-          if (base && bf16)
-            for (int bx = 0; bx < 2; ++bx) {
-              tma_load_2d(stage + bx * B_WBOX, &F.wmap[p], kc * B_KC + 64 * bx, ot * 128, &tail->full[s]);
-              tma_load_2d(stage + 2 * B_WBOX + bx * B_XBOX, &F.xmap[lin.input], kc * B_KC + 64 * bx, tb,
-                          &tail->full[s]);
-            }
+          if (base && bf16) {
+            tma_load_2d(stage, &F.wmap[p], kc * B_KC, ot * 128, &tail->full[s]);
+            tma_load_2d(stage + B_WBOX, &F.xmap[lin.input], kc * B_KC, tb, &tail->full[s]);
+          }
         }
         __syncwarp();
         ++seq;
@@ -1330,29 +1310,27 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ D
         for (int q = 0; q < 4; ++q) acc[a][q] = 0.f;
     }
     if (d.kind == 0) {
-      // rows 16w.. of W and the block's tokens, 128 columns in two 64-column boxes stored with the
-      // 128-byte swizzle (16-byte chunk c of row r at chunk c ^ (r & 7))
+      // rows 16w.. of W and the block's tokens, 64 columns, stored with the 128-byte swizzle
+      // (16-byte chunk c of row r at chunk c ^ (r & 7))
       const int ntv = (d.Tb + 7) >> 3;
       const int r0 = 16 * warp + g, r1 = r0 + 8;
-      uint4 wa[4], wb[4];
+      uint4 wa[2], wb[2];
 #pragma unroll
-      for (int k32 = 0; k32 < 4; ++k32) {
-        const uint8_t* box = stage + (k32 >> 1) * B_WBOX;
-        const int c = 4 * (k32 & 1) + t;
-        wa[k32] = *reinterpret_cast<const uint4*>(box + r0 * 128 + ((c ^ (r0 & 7)) << 4));
-        wb[k32] = *reinterpret_cast<const uint4*>(box + r1 * 128 + ((c ^ (r1 & 7)) << 4));
+      for (int k32 = 0; k32 < 2; ++k32) {
+        const int c = 4 * k32 + t;
+        wa[k32] = *reinterpret_cast<const uint4*>(stage + r0 * 128 + ((c ^ (r0 & 7)) << 4));
+        wb[k32] = *reinterpret_cast<const uint4*>(stage + r1 * 128 + ((c ^ (r1 & 7)) << 4));
       }
-      // each 128-column chunk is summed in a fresh MMA chain, then added with an IEEE fp32 add
+      // each 64-column chunk is summed in a fresh MMA chain, then added with an IEEE fp32 add
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt) {
         if (nt < ntv) {
           const int xr = 8 * nt + g;
           float part[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-          for (int k32 = 0; k32 < 4; ++k32) {
-            const uint8_t* box = stage + 2 * B_WBOX + (k32 >> 1) * B_XBOX;
-            const int c = 4 * (k32 & 1) + t;
-            const uint4 xv = *reinterpret_cast<const uint4*>(box + xr * 128 + ((c ^ (xr & 7)) << 4));
+          for (int k32 = 0; k32 < 2; ++k32) {
+            const int c = 4 * k32 + t;
+            const uint4 xv = *reinterpret_cast<const uint4*>(stage + B_WBOX + xr * 128 + ((c ^ (xr & 7)) << 4));
             mma_bf16(part, wa[k32].x, wb[k32].x, wa[k32].y, wb[k32].y, xv.x, xv.y);
             mma_bf16(part, wa[k32].z, wb[k32].z, wa[k32].w, wb[k32].w, xv.z, xv.w);
           }
@@ -1437,13 +1415,14 @@ __global__ void k_unpack_u(const uint8_t* blob, DcLayout L, int bi, uint8_t* out
   if (B.bits == 8) {
     if (id >= (int64_t)L.d_out * B.rank) return;
     const int o = (int)(id / B.rank), i = (int)(id % B.rank);
-    out[(int64_t)(B.r0 + i) * L.d_out + o] = blob[B.u_off + id];
+    const int go = o >> 7;
+    out[(int64_t)(B.r0 + i) * L.d_out + o] = blob[L.u_off + (int64_t)go * L.u_unit + B.u_boff + (int64_t)(o & 127) * B.rank + i];
     return;
   }
   if (id >= (int64_t)(L.d_out / 16) * 32) return;
   const int lane = (int)(id & 31), ot = (int)(id >> 5);
   const int g = lane >> 2, t = lane & 3;
-  const uint8_t* ub = blob + B.u_off + (int64_t)ot * B.u_otile_bytes;
+  const uint8_t* ub = blob + L.u_off + (int64_t)(ot >> 3) * L.u_unit + B.u_boff + (int64_t)(ot & 7) * B.u_otile_bytes;
   auto put = [&](uint32_t reg, int j, int rank_base) {
     for (int b = 0; b < 4; ++b) {
       const int rank = rank_base + 8 * t + 4 * (j >> 1) + b;

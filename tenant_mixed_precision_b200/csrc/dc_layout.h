@@ -45,9 +45,12 @@
 //                                 byte b;
 //   the last step of a band may be partial: only lanes with 8t < valid ranks are stored
 //   (ranks inside a lane padded to 8 with code 0).
-// 8-bit bands of U are small (the top singular vectors) and are stored row-major [d_out][R8]
-// as bytes for a scalar path.
-// U meta: [d_out/128][r4] fp16 pairs (scale, zero), r4 = r rounded up to a multiple of 4.
+// 8-bit bands of U are small (the top singular vectors) and are stored row-major (128 rows x R8
+// bytes per 128-row group) for a scalar path.
+// The U side is grouped by 128-row output group (= the quantisation group along d_out): group go
+// holds, contiguously, every band's codes of its 128 rows (the eight 16-row tiles of a 2/3-bit
+// band one after the other) followed by the U meta of the group: r4 fp16 pairs (scale, zero),
+// r4 = r rounded up to a multiple of 4.  One 128-row group is one contiguous run of bytes.
 #pragma once
 #include <stdint.h>
 
@@ -71,8 +74,9 @@ struct DcBand {
   int32_t u_last;      // U: valid ranks of the last shift-layout step (32 if it is full)
   int64_t v_off;       // V codes of the band
   int64_t v_tile_bytes;// bytes of one full 16-row tile (codes and meta of every block)
-  int64_t u_off;       // U codes of the band
+  int64_t u_boff;      // offset of the band's codes inside one 128-row group's run
   int64_t u_otile_bytes; // bytes per 16-row output tile (MMA bands); R8 for 8-bit bands
+  int64_t u_region;    // bytes of the band inside one 128-row group's run
 };
 
 struct DcLayout {
@@ -84,7 +88,10 @@ struct DcLayout {
   int32_t bsm_total;   // extent of the U-stage B staging (ranks, padded)
   int32_t valid;       // 1 if the descriptor is valid
   int32_t r4;          // U meta row stride (entries)
-  int64_t s_off, u_meta_off, bytes;
+  int64_t s_off, bytes;
+  int64_t u_off;       // start of the U part (128-row group runs)
+  int64_t u_unit;      // bytes of one 128-row group's run
+  int64_t u_meta_in;   // offset of the U meta inside a run
   int64_t dev_base;    // device address of the blob (filled where a layout is bound to a blob)
   DcBand band[DC_MAX_BANDS];
 };
@@ -134,7 +141,9 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   L.bytes = 0;
   L.s_off = 0;
   L.dev_base = 0;
-  L.u_meta_off = 0;
+  L.u_off = 0;
+  L.u_unit = 0;
+  L.u_meta_in = 0;
   L.bsm_total = 0;
   L.r4 = 0;
   L.groups_in = d.d_in / DC_GROUP;
@@ -168,18 +177,20 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
     int64_t sz = B.v_tile_bytes * (B.v_tiles - 1) + dc_v_block_bytes(B.bits, last_rows, L.groups_in);
     off = dc_align(off + sz, 256);
   }
-  // U codes
+  // U: runs of 128-row groups [band codes ...][meta]
   int32_t bsm = 0;
+  int64_t in_unit = 0;
   for (int i = 0; i < L.n_bands; ++i) {
     DcBand& B = L.band[i];
-    B.u_off = off;
+    B.u_boff = in_unit;
     B.bsm_off = bsm;
     if (B.bits == 8) {
       B.u_quads = 0;
       B.u_steps = 0;
       B.u_last = 0;
       B.u_otile_bytes = B.rank;
-      off = dc_align(off + (int64_t)d.d_out * B.rank, 256);
+      B.u_region = dc_align((int64_t)128 * B.rank, 16);
+      in_unit += B.u_region;
       continue;
     }
     B.u_quads = B.bits == 2 ? B.rank / 128 : 0;
@@ -193,14 +204,16 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
       ot += dc_u_step_bytes(B.bits, dc_u_step_lanes(valid));
     }
     B.u_otile_bytes = ot;
-    off = dc_align(off + ot * (d.d_out / 16), 256);
+    B.u_region = 8 * ot;
+    in_unit += B.u_region;
     bsm += (int32_t)dc_align(B.rank, 32);
   }
   L.bsm_total = bsm;
-  // U meta
   L.r4 = (int32_t)dc_align(r, 4);
-  L.u_meta_off = off;
-  off = dc_align(off + (int64_t)L.groups_out * L.r4 * 4, 256);
+  L.u_meta_in = in_unit;
+  L.u_unit = in_unit + (int64_t)L.r4 * 4;
+  L.u_off = off;
+  off = dc_align(off + L.u_unit * L.groups_out, 256);
   L.bytes = off;
   L.valid = 1;
   return L;

@@ -18,9 +18,6 @@ DC_HD int64_t dc_v_band_bytes(const DcLayout& L, const DcBand& B) {
   int32_t last_rows = B.rank - 16 * (B.v_tiles - 1);
   return B.v_tile_bytes * (B.v_tiles - 1) + dc_v_block_bytes(B.bits, last_rows, L.groups_in);
 }
-DC_HD int64_t dc_u_band_bytes(const DcLayout& L, const DcBand& B) {
-  return B.bits == 8 ? (int64_t)L.d_out * B.rank : B.u_otile_bytes * (L.d_out / 16);
-}
 
 DC_HD uint32_t dc_cv(const DcLayout& L, const DcPlain& P, int32_t rank, int32_t k) {
   return P.cv[(int64_t)rank * L.d_in + k];
@@ -109,21 +106,21 @@ DC_HD uint32_t dc_pack_v_word(const DcLayout& L, const DcBand& B, int64_t off, c
   return w;
 }
 
-// Word at byte offset `off` inside the U codes of band B.
-DC_HD uint32_t dc_pack_u_word(const DcLayout& L, const DcBand& B, int64_t off, const DcPlain& P) {
+// Word at byte offset `off` inside band B's codes of the 128-row group `go`.
+DC_HD uint32_t dc_pack_u_word(const DcLayout& L, const DcBand& B, int32_t go, int64_t off, const DcPlain& P) {
   uint32_t w = 0;
   if (B.bits == 8) {
     for (int b = 0; b < 4; ++b) {
       const int64_t idx = off + b;
       const int64_t o = idx / B.rank;
       const int32_t i = (int32_t)(idx % B.rank);
-      if (o < L.d_out) w |= dc_cu(L, P, B.r0 + i, (int32_t)o) << (8 * b);
+      if (o < 128) w |= dc_cu(L, P, B.r0 + i, (int32_t)(128 * go + o)) << (8 * b);
     }
     return w;
   }
-  const int32_t ot = (int32_t)(off / B.u_otile_bytes);
+  const int32_t ot = (int32_t)(off / B.u_otile_bytes);  // 16-row tile inside the group
   int64_t x = off - (int64_t)ot * B.u_otile_bytes;
-  const int32_t o0 = 16 * ot;
+  const int32_t o0 = 128 * go + 16 * ot;
   if (x < (int64_t)512 * B.u_quads) {  // mask layout quads
     const int32_t q = (int32_t)(x / 512);
     const int32_t y = (int32_t)(x % 512);
@@ -193,14 +190,21 @@ DC_HD uint32_t dc_pack_word(const DcLayout& L, int64_t off, const DcPlain& P) {
   for (int i = 0; i < L.n_bands; ++i) {
     const DcBand& B = L.band[i];
     if (off >= B.v_off && off < B.v_off + dc_v_band_bytes(L, B)) return dc_pack_v_word(L, B, off - B.v_off, P);
-    if (off >= B.u_off && off < B.u_off + dc_u_band_bytes(L, B)) return dc_pack_u_word(L, B, off - B.u_off, P);
   }
-  if (off >= L.u_meta_off && off < L.u_meta_off + (int64_t)L.groups_out * L.r4 * 4) {
-    const int64_t e = (off - L.u_meta_off) / 4;
-    const int32_t go = (int32_t)(e / L.r4), i = (int32_t)(e % L.r4);
-    if (i >= L.r) return 0u;
-    const uint16_t* sz = P.szu + ((int64_t)i * L.groups_out + go) * 2;
-    return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
+  if (off >= L.u_off && off < L.u_off + L.u_unit * L.groups_out) {
+    const int64_t rel = off - L.u_off;
+    const int32_t go = (int32_t)(rel / L.u_unit);
+    const int64_t in = rel - (int64_t)go * L.u_unit;
+    if (in >= L.u_meta_in) {
+      const int32_t i = (int32_t)((in - L.u_meta_in) / 4);
+      if (i >= L.r) return 0u;
+      const uint16_t* sz = P.szu + ((int64_t)i * L.groups_out + go) * 2;
+      return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
+    }
+    for (int i = 0; i < L.n_bands; ++i) {
+      const DcBand& B = L.band[i];
+      if (in >= B.u_boff && in < B.u_boff + B.u_region) return dc_pack_u_word(L, B, go, in - B.u_boff, P);
+    }
   }
   return 0u;
 }
