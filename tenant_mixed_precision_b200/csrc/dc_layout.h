@@ -8,7 +8,7 @@
 // shared memory with 1-D bulk copies (every region below starts on 16 bytes and is a multiple of
 // 16 bytes long):
 //
-//   [S fp32 r] [V codes + V meta, band by band] [U codes, band by band] [U meta]
+//   [S fp32 r] [V codes + V meta, band by band] [U runs: one per 128-row output group]
 //
 // V side (rank reduction t = S * (V_hat^T x)): the kernel's MMA tile is 16 ranks x 32 columns of
 // d_in (mma.m16n8k32, u8 codes).  Ranks of a band are cut into tiles of 16 (the last may be
