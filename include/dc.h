@@ -178,6 +178,38 @@ dc_status dc_delta_linear_segmented(const dc_linear* lin, const void* x, void* y
                                     int32_t dtype_out, int32_t flags, void* ws, size_t ws_bytes,
                                     void* stream);
 
+/* Allocation-free variant of dc_delta_linear_segmented.  The pages have no counterpart: this
+ * is a serving-runtime convenience, not part of the method.
+ *
+ * Some callers cannot hand the library a workspace per call: a plain C host program with no
+ * caching allocator (cudaMalloc and cudaFree synchronise the whole device, which would stall
+ * every other stream once per call), or a serving runtime whose device memory plan is fixed at
+ * start-up and forbids allocation on the request path.  This entry point serves them from one
+ * workspace compiled into the library as a static device array of DC_STATIC_WORKSPACE_BYTES
+ * (16 MiB) per device, enough for one linear at decode sizes (e.g. 11008 x 4096 at 1/16 with
+ * T = 64 needs about 7 MB).  It allocates nothing and calls no allocating library.
+ *
+ * - Arguments, layouts and results are those of dc_delta_linear_segmented without ws/ws_bytes.
+ *   flags may hold DC_BASE and DC_DELTA; DC_REUSE_ROUTING is rejected (DC_ERR_INVALID_ARG):
+ *   the routing is rebuilt on every call.
+ * - A request whose workspace (dc_workspace_size(T, lin->max_rank, max(d_in, d_out), 1,
+ *   lin->n_tenants)) exceeds DC_STATIC_WORKSPACE_BYTES is rejected with DC_ERR_WORKSPACE before
+ *   anything is launched.
+ * - Nothing has to be zeroed by the caller: the array is zero when the library's device code is
+ *   loaded, and every call resets the status word and the work counters it uses.
+ * - The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ *   and keeps it; make that first call on each device outside any stream capture.
+ * - There is one array per device, shared by every caller in the process: two calls on the same
+ *   device that can overlap (different streams, or different threads without ordering) race on
+ *   it and give wrong results.  Serialise the calls on a device.
+ * - host_status: NULL, or where to store the device status word of this call (then the call
+ *   waits for the stream and clears the word, like dc_read_device_status). */
+#define DC_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
+dc_status dc_delta_linear_segmented_static(const dc_linear* lin, const void* x, void* y,
+                                           const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
+                                           int32_t dtype_out, int32_t flags, void* stream,
+                                           int32_t* host_status);
+
 /* The seven projections of one Llama-style decoder layer in one call, sharing one routing:
  * lin[0..6] = q, k, v, o, gate, up, down.  q, k, v, gate and up read x_h [T, hidden]; o reads
  * x_o [T, hidden]; down reads x_f [T, ffn].  y[p] receives [T, lin[p].d_out]. */

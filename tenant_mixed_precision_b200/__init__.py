@@ -76,6 +76,7 @@ def _load():
         "dc_build_segments": (I32, [VP, I32, I32, VP, SZ, VP]),
         "dc_read_segments": (I32, [VP, I32, VP, VP, VP, VP, VP]),
         "dc_delta_linear_segmented": (I32, [P(dc_linear), VP, VP, VP, I32, I32, I32, I32, VP, SZ, VP]),
+        "dc_delta_linear_segmented_static": (I32, [P(dc_linear), VP, VP, VP, I32, I32, I32, I32, VP, P(I32)]),
         "dc_layer_forward": (I32, [P(dc_linear), VP, VP, VP, P(VP), VP, I32, I32, I32, I32, VP, SZ, VP]),
         "dc_unpack_codes_debug": (I32, [P(dc_delta_handle), I32, VP, VP]),
         "dc_read_device_status": (I32, [VP, VP, P(I32)]),
@@ -99,6 +100,7 @@ def exported_symbols() -> list[str]:
     return ["dc_last_error", "dc_version", "dc_packed_size", "dc_quantize_rtn", "dc_pack_upload",
             "dc_quantize_pack_device", "dc_quantize_scratch_size", "dc_tenant_table_upload",
             "dc_workspace_size", "dc_build_segments", "dc_read_segments", "dc_delta_linear_segmented",
+            "dc_delta_linear_segmented_static",
             "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status", "dc_profile_begin",
             "dc_profile_end"]
 
@@ -256,6 +258,22 @@ def dc_delta_linear_segmented(lin: dc_linear, x, y, tenant_ids, T: int, flags: i
     _check(_load().dc_delta_linear_segmented(C.byref(lin), _ptr(x), _ptr(y), _ptr(tenant_ids), T, _dtype_code(x),
                                              _dtype_code(y), flags, _ptr(ws), ws.numel() * ws.element_size(),
                                              _stream(stream)))
+
+
+STATIC_WORKSPACE_BYTES = 16 << 20  # DC_STATIC_WORKSPACE_BYTES
+
+
+def dc_delta_linear_segmented_static(lin: dc_linear, x, y, tenant_ids, T: int, flags: int, stream=None,
+                                     read_status: bool = False):
+    """dc_delta_linear_segmented on the library's static workspace (no workspace argument).
+
+    Returns the device status word of the call when read_status is set (the call then waits for
+    the stream), else None."""
+    v = C.c_int32(0)
+    _check(_load().dc_delta_linear_segmented_static(C.byref(lin), _ptr(x), _ptr(y), _ptr(tenant_ids), T,
+                                                    _dtype_code(x), _dtype_code(y), flags, _stream(stream),
+                                                    C.byref(v) if read_status else None))
+    return v.value if read_status else None
 
 
 def dc_layer_forward(lins, x_h, x_o, x_f, ys, tenant_ids, T: int, flags: int, ws, stream=None):

@@ -25,6 +25,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "dc.h"
 #include "dc_internal.h"
@@ -1907,4 +1908,56 @@ extern "C" dc_status dc_read_device_status(void* ws, void* stream, int32_t* host
   if (st) return st;
   *host_status = v;
   return dc_cuda_check(cudaMemsetAsync(ws, 0, 4, s), "status clear");
+}
+
+// ---------------------------------------------------------------------------------------------
+// Allocation-free serving of one linear from a workspace compiled into the library.  For callers
+// that cannot allocate per call (no caching allocator, or a device memory plan fixed at start-up):
+// the workspace is a static device array, and its device address is looked up once per device.
+// ---------------------------------------------------------------------------------------------
+static __device__ __align__(256) uint8_t dc_static_ws[DC_STATIC_WORKSPACE_BYTES];
+
+namespace {
+constexpr int kStaticMaxDevices = 64;
+std::mutex g_static_mu;
+void* g_static_ptr[kStaticMaxDevices];  // device address of dc_static_ws per device, once looked up
+}  // namespace
+
+extern "C" dc_status dc_delta_linear_segmented_static(const dc_linear* lin, const void* x, void* y,
+                                                      const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
+                                                      int32_t dtype_out, int32_t flags, void* stream,
+                                                      int32_t* host_status) {
+  dc_clear_error();
+  if (!lin) return dc_fail(DC_ERR_INVALID_ARG, "null linear");
+  if (flags & DC_REUSE_ROUTING)
+    return dc_fail(DC_ERR_INVALID_ARG, "the static workspace rebuilds the routing on every call (no DC_REUSE_ROUTING)");
+  if (T < 0) return dc_fail(DC_ERR_INVALID_ARG, "negative T");
+  if (T == 0) return DC_OK;
+  const size_t need =
+      dc_workspace_size(T, lin->max_rank, std::max(lin->d_in, lin->d_out), 1, lin->n_tenants);
+  if (need == 0) return dc_fail(DC_ERR_INVALID_ARG, "invalid sizes in the linear");
+  if (need > DC_STATIC_WORKSPACE_BYTES)
+    return dc_fail(DC_ERR_WORKSPACE,
+                   "this request needs %zu bytes of workspace; the static workspace holds %zu "
+                   "(use dc_delta_linear_segmented with a caller workspace)",
+                   need, (size_t)DC_STATIC_WORKSPACE_BYTES);
+  int dev = 0;
+  dc_status st = dc_cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
+  if (st) return st;
+  if (dev < 0 || dev >= kStaticMaxDevices) return dc_fail(DC_ERR_UNSUPPORTED, "device index %d", dev);
+  void* ws = nullptr;
+  {
+    std::lock_guard<std::mutex> lock(g_static_mu);
+    if (!g_static_ptr[dev]) {
+      void* p = nullptr;
+      st = dc_cuda_check(cudaGetSymbolAddress(&p, dc_static_ws), "cudaGetSymbolAddress(static workspace)");
+      if (st) return st;
+      g_static_ptr[dev] = p;
+    }
+    ws = g_static_ptr[dev];
+  }
+  st = dc_delta_linear_segmented(lin, x, y, tenant_ids_dev, T, dtype_in, dtype_out, flags, ws,
+                                 DC_STATIC_WORKSPACE_BYTES, stream);
+  if (st || !host_status) return st;
+  return dc_read_device_status(ws, stream, host_status);
 }
