@@ -2,6 +2,7 @@
 // the host packer and the uploads.  No device memory is allocated here.
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdarg>
 #include <cstdio>
@@ -209,7 +210,15 @@ extern "C" dc_status dc_pack_upload(const dc_factor_desc* desc, const uint8_t* c
   if (dev_bytes < (size_t)L.bytes)
     return dc_fail(DC_ERR_WORKSPACE, "destination holds %zu bytes, need %lld", dev_bytes, (long long)L.bytes);
   std::vector<uint8_t> blob((size_t)L.bytes, 0);
-  DcPlain P{codes_u, codes_v, sz_u, sz_v, S};
+  // bound on the U scales of the 2/3-bit bands (scales are positive fp16 values)
+  double umax = 0.0;
+  for (int b = 0; b < L.n_bands; ++b) {
+    const DcBand& B = L.band[b];
+    if (B.bits == 8) continue;
+    for (int64_t i = (int64_t)B.r0 * L.groups_out; i < (int64_t)(B.r0 + B.rank) * L.groups_out; ++i)
+      umax = std::max(umax, std::fabs(dc_f16_to_f64(sz_u[2 * i])));
+  }
+  DcPlain P{codes_u, codes_v, sz_u, sz_v, S, (float)umax};
   dc_pack_host(L, P, blob.data());
   cudaStream_t s = (cudaStream_t)stream;
   st = dc_cuda_check(cudaMemcpyAsync(dev_dst, blob.data(), blob.size(), cudaMemcpyHostToDevice, s), "upload");

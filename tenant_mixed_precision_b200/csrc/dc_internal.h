@@ -51,23 +51,24 @@ struct alignas(16) DcVItem {
 
 // One (linear, segment) record for the output kernel, self-contained.
 struct DcUBand {
-  int32_t bits, rank, r0, bsm_off;
-  int32_t quads, steps, last, region;  // region: bytes of the band inside one 128-row group's run
-  int64_t boff;                        // offset of the band inside a run
-  int32_t otile;                       // bytes per 16-row tile (2/3-bit) or R8 (8-bit)
-  int32_t pad;
+  int32_t bits, rank, r0;
+  int32_t quads, steps, last;  // U geometry of the band (dc_layout.h)
+  int32_t nblk, full;          // blocks per 128-row group and bytes of a full block
+  int32_t boff;                // offset of the band inside a run
+  int32_t pad[3];
 };
 struct alignas(16) DcURec {  // moved with 16-byte vector loads and stores
   int64_t blob;
   int64_t u_off;  // start of the 128-row group runs (blob-relative)
-  int32_t valid, tenant, st, len, r, r4, n_bands, u_unit, u_meta_in, pad[3];
+  int32_t valid, tenant, st, len, r, n_bands, u_unit;
+  float umax;     // bound on the U scales of the 2/3-bit bands
   DcUBand band[DC_MAX_BANDS];
 };
 
 // Workspace layout (byte offsets from the workspace base).
 struct DcWs {
   int32_t T, max_rank, max_d_in, n_lin, n_in, r_stride, max_items, max_tenants, nkb, pad;
-  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, total;
+  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, total;
 };
 
 DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, int32_t max_tenants);

@@ -133,6 +133,7 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.tws = take((int64_t)n_lin * T * W.r_stride * 4);
   W.yd = take((int64_t)n_lin * T * W.max_d_in * 4);
   W.dflag = take((int64_t)n_lin * T);
+  W.tmax = take((int64_t)n_lin * T * 4);
   W.total = off;
   return W;
 }
@@ -156,7 +157,7 @@ struct DcFwd {
   DcLinDev lin[7];
   const void* x[3];
   int32_t dx[3];
-  int32_t n_lin, T, dtype_in, dtype_out, flags, bsm_max;
+  int32_t n_lin, T, dtype_in, dtype_out, flags, pad;
   int32_t order[7];        // launch order of the linears in the U kernel (largest first)
   int32_t tile_prefix[8];  // cumulative 128-row output tiles in that order
   DcWs ws;
@@ -175,6 +176,7 @@ struct WsPtr {
   float* tws;
   float* yd;
   uint8_t* dflag;
+  int* tmax;  // per (linear, sorted token): max |t| over the 2/3-bit ranks, as fp32 bits
 };
 __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   WsPtr p;
@@ -190,6 +192,7 @@ __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   p.tws = (float*)(ws + W.tws);
   p.yd = (float*)(ws + W.yd);
   p.dflag = ws + W.dflag;
+  p.tmax = (int*)(ws + W.tmax);
   return p;
 }
 
@@ -275,17 +278,21 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
   R.tenant = tau;
   R.st = st;
   R.len = len;
-  R.r = R.r4 = R.n_bands = R.u_unit = R.u_meta_in = 0;
+  R.r = R.n_bands = R.u_unit = 0;
+  R.umax = 0.f;
   R.u_off = 0;
-  R.pad[0] = R.pad[1] = R.pad[2] = 0;
+  for (int b = 0; b < DC_MAX_BANDS; ++b) {
+    DcUBand& U = R.band[b];
+    U.bits = U.rank = U.r0 = U.quads = U.steps = U.last = U.nblk = U.full = U.boff = 0;
+    U.pad[0] = U.pad[1] = U.pad[2] = 0;
+  }
   DcLayout L;
   L.valid = 0;
   if (tau < F.lin[p].n_tenants) {
     const dc_delta_handle* h = F.lin[p].tenants + tau;
     if (h->dev_base != 0) {
       L = dc_layout(h->desc);
-      if (!L.valid || L.d_out != F.lin[p].d_out || L.d_in != F.lin[p].d_in || L.r > W.r_stride ||
-          L.bsm_total > F.bsm_max) {
+      if (!L.valid || L.d_out != F.lin[p].d_out || L.d_in != F.lin[p].d_in || L.r > W.r_stride) {
         L.valid = 0;
         set_status(P.st, DC_ERR_SHAPE);
       }
@@ -294,30 +301,22 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
       R.blob = (int64_t)h->dev_base;
       R.valid = 1;
       R.r = L.r;
-      R.r4 = L.r4;
       R.n_bands = L.n_bands;
       R.u_off = L.u_off;
       R.u_unit = (int32_t)L.u_unit;
-      R.u_meta_in = (int32_t)L.u_meta_in;
-      for (int b = 0; b < DC_MAX_BANDS; ++b) {
+      R.umax = *reinterpret_cast<const float*>(reinterpret_cast<const uint8_t*>(h->dev_base) + L.umax_off);
+      for (int b = 0; b < L.n_bands; ++b) {
         DcUBand& U = R.band[b];
-        if (b >= L.n_bands) {
-          U.bits = U.rank = U.r0 = U.bsm_off = U.quads = U.steps = U.last = U.region = U.otile = U.pad = 0;
-          U.boff = 0;
-          continue;
-        }
         const DcBand& B = L.band[b];
         U.bits = B.bits;
         U.rank = B.rank;
         U.r0 = B.r0;
-        U.bsm_off = B.bsm_off;
         U.quads = B.u_quads;
         U.steps = B.u_steps;
         U.last = B.u_last;
-        U.otile = (int32_t)B.u_otile_bytes;
-        U.region = (int32_t)B.u_region;
-        U.boff = B.u_boff;
-        U.pad = 0;
+        U.nblk = B.u_nblk;
+        U.full = B.u_full;
+        U.boff = (int32_t)B.u_boff;
       }
     }
   }
@@ -752,6 +751,7 @@ __global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__
         // combine the three limbs (lane t holds limb t), scale by 2^-e and S, store t
         const float lw = (float)(1 << (8 * min(t, 2)));
         const float* S = reinterpret_cast<const float*>(d.sbase);
+        float tmx[DC_V_TOKS] = {0.f, 0.f, 0.f, 0.f};  // max |t| per pass token over this warp's rows
 #pragma unroll
         for (int pr = 0; pr < 2; ++pr)
 #pragma unroll
@@ -765,9 +765,22 @@ __global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__
               const int rl = 16 * warp + row;  // row within the item
               const int tok = d.tok0 + tk;
               const int e = P.xe[d.m * T + tok];
-              P.tws[((int64_t)d.p * T + tok) * F.ws.r_stride + d.rank0 + rl] = ldexpf(v, -e) * S[rl];
+              const float tv = ldexpf(v, -e) * S[rl];
+              P.tws[((int64_t)d.p * T + tok) * F.ws.r_stride + d.rank0 + rl] = tv;
+              tmx[tk] = fmaxf(tmx[tk], fabsf(tv));
             }
           }
+        if (d.bits != 8) {  // bound for the output kernel's fixed-point exponent (2/3-bit ranks)
+#pragma unroll
+          for (int tk = 0; tk < DC_V_TOKS; ++tk) {
+            float m = tmx[tk];
+            m = fmaxf(m, __shfl_xor_sync(FULLMASK, m, 4));
+            m = fmaxf(m, __shfl_xor_sync(FULLMASK, m, 8));
+            m = fmaxf(m, __shfl_xor_sync(FULLMASK, m, 16));
+            if (lane == 0 && tk < d.ntok && m > 0.f)
+              atomicMax(P.tmax + d.p * T + d.tok0 + tk, __float_as_int(m));
+          }
+        }
       }
     }
     __syncwarp();
@@ -778,47 +791,85 @@ __global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__
 
 // ---------------------------------------------------------------------------------------------
 // k_udelta: ydelta[token, row] = (U_hat (scale * t))[row] for every token of every segment with a
-// delta.  Persistent CTAs of 8 consumer warps + 1 producer warp over items (linear, segment,
-// 128-row output group); segments partition the tokens, so items write disjoint outputs.  Per
-// 4-token pass the producer streams the item's U_hat codes of every band, the U meta of its
-// 128-row group and the pass's t rows into a shared-memory stage; consumer warp w owns rows
-// 16w..16w+15 of the group.
+// delta.  Work is taken from a global counter in chunks of (linear, segment, up to U_CHUNK
+// consecutive 128-row output groups).  For each pass of <= 4 tokens and each group of the chunk
+// the producer warp streams the group's U blocks in batches of consecutive blocks (codes of the
+// eight 16-row tiles and the meta of the blocks' ranks: one bulk copy) together with the pass's
+// t values of the batch's ranks (one copy per token) through a ring of shared-memory stages.
+// Consumer warp w owns rows 16w..16w+15 of the group.
+//
+// Arithmetic of a (group, pass) unit: B = scale * t is written, per token, as the fixed-point
+// integer rint(B * 2^e) with e fixed by the bound umax * max|t| (so |B * 2^e| < 2^21): one fp32
+// FMA with the constant 1.5 * 2^23 leaves rint(B * 2^e) + 2^22 in the low 23 bits of the result,
+// whose three low bytes are the unsigned limbs of the operand.  The tensor cores multiply the u8
+// codes by those u8 limbs exactly (mma m16n8k32 u8.u8 -> s32); B column 6 is all ones, giving
+// the codes' row sums, which remove the 2^22 bias.  The zero points are removed in fp32
+// (sum over ranks of zero * scale * t), then the exponent.  8-bit bands use a scalar fp32 path.
 // ---------------------------------------------------------------------------------------------
-#define U_STAGES 2
-#define U_STAGE_BYTES (100 * 1024)
+#define U_STAGES 4
+#define U_STAGE_BYTES 24576  // a batch of blocks (codes + meta) and the t windows of its tokens
+#define U_CTAS_PER_SM 2      // two CTAs per SM: their producers' and consumers' stalls overlap
+#define U_MAXSUB 8           // blocks per batch
+#define U_MAXBLK 64          // blocks per (linear, tenant) U run of one group
+#define U_CHUNK 4            // 128-row output groups per chunk of work
+#define U_BROW 288           // row stride of the staged limb matrix (rows g and g+4 on different banks)
+#define U_BBUF (12 * U_BROW) // one limb matrix: 2 token pairs x (3 limbs x 2 tokens)
+#define U_BCONST (2 * U_BROW) // B columns 6 and 7 of every step: a row of ones and a row of zeros
 #define U_CONSUMERS 8
 #define U_THREADS (32 * (U_CONSUMERS + 1))
+#define U_MAGIC 12582912.0f  // 1.5 * 2^23
 
-struct UBandD {
-  int bits, rank, r0, bsm_off, quads, steps, last, otile, off;
-};
 struct UDesc {
-  int kind;  // 1 delta pass, 2 end
-  int p, ot, tok0, ntok;
-  int n_bands, r, off_meta, off_t, tstride, error;
-  UBandD band[DC_MAX_BANDS];
+  int kind;              // 1 batch, 2 end
+  int p, go, tok0, ntok;
+  int nsub;              // blocks in the batch
+  int code_bytes;        // bytes of the batch's blocks (the t windows follow)
+  int tfl;               // floats per token t window
+  int t_shift;           // position of the batch's first rank inside the t window
+  int ufirst, ulast;     // the batch opens / closes its (group, pass) unit
+  int error;
+  int sub[U_MAXSUB][2];  // per block: bits | nq << 4 | ns << 8 | last << 16, and nr | tile_bytes << 16
+  float pe[DC_V_TOKS];   // 2^e per pass token
+  float ie[DC_V_TOKS];   // 2^-e
+};
+
+struct UBlkE {  // producer-side table of a run's blocks
+  int off, bytes, p0, p1, nr, r0;
 };
 
 struct USmemTail {
   UDesc desc[U_STAGES];
   uint64_t full[U_STAGES];
   uint64_t empty[U_STAGES];
-  DcURec rec;  // producer: record of the current segment
-  int exps[DC_V_TOKS];
-  int zc[2][3][2];
-  float red[U_CONSUMERS][DC_V_TOKS];
+  DcURec rec;                    // producer: record of the current chunk
+  UBlkE tbl[U_MAXBLK];           // producer: blocks of the current chunk's runs
+  int bfirst[U_MAXBLK + 1];      // producer: batches of the current pass (first block of each)
+  int nbatch;
+  float zpart[2][U_CONSUMERS][DC_V_TOKS];  // per-warp zero-point sums (unit parity)
+  float s8[U_CONSUMERS][16][DC_V_TOKS];    // 8-bit band partials of a unit
 };
 
-// item u -> (linear p, segment sg, output group ot); linears in F.order, segment-major inside a linear
-__device__ __forceinline__ bool ud_item(const DcFwd& F, int nseg, int u, int& p, int& sg, int& ot) {
+// D += A(u8, 16x32, row) * B(u8, 32x8, col), int32 accumulate.
+__device__ __forceinline__ void mma_u8u8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// chunk u -> (linear p, segment sg, first group go0, groups ngo); linears in F.order
+__device__ __forceinline__ bool ud_chunk(const DcFwd& F, int nseg, int u, int& p, int& sg, int& go0, int& ngo) {
   for (int i = 0; i < F.n_lin; ++i) {
     const int q = F.order[i];
-    const int n_ot = F.lin[q].d_out / 128;
-    const int cnt = nseg * n_ot;
+    const int G = F.lin[q].d_out / 128;
+    const int nc = (G + U_CHUNK - 1) / U_CHUNK;
+    const int cnt = nseg * nc;
     if (u < cnt) {
       p = q;
-      sg = u / n_ot;
-      ot = u % n_ot;
+      sg = u / nc;
+      go0 = (u % nc) * U_CHUNK;
+      ngo = min(U_CHUNK, G - go0);
       return true;
     }
     u -= cnt;
@@ -826,215 +877,73 @@ __device__ __forceinline__ bool ud_item(const DcFwd& F, int nseg, int u, int& p,
   return false;
 }
 
-template <int NTOK>
-__device__ __forceinline__ void ud_pass(const DcFwd& F, const WsPtr& P, const UDesc& d, const uint8_t* stage,
-                                        uint8_t* bsm, USmemTail* tail, int warp, int lane) {
-  constexpr int NPAIR = (NTOK + 1) / 2;
-  const int tid = threadIdx.x;  // 0..255
-  const int g = lane >> 2, t = lane & 3;
-  const uint8_t* umeta = stage + d.off_meta;
-  const float* tst = reinterpret_cast<const float*>(stage + d.off_t);
-  const int T = F.ws.T;
-  // ---- B = scale * t: per-token exponent from the largest |B| over the 2/3-bit bands
-  float mx[NTOK];
-#pragma unroll
-  for (int q = 0; q < NTOK; ++q) mx[q] = 0.f;
-  for (int b = 0; b < d.n_bands; ++b) {
-    const UBandD& Bd = d.band[b];
-    if (Bd.bits == 8) continue;
-    for (int i = tid; i < Bd.rank; i += 32 * U_CONSUMERS) {
-      const int r = Bd.r0 + i;
-      const float sc = __low2float(*reinterpret_cast<const __half2*>(umeta + 4 * r));
-#pragma unroll
-      for (int q = 0; q < NTOK; ++q) mx[q] = fmaxf(mx[q], fabsf(sc * tst[q * d.tstride + r]));
-    }
-  }
-#pragma unroll
-  for (int q = 0; q < NTOK; ++q) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) mx[q] = fmaxf(mx[q], __shfl_xor_sync(FULLMASK, mx[q], o));
-    if (lane == 0) tail->red[warp][q] = mx[q];
-  }
-  if (tid < 12) (&tail->zc[0][0][0])[tid] = 0;
-  named_bar(1, 32 * U_CONSUMERS);
-  if (tid < NTOK) {
-    float m = 0.f;
-#pragma unroll
-    for (int ww = 0; ww < U_CONSUMERS; ++ww) m = fmaxf(m, tail->red[ww][tid]);
-    int e = 0;
-    if (m > 0.f) {
-      int E;
-      frexpf(m, &E);
-      e = 22 - E;
-    }
-    tail->exps[tid] = e;
-  }
-  named_bar(1, 32 * U_CONSUMERS);
-  // ---- limbs of B into the staging buffer, 4 consecutive ranks per thread (ranks past the band's
-  //      end up to its 32-rank padding are written as zeros); zero-point correction sums
-  int zc[NPAIR][3][2];
-#pragma unroll
-  for (int a = 0; a < NPAIR; ++a)
-#pragma unroll
-    for (int b = 0; b < 3; ++b) zc[a][b][0] = zc[a][b][1] = 0;
-  float pe[NTOK];
-#pragma unroll
-  for (int q = 0; q < NTOK; ++q) pe[q] = ldexpf(1.f, tail->exps[q]);
-  for (int b = 0; b < d.n_bands; ++b) {
-    const UBandD& Bd = d.band[b];
-    if (Bd.bits == 8) continue;
-    const int padded = (Bd.rank + 31) & ~31;
-    for (int i4 = 4 * tid; i4 < padded; i4 += 4 * 32 * U_CONSUMERS) {
-      float sc[4];
-      int z[4];
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        const bool ok = i4 + c < Bd.rank;
-        const __half2 mz = *reinterpret_cast<const __half2*>(umeta + 4 * (Bd.r0 + (ok ? i4 + c : 0)));
-        sc[c] = ok ? __low2float(mz) : 0.f;
-        z[c] = ok ? (int)__high2float(mz) : 0;
-      }
-#pragma unroll
-      for (int q = 0; q < NTOK; ++q) {
-        uint32_t w0 = 0, w1 = 0, w2 = 0;
-        const int pr = q >> 1, tk = q & 1;
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int rr = Bd.r0 + (i4 + c < Bd.rank ? i4 + c : 0);
-          const int bi = __float2int_rn(sc[c] * tst[q * d.tstride + rr] * pe[q]);
-          const int l0 = sext8(bi);
-          const int x1 = (bi - l0) >> 8;
-          const int l1 = sext8(x1);
-          const int l2 = (x1 - l1) >> 8;
-          w0 |= (uint32_t)(l0 & 0xff) << (8 * c);
-          w1 |= (uint32_t)(l1 & 0xff) << (8 * c);
-          w2 |= (uint32_t)(l2 & 0xff) << (8 * c);
-          zc[pr][0][tk] += z[c] * l0;
-          zc[pr][1][tk] += z[c] * l1;
-          zc[pr][2][tk] += z[c] * l2;
-        }
-        uint8_t* col = bsm + (int64_t)(pr * 6) * F.bsm_max + Bd.bsm_off + i4;
-        *reinterpret_cast<uint32_t*>(col + (0 * 2 + tk) * F.bsm_max) = w0;
-        *reinterpret_cast<uint32_t*>(col + (1 * 2 + tk) * F.bsm_max) = w1;
-        *reinterpret_cast<uint32_t*>(col + (2 * 2 + tk) * F.bsm_max) = w2;
-      }
-    }
-  }
-#pragma unroll
-  for (int a = 0; a < NPAIR; ++a)
-#pragma unroll
-    for (int b = 0; b < 3; ++b)
-#pragma unroll
-      for (int k = 0; k < 2; ++k) {
-        if (2 * a + k >= NTOK) continue;
-        int v = zc[a][b][k];
-#pragma unroll
-        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
-        if (lane == 0 && v != 0) atomicAdd(&tail->zc[a][b][k], v);
-      }
-  named_bar(1, 32 * U_CONSUMERS);
-  // ---- MMA over the rank steps of every 2/3-bit band (codes of this warp's 16 rows)
-  int C[NPAIR][4][4];  // [pair][position][reg]
-#pragma unroll
-  for (int a = 0; a < NPAIR; ++a)
-#pragma unroll
-    for (int b = 0; b < 4; ++b)
-#pragma unroll
-      for (int q = 0; q < 4; ++q) C[a][b][q] = 0;
-  float s8v[NPAIR];  // 8-bit band contribution of lane t: (row g + 8*(t>>1), token t&1) per pair
-#pragma unroll
-  for (int a = 0; a < NPAIR; ++a) s8v[a] = 0.f;
-  const bool bl = g < 6;  // B columns 2*limb + token; columns 6 and 7 are zero
-  for (int b = 0; b < d.n_bands; ++b) {
-    const UBandD& Bd = d.band[b];
-    if (Bd.bits == 8) {
-      const int row = g + 8 * (t >> 1);
-      const uint8_t* ur = stage + Bd.off + (16 * warp + row) * Bd.rank;
-#pragma unroll
-      for (int pr = 0; pr < NPAIR; ++pr) {
-        const int q = 2 * pr + (t & 1);
-        if (q >= NTOK) continue;
-        float sum = 0.f;
-        for (int i = 0; i < Bd.rank; ++i) {
-          const __half2 mz = *reinterpret_cast<const __half2*>(umeta + 4 * (Bd.r0 + i));
-          sum = fmaf(((float)ur[i] - __high2float(mz)) * __low2float(mz), tst[q * d.tstride + Bd.r0 + i], sum);
-        }
-        s8v[pr] += sum;
-      }
-      continue;
-    }
-    const uint8_t* ub = stage + Bd.off + (int64_t)warp * Bd.otile;
-    const uint8_t* bcol = bsm + (int64_t)(bl ? g : 0) * F.bsm_max + Bd.bsm_off + 8 * t;
-#pragma unroll 2
-    for (int q = 0; q < Bd.quads; ++q) {
-      const uint4 wq = *reinterpret_cast<const uint4*>(ub + 512 * q + 16 * lane);
-#pragma unroll
-      for (int ps = 0; ps < 4; ++ps) {
-        const int step = 4 * q + ps;
-        const uint32_t msk = 0x03030303u << (2 * ps);
-        const uint32_t a0 = wq.x & msk, a1 = wq.y & msk, a2 = wq.z & msk, a3 = wq.w & msk;
-#pragma unroll
-        for (int pr = 0; pr < NPAIR; ++pr) {
-          const uint2 bb = bl ? *reinterpret_cast<const uint2*>(bcol + (int64_t)(6 * pr) * F.bsm_max + 32 * step)
-                              : make_uint2(0, 0);
-          mma_u8s8(C[pr][ps], a0, a1, a2, a3, bb.x, bb.y);
-        }
-      }
-    }
-    const uint8_t* sb = ub + (int64_t)512 * Bd.quads;
-    for (int sidx = 0; sidx < Bd.steps; ++sidx) {
-      const int valid = (sidx == Bd.steps - 1) ? Bd.last : 32;
-      const int nl = dc_u_step_lanes(valid);
-      const int ntv = nl / 8;
-      uint32_t wv = 0, hv = 0;
-      if (t < ntv) {
-        wv = *reinterpret_cast<const uint32_t*>(sb + 4 * (g * ntv + t));
-        if (Bd.bits == 3) hv = *reinterpret_cast<const uint16_t*>(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t));
-      }
-      uint32_t a[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        a[j] = reg_shift2(wv, j);
-        if (Bd.bits == 3) a[j] |= u_reg_hi3(hv, j);
-      }
-      const int step = 4 * Bd.quads + sidx;
-#pragma unroll
-      for (int pr = 0; pr < NPAIR; ++pr) {
-        const uint2 bb = bl ? *reinterpret_cast<const uint2*>(bcol + (int64_t)(6 * pr) * F.bsm_max + 32 * step)
-                            : make_uint2(0, 0);
-        mma_u8s8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
-      }
-      sb += dc_u_step_bytes(Bd.bits, nl);
-    }
-  }
-  // ---- combine positions and limbs (lane t holds limb t of pair tokens 0, 1); write ydelta
-  const float lw = (float)(1 << (8 * min(t, 2)));
-  float* yd = P.yd + (int64_t)d.p * T * F.ws.max_d_in;
-#pragma unroll
-  for (int pr = 0; pr < NPAIR; ++pr)
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int tk = q & 1;
-      const int qq = 2 * pr + tk;
-      if (qq >= NTOK) continue;
-      const int cl = C[pr][0][q] + (C[pr][1][q] >> 2) + (C[pr][2][q] >> 4) + (C[pr][3][q] >> 6);
-      float v = t < 3 ? (float)(cl - tail->zc[pr][t][tk]) * lw : 0.f;
-      v += __shfl_xor_sync(FULLMASK, v, 1);
-      v += __shfl_xor_sync(FULLMASK, v, 2);
-      v = ldexpf(v, -tail->exps[qq]);
-      v += __shfl_sync(FULLMASK, s8v[pr], (lane & ~3) | q);
-      if (t == 0) {
-        const int row = d.ot * 128 + 16 * warp + g + 8 * (q >> 1);
-        yd[(int64_t)(d.tok0 + qq) * F.ws.max_d_in + row] = v;
-      }
-    }
-  named_bar(1, 32 * U_CONSUMERS);  // the staging buffer is reused by the next pass
+// Exponent e of a pass token from the bound umax * max|t|: |scale * t * 2^e| < 2^21.
+__device__ __forceinline__ int ud_exponent(float umax, int tmax_bits) {
+  const float bound = umax * __int_as_float(tmax_bits);
+  if (!(bound > 0.f)) return 0;
+  int E;
+  frexpf(bound, &E);
+  return max(-120, min(120, 21 - E));
 }
 
-__global__ void __launch_bounds__(U_THREADS, 1) k_udelta(const __grid_constant__ DcFwd F, uint8_t* ws) {
+// MMA over one block for this warp's 16-row tile.  C[pair][position][reg].
+template <int NPAIR>
+__device__ __forceinline__ void ud_mma(const uint8_t* blk, int bits, int nq, int ns, int last, int tile_bytes,
+                                       const uint8_t* bsm, const uint8_t* bconst, int (&C)[2][4][4], int warp,
+                                       int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  const uint8_t* ub = blk + warp * tile_bytes;
+  // B column g: limb rows 0..5 of pair 0 (pair 1 six rows further), column 6 a row of ones (the
+  // codes' row sums), column 7 a row of zeros; both constant rows sit after the two limb matrices
+  const uint8_t* brow = (g < 6 ? bsm + g * U_BROW : bconst + (g - 6) * U_BROW) + 8 * t;
+  const int pstride = g < 6 ? 6 * U_BROW : 0;
+#pragma unroll 2
+  for (int q = 0; q < nq; ++q) {
+    const uint4 wq = *reinterpret_cast<const uint4*>(ub + 512 * q + 16 * lane);
+#pragma unroll
+    for (int ps = 0; ps < 4; ++ps) {
+      const int step = 4 * q + ps;
+      const uint32_t msk = 0x03030303u << (2 * ps);
+      const uint32_t a0 = wq.x & msk, a1 = wq.y & msk, a2 = wq.z & msk, a3 = wq.w & msk;
+#pragma unroll
+      for (int pr = 0; pr < NPAIR; ++pr) {
+        const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * step);
+        mma_u8u8(C[pr][ps], a0, a1, a2, a3, bb.x, bb.y);
+      }
+    }
+  }
+  const uint8_t* sb = ub + 512 * nq;
+#pragma unroll 1
+  for (int si = 0; si < ns; ++si) {
+    const int valid = (si == ns - 1) ? last : 32;
+    const int nl = dc_u_step_lanes(valid);
+    const int ntv = nl / 8;
+    uint32_t wv = 0, hv = 0;
+    if (t < ntv) {
+      wv = *reinterpret_cast<const uint32_t*>(sb + 4 * (g * ntv + t));
+      if (bits == 3) hv = *reinterpret_cast<const uint16_t*>(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t));
+    }
+    uint32_t a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a[j] = reg_shift2(wv, j);
+      if (bits == 3) a[j] |= u_reg_hi3(hv, j);
+    }
+    const int step = 4 * nq + si;
+#pragma unroll
+    for (int pr = 0; pr < NPAIR; ++pr) {
+      const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * step);
+      mma_u8u8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
+    }
+    sb += dc_u_step_bytes(bits, nl);
+  }
+}
+
+__global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __grid_constant__ DcFwd F, uint8_t* ws) {
   extern __shared__ __align__(128) uint8_t usm[];
-  uint8_t* bsm = usm + U_STAGES * U_STAGE_BYTES;
-  USmemTail* tail = reinterpret_cast<USmemTail*>(bsm + 12 * F.bsm_max);
+  uint8_t* bsm = usm + U_STAGES * U_STAGE_BYTES;  // two limb matrices, then the constant rows
+  uint8_t* bconst = bsm + 2 * U_BBUF;
+  USmemTail* tail = reinterpret_cast<USmemTail*>(bconst + U_BCONST);
   WsPtr P = ws_ptr(F.ws, ws);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = F.ws.T;
@@ -1045,83 +954,162 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_udelta(const __grid_constant__
     }
     fence_mbar_init();
   }
+  for (int i = threadIdx.x; i < U_BCONST / 4; i += blockDim.x)
+    reinterpret_cast<uint32_t*>(bconst)[i] = i < U_BROW / 4 ? 0x01010101u : 0u;
   __syncthreads();
   if (warp == U_CONSUMERS) {
     // ---------------- producer warp
     const int nseg = P.st[DC_WS_NSEG];
     constexpr int REC_VEC = sizeof(DcURec) / 16;
     uint32_t seq = 0;
-    int cur_p = -1, cur_sg = -1;
     auto acquire = [&](int& s) -> bool {
       s = seq % U_STAGES;
       if (seq >= U_STAGES && !mbar_wait(&tail->empty[s], ((seq / U_STAGES) - 1) & 1)) {
         set_status(P.st, DC_ERR_CUDA);
         return false;
       }
-      fence_proxy_async();
+      
       return true;
     };
-    for (;;) {
+    // next chunk: index, its record (lanes 0..14) and the tmax words of its first pass (lanes 0..3)
+    auto grab = [&](int& p, int& sg, int& go0, int& ngo, uint4& rv, int& tm) -> bool {
       int u = 0;
       if (lane == 0) u = atomicAdd(P.st + DC_WS_UCOUNTER, 1);
       u = __shfl_sync(FULLMASK, u, 0);
-      int p = 0, sg = 0, ot = 0;
-      if (nseg == 0 || !ud_item(F, nseg, u, p, sg, ot)) {
-        int s;
-        if (!acquire(s)) return;
-        if (lane == 0) {
-          tail->desc[s].kind = 2;
-          mbar_arrive(&tail->full[s]);
-        }
-        return;
-      }
-      if (p != cur_p || sg != cur_sg) {
-        const uint4 v = lane < REC_VEC ? ldg128(reinterpret_cast<const uint8_t*>(P.urecs + (int64_t)p * T + sg) + 16 * lane)
-                                       : make_uint4(0, 0, 0, 0);
-        __syncwarp();
-        if (lane < REC_VEC) reinterpret_cast<uint4*>(&tail->rec)[lane] = v;
-        __syncwarp();
-        cur_p = p, cur_sg = sg;
-      }
+      if (nseg == 0 || !ud_chunk(F, nseg, u, p, sg, go0, ngo)) return false;
+      rv = lane < REC_VEC ? ldg128(reinterpret_cast<const uint8_t*>(P.urecs + (int64_t)p * T + sg) + 16 * lane)
+                          : make_uint4(0, 0, 0, 0);
+      const int st0 = P.segs[3 * sg + 1], len = P.segs[3 * sg + 2];
+      tm = lane < min(DC_V_TOKS, len) ? P.tmax[p * T + st0 + lane] : 0;
+      return true;
+    };
+    int p = 0, sg = 0, go0 = 0, ngo = 0, tm = 0;
+    uint4 rv = make_uint4(0, 0, 0, 0);
+    bool have = grab(p, sg, go0, ngo, rv, tm);
+    while (have) {
+      __syncwarp();
+      if (lane < REC_VEC) reinterpret_cast<uint4*>(&tail->rec)[lane] = rv;
+      __syncwarp();
+      const int cp = p, cgo0 = go0, cngo = ngo;
+      int ctm = tm;
+      int np = 0, nsg = 0, ngo0 = 0, nngo = 0, ntm = 0;
+      uint4 nrv = make_uint4(0, 0, 0, 0);
+      const bool nhave = grab(np, nsg, ngo0, nngo, nrv, ntm);
       const DcURec& R = tail->rec;
-      if (!R.valid) continue;
-      const uint8_t* blob = reinterpret_cast<const uint8_t*>(R.blob);
-      for (int pt0 = R.st; pt0 < R.st + R.len; pt0 += DC_V_TOKS) {
-        const int ntok = min(DC_V_TOKS, R.st + R.len - pt0);
-        int s;
-        if (!acquire(s)) return;
-        uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
-        const int off_t = R.u_unit;  // a multiple of 16
-        const int tstride = F.ws.r_stride;
-        const int total = off_t + ntok * tstride * 4;
-        const bool fits = total <= U_STAGE_BYTES;
-        if (lane == 0) {
-          UDesc& d = tail->desc[s];
-          d.kind = 1;
-          d.p = p, d.ot = ot, d.tok0 = pt0, d.ntok = ntok;
-          d.n_bands = R.n_bands, d.r = R.r, d.off_meta = R.u_meta_in, d.off_t = off_t, d.tstride = tstride;
-          d.error = fits ? 0 : 1;
-          for (int b = 0; b < DC_MAX_BANDS; ++b) {
-            const DcUBand& B = R.band[b];
-            d.band[b] = UBandD{B.bits, B.rank, B.r0, B.bsm_off, B.quads, B.steps, B.last, B.otile, (int)B.boff};
-          }
-          if (!fits) set_status(P.st, DC_ERR_UNSUPPORTED);
-          if (fits) {
-            mbar_arrive_expect_tx(&tail->full[s], (uint32_t)total);
-            bulk_g2s(stage, blob + R.u_off + (int64_t)ot * R.u_unit, (uint32_t)R.u_unit, &tail->full[s]);
-            bulk_g2s(stage + off_t, P.tws + ((int64_t)p * T + pt0) * tstride, (uint32_t)(ntok * tstride * 4),
-                     &tail->full[s]);
-          } else {
-            mbar_arrive(&tail->full[s]);
-          }
+      int NB = 0;
+      for (int b = 0; b < R.n_bands; ++b) NB += R.band[b].nblk;
+      if (NB > U_MAXBLK) {
+        set_status(P.st, DC_ERR_UNSUPPORTED);
+      } else if (R.valid) {
+        // block table of the run, one lane per block
+        for (int i = lane; i < NB; i += 32) {
+          int b = 0, k = i;
+          while (k >= R.band[b].nblk) k -= R.band[b++].nblk;
+          const DcUBand& UB = R.band[b];
+          DcBand B;
+          B.bits = UB.bits, B.rank = UB.rank, B.r0 = UB.r0;
+          B.u_quads = UB.quads, B.u_steps = UB.steps, B.u_last = UB.last;
+          const DcUBlk K = dc_u_block(B, k);
+          UBlkE& E = tail->tbl[i];
+          E.off = UB.boff + k * UB.full;
+          E.bytes = K.bytes;
+          E.p0 = UB.bits | (K.nq << 4) | (K.ns << 8) | (K.last << 16);
+          E.p1 = K.nr | (K.tile_bytes << 16);
+          E.nr = K.nr;
+          E.r0 = UB.r0 + K.rr0;
         }
         __syncwarp();
-        ++seq;
+        const uint8_t* runs = reinterpret_cast<const uint8_t*>(R.blob) + R.u_off;
+        for (int pt0 = R.st; pt0 < R.st + R.len; pt0 += DC_V_TOKS) {
+          const int ntok = min(DC_V_TOKS, R.st + R.len - pt0);
+          if (pt0 != R.st) ctm = lane < ntok ? P.tmax[cp * T + pt0 + lane] : 0;
+          const int e = ud_exponent(R.umax, ctm);  // lane q: token q
+          const float pe = ldexpf(1.f, e), ie = ldexpf(1.f, -e);
+          if (lane == 0) {  // batches of consecutive blocks that fit a stage with this pass's t windows
+            int nbt = 0, i = 0;
+            while (i < NB) {
+              tail->bfirst[nbt++] = i;
+              int cb = 0, j = i;
+              while (j < NB && j - i < U_MAXSUB) {
+                const int w0 = tail->tbl[i].r0 & ~3;
+                const int tfl = (int)dc_align(tail->tbl[j].r0 + tail->tbl[j].nr, 4) - w0;
+                if (j > i && cb + tail->tbl[j].bytes + ntok * 4 * tfl > U_STAGE_BYTES) break;
+                cb += tail->tbl[j].bytes;
+                ++j;
+              }
+              i = j;
+            }
+            tail->bfirst[nbt] = NB;
+            tail->nbatch = nbt;
+          }
+          __syncwarp();
+          const int nbatch = tail->nbatch;
+          for (int go = cgo0; go < cgo0 + cngo; ++go) {
+            for (int j = 0; j < nbatch; ++j) {
+              const int f = tail->bfirst[j], nsub = tail->bfirst[j + 1] - f;
+              const UBlkE& E0 = tail->tbl[f];
+              const UBlkE& E1 = tail->tbl[f + nsub - 1];
+              const int code_bytes = E1.off + E1.bytes - E0.off;
+              const int w0 = E0.r0 & ~3;
+              const int tfl = (int)dc_align(E1.r0 + E1.nr, 4) - w0;
+              const bool fits = code_bytes + ntok * 4 * tfl <= U_STAGE_BYTES;
+              int s;
+              if (!acquire(s)) return;
+              uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
+              UDesc& d = tail->desc[s];
+              if (lane < 2 * nsub) d.sub[lane >> 1][lane & 1] = (lane & 1) ? tail->tbl[f + (lane >> 1)].p1
+                                                                            : tail->tbl[f + (lane >> 1)].p0;
+              if (lane < DC_V_TOKS) {
+                d.pe[lane] = pe;
+                d.ie[lane] = ie;
+              }
+              if (lane == 0) {
+                d.kind = 1;
+                d.p = cp, d.go = go, d.tok0 = pt0, d.ntok = ntok;
+                d.nsub = nsub, d.code_bytes = code_bytes, d.tfl = tfl, d.t_shift = E0.r0 - w0;
+                d.ufirst = j == 0, d.ulast = j == nbatch - 1;
+                d.error = fits ? 0 : 1;
+                if (fits) {
+                  mbar_arrive_expect_tx(&tail->full[s], (uint32_t)(code_bytes + ntok * 4 * tfl));
+                } else {
+                  set_status(P.st, DC_ERR_UNSUPPORTED);
+                  mbar_arrive(&tail->full[s]);
+                }
+              }
+              __syncwarp();
+              if (fits) {
+                if (lane == 0) {
+                  bulk_g2s(stage, runs + (int64_t)go * R.u_unit + E0.off, (uint32_t)code_bytes, &tail->full[s]);
+                } else if (lane <= ntok) {
+                  const int q = lane - 1;
+                  const float* src = P.tws + ((int64_t)cp * T + pt0 + q) * F.ws.r_stride + w0;
+                  bulk_g2s(stage + code_bytes + q * 4 * tfl, src, (uint32_t)(4 * tfl), &tail->full[s]);
+                }
+              }
+              __syncwarp();
+              ++seq;
+            }
+          }
+        }
       }
+      p = np, sg = nsg, go0 = ngo0, ngo = nngo, rv = nrv, tm = ntm;
+      have = nhave;
     }
+    int s;
+    if (!acquire(s)) return;
+    if (lane == 0) {
+      tail->desc[s].kind = 2;
+      mbar_arrive(&tail->full[s]);
+    }
+    return;
   }
   // ---------------- consumer warps
-  uint32_t seq = 0;
+  const int tid = threadIdx.x;  // 0..255
+  const int g = lane >> 2, t = lane & 3;
+  int C[2][4][4];
+  float zc[DC_V_TOKS];
+  float s8[2];
+  uint32_t seq = 0, nmma = 0, unit = 0;
   for (;;) {
     const int s = seq % U_STAGES;
     if (!mbar_wait(&tail->full[s], (seq / U_STAGES) & 1)) {
@@ -1131,17 +1119,133 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_udelta(const __grid_constant__
     const UDesc& d = tail->desc[s];
     if (d.kind == 2) return;
     const uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
+    const int ntok = d.ntok;
+    if (d.ufirst) {
+#pragma unroll
+      for (int a = 0; a < 2; ++a)
+#pragma unroll
+        for (int b = 0; b < 4; ++b)
+#pragma unroll
+          for (int q = 0; q < 4; ++q) C[a][b][q] = 0;
+#pragma unroll
+      for (int q = 0; q < DC_V_TOKS; ++q) zc[q] = 0.f;
+      s8[0] = s8[1] = 0.f;
+    }
     if (!d.error) {
-      switch (d.ntok) {
-        case 1: ud_pass<1>(F, P, d, stage, bsm, tail, warp, lane); break;
-        case 2: ud_pass<2>(F, P, d, stage, bsm, tail, warp, lane); break;
-        case 3: ud_pass<3>(F, P, d, stage, bsm, tail, warp, lane); break;
-        default: ud_pass<4>(F, P, d, stage, bsm, tail, warp, lane); break;
+      const float* tw = reinterpret_cast<const float*>(stage + d.code_bytes);
+      const int tfl = d.tfl;
+      float pe[DC_V_TOKS];
+#pragma unroll
+      for (int q = 0; q < DC_V_TOKS; ++q) pe[q] = d.pe[q];
+      int off = 0, ro = d.t_shift;
+      for (int i = 0; i < d.nsub; ++i) {
+        const int p0 = d.sub[i][0], p1 = d.sub[i][1];
+        const int bits = p0 & 15, nq = (p0 >> 4) & 15, ns = (p0 >> 8) & 255, last = p0 >> 16;
+        const int nr = p1 & 0xffff, tile_bytes = p1 >> 16;
+        const int code_bytes = bits == 8 ? (int)dc_align((int64_t)128 * nr, 16) : 8 * tile_bytes;
+        const uint8_t* blk = stage + off;
+        const uint8_t* meta = blk + code_bytes;
+        if (bits != 8) {
+          // ---- limbs of scale * t * 2^e for rank tid of the block, every pass token
+          uint8_t* bb = bsm + (nmma & 1) * U_BBUF;
+          if (tid < nr) {
+            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * tid);
+            const float sc = __low2float(mz), zs = sc * __high2float(mz);
+#pragma unroll
+            for (int q = 0; q < DC_V_TOKS; ++q) {
+              if (q < ntok) {
+                const float tq = tw[q * tfl + ro + tid];
+                const uint32_t v = __float_as_uint(fmaf(sc, tq * pe[q], U_MAGIC));
+                uint8_t* col = bb + (6 * (q >> 1) + (q & 1)) * U_BROW + tid;
+                col[0] = (uint8_t)v;
+                col[2 * U_BROW] = (uint8_t)(v >> 8);
+                col[4 * U_BROW] = (uint8_t)(v >> 16);
+                zc[q] = fmaf(zs, tq, zc[q]);
+              }
+            }
+          }
+          named_bar(1, 32 * U_CONSUMERS);
+          if (ntok > 2)
+            ud_mma<2>(blk, bits, nq, ns, last, tile_bytes, bb, bconst, C, warp, lane);
+          else
+            ud_mma<1>(blk, bits, nq, ns, last, tile_bytes, bb, bconst, C, warp, lane);
+          ++nmma;
+        } else {
+          // ---- 8-bit band: scalar fp32, lane = (row lane & 15, tokens 2 (lane >> 4) + {0, 1})
+          const int row = lane & 15, th = lane >> 4;
+          const uint8_t* cr = blk + (16 * warp + row) * nr;
+          for (int k = 0; k < nr; ++k) {
+            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
+            const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = 2 * th + h;
+              if (q < ntok) s8[h] = fmaf(f, tw[q * tfl + ro + k], s8[h]);
+            }
+          }
+        }
+        off += code_bytes + (int)dc_align((int64_t)4 * nr, 16);
+        ro += nr;
       }
     }
+    const bool ulast = d.ulast;
+    const int p = d.p, go = d.go, tok0 = d.tok0;
+    float ie[DC_V_TOKS];
+#pragma unroll
+    for (int q = 0; q < DC_V_TOKS; ++q) ie[q] = d.ie[q];
     __syncwarp();
     if (lane == 0) mbar_arrive(&tail->empty[s]);
     ++seq;
+    if (!ulast) continue;
+    // ---- epilogue of the (group, pass) unit; sums in a fixed order (deterministic)
+    float (*zp)[DC_V_TOKS] = tail->zpart[unit & 1];
+#pragma unroll
+    for (int q = 0; q < DC_V_TOKS; ++q) {
+      float v = zc[q];
+#pragma unroll
+      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
+      if (lane == 0) zp[warp][q] = v;
+    }
+    {
+      const int row = lane & 15, th = lane >> 4;
+      tail->s8[warp][row][2 * th] = s8[0];
+      tail->s8[warp][row][2 * th + 1] = s8[1];
+    }
+    named_bar(2, 32 * U_CONSUMERS);
+    float zs[DC_V_TOKS];
+#pragma unroll
+    for (int q = 0; q < DC_V_TOKS; ++q) {
+      float v = 0.f;
+      if (q < ntok) {
+#pragma unroll
+        for (int w = 0; w < U_CONSUMERS; ++w) v += zp[w][q];
+      }
+      zs[q] = v;
+    }
+#pragma unroll
+    for (int pr = 0; pr < 2; ++pr) {
+      if (2 * pr >= ntok) continue;
+      int Ct[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r)
+        Ct[r] = C[pr][0][r] + (C[pr][1][r] >> 2) + (C[pr][2][r] >> 4) + (C[pr][3][r] >> 6);
+      // lane t holds limb t (t < 3) or the row sums (t = 3, regs 0 and 2)
+      const int rs0 = __shfl_down_sync(FULLMASK, Ct[0], 3), rs1 = __shfl_down_sync(FULLMASK, Ct[2], 3);
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int l1 = __shfl_down_sync(FULLMASK, Ct[r], 1);
+        const int l2 = __shfl_down_sync(FULLMASK, Ct[r], 2);
+        const int q = 2 * pr + (r & 1);
+        const int rl = g + 8 * (r >> 1);
+        if (t == 0 && q < ntok) {
+          const int rsum = (r >> 1) ? rs1 : rs0;
+          const float v = (float)(l2 - 64 * rsum) * 65536.f + (float)l1 * 256.f + (float)Ct[r];
+          const float y = fmaf(v, ie[q], -zs[q]) + tail->s8[warp][rl][q];
+          P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + 16 * warp + rl] = y;
+        }
+      }
+    }
+    ++unit;
   }
 }
 
@@ -1413,43 +1517,41 @@ __global__ void k_unpack_v(const uint8_t* blob, DcLayout L, int bi, uint8_t* out
 __global__ void k_unpack_u(const uint8_t* blob, DcLayout L, int bi, uint8_t* out) {
   const DcBand& B = L.band[bi];
   const int64_t id = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (id >= (int64_t)B.rank * L.d_out) return;
+  const int i = (int)(id / L.d_out), o = (int)(id % L.d_out);  // rank inside the band, output row
+  const uint8_t* band = blob + L.u_off + (int64_t)(o >> 7) * L.u_unit + B.u_boff;
+  uint32_t code;
   if (B.bits == 8) {
-    if (id >= (int64_t)L.d_out * B.rank) return;
-    const int o = (int)(id / B.rank), i = (int)(id % B.rank);
-    const int go = o >> 7;
-    out[(int64_t)(B.r0 + i) * L.d_out + o] = blob[L.u_off + (int64_t)go * L.u_unit + B.u_boff + (int64_t)(o & 127) * B.rank + i];
-    return;
-  }
-  if (id >= (int64_t)(L.d_out / 16) * 32) return;
-  const int lane = (int)(id & 31), ot = (int)(id >> 5);
-  const int g = lane >> 2, t = lane & 3;
-  const uint8_t* ub = blob + L.u_off + (int64_t)(ot >> 3) * L.u_unit + B.u_boff + (int64_t)(ot & 7) * B.u_otile_bytes;
-  auto put = [&](uint32_t reg, int j, int rank_base) {
-    for (int b = 0; b < 4; ++b) {
-      const int rank = rank_base + 8 * t + 4 * (j >> 1) + b;
-      if (rank < B.rank) out[(int64_t)(B.r0 + rank) * L.d_out + 16 * ot + g + 8 * (j & 1)] = (uint8_t)(reg >> (8 * b));
+    const int k = i / 64;
+    const DcUBlk K = dc_u_block(B, k);
+    code = band[(int64_t)k * B.u_full + (o & 127) * K.nr + (i - K.rr0)];
+  } else {
+    const int Q = B.u_quads;
+    const bool in_quad = i < 128 * Q;
+    const int k = B.bits == 3 ? i / 256 : (in_quad && (i / 128) / 2 < Q / 2 ? (i / 128) / 2 : B.u_nblk - 1);
+    const DcUBlk K = dc_u_block(B, k);
+    const int r16 = o & 15, g = r16 & 7, jrow = r16 >> 3;
+    const uint8_t* tile = band + (int64_t)k * B.u_full + ((o & 127) >> 4) * K.tile_bytes;
+    if (in_quad) {
+      const int q = i / 128, pp = (i % 128) / 32, w32 = i % 32;
+      const int t = w32 / 8, jhi = (w32 % 8) / 4, b = w32 % 4;
+      const int j = jrow + 2 * jhi, ln = 4 * g + t;
+      const uint32_t w = ldg32(tile + 512 * (q - K.q0) + 16 * ln + 4 * j);
+      code = (w >> (8 * b + 2 * pp)) & 3u;
+    } else {
+      const int sidx = (i - 128 * Q) / 32, w32 = (i - 128 * Q) % 32;
+      const uint8_t* sb = tile + 512 * K.nq;
+      for (int s2 = K.s0; s2 < sidx; ++s2)
+        sb += dc_u_step_bytes(B.bits, dc_u_step_lanes(s2 == B.u_steps - 1 ? B.u_last : 32));
+      const int valid = sidx == B.u_steps - 1 ? B.u_last : 32;
+      const int nl = dc_u_step_lanes(valid), ntv = nl / 8;
+      const int t = w32 / 8, jhi = (w32 % 8) / 4, b = w32 % 4;
+      const int j = jrow + 2 * jhi, idx = g * ntv + t;
+      code = (ldg32(sb + 4 * idx) >> (8 * b + 2 * j)) & 3u;
+      if (B.bits == 3) code |= ((ldg16(sb + dc_align((int64_t)nl * 4, 16) + 2 * idx) >> (4 * j + b)) & 1u) << 2;
     }
-  };
-  for (int q = 0; q < B.u_quads; ++q) {
-    const uint4 wq = ldg128(ub + 512 * q + 16 * lane);
-    for (int ps = 0; ps < 4; ++ps)
-      for (int j = 0; j < 4; ++j) put(u_reg_mask2(wsel(wq, j), ps) >> (2 * ps), j, 128 * q + 32 * ps);
   }
-  const uint8_t* sb = ub + (int64_t)512 * B.u_quads;
-  for (int s = 0; s < B.u_steps; ++s) {
-    const int valid = (s == B.u_steps - 1) ? B.u_last : 32;
-    const int nl = dc_u_step_lanes(valid), ntv = nl / 8;
-    if (t < ntv) {
-      const uint32_t wv = ldg32(sb + 4 * (g * ntv + t));
-      const uint32_t hv = B.bits == 3 ? ldg16(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t)) : 0u;
-      for (int j = 0; j < 4; ++j) {
-        uint32_t r = reg_shift2(wv, j);
-        if (B.bits == 3) r |= u_reg_hi3(hv, j);
-        put(r, j, 128 * B.u_quads + 32 * s);
-      }
-    }
-    sb += dc_u_step_bytes(B.bits, nl);
-  }
+  out[(int64_t)(B.r0 + i) * L.d_out + o] = (uint8_t)code;
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1517,6 +1619,26 @@ __global__ void k_pack_words(DcLayout L, DcPlain Pl, uint32_t* dst) {
   const int64_t nw = L.bytes / 4;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nw; i += (int64_t)gridDim.x * blockDim.x)
     dst[i] = dc_pack_word(L, i * 4, Pl);
+}
+
+// Largest U scale over the 2/3-bit bands and every output group -> the blob's bound word.
+__global__ void k_umax(DcLayout L, const uint16_t* __restrict__ szu, float* dst) {
+  __shared__ float red[32];
+  float m = 0.f;
+  for (int b = 0; b < L.n_bands; ++b) {
+    const DcBand& B = L.band[b];
+    if (B.bits == 8) continue;
+    const int64_t a = (int64_t)B.r0 * L.groups_out, e = (int64_t)(B.r0 + B.rank) * L.groups_out;
+    for (int64_t i = a + threadIdx.x; i < e; i += blockDim.x)
+      m = fmaxf(m, fabsf(__half2float(__ushort_as_half(szu[2 * i]))));
+  }
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULLMASK, m, o));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) m = fmaxf(m, red[w]);
+    *dst = m;
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1622,11 +1744,14 @@ extern "C" dc_status dc_quantize_pack_device(const dc_factor_desc* desc, const f
     st = dc_cuda_check(cudaGetLastError(), "quantise kernel");
     if (st) return st;
   }
-  DcPlain Pl{cu, cv, szu, szv, S_dev};
+  DcPlain Pl{cu, cv, szu, szv, S_dev, 0.f};  // the bound word is written by k_umax
   const int64_t nw = L.bytes / 4;
   const unsigned blocks = (unsigned)std::min<int64_t>((nw + 255) / 256, 148 * 64);
   k_pack_words<<<blocks, 256, 0, s>>>(L, Pl, (uint32_t*)dev_dst);
   st = dc_cuda_check(cudaGetLastError(), "pack kernel");
+  if (st) return st;
+  k_umax<<<1, 256, 0, s>>>(L, szu, (float*)((uint8_t*)dev_dst + L.umax_off));
+  st = dc_cuda_check(cudaGetLastError(), "scale bound kernel");
   if (st) return st;
   dc_fill_handle(desc, L, dev_dst, out);
   return DC_OK;
@@ -1714,7 +1839,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   F.dtype_in = dtype_in;
   F.dtype_out = dtype_out;
   F.flags = flags;
-  int max_rank = 0, max_d_in = 0, max_ten = 0, bsm_max = 32;
+  int max_rank = 0, max_d_in = 0, max_ten = 0;
   const int n_in = n_lin == 7 ? 3 : 1;
   for (int m = 0; m < n_in; ++m) {
     F.x[m] = xs[m];
@@ -1741,7 +1866,6 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     max_rank = std::max(max_rank, l.max_rank);
     max_ten = std::max(max_ten, l.n_tenants);
     max_d_in = std::max(max_d_in, l.d_out);  // the workspace's per-token rows also hold outputs
-    bsm_max = std::max(bsm_max, (int)dc_align(dc_align(l.max_rank, 32) + 32 * DC_MAX_BANDS, 128) + 32);
     F.lin[p].W = l.W_base;
     F.lin[p].tenants = l.tenants_dev;
     F.lin[p].y = ys[p];
@@ -1751,7 +1875,6 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     F.lin[p].w_dtype = l.w_dtype;
     F.lin[p].input = m;
   }
-  F.bsm_max = bsm_max;
   F.ws = dc_ws_layout(T, max_rank, max_d_in, n_lin, max_ten);
   if (ws_bytes < (size_t)F.ws.total)
     return dc_fail(DC_ERR_WORKSPACE, "workspace holds %zu bytes, need %lld", ws_bytes, (long long)F.ws.total);
@@ -1795,6 +1918,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   if (st) return st;
   st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.dflag, 0, (size_t)n_lin * T, s), "flag reset");
   if (st) return st;
+  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.tmax, 0, (size_t)n_lin * T * 4, s), "bound reset");
+  if (st) return st;
   const int nb_items = (T + 255) / 256;
   k_prep<<<dim3(T + nb_items, std::max(n_in, n_lin)), 256, 0, s>>>(F, (uint8_t*)ws);
   prof_after(s);
@@ -1822,7 +1947,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (st) return st;
   }
   if (flags & DC_DELTA) {
-    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + (size_t)12 * bsm_max + sizeof(USmemTail);
+    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_BBUF + U_BCONST + sizeof(USmemTail);
     if (usmem > 227 * 1024)
       return dc_fail(DC_ERR_UNSUPPORTED, "max_rank %d needs %zu bytes of shared memory", max_rank, usmem);
     static size_t usmem_set = 0;
@@ -1832,7 +1957,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
       usmem_set = usmem;
     }
     prof_before(s, 3);
-    k_udelta<<<n_sm, U_THREADS, usmem, s>>>(F, (uint8_t*)ws);
+    k_udelta<<<U_CTAS_PER_SM * n_sm, U_THREADS, usmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "delta output kernel");
     if (st) return st;
@@ -1886,7 +2011,7 @@ extern "C" dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t whi
       const int64_t n = (int64_t)B.v_tiles * L.nkb * 64;
       k_unpack_v<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(blob, L, b, out_dev);
     } else if (which == 0) {
-      const int64_t n = B.bits == 8 ? (int64_t)L.d_out * B.rank : (int64_t)(L.d_out / 16) * 32;
+      const int64_t n = (int64_t)L.d_out * B.rank;
       k_unpack_u<<<(unsigned)((n + 127) / 128), 128, 0, s>>>(blob, L, b, out_dev);
     } else {
       return dc_fail(DC_ERR_INVALID_ARG, "which must be 0 (U) or 1 (V)");

@@ -45,12 +45,19 @@
 //                                 byte b;
 //   the last step of a band may be partial: only lanes with 8t < valid ranks are stored
 //   (ranks inside a lane padded to 8 with code 0).
-// 8-bit bands of U are small (the top singular vectors) and are stored row-major (128 rows x R8
-// bytes per 128-row group) for a scalar path.
-// The U side is grouped by 128-row output group (= the quantisation group along d_out): group go
-// holds, contiguously, every band's codes of its 128 rows (the eight 16-row tiles of a 2/3-bit
-// band one after the other) followed by the U meta of the group: r4 fp16 pairs (scale, zero),
-// r4 = r rounded up to a multiple of 4.  One 128-row group is one contiguous run of bytes.
+// The U side is grouped by 128-row output group (= the quantisation group along d_out): the run
+// of group go holds every band's codes and meta for its 128 rows, and is one contiguous run of
+// bytes.  Inside the run each band is cut into blocks of at most 8 steps (256 ranks): a 2-bit
+// band into blocks of 2 quads plus one tail block (a leftover quad and the shift-layout steps),
+// a 3-bit band into blocks of 8 steps, an 8-bit band into blocks of 64 ranks.  A block is
+//   [tile 0 codes][tile 1 codes] ... [tile 7 codes][meta: nr fp16 pairs (scale, zero)]
+// for 2/3-bit bands (a tile = the 16-row MMA tile: the block's quads, then its shift steps) and
+//   [128 rows x nr code bytes, row-major][meta]
+// for 8-bit bands (a scalar path).  Every block but a band's last has the band's full-block
+// size, so block k of a band starts at k * full_bytes.  One block is one bulk copy.
+// After S (fp32, r entries, padded to r4 = r rounded up to 4) the blob holds one fp32: the
+// largest U scale over the 2/3-bit bands and every output group (a bound used to pick the
+// fixed-point exponent of scale * t without a pass over the data).
 #pragma once
 #include <stdint.h>
 
@@ -66,17 +73,17 @@ struct DcBand {
   int32_t bits;        // 2, 3 or 8
   int32_t rank;        // ranks in the band
   int32_t r0;          // first rank of the band (index into S, t and U meta)
-  int32_t bsm_off;     // offset of the band in the U-stage staging of B (multiple of 32)
   int32_t v_tiles;     // ceil(rank / 16)
   int32_t v_group;     // tiles per group (8, 5 or 2)
   int32_t u_quads;     // U: full 4-step quads in the mask layout (2-bit only)
   int32_t u_steps;     // U: steps in the shift layout after the quads (incl. a partial last one)
   int32_t u_last;      // U: valid ranks of the last shift-layout step (32 if it is full)
+  int32_t u_nblk;      // U: blocks of the band inside one 128-row group's run
+  int32_t u_full;      // U: bytes of a full block (every block but the last)
   int64_t v_off;       // V codes of the band
   int64_t v_tile_bytes;// bytes of one full 16-row tile (codes and meta of every block)
-  int64_t u_boff;      // offset of the band's codes inside one 128-row group's run
-  int64_t u_otile_bytes; // bytes per 16-row output tile (MMA bands); R8 for 8-bit bands
-  int64_t u_region;    // bytes of the band inside one 128-row group's run
+  int64_t u_boff;      // offset of the band inside one 128-row group's run
+  int64_t u_bytes;     // bytes of the band inside one 128-row group's run
 };
 
 struct DcLayout {
@@ -85,15 +92,26 @@ struct DcLayout {
   int32_t groups_out;  // d_out / 128
   int32_t nkb;         // ceil(groups_in / 4) blocks of 512 columns
   int32_t tail_groups; // groups in the last block (1..4)
-  int32_t bsm_total;   // extent of the U-stage B staging (ranks, padded)
   int32_t valid;       // 1 if the descriptor is valid
-  int32_t r4;          // U meta row stride (entries)
+  int32_t r4;          // r rounded up to a multiple of 4
   int64_t s_off, bytes;
+  int64_t umax_off;    // fp32 bound on the U scales of the 2/3-bit bands
   int64_t u_off;       // start of the U part (128-row group runs)
   int64_t u_unit;      // bytes of one 128-row group's run
-  int64_t u_meta_in;   // offset of the U meta inside a run
   int64_t dev_base;    // device address of the blob (filled where a layout is bound to a blob)
   DcBand band[DC_MAX_BANDS];
+};
+
+// Geometry of block k of a band's U codes inside a 128-row group's run.
+struct DcUBlk {
+  int32_t nq, q0;      // quads (mask layout) in the block and the band's first one among them
+  int32_t ns, s0;      // shift-layout steps in the block and the band's first one among them
+  int32_t last;        // valid ranks of the block's final shift step (32 if full or none)
+  int32_t nr;          // valid ranks of the block
+  int32_t rr0;         // first rank of the block inside the band
+  int32_t tile_bytes;  // bytes of one 16-row tile (2/3-bit bands)
+  int32_t code_bytes;  // codes of the block (multiple of 16)
+  int32_t bytes;       // codes + meta (multiple of 16)
 };
 
 DC_HD int64_t dc_align(int64_t x, int64_t a) { return (x + a - 1) / a * a; }
@@ -130,6 +148,57 @@ DC_HD bool dc_bits_ok(int32_t b) { return b == 0 || b == 2 || b == 3 || b == 8; 
 // tiles of 16 ranks per group (= per serving work item) for a bit width
 DC_HD int32_t dc_v_group_tiles(int32_t bits) { return bits == 2 ? 8 : (bits == 3 ? 5 : 2); }
 
+// Block k of band B (u_quads/u_steps/u_last must be set).
+DC_HD DcUBlk dc_u_block(const DcBand& B, int32_t k) {
+  DcUBlk K;
+  K.nq = K.q0 = K.ns = K.s0 = 0;
+  K.last = 32;
+  K.tile_bytes = 0;
+  if (B.bits == 8) {
+    K.rr0 = 64 * k;
+    K.nr = dc_min(64, B.rank - K.rr0);
+    K.code_bytes = (int32_t)dc_align((int64_t)128 * K.nr, 16);
+    K.bytes = K.code_bytes + (int32_t)dc_align((int64_t)4 * K.nr, 16);
+    return K;
+  }
+  if (B.bits == 2) {
+    const int32_t nfull = B.u_quads / 2;
+    if (k < nfull) {
+      K.nq = 2;
+      K.q0 = 2 * k;
+    } else {
+      K.nq = B.u_quads % 2;
+      K.q0 = 2 * nfull;
+      K.ns = B.u_steps;
+      K.s0 = 0;
+    }
+    K.rr0 = 256 * k;
+  } else {
+    K.s0 = 8 * k;
+    K.ns = dc_min(8, B.u_steps - K.s0);
+    K.rr0 = 256 * k;
+  }
+  int32_t nr = 128 * K.nq;
+  int32_t tb = 512 * K.nq;
+  for (int32_t s = K.s0; s < K.s0 + K.ns; ++s) {
+    const int32_t valid = (s == B.u_steps - 1) ? B.u_last : 32;
+    nr += valid;
+    tb += (int32_t)dc_u_step_bytes(B.bits, dc_u_step_lanes(valid));
+    if (s == K.s0 + K.ns - 1) K.last = valid;
+  }
+  K.nr = nr;
+  K.tile_bytes = tb;
+  K.code_bytes = 8 * tb;
+  K.bytes = K.code_bytes + (int32_t)dc_align((int64_t)4 * nr, 16);
+  return K;
+}
+
+DC_HD int32_t dc_u_nblk(const DcBand& B) {
+  if (B.bits == 8) return (B.rank + 63) / 64;
+  if (B.bits == 2) return B.u_quads / 2 + ((B.u_quads % 2 + B.u_steps) > 0 ? 1 : 0);
+  return (B.u_steps + 7) / 8;
+}
+
 // Compute the layout of a descriptor; layout.valid = 0 on an invalid descriptor.
 DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   DcLayout L;
@@ -143,8 +212,7 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   L.dev_base = 0;
   L.u_off = 0;
   L.u_unit = 0;
-  L.u_meta_in = 0;
-  L.bsm_total = 0;
+  L.umax_off = 0;
   L.r4 = 0;
   L.groups_in = d.d_in / DC_GROUP;
   L.groups_out = d.d_out / DC_GROUP;
@@ -165,7 +233,9 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
   int32_t cap = d.d_out < d.d_in ? d.d_out : d.d_in;
   if (r > cap) return L;
   L.r = r;
-  int64_t off = dc_align((int64_t)r * 4, 256);  // S
+  L.r4 = (int32_t)dc_align(r, 4);
+  L.umax_off = (int64_t)L.r4 * 4;
+  int64_t off = dc_align(L.umax_off + 4, 256);  // S, then the U scale bound
   // V codes with inline meta
   for (int i = 0; i < L.n_bands; ++i) {
     DcBand& B = L.band[i];
@@ -177,41 +247,27 @@ DC_HD DcLayout dc_layout(const dc_factor_desc& d) {
     int64_t sz = B.v_tile_bytes * (B.v_tiles - 1) + dc_v_block_bytes(B.bits, last_rows, L.groups_in);
     off = dc_align(off + sz, 256);
   }
-  // U: runs of 128-row groups [band codes ...][meta]
-  int32_t bsm = 0;
+  // U: runs of 128-row groups, band by band, blocks inside a band
   int64_t in_unit = 0;
   for (int i = 0; i < L.n_bands; ++i) {
     DcBand& B = L.band[i];
-    B.u_boff = in_unit;
-    B.bsm_off = bsm;
     if (B.bits == 8) {
-      B.u_quads = 0;
-      B.u_steps = 0;
-      B.u_last = 0;
-      B.u_otile_bytes = B.rank;
-      B.u_region = dc_align((int64_t)128 * B.rank, 16);
-      in_unit += B.u_region;
-      continue;
+      B.u_quads = B.u_steps = 0;
+      B.u_last = 32;
+    } else {
+      B.u_quads = B.bits == 2 ? B.rank / 128 : 0;
+      int32_t rest = B.rank - 128 * B.u_quads;
+      B.u_steps = (rest + 31) / 32;
+      B.u_last = rest - 32 * (B.u_steps - 1);
+      if (B.u_steps == 0) B.u_last = 32;
     }
-    B.u_quads = B.bits == 2 ? B.rank / 128 : 0;
-    int32_t rest = B.rank - 128 * B.u_quads;
-    B.u_steps = (rest + 31) / 32;
-    B.u_last = rest - 32 * (B.u_steps - 1);
-    if (B.u_steps == 0) B.u_last = 32;
-    int64_t ot = (int64_t)B.u_quads * 512;
-    for (int s = 0; s < B.u_steps; ++s) {
-      int32_t valid = (s == B.u_steps - 1) ? B.u_last : 32;
-      ot += dc_u_step_bytes(B.bits, dc_u_step_lanes(valid));
-    }
-    B.u_otile_bytes = ot;
-    B.u_region = 8 * ot;
-    in_unit += B.u_region;
-    bsm += (int32_t)dc_align(B.rank, 32);
+    B.u_nblk = dc_u_nblk(B);
+    B.u_full = dc_u_block(B, 0).bytes;
+    B.u_boff = in_unit;
+    B.u_bytes = (int64_t)(B.u_nblk - 1) * B.u_full + dc_u_block(B, B.u_nblk - 1).bytes;
+    in_unit += B.u_bytes;
   }
-  L.bsm_total = bsm;
-  L.r4 = (int32_t)dc_align(r, 4);
-  L.u_meta_in = in_unit;
-  L.u_unit = in_unit + (int64_t)L.r4 * 4;
+  L.u_unit = in_unit;
   L.u_off = off;
   off = dc_align(off + L.u_unit * L.groups_out, 256);
   L.bytes = off;

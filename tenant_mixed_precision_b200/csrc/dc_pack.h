@@ -12,7 +12,9 @@ struct DcPlain {
   const uint16_t* szu;  // [r][d_out/128][2] fp16 (scale, zero)
   const uint16_t* szv;  // [r][d_in/128][2]
   const float* S;       // [r]
+  float umax;           // largest U scale over the 2/3-bit bands and every output group
 };
+
 
 DC_HD int64_t dc_v_band_bytes(const DcLayout& L, const DcBand& B) {
   int32_t last_rows = B.rank - 16 * (B.v_tiles - 1);
@@ -106,23 +108,33 @@ DC_HD uint32_t dc_pack_v_word(const DcLayout& L, const DcBand& B, int64_t off, c
   return w;
 }
 
-// Word at byte offset `off` inside band B's codes of the 128-row group `go`.
+// Word at byte offset `off` inside band B's part of the 128-row group `go`'s run.
 DC_HD uint32_t dc_pack_u_word(const DcLayout& L, const DcBand& B, int32_t go, int64_t off, const DcPlain& P) {
+  int32_t k = (int32_t)(off / B.u_full);
+  if (k > B.u_nblk - 1) k = B.u_nblk - 1;
+  const DcUBlk K = dc_u_block(B, k);
+  const int64_t lo = off - (int64_t)k * B.u_full;
+  if (lo >= K.code_bytes) {  // meta of the block's ranks
+    const int32_t i = (int32_t)((lo - K.code_bytes) / 4);
+    if (i >= K.nr) return 0u;
+    const uint16_t* sz = P.szu + ((int64_t)(B.r0 + K.rr0 + i) * L.groups_out + go) * 2;
+    return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
+  }
   uint32_t w = 0;
-  if (B.bits == 8) {
+  if (B.bits == 8) {  // row-major 128 x nr
     for (int b = 0; b < 4; ++b) {
-      const int64_t idx = off + b;
-      const int64_t o = idx / B.rank;
-      const int32_t i = (int32_t)(idx % B.rank);
-      if (o < 128) w |= dc_cu(L, P, B.r0 + i, (int32_t)(128 * go + o)) << (8 * b);
+      const int64_t idx = lo + b;
+      const int64_t o = idx / K.nr;
+      const int32_t i = (int32_t)(idx % K.nr);
+      if (o < 128) w |= dc_cu(L, P, B.r0 + K.rr0 + i, (int32_t)(128 * go + o)) << (8 * b);
     }
     return w;
   }
-  const int32_t ot = (int32_t)(off / B.u_otile_bytes);  // 16-row tile inside the group
-  int64_t x = off - (int64_t)ot * B.u_otile_bytes;
+  const int32_t ot = (int32_t)(lo / K.tile_bytes);  // 16-row tile inside the group
+  int64_t x = lo - (int64_t)ot * K.tile_bytes;
   const int32_t o0 = 128 * go + 16 * ot;
-  if (x < (int64_t)512 * B.u_quads) {  // mask layout quads
-    const int32_t q = (int32_t)(x / 512);
+  if (x < (int64_t)512 * K.nq) {  // mask layout quads
+    const int32_t q = K.q0 + (int32_t)(x / 512);
     const int32_t y = (int32_t)(x % 512);
     const int32_t lane = y / 16, j = (y % 16) / 4;
     const int32_t g = lane >> 2, t = lane & 3;
@@ -134,8 +146,8 @@ DC_HD uint32_t dc_pack_u_word(const DcLayout& L, const DcBand& B, int32_t go, in
       }
     return w;
   }
-  x -= (int64_t)512 * B.u_quads;
-  for (int s = 0; s < B.u_steps; ++s) {
+  x -= (int64_t)512 * K.nq;
+  for (int s = K.s0; s < K.s0 + K.ns; ++s) {
     const int32_t valid = (s == B.u_steps - 1) ? B.u_last : 32;
     const int32_t nl = dc_u_step_lanes(valid);
     const int32_t ntv = nl / 8;
@@ -175,18 +187,20 @@ DC_HD uint32_t dc_pack_u_word(const DcLayout& L, const DcBand& B, int32_t go, in
   return 0u;
 }
 
+DC_HD uint32_t dc_f32_bits(float f) {
+  uint32_t u;
+#if defined(__CUDA_ARCH__)
+  u = __float_as_uint(f);
+#else
+  __builtin_memcpy(&u, &f, 4);
+#endif
+  return u;
+}
+
 // Word at byte offset `off` of the whole blob.
 DC_HD uint32_t dc_pack_word(const DcLayout& L, int64_t off, const DcPlain& P) {
-  if (off < (int64_t)L.r * 4) {
-    const float f = P.S[off / 4];
-    uint32_t u;
-#if defined(__CUDA_ARCH__)
-    u = __float_as_uint(f);
-#else
-    __builtin_memcpy(&u, &f, 4);
-#endif
-    return u;
-  }
+  if (off < (int64_t)L.r * 4) return dc_f32_bits(P.S[off / 4]);
+  if (off == L.umax_off) return dc_f32_bits(P.umax);
   for (int i = 0; i < L.n_bands; ++i) {
     const DcBand& B = L.band[i];
     if (off >= B.v_off && off < B.v_off + dc_v_band_bytes(L, B)) return dc_pack_v_word(L, B, off - B.v_off, P);
@@ -195,15 +209,9 @@ DC_HD uint32_t dc_pack_word(const DcLayout& L, int64_t off, const DcPlain& P) {
     const int64_t rel = off - L.u_off;
     const int32_t go = (int32_t)(rel / L.u_unit);
     const int64_t in = rel - (int64_t)go * L.u_unit;
-    if (in >= L.u_meta_in) {
-      const int32_t i = (int32_t)((in - L.u_meta_in) / 4);
-      if (i >= L.r) return 0u;
-      const uint16_t* sz = P.szu + ((int64_t)i * L.groups_out + go) * 2;
-      return (uint32_t)sz[0] | ((uint32_t)sz[1] << 16);
-    }
     for (int i = 0; i < L.n_bands; ++i) {
       const DcBand& B = L.band[i];
-      if (in >= B.u_boff && in < B.u_boff + B.u_region) return dc_pack_u_word(L, B, go, in - B.u_boff, P);
+      if (in >= B.u_boff && in < B.u_boff + B.u_bytes) return dc_pack_u_word(L, B, go, in - B.u_boff, P);
     }
   }
   return 0u;
