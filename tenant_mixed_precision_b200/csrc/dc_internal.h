@@ -68,7 +68,13 @@ struct alignas(16) DcURec {  // moved with 16-byte vector loads and stores
 // Workspace layout (byte offsets from the workspace base).
 struct DcWs {
   int32_t T, max_rank, max_d_in, n_lin, n_in, r_stride, max_items, max_tenants, nkb, pad;
-  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, total;
+  int32_t bt_nb;     // token block of the tensor-core backbone (multiple of 16, <= 256)
+  int32_t bt_units;  // upper bound on its (linear, 128-row tile, token block) units
+  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, bt_part, bt_cnt, total;
 };
+
+// Tensor-core backbone: CTAs of the persistent grid (at most; 148 SMs on B200) and the partial
+// tiles they may leave for split units (two per CTA: its first and its last unit).
+#define DC_BT_MAX_CTAS 148
 
 DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, int32_t max_tenants);

@@ -32,6 +32,7 @@
 #include "dc_layout.h"
 #include "dc_pack.h"
 #include "dc_tma.h"
+#include "dc_umma.h"
 
 #define FULLMASK 0xffffffffu
 
@@ -134,6 +135,10 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.yd = take((int64_t)n_lin * T * W.max_d_in * 4);
   W.dflag = take((int64_t)n_lin * T);
   W.tmax = take((int64_t)n_lin * T * 4);
+  W.bt_nb = T <= 256 ? (int32_t)dc_align(T > 0 ? T : 1, 16) : 256;
+  W.bt_units = n_lin * (W.max_d_in / 128) * (int32_t)((T + W.bt_nb - 1) / W.bt_nb);
+  W.bt_part = take((int64_t)2 * DC_BT_MAX_CTAS * 128 * W.bt_nb * 4);
+  W.bt_cnt = take((int64_t)W.bt_units * 4);
   W.total = off;
   return W;
 }
@@ -160,6 +165,9 @@ struct DcFwd {
   int32_t n_lin, T, dtype_in, dtype_out, flags, pad;
   int32_t order[7];        // launch order of the linears in the U kernel (largest first)
   int32_t tile_prefix[8];  // cumulative 128-row output tiles in that order
+  int64_t bt_chunk_prefix[8];  // tensor-core backbone: cumulative 64-column chunks of all units, same order
+  int64_t bt_total;            // total chunks
+  int32_t bt_ntb, bt_ns, bt_grid, bt_pad;  // token blocks, pipeline stages, CTAs
   DcWs ws;
 };
 
@@ -1476,6 +1484,292 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ D
 }
 
 // ---------------------------------------------------------------------------------------------
+// k_base_tc: y = W_base x (+ ydelta) on the tcgen05 tensor cores, for bf16 backbones.
+// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens); its K is cut
+// into 64-column chunks.  The units' chunks, largest-K linears first, form one sequence that is
+// split evenly over the persistent CTAs (stream-K), so every CTA moves the same number of bytes
+// whatever the tile count.  Per CTA: warp 0 loads each chunk's W slice (128 x 64) and activation
+// slice (NB x 64) with 2-D TMA into a ring of stages; warp 1 owns two NB-column fp32
+// accumulators in Tensor Memory and, from one thread, issues 4 MMAs (M 128, N NB, K 16) per
+// chunk, releasing the stage with a commit; warps 2-5 (one TMEM lane quarter each, lane = output
+// row) drain a finished accumulator.  A unit shared by several CTAs leaves fp32 partial tiles;
+// the last contributor to arrive (a counter per unit) adds them in k order, so the result does
+// not depend on timing.  The epilogue adds the delta and writes y in the tokens' original order.
+// ---------------------------------------------------------------------------------------------
+#define BT_THREADS 192
+#define BT_MAX_STAGES 8
+#define BT_A_BYTES 16384  // 128 rows x 64 bf16
+
+struct BtTail {
+  uint64_t full[BT_MAX_STAGES];
+  uint64_t empty[BT_MAX_STAGES];
+  uint64_t acc_full[2];
+  uint64_t acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+  int last_flag;
+  int perm[256];    // epilogue: original position of each token of the unit's block (-1: none)
+  uint8_t dfl[256]; // epilogue: the token has a delta
+};
+
+__device__ __forceinline__ int64_t bt_g0(const DcFwd& F, int c) { return (int64_t)c * F.bt_total / F.bt_grid; }
+
+// CTA whose chunk range holds global chunk g
+__device__ __forceinline__ int bt_cta_of(const DcFwd& F, int64_t g) {
+  int c = (int)(g * F.bt_grid / F.bt_total);
+  while (c + 1 < F.bt_grid && bt_g0(F, c + 1) <= g) ++c;
+  while (c > 0 && bt_g0(F, c) > g) --c;
+  return c;
+}
+
+struct BtSeg {
+  int u, slot, ot, tb, K;  // unit, linear order slot, tile, token block, chunks of the unit
+  int64_t ustart;          // global index of the unit's first chunk
+  int k0, k1;              // chunk range of this segment inside the unit
+};
+
+__device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1) {
+  BtSeg S;
+  int slot = 0;
+  while (slot + 1 < F.n_lin && g >= F.bt_chunk_prefix[slot + 1]) ++slot;
+  S.slot = slot;
+  S.K = F.lin[F.order[slot]].d_in / 64;
+  const int64_t local = (g - F.bt_chunk_prefix[slot]) / S.K;
+  S.u = (int)(F.tile_prefix[slot] * (int64_t)F.bt_ntb + local);
+  S.ot = (int)(local / F.bt_ntb);
+  S.tb = (int)(local % F.bt_ntb);
+  S.ustart = F.bt_chunk_prefix[slot] + local * S.K;
+  S.k0 = (int)(g - S.ustart);
+  S.k1 = (int)min((int64_t)S.K, g1 - S.ustart);
+  return S;
+}
+
+__device__ __forceinline__ bool bt_aborted(BtTail* tail) { return *reinterpret_cast<volatile int*>(&tail->abort) != 0; }
+
+// AND of `ok` over the `count` threads of named barrier `id` (all of them take part).
+__device__ __forceinline__ bool bar_and(int id, int count, bool ok) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+               : "=r"(r)
+               : "r"((uint32_t)ok), "r"(id), "r"(count)
+               : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ bool bt_wait(uint64_t* bar, uint32_t parity, BtTail* tail, int* st) {
+  if (bt_aborted(tail)) return false;
+  if (mbar_wait(bar, parity)) return true;
+  tail->abort = 1;
+  set_status(st, DC_ERR_CUDA);
+  return false;
+}
+
+__global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  extern __shared__ __align__(1024) uint8_t bt_raw[];
+  uint8_t* sm = bt_raw + ((1024 - (smem_u32(bt_raw) & 1023)) & 1023);  // 1024-aligned (swizzled tiles)
+  const int NB = F.ws.bt_nb, NS = F.bt_ns;
+  const int stage_bytes = BT_A_BYTES + NB * 128;
+  BtTail* tail = reinterpret_cast<BtTail*>(sm + (size_t)NS * stage_bytes);
+  WsPtr P = ws_ptr(F.ws, ws);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = F.ws.T;
+  const int c = blockIdx.x;
+  const int64_t g0 = bt_g0(F, c), g1 = bt_g0(F, c + 1);
+  uint32_t ncols = 32;
+  while (ncols < (uint32_t)(2 * NB)) ncols <<= 1;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&tail->full[s], 1);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->acc_full[b], 1);
+      mbar_init(&tail->acc_empty[b], 4);
+    }
+    tail->abort = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&tail->tmem_base), ncols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tail->tmem_base;
+  if (warp == 0) {
+    // ---------------- TMA producer
+    uint32_t seq = 0;
+    for (int64_t g = g0; g < g1 && !bt_aborted(tail);) {
+      const BtSeg S = bt_seg_at(F, g, g1);
+      const int p = F.order[S.slot];
+      const int m = F.lin[p].input;
+      for (int k = S.k0; k < S.k1; ++k, ++seq) {
+        const int s = seq % NS;
+        if (seq >= (uint32_t)NS && !bt_wait(&tail->empty[s], ((seq / NS) - 1) & 1, tail, P.st)) break;
+        if (lane == 0) {
+          uint8_t* st = sm + (size_t)s * stage_bytes;
+          mbar_arrive_expect_tx(&tail->full[s], (uint32_t)stage_bytes);
+          tma_load_2d(st, &F.wmap[p], k * 64, S.ot * 128, &tail->full[s]);
+          tma_load_2d(st + BT_A_BYTES, &F.xmap[m], k * 64, S.tb * NB, &tail->full[s]);
+        }
+        __syncwarp();
+      }
+      g = S.ustart + S.k1;
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (one thread)
+    const uint32_t idesc = umma_idesc_bf16(128, NB);
+    uint32_t seq = 0, segi = 0;
+    for (int64_t g = g0; g < g1 && !bt_aborted(tail); ++segi) {
+      const BtSeg S = bt_seg_at(F, g, g1);
+      const int b = segi & 1;
+      if (segi >= 2 && !bt_wait(&tail->acc_empty[b], ((segi >> 1) - 1) & 1, tail, P.st)) break;
+      tc_fence_after();
+      const uint32_t dt = tbase + (uint32_t)(b * NB);
+      bool ok = true;
+      for (int k = S.k0; k < S.k1; ++k, ++seq) {
+        const int s = seq % NS;
+        if (!bt_wait(&tail->full[s], (seq / NS) & 1, tail, P.st)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sm + (size_t)s * stage_bytes);
+          const uint64_t ad = umma_desc_sw128(a0), bd = umma_desc_sw128(a0 + BT_A_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)  // K = 16 per MMA: 32 bytes further inside the swizzle atom
+            umma_bf16(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (k > S.k0 || kk > 0) ? 1u : 0u);
+          umma_commit(smem_u32(&tail->empty[s]));  // the stage is free once these MMAs have read it
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(&tail->acc_full[b]));  // accumulator complete
+      __syncwarp();
+      g = S.ustart + S.k1;
+    }
+  } else {
+    // ---------------- epilogue warpgroup (warps 2-5): TMEM lane quarter warp % 4
+    const int q4 = warp & 3;
+    const int row = 32 * q4 + lane;  // output row inside the tile
+    const bool delta = (F.flags & DC_DELTA) != 0;
+    float* part_base = reinterpret_cast<float*>(ws + F.ws.bt_part);
+    int* cnt = reinterpret_cast<int*>(ws + F.ws.bt_cnt);
+    uint32_t segi = 0;
+    // The four warps leave the loop together: the outcome of every wait is agreed through a
+    // reducing named barrier, so no warp is left waiting at a barrier the others skipped.
+    for (int64_t g = g0; g < g1; ++segi) {
+      const BtSeg S = bt_seg_at(F, g, g1);
+      const int b = segi & 1;
+      const bool okw = bt_wait(&tail->acc_full[b], (segi >> 1) & 1, tail, P.st);
+      if (!bar_and(1, 128, okw)) break;
+      tc_fence_after();
+      const int p = F.order[S.slot];
+      const DcLinDev& lin = F.lin[p];
+      const bool whole = S.k0 == 0 && S.k1 == S.K;
+      const int my_slot = S.ustart <= bt_g0(F, c) ? 0 : 1;  // 0: the CTA's first unit, 1: its last
+      float* mypart = part_base + ((int64_t)(2 * c + my_slot) * NB) * 128;
+      const uint32_t ta = tbase + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * NB);
+      const int orow = S.ot * 128 + row;
+      const int et = threadIdx.x - 64;  // 0..127
+      // destinations of the block's tokens, staged once per unit
+      for (int col = et; col < NB; col += 128) {
+        const int ts = S.tb * NB + col;
+        tail->perm[col] = ts < T ? P.perm[ts] : -1;
+        tail->dfl[col] = (delta && ts < T) ? P.dflag[(int64_t)p * T + ts] : 0;
+      }
+      named_bar(1, 128);
+      const float* ydp = P.yd + (int64_t)p * T * F.ws.max_d_in + orow;
+      for (int cb = 0; cb < NB; cb += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + cb, r);
+        tmem_ld_wait();
+        if (whole) {
+          float yv[16];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int col = cb + j;
+            yv[j] = __uint_as_float(r[j]);
+            if (tail->dfl[col]) yv[j] += ydp[(int64_t)(S.tb * NB + col) * F.ws.max_d_in];
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int dst = tail->perm[cb + j];
+            if (dst >= 0) {
+              const int64_t o = (int64_t)dst * lin.d_out + orow;
+              if (F.dtype_out == DC_DTYPE_F32)
+                reinterpret_cast<float*>(lin.y)[o] = yv[j];
+              else
+                reinterpret_cast<__nv_bfloat16*>(lin.y)[o] = __float2bfloat16_rn(yv[j]);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) mypart[(cb + j) * 128 + row] = __uint_as_float(r[j]);
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->acc_empty[b]);  // the accumulator may be overwritten
+      if (!whole) {
+        // hand the partial over; the last contributor of the unit finishes it
+        __threadfence();
+        named_bar(1, 128);
+        const int c0 = bt_cta_of(F, S.ustart), c1 = bt_cta_of(F, S.ustart + S.K - 1);
+        if (et == 0) {
+          const int old = atomicAdd(cnt + S.u, 1);
+          tail->last_flag = old == c1 - c0;
+          __threadfence();
+        }
+        named_bar(1, 128);
+        if (tail->last_flag) {
+          for (int cb = 0; cb < NB; cb += 16) {
+            float yv[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) yv[j] = 0.f;
+            for (int cc = c0; cc <= c1; ++cc) {  // k order
+              const int sl = S.ustart <= bt_g0(F, cc) ? 0 : 1;
+              const float* pp = part_base + ((int64_t)(2 * cc + sl) * NB + cb) * 128 + row;
+              float pv[16];
+#pragma unroll
+              for (int j = 0; j < 16; ++j) pv[j] = __ldcg(pp + j * 128);
+#pragma unroll
+              for (int j = 0; j < 16; ++j) yv[j] += pv[j];
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int col = cb + j;
+              if (tail->dfl[col]) yv[j] += ydp[(int64_t)(S.tb * NB + col) * F.ws.max_d_in];
+            }
+#pragma unroll
+            for (int j = 0; j < 16; ++j) {
+              const int dst = tail->perm[cb + j];
+              if (dst >= 0) {
+                const int64_t o = (int64_t)dst * lin.d_out + orow;
+                if (F.dtype_out == DC_DTYPE_F32)
+                  reinterpret_cast<float*>(lin.y)[o] = yv[j];
+                else
+                  reinterpret_cast<__nv_bfloat16*>(lin.y)[o] = __float2bfloat16_rn(yv[j]);
+              }
+            }
+          }
+        }
+      }
+      g = S.ustart + S.k1;
+    }
+  }
+  // every role has left its loop (all waits are bounded); release Tensor Memory
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, ncols);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Debug unpacker: the integer codes back out of the packed layout with the extraction helpers
 // the serving kernels use.  One thread per (V: tile, block, half, lane) or (U: o-tile16, lane).
 // ---------------------------------------------------------------------------------------------
@@ -1878,6 +2172,9 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   F.ws = dc_ws_layout(T, max_rank, max_d_in, n_lin, max_ten);
   if (ws_bytes < (size_t)F.ws.total)
     return dc_fail(DC_ERR_WORKSPACE, "workspace holds %zu bytes, need %lld", ws_bytes, (long long)F.ws.total);
+  // bf16 backbones with bf16 activations run on the tcgen05 tensor cores
+  bool use_tc = (flags & DC_BASE) && dtype_in == DC_DTYPE_BF16;
+  for (int p = 0; p < n_lin; ++p) use_tc = use_tc && lins[p].w_dtype == DC_DTYPE_BF16;
   if (flags & DC_BASE) {
     for (int p = 0; p < n_lin; ++p)
       if (lins[p].w_dtype == DC_DTYPE_BF16) {
@@ -1887,7 +2184,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (dtype_in == DC_DTYPE_BF16)
       for (int m = 0; m < n_in; ++m) {
         const uint8_t* xb = (const uint8_t*)ws + F.ws.xsort + (int64_t)m * T * F.ws.max_d_in * 2;
-        dc_status st0 = encode_bf16_map(&F.xmap[m], xb, dxs[m], T, F.ws.max_d_in, std::min(64, T));
+        dc_status st0 = encode_bf16_map(&F.xmap[m], xb, dxs[m], T, F.ws.max_d_in, use_tc ? F.ws.bt_nb : std::min(64, T));
         if (st0) return st0;
       }
   }
@@ -1961,6 +2258,32 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "delta output kernel");
     if (st) return st;
+  }
+  if (use_tc) {
+    F.bt_ntb = (T + F.ws.bt_nb - 1) / F.ws.bt_nb;
+    F.bt_chunk_prefix[0] = 0;
+    for (int i = 0; i < n_lin; ++i) {
+      const dc_linear& l = lins[ord[i]];
+      F.bt_chunk_prefix[i + 1] = F.bt_chunk_prefix[i] + (int64_t)(l.d_out / 128) * F.bt_ntb * (l.d_in / 64);
+    }
+    F.bt_total = F.bt_chunk_prefix[n_lin];
+    const int stage_bytes = BT_A_BYTES + F.ws.bt_nb * 128;
+    F.bt_ns = std::min(BT_MAX_STAGES, (int)((200 * 1024) / stage_bytes));
+    F.bt_grid = (int)std::min<int64_t>(std::min(n_sm, DC_BT_MAX_CTAS), F.bt_total);
+    const size_t tsmem = 1024 + (size_t)F.bt_ns * stage_bytes + sizeof(BtTail);
+    static size_t tset = 0;
+    if (tsmem > tset) {
+      st = dc_cuda_check(cudaFuncSetAttribute(k_base_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem),
+                         "smem attr");
+      if (st) return st;
+      tset = tsmem;
+    }
+    st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.bt_cnt, 0, (size_t)F.ws.bt_units * 4, s), "unit counters");
+    if (st) return st;
+    prof_before(s, 4);
+    k_base_tc<<<F.bt_grid, BT_THREADS, tsmem, s>>>(F, (uint8_t*)ws);
+    prof_after(s);
+    return dc_cuda_check(cudaGetLastError(), "tensor-core output kernel");
   }
   const size_t bsmem = 1024 + (size_t)B_STAGES * B_STAGE_BYTES + sizeof(BSmemTail);
   static bool bset = false;
