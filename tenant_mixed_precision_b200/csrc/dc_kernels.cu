@@ -463,7 +463,8 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
 // the pass's tokens -- into a ring of shared-memory stages with bulk copies; consumer warp w
 // decodes tile w from shared memory into u8 MMA operands.
 // ---------------------------------------------------------------------------------------------
-#define V_STAGES 8
+#define V_STAGES 4
+#define V_CTAS_PER_SM 2  // two CTAs per SM: twice the warps to hide the consumers' latencies
 #define V_A_BYTES 18432   // one block of the item's tiles: 8 x 2304 (2-bit), 5 x 3328 (3-bit), 2 x 8448 (8-bit)
 #define V_XTOK DC_XBLK    // one token's limb block in shared memory (1616: offsets tokens by 20 banks)
 #define V_X_BYTES (4 * V_XTOK)
@@ -634,7 +635,7 @@ __device__ __forceinline__ uint4 ldg128_item(const DcVItem* it, int lane) {
   return ldg128(reinterpret_cast<const uint8_t*>(it) + 16 * lane);
 }
 
-__global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__ DcFwd F, uint8_t* ws) {
+__global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __grid_constant__ DcFwd F, uint8_t* ws) {
   extern __shared__ __align__(128) uint8_t vsm[];
   VSmemTail* tail = reinterpret_cast<VSmemTail*>(vsm + V_STAGES * V_STAGE_BYTES);
   WsPtr P = ws_ptr(F.ws, ws);
@@ -677,7 +678,7 @@ __global__ void __launch_bounds__(V_THREADS, 1) k_vstage(const __grid_constant__
           set_status(P.st, DC_ERR_CUDA);
           return;
         }
-        fence_proxy_async();
+        
         uint8_t* stage = vsm + (size_t)s * V_STAGE_BYTES;
         if (end) {
           if (lane == 0) {
@@ -2238,7 +2239,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
       vset = true;
     }
     prof_before(s, 2);
-    k_vstage<<<n_sm, V_THREADS, vsmem, s>>>(F, (uint8_t*)ws);
+    k_vstage<<<V_CTAS_PER_SM * n_sm, V_THREADS, vsmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "rank-reduction kernel");
     if (st) return st;
