@@ -816,7 +816,7 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
 // (sum over ranks of zero * scale * t), then the exponent.  8-bit bands use a scalar fp32 path.
 // ---------------------------------------------------------------------------------------------
 #define U_STAGES 4
-#define U_STAGE_BYTES 24576  // a batch of blocks (codes + meta) and the t windows of its tokens
+#define U_STAGE_BYTES 22528  // a batch of blocks (codes + meta) and the t windows of its tokens
 #define U_CTAS_PER_SM 2      // two CTAs per SM: their producers' and consumers' stalls overlap
 #define U_MAXSUB 8           // blocks per batch
 #define U_MAXBLK 64          // blocks per (linear, tenant) U run of one group
@@ -854,8 +854,10 @@ struct USmemTail {
   UBlkE tbl[U_MAXBLK];           // producer: blocks of the current chunk's runs
   int bfirst[U_MAXBLK + 1];      // producer: batches of the current pass (first block of each)
   int nbatch;
-  float zpart[2][U_CONSUMERS][DC_V_TOKS];  // per-warp zero-point sums (unit parity)
+  float zpart[U_CONSUMERS][DC_V_TOKS];     // per-warp zero-point sums of a unit
   float s8[U_CONSUMERS][16][DC_V_TOKS];    // 8-bit band partials of a unit
+  int cbuf[U_CONSUMERS][2][16][8];         // combined integer MMA results of a unit: [warp][pair][row][col]
+  float uie[DC_V_TOKS];                    // 2^-e of the unit's tokens
 };
 
 // D += A(u8, 16x32, row) * B(u8, 32x8, col), int32 accumulate.
@@ -906,7 +908,28 @@ __device__ __forceinline__ void ud_mma(const uint8_t* blk, int bits, int nq, int
   // codes' row sums), column 7 a row of zeros; both constant rows sit after the two limb matrices
   const uint8_t* brow = (g < 6 ? bsm + g * U_BROW : bconst + (g - 6) * U_BROW) + 8 * t;
   const int pstride = g < 6 ? 6 * U_BROW : 0;
-#pragma unroll 2
+  if (ns == 0) {  // 2-bit block: one or two quads in straight-line code
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      if (q >= nq) break;
+      const uint4 wq = *reinterpret_cast<const uint4*>(ub + 512 * q + 16 * lane);
+      uint2 bq[NPAIR][4];
+#pragma unroll
+      for (int pr = 0; pr < NPAIR; ++pr)
+#pragma unroll
+        for (int ps = 0; ps < 4; ++ps)
+          bq[pr][ps] = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * (4 * q + ps));
+#pragma unroll
+      for (int ps = 0; ps < 4; ++ps) {
+        const uint32_t msk = 0x03030303u << (2 * ps);
+#pragma unroll
+        for (int pr = 0; pr < NPAIR; ++pr)
+          mma_u8u8(C[pr][ps], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bq[pr][ps].x, bq[pr][ps].y);
+      }
+    }
+    return;
+  }
+#pragma unroll 1
   for (int q = 0; q < nq; ++q) {
     const uint4 wq = *reinterpret_cast<const uint4*>(ub + 512 * q + 16 * lane);
 #pragma unroll
@@ -1206,30 +1229,35 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     if (lane == 0) mbar_arrive(&tail->empty[s]);
     ++seq;
     if (!ulast) continue;
-    // ---- epilogue of the (group, pass) unit; sums in a fixed order (deterministic)
-    float (*zp)[DC_V_TOKS] = tail->zpart[unit & 1];
+    // ---- epilogue of the (group, pass) unit.  Phase 1: per-warp zero-point sums, 8-bit partials
+    // and the integer MMA results (positions combined) go to shared memory; phase 2: every
+    // thread finishes (row, token) outputs.  Sums run in a fixed order (deterministic).
+    float zw[DC_V_TOKS];
 #pragma unroll
     for (int q = 0; q < DC_V_TOKS; ++q) {
-      float v = zc[q];
+      float v = 0.f;
+      if (q < ntok) {
+        v = zc[q];
 #pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
-      if (lane == 0) zp[warp][q] = v;
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
+      }
+      zw[q] = v;
+    }
+    named_bar(2, 32 * U_CONSUMERS);  // the previous unit's phase 2 is over
+    if (lane < DC_V_TOKS) {
+      float v = zw[0], e = ie[0];
+#pragma unroll
+      for (int q = 1; q < DC_V_TOKS; ++q) {
+        v = lane == q ? zw[q] : v;
+        e = lane == q ? ie[q] : e;
+      }
+      tail->zpart[warp][lane] = v;
+      if (warp == 0) tail->uie[lane] = e;
     }
     {
       const int row = lane & 15, th = lane >> 4;
       tail->s8[warp][row][2 * th] = s8[0];
       tail->s8[warp][row][2 * th + 1] = s8[1];
-    }
-    named_bar(2, 32 * U_CONSUMERS);
-    float zs[DC_V_TOKS];
-#pragma unroll
-    for (int q = 0; q < DC_V_TOKS; ++q) {
-      float v = 0.f;
-      if (q < ntok) {
-#pragma unroll
-        for (int w = 0; w < U_CONSUMERS; ++w) v += zp[w][q];
-      }
-      zs[q] = v;
     }
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
@@ -1238,21 +1266,21 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
 #pragma unroll
       for (int r = 0; r < 4; ++r)
         Ct[r] = C[pr][0][r] + (C[pr][1][r] >> 2) + (C[pr][2][r] >> 4) + (C[pr][3][r] >> 6);
-      // lane t holds limb t (t < 3) or the row sums (t = 3, regs 0 and 2)
-      const int rs0 = __shfl_down_sync(FULLMASK, Ct[0], 3), rs1 = __shfl_down_sync(FULLMASK, Ct[2], 3);
+      *reinterpret_cast<int2*>(&tail->cbuf[warp][pr][g][2 * t]) = make_int2(Ct[0], Ct[1]);
+      *reinterpret_cast<int2*>(&tail->cbuf[warp][pr][g + 8][2 * t]) = make_int2(Ct[2], Ct[3]);
+    }
+    named_bar(2, 32 * U_CONSUMERS);
+    // cbuf columns: 2 limb + token-in-pair for limbs 0..2, column 6 = the codes' row sum
+    for (int idx = tid; idx < 128 * ntok; idx += 32 * U_CONSUMERS) {
+      const int row = idx & 127, q = idx >> 7;
+      const int w = row >> 4, rr = row & 15, pr = q >> 1, tk = q & 1;
+      const int* cr = tail->cbuf[w][pr][rr];
+      const float v = (float)(cr[4 + tk] - 64 * cr[6]) * 65536.f + (float)cr[2 + tk] * 256.f + (float)cr[tk];
+      float zs = 0.f;
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int l1 = __shfl_down_sync(FULLMASK, Ct[r], 1);
-        const int l2 = __shfl_down_sync(FULLMASK, Ct[r], 2);
-        const int q = 2 * pr + (r & 1);
-        const int rl = g + 8 * (r >> 1);
-        if (t == 0 && q < ntok) {
-          const int rsum = (r >> 1) ? rs1 : rs0;
-          const float v = (float)(l2 - 64 * rsum) * 65536.f + (float)l1 * 256.f + (float)Ct[r];
-          const float y = fmaf(v, ie[q], -zs[q]) + tail->s8[warp][rl][q];
-          P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + 16 * warp + rl] = y;
-        }
-      }
+      for (int ww = 0; ww < U_CONSUMERS; ++ww) zs += tail->zpart[ww][q];
+      const float y = fmaf(v, tail->uie[q], -zs) + tail->s8[w][rr][q];
+      P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + row] = y;
     }
     ++unit;
   }

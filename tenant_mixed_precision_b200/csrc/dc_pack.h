@@ -142,7 +142,7 @@ DC_HD uint32_t dc_pack_u_word(const DcLayout& L, const DcBand& B, int32_t go, in
     for (int p = 0; p < 4; ++p)
       for (int b = 0; b < 4; ++b) {
         const int32_t rank = 128 * q + 32 * p + 8 * t + 4 * (j >> 1) + b;
-        w |= (dc_cu(L, P, B.r0 + rank, o) & 3u) << (8 * b + 2 * p);
+        if (rank < B.rank) w |= (dc_cu(L, P, B.r0 + rank, o) & 3u) << (8 * b + 2 * p);
       }
     return w;
   }
