@@ -371,6 +371,123 @@ def run_gpu(args):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# Prefill workload (13B shapes): tokens/s against the tensor roofline
+# ------------------------------------------------------------------------------------------------
+PREFILL_METRIC = "tokens/s and % of tensor roofline, 16-tenant 13B mixed-precision delta prefill"
+PREFILL = dict(name="llama2-13b linear stack prefill, 16 resident tenant deltas at 1/16, 2048 tokens in "
+                    "per-tenant segments of 32-256", hidden=5120, ffn=13824, layers=40, n_tenants=16, T=2048,
+               seed=20244, ids_seed=4)
+
+
+def _bf16_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return float(d.get("bf16_tflops_sustained", 1400.0)), "measured bf16_tflops_sustained"
+    return 1400.0, "fallback sustained bf16"
+
+
+def run_prefill(args):
+    import numpy as np
+    import torch
+
+    import tenant_mixed_precision_b200 as dc
+    from tenant_mixed_precision_b200 import plans, synth
+    from tenant_mixed_precision_b200.stack import DeltaStack
+    from tenant_mixed_precision_b200.synth_stack import populate
+
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if rank != 0:
+        return 0
+    torch.cuda.set_device(local)
+    W = dict(PREFILL)
+    if args.layers:
+        W["layers"] = args.layers
+    T = W["T"]
+
+    def plan_fn(l, p, d_out, d_in, t):
+        return plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+
+    t_setup = time.time()
+    stack = DeltaStack(W["hidden"], W["ffn"], W["layers"], W["n_tenants"], T, plan_fn, out_dtype=torch.bfloat16)
+    populate(stack, W["seed"], s0=0.02 * math.sqrt(W["hidden"]))
+    ids = synth.prefill_segments(np.random.default_rng(W["ids_seed"]), T, W["n_tenants"])
+    ids_dev = torch.from_numpy(ids).cuda()
+    setup_s = time.time() - t_setup
+    stream = torch.cuda.Stream()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        stack.forward(ids_dev, T)
+    stream.synchronize()
+    assert dc.dc_read_device_status(stack.ws, stream) == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        stack.forward(ids_dev, T)
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        ev0.record(stream)
+        for _ in range(args.steps):
+            graph.replay()
+        ev1.record(stream)
+    ev1.synchronize()
+    ck = clocks.stop()
+    ms_per_step = ev0.elapsed_time(ev1) / args.steps
+    status = dc.dc_read_device_status(stack.ws, stream)
+    # per-kernel times (eager, CUDA events on the launching stream)
+    n_prof = 2
+    cap = n_prof * (1 + 4 * W["layers"]) + 8
+    dc.dc_profile_begin(cap)
+    with torch.cuda.stream(stream):
+        for _ in range(n_prof):
+            stack.forward(ids_dev, T)
+    rec = dc.dc_profile_end(cap)
+    per = {}
+    for kind, m in rec:
+        per.setdefault(kind, []).append(m)
+    # algorithmic flops: backbone 2 T d_out d_in, delta 2 r (d_in + d_out) per token of a tenant
+    base_flops = delta_flops = 0.0
+    for l in range(W["layers"]):
+        for p, (d_out, d_in) in enumerate(stack.shapes):
+            base_flops += 2.0 * T * d_out * d_in
+            for t in ids.tolist():
+                desc = stack.descs.get((l, p, int(t)))
+                if desc is not None:
+                    r = sum(desc.rank[i] for i in range(desc.n_bands) if desc.bits[i])
+                    delta_flops += 2.0 * r * (d_in + d_out)
+    peak, peak_kind = _bf16_peak()
+    tf = (base_flops + delta_flops) / (ms_per_step * 1e-3) / 1e12
+    base_ms = sum(per.get("backbone_output", [0])) / n_prof
+    base_tf = base_flops / (base_ms * 1e-3) / 1e12 if base_ms else None
+    line = {
+        "metric": PREFILL_METRIC, "value": T / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 backbone, u8xs8->s32 delta", "data": "synthetic",
+        "config": {"workload": W["name"], "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
+                   "tenants_resident": W["n_tenants"], "T": T,
+                   "segments": int(1 + np.count_nonzero(np.diff(ids))), "distinct_tenants": len(set(ids.tolist())),
+                   "cuda_graph": True},
+        "step_tensor": {"algorithmic_tflop": (base_flops + delta_flops) / 1e12, "base_tflop": base_flops / 1e12,
+                        "delta_tflop": delta_flops / 1e12, "achieved_tflops": tf, "peak_tflops": peak,
+                        "frac": tf / peak, "peak_source": peak_kind},
+        "roofline": {"bound": "tensor", "kernel": "k_base_tc", "achieved": base_tf, "peak": peak, "unit": "TFLOP/s",
+                     "frac": (base_tf / peak) if base_tf else None, "peak_source": peak_kind, "traffic": None},
+        "kernel_ms_per_step": {k: sum(v) / n_prof for k, v in per.items()},
+        "gpu_launches": (1 + 4 * W["layers"]) * args.steps,
+        "clocks": ck, "device_status": status, "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -381,11 +498,15 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=0, help="smaller stack for profiling captures (default: 32)")
     ap.add_argument("--tenants", type=int, default=0, help="fewer resident tenants (default: 50)")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
+                    help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill pass")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "prefill":
+        return run_prefill(args)
     return run_gpu(args)
 
 
