@@ -444,7 +444,7 @@ def run_prefill(args):
     status = dc.dc_read_device_status(stack.ws, stream)
     # per-kernel times (eager, CUDA events on the launching stream)
     n_prof = 2
-    cap = n_prof * (1 + 4 * W["layers"]) + 8
+    cap = n_prof * (1 + 8 * W["layers"]) + 8  # up to 6 launches per layer on the prefill path
     dc.dc_profile_begin(cap)
     with torch.cuda.stream(stream):
         for _ in range(n_prof):
@@ -481,7 +481,7 @@ def run_prefill(args):
         "roofline": {"bound": "tensor", "kernel": "k_base_tc", "achieved": base_tf, "peak": peak, "unit": "TFLOP/s",
                      "frac": (base_tf / peak) if base_tf else None, "peak_source": peak_kind, "traffic": None},
         "kernel_ms_per_step": {k: sum(v) / n_prof for k, v in per.items()},
-        "gpu_launches": (1 + 4 * W["layers"]) * args.steps,
+        "gpu_launches": (1 + 6 * W["layers"]) * args.steps,
         "clocks": ck, "device_status": status, "setup_s": setup_s,
     }
     print(json.dumps(line), flush=True)

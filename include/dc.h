@@ -60,8 +60,11 @@ enum { DC_DTYPE_F32 = 0, DC_DTYPE_BF16 = 1 };
 enum {
   DC_BASE = 1,          /* add W_base x                                                  */
   DC_DELTA = 2,         /* add U_hat (S * (V_hat^T x)) of the token's tenant             */
-  DC_REUSE_ROUTING = 4  /* skip dc_build_segments: the workspace already holds the routing
+  DC_REUSE_ROUTING = 4, /* skip dc_build_segments: the workspace already holds the routing
                            of these tenant ids (e.g. every layer after the first)        */
+  DC_DECODE_ONLY = 8    /* serve every segment with the decode kernels, also segments of 64
+                           or more tokens that would take the tensor-core prefill path
+                           (for comparisons and tests)                                   */
 };
 
 #define DC_MAX_BANDS 4

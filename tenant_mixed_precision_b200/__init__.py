@@ -22,7 +22,7 @@ SYNTH_LIB_PATH = os.path.join(_HERE, "libdc_synth.so")
 DC_OK, DC_ERR_INVALID_ARG, DC_ERR_SHAPE, DC_ERR_BITS, DC_ERR_ALIGN = 0, 1, 2, 3, 4
 DC_ERR_WORKSPACE, DC_ERR_TENANT, DC_ERR_CUDA, DC_ERR_UNSUPPORTED = 5, 6, 7, 8
 DC_DTYPE_F32, DC_DTYPE_BF16 = 0, 1
-DC_BASE, DC_DELTA, DC_REUSE_ROUTING = 1, 2, 4
+DC_BASE, DC_DELTA, DC_REUSE_ROUTING, DC_DECODE_ONLY = 1, 2, 4, 8
 DC_MAX_BANDS = 4
 DC_GROUP = 128
 

@@ -70,8 +70,17 @@ struct DcWs {
   int32_t T, max_rank, max_d_in, n_lin, n_in, r_stride, max_items, max_tenants, nkb, pad;
   int32_t bt_nb;     // token block of the tensor-core backbone (multiple of 16, <= 256)
   int32_t bt_units;  // upper bound on its (linear, 128-row tile, token block) units
-  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, bt_part, bt_cnt, total;
+  int32_t tcols;     // columns of the bf16 t planes: every band starts on a multiple of 64
+  int32_t pad2;
+  int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, bt_part, bt_cnt;
+  int64_t tseg;      // per tenant-sorted token: its segment
+  int64_t thl;       // bf16 t, high and low parts: [2][n_lin][T][tcols]
+  int64_t total;
 };
+
+// Segments of at least DC_PF_MIN tokens take the tensor-core (prefill) delta path when the batch
+// has at least that many tokens.
+#define DC_PF_MIN 64
 
 // Tensor-core backbone: CTAs of the persistent grid (at most; 148 SMs on B200) and the partial
 // tiles they may leave for split units (two per CTA: its first and its last unit).

@@ -139,6 +139,9 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.bt_units = n_lin * (W.max_d_in / 128) * (int32_t)((T + W.bt_nb - 1) / W.bt_nb);
   W.bt_part = take((int64_t)2 * DC_BT_MAX_CTAS * 128 * W.bt_nb * 4);
   W.bt_cnt = take((int64_t)W.bt_units * 4);
+  W.tseg = take((int64_t)T * 4);
+  W.tcols = (int32_t)dc_align(max_rank > 0 ? max_rank : 1, 64) + 64 * (DC_MAX_BANDS - 1);
+  W.thl = T >= DC_PF_MIN ? take((int64_t)2 * n_lin * T * W.tcols * 2) : take(0);
   W.total = off;
   return W;
 }
@@ -168,6 +171,8 @@ struct DcFwd {
   int64_t bt_chunk_prefix[8];  // tensor-core backbone: cumulative 64-column chunks of all units, same order
   int64_t bt_total;            // total chunks
   int32_t bt_ntb, bt_ns, bt_grid, bt_pad;  // token blocks, pipeline stages, CTAs
+  CUtensorMap tmap;            // prefill path: bf16 t planes [2 n_lin T rows x tcols], box 64 x 256
+  int32_t pf;                  // segments of >= DC_PF_MIN tokens take the prefill delta path
   DcWs ws;
 };
 
@@ -185,6 +190,8 @@ struct WsPtr {
   float* yd;
   uint8_t* dflag;
   int* tmax;  // per (linear, sorted token): max |t| over the 2/3-bit ranks, as fp32 bits
+  int* tseg;  // per sorted token: its segment
+  __nv_bfloat16* thl;  // t as bf16 high and low parts (prefill path)
 };
 __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   WsPtr p;
@@ -201,6 +208,8 @@ __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   p.yd = (float*)(ws + W.yd);
   p.dflag = ws + W.dflag;
   p.tmax = (int*)(ws + W.tmax);
+  p.tseg = (int*)(ws + W.tseg);
+  p.thl = (__nv_bfloat16*)(ws + W.thl);
   return p;
 }
 
@@ -330,6 +339,8 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
   }
   P.urecs[(int64_t)p * W.T + s] = R;
   for (int k = 0; k < len; ++k) P.dflag[(int64_t)p * W.T + st + k] = (uint8_t)R.valid;
+  if (p == 0)
+    for (int k = 0; k < len; ++k) P.tseg[st + k] = s;
   if (!R.valid || !(F.flags & DC_DELTA)) return;
   const int passes = (len + DC_V_TOKS - 1) / DC_V_TOKS;
   int per_pass = 0;
@@ -1032,7 +1043,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       for (int b = 0; b < R.n_bands; ++b) NB += R.band[b].nblk;
       if (NB > U_MAXBLK) {
         set_status(P.st, DC_ERR_UNSUPPORTED);
-      } else if (R.valid) {
+      } else if (R.valid && !(F.pf && R.len >= DC_PF_MIN)) {  // long segments: k_upre
         // block table of the run, one lane per block
         for (int i = lane; i < NB; i += 32) {
           int b = 0, k = i;
@@ -1799,6 +1810,452 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
 }
 
 // ---------------------------------------------------------------------------------------------
+// Prefill delta path (segments of at least DC_PF_MIN tokens), tcgen05 tensor cores.
+//
+// k_thl: t of every token of such a segment as two bf16 planes, t = hi + lo to ~16 bits, in the
+// layout the U-side kernel loads with TMA: [plane][linear][token][tcols], band b of the tenant
+// starting at column sum_{b' < b} align(rank_b', 64) (zeros in the padding).
+// ---------------------------------------------------------------------------------------------
+__device__ __forceinline__ int pf_band_col(const DcURec& R, int b) {
+  int c = 0;
+  for (int i = 0; i < b; ++i) c += (R.band[i].rank + 63) & ~63;
+  return c;
+}
+
+__global__ void __launch_bounds__(256) k_thl(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  WsPtr P = ws_ptr(F.ws, ws);
+  const int T = F.ws.T;
+  const int p = blockIdx.y, tok = blockIdx.x;
+  if (p >= F.n_lin || tok >= T) return;
+  const int sg = P.tseg[tok];
+  const DcURec& R = P.urecs[(int64_t)p * T + sg];
+  if (!R.valid || R.len < DC_PF_MIN) return;
+  const float* tr = P.tws + ((int64_t)p * T + tok) * F.ws.r_stride;
+  __nv_bfloat16* hi = P.thl + ((int64_t)p * T + tok) * F.ws.tcols;
+  __nv_bfloat16* lo = hi + (int64_t)F.n_lin * T * F.ws.tcols;
+  int col = 0;
+  for (int b = 0; b < R.n_bands; ++b) {
+    const int rb = R.band[b].rank, padded = (rb + 63) & ~63;
+    for (int i = threadIdx.x; i < padded; i += blockDim.x) {
+      const float v = i < rb ? tr[R.band[b].r0 + i] : 0.f;
+      const __nv_bfloat16 h = __float2bfloat16_rn(v);
+      hi[col + i] = h;
+      lo[col + i] = __float2bfloat16_rn(v - __bfloat162float(h));
+    }
+    col += padded;
+  }
+}
+
+// One 16-byte chunk (8 consecutive K columns) of a 128-byte-swizzled K-major bf16 tile row.
+__device__ __forceinline__ void sw128_store(uint8_t* tile, int row, int chunk, uint4 v) {
+  *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = v;
+}
+
+// bf16 high and low parts of (c - z) * s for 8 codes (4 bytes of r0, then 4 of r1).
+__device__ __forceinline__ void pf_dequant8(uint32_t r0, uint32_t r1, const float (&s)[8], const float (&z)[8],
+                                            uint4& hv, uint4& lv) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    float v[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int idx = 2 * k + e;
+      const uint32_t c = ((idx < 4 ? r0 : r1) >> (8 * (idx & 3))) & 0xffu;
+      v[e] = ((float)c - z[idx]) * s[idx];
+    }
+    const __nv_bfloat162 hb = __floats2bfloat162_rn(v[0], v[1]);
+    const float2 hf = __bfloat1622float2(hb);
+    const __nv_bfloat162 lb = __floats2bfloat162_rn(v[0] - hf.x, v[1] - hf.y);
+    h[k] = *reinterpret_cast<const uint32_t*>(&hb);
+    l[k] = *reinterpret_cast<const uint32_t*>(&lb);
+  }
+  hv = make_uint4(h[0], h[1], h[2], h[3]);
+  lv = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_upre: ydelta = U_hat t for segments of at least DC_PF_MIN tokens, on tcgen05.
+// Unit = (linear p, long segment, 128-row output group go); the segment's tokens are taken in
+// tiles of up to 256 (the MMA N).  K = the tenant's ranks, band by band, in chunks of 64.
+//   warp 0     TMA: per chunk the t planes (hi, lo: 256 tokens x 64 ranks each); per U block the
+//              block's bytes (codes of the eight 16-row tiles + meta) into a two-slot ring
+//   warps 1-4  expansion: (c - z) * scale of the chunk's 128 x 64 codes as bf16 hi and lo
+//              (128-byte-swizzled K-major tiles), from the staged block
+//   warp 5     TMEM owner and MMA issuer: D[row][token] += Uhi thi + Uhi tlo + Ulo thi
+//              (M 128, N tokens, K 16 per instruction), two accumulators
+//   warps 6-9  epilogue: TMEM lane = output row, writes ydelta
+// Units are dealt to the persistent CTAs round robin; every wait is bounded.
+// ---------------------------------------------------------------------------------------------
+#define UP_THREADS 320
+#define UP_A_BYTES 16384                  // 128 rows x 64 bf16
+#define UP_B_BYTES 32768                  // 256 tokens x 64 bf16
+#define UP_STAGE_BYTES (2 * UP_A_BYTES + 2 * UP_B_BYTES)
+#define UP_STAGES 2
+#define UP_BLK_BYTES 13312                // largest U block (3-bit, 8 steps, with meta)
+#define UP_MAX_LONG 256
+
+struct UpTail {
+  uint64_t full_b[UP_STAGES], full_a[UP_STAGES], empty[UP_STAGES];
+  uint64_t blk_full[2], blk_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+  int nlong;
+  int lseg[UP_MAX_LONG];
+};
+
+struct UpChunk {
+  int b, c0;   // band, first band-relative rank of the chunk
+  int k;       // U block of the band holding it
+};
+
+// Chunk i of a record (band by band, 64 ranks each); false past the last one.
+__device__ __forceinline__ bool up_chunk(const DcURec& R, int i, UpChunk& C) {
+  for (int b = 0; b < R.n_bands; ++b) {
+    const int n = (R.band[b].rank + 63) / 64;
+    if (i < n) {
+      const DcUBand& UB = R.band[b];
+      C.b = b;
+      C.c0 = 64 * i;
+      if (UB.bits == 8 || UB.bits == 3) {
+        C.k = C.c0 / (UB.bits == 8 ? 64 : 256);
+      } else {
+        const int qi = C.c0 / 128;
+        C.k = (C.c0 < 128 * UB.quads && qi < 2 * (UB.quads / 2)) ? qi / 2 : UB.nblk - 1;
+      }
+      return true;
+    }
+    i -= n;
+  }
+  return false;
+}
+
+__device__ __forceinline__ DcBand up_band(const DcUBand& UB) {
+  DcBand B;
+  B.bits = UB.bits, B.rank = UB.rank, B.r0 = UB.r0;
+  B.u_quads = UB.quads, B.u_steps = UB.steps, B.u_last = UB.last;
+  return B;
+}
+
+// Unit u -> (linear p, long segment index, group go); false past the last unit.
+__device__ __forceinline__ bool up_unit(const DcFwd& F, int nlong, int u, int& p, int& j, int& go) {
+  for (int i = 0; i < F.n_lin; ++i) {
+    const int q = F.order[i];
+    const int G = F.lin[q].d_out / 128;
+    const int cnt = nlong * G;
+    if (u < cnt) {
+      p = q;
+      j = u / G;
+      go = u % G;
+      return true;
+    }
+    u -= cnt;
+  }
+  return false;
+}
+
+// Expand ranks [c0, c0 + 64) of band UB for the 16-row tile `tile` of the staged block `blk`
+// (block k of the band) into the bf16 tiles ahi / alo (rows 16 tile + g and + g + 8).
+__device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand& UB, int k, int c0, int tile,
+                                               int lane, uint8_t* ahi, uint8_t* alo) {
+  const int g = lane >> 2, t = lane & 3;
+  const DcBand B = up_band(UB);
+  const DcUBlk K = dc_u_block(B, k);
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const int rs = c0 + 32 * s;  // first band-relative rank of the step
+    uint32_t a[4] = {0u, 0u, 0u, 0u};
+    float sc[8], zz[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sc[e] = zz[e] = 0.f;
+    if (rs < UB.rank) {
+      if (UB.bits == 8) {
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+          for (int b = 0; b < 4; ++b) {
+            const int i = rs + 8 * t + 4 * (jj >> 1) + b;
+            const int row = 16 * tile + g + 8 * (jj & 1);
+            const uint32_t c = i < UB.rank ? blk[row * K.nr + (i - K.rr0)] : 0u;
+            a[jj] |= c << (8 * b);
+          }
+      } else if (UB.bits == 2 && rs < 128 * UB.quads) {
+        const int qb = rs / 128 - K.q0, ps = (rs % 128) / 32;
+        const uint4 wq = *reinterpret_cast<const uint4*>(blk + tile * K.tile_bytes + 512 * qb + 16 * lane);
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) a[jj] = (wsel(wq, jj) >> (2 * ps)) & 0x03030303u;
+      } else {
+        const int si = (rs - 128 * UB.quads) / 32;  // shift-layout step of the band
+        const uint8_t* sb = blk + tile * K.tile_bytes + 512 * K.nq;
+        for (int s2 = K.s0; s2 < si; ++s2)
+          sb += dc_u_step_bytes(UB.bits, dc_u_step_lanes(s2 == UB.steps - 1 ? UB.last : 32));
+        const int valid = si == UB.steps - 1 ? UB.last : 32;
+        const int nl = dc_u_step_lanes(valid), ntv = nl / 8;
+        uint32_t wv = 0, hv = 0;
+        if (t < ntv) {
+          wv = *reinterpret_cast<const uint32_t*>(sb + 4 * (g * ntv + t));
+          if (UB.bits == 3) hv = *reinterpret_cast<const uint16_t*>(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t));
+        }
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          a[jj] = reg_shift2(wv, jj);
+          if (UB.bits == 3) a[jj] |= u_reg_hi3(hv, jj);
+        }
+      }
+      const uint8_t* meta = blk + K.code_bytes;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int i = rs + 8 * t + e;
+        if (i < UB.rank) {
+          const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * (i - K.rr0));
+          sc[e] = __low2float(mz);
+          zz[e] = __high2float(mz);
+        }
+      }
+    }
+    uint4 hv, lv;
+    pf_dequant8(a[0], a[2], sc, zz, hv, lv);  // row g: ranks 8t .. 8t + 7
+    sw128_store(ahi, 16 * tile + g, 4 * s + t, hv);
+    sw128_store(alo, 16 * tile + g, 4 * s + t, lv);
+    pf_dequant8(a[1], a[3], sc, zz, hv, lv);  // row g + 8
+    sw128_store(ahi, 16 * tile + g + 8, 4 * s + t, hv);
+    sw128_store(alo, 16 * tile + g + 8, 4 * s + t, lv);
+  }
+}
+
+__device__ __forceinline__ bool up_aborted(UpTail* tail) { return *reinterpret_cast<volatile int*>(&tail->abort) != 0; }
+
+__device__ __forceinline__ bool up_wait(uint64_t* bar, uint32_t parity, UpTail* tail, int* st) {
+  if (up_aborted(tail)) return false;
+  if (mbar_wait(bar, parity)) return true;
+  tail->abort = 1;
+  set_status(st, DC_ERR_CUDA);
+  return false;
+}
+
+// Next (unit, token tile) of this CTA's sequence; the same for every role.
+struct UpIter {
+  int u, tt;  // current unit (-1 before the first) and token tile
+};
+__device__ __forceinline__ bool up_next(const DcFwd& F, const WsPtr& P, const UpTail* tail, UpIter& it, int& p,
+                                        int& go, const DcURec*& R, int& tok0, int& ntok) {
+  const int T = F.ws.T;
+  for (;;) {
+    if (it.u >= 0) {
+      int j;
+      if (!up_unit(F, tail->nlong, it.u, p, j, go)) return false;
+      R = P.urecs + (int64_t)p * T + tail->lseg[j];
+      if (R->valid && 256 * (it.tt + 1) < R->len) {
+        ++it.tt;
+        tok0 = R->st + 256 * it.tt;
+        ntok = min(256, R->st + R->len - tok0);
+        return true;
+      }
+      it.u += gridDim.x;
+    } else {
+      it.u = blockIdx.x;
+    }
+    it.tt = 0;
+    int j;
+    if (!up_unit(F, tail->nlong, it.u, p, j, go)) return false;
+    R = P.urecs + (int64_t)p * T + tail->lseg[j];
+    if (!R->valid) {
+      it.tt = 1 << 20;  // skip: the next call moves to the next unit
+      continue;
+    }
+    tok0 = R->st;
+    ntok = min(256, R->len);
+    return true;
+  }
+}
+
+__global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  extern __shared__ __align__(1024) uint8_t up_raw[];
+  uint8_t* sm = up_raw + ((1024 - (smem_u32(up_raw) & 1023)) & 1023);
+  uint8_t* blkring = sm + UP_STAGES * UP_STAGE_BYTES;
+  UpTail* tail = reinterpret_cast<UpTail*>(blkring + 2 * UP_BLK_BYTES);
+  WsPtr P = ws_ptr(F.ws, ws);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = F.ws.T;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < UP_STAGES; ++s) {
+      mbar_init(&tail->full_b[s], 1);
+      mbar_init(&tail->full_a[s], 4);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->blk_full[b], 1);
+      mbar_init(&tail->blk_empty[b], 4);
+      mbar_init(&tail->acc_full[b], 1);
+      mbar_init(&tail->acc_empty[b], 4);
+    }
+    tail->abort = 0;
+    const int nseg = P.st[DC_WS_NSEG];  // long segments, in segment order
+    int n = 0;
+    for (int sg = 0; sg < nseg && n < UP_MAX_LONG; ++sg)
+      if (P.segs[3 * sg] >= 0 && P.segs[3 * sg + 2] >= DC_PF_MIN) tail->lseg[n++] = sg;
+    tail->nlong = n;
+    fence_mbar_init();
+  }
+  if (warp == 5) {
+    tmem_alloc(smem_u32(&tail->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tail->tmem_base;
+  UpIter it{-1, 0};
+  int p = 0, go = 0, tok0 = 0, ntok = 0;
+  const DcURec* R = nullptr;
+  if (warp == 0) {
+    // ---------------- TMA producer: t planes per chunk, U blocks into the ring
+    uint32_t seq = 0, bseq = 0;
+    while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
+      const uint8_t* run = reinterpret_cast<const uint8_t*>(R->blob) + R->u_off + (int64_t)go * R->u_unit;
+      int lb = -1, lk = -1;
+      UpChunk C;
+      for (int ci = 0; up_chunk(*R, ci, C); ++ci, ++seq) {
+        if (C.b != lb || C.k != lk) {  // a new U block
+          lb = C.b, lk = C.k;
+          const int bs = bseq & 1;
+          if (bseq >= 2 && !up_wait(&tail->blk_empty[bs], ((bseq >> 1) - 1) & 1, tail, P.st)) break;
+          const DcUBand& UB = R->band[C.b];
+          const int bytes = dc_u_block(up_band(UB), C.k).bytes;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(&tail->blk_full[bs], (uint32_t)bytes);
+            bulk_g2s(blkring + bs * UP_BLK_BYTES, run + UB.boff + (int64_t)C.k * UB.full, (uint32_t)bytes,
+                     &tail->blk_full[bs]);
+          }
+          __syncwarp();
+          ++bseq;
+        }
+        const int s = seq % UP_STAGES;
+        if (seq >= UP_STAGES && !up_wait(&tail->empty[s], ((seq / UP_STAGES) - 1) & 1, tail, P.st)) break;
+        if (lane == 0) {
+          uint8_t* st = sm + (size_t)s * UP_STAGE_BYTES + 2 * UP_A_BYTES;
+          const int col = pf_band_col(*R, C.b) + C.c0;
+          const int row = p * T + tok0;
+          mbar_arrive_expect_tx(&tail->full_b[s], (uint32_t)(2 * UP_B_BYTES));
+          tma_load_2d(st, &F.tmap, col, row, &tail->full_b[s]);
+          tma_load_2d(st + UP_B_BYTES, &F.tmap, col, F.n_lin * T + row, &tail->full_b[s]);
+        }
+        __syncwarp();
+      }
+    }
+  } else if (warp <= 4) {
+    // ---------------- expansion warps: tiles 2 (warp - 1) and 2 (warp - 1) + 1
+    const int e = warp - 1;
+    uint32_t seq = 0, bseq = 0;
+    while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
+      int lb = -1, lk = -1;
+      UpChunk C;
+      bool ok = true;
+      for (int ci = 0; up_chunk(*R, ci, C); ++ci, ++seq) {
+        if (C.b != lb || C.k != lk) {
+          if (lb >= 0) {  // the previous block is done
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tail->blk_empty[(bseq - 1) & 1]);
+          }
+          lb = C.b, lk = C.k;
+          if (!up_wait(&tail->blk_full[bseq & 1], (bseq >> 1) & 1, tail, P.st)) {
+            ok = false;
+            break;
+          }
+          ++bseq;
+        }
+        const int s = seq % UP_STAGES;
+        if (seq >= UP_STAGES && !up_wait(&tail->empty[s], ((seq / UP_STAGES) - 1) & 1, tail, P.st)) {
+          ok = false;
+          break;
+        }
+        uint8_t* ahi = sm + (size_t)s * UP_STAGE_BYTES;
+        const uint8_t* blk = blkring + ((bseq - 1) & 1) * UP_BLK_BYTES;
+        const DcUBand UB = R->band[C.b];
+        for (int tl = 0; tl < 2; ++tl) up_expand_tile(blk, UB, C.k, C.c0, 2 * e + tl, lane, ahi, ahi + UP_A_BYTES);
+        fence_proxy_async();  // generic-proxy writes -> tensor-core (async proxy) reads
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->full_a[s]);
+      }
+      if (!ok) break;
+      __syncwarp();
+      if (lb >= 0 && lane == 0) mbar_arrive(&tail->blk_empty[(bseq - 1) & 1]);
+    }
+  } else if (warp == 5) {
+    // ---------------- MMA issuer
+    uint32_t seq = 0, unit = 0;
+    while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
+      const int N = (ntok + 15) & ~15;
+      const uint32_t idesc = umma_idesc_bf16(128, N);
+      const int b = unit & 1;
+      if (unit >= 2 && !up_wait(&tail->acc_empty[b], ((unit >> 1) - 1) & 1, tail, P.st)) break;
+      tc_fence_after();
+      const uint32_t dt = tbase + (uint32_t)(b * 256);
+      UpChunk C;
+      bool ok = true;
+      for (int ci = 0; up_chunk(*R, ci, C); ++ci, ++seq) {
+        const int s = seq % UP_STAGES;
+        const uint32_t ph = (seq / UP_STAGES) & 1;
+        if (!up_wait(&tail->full_b[s], ph, tail, P.st) || !up_wait(&tail->full_a[s], ph, tail, P.st)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        if (lane == 0) {
+          const uint32_t a0 = smem_u32(sm + (size_t)s * UP_STAGE_BYTES);
+          const uint64_t ah = umma_desc_sw128(a0), al = umma_desc_sw128(a0 + UP_A_BYTES);
+          const uint64_t bh = umma_desc_sw128(a0 + 2 * UP_A_BYTES), bl = umma_desc_sw128(a0 + 2 * UP_A_BYTES + UP_B_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) {
+            const uint64_t o = (uint64_t)(2 * kk);  // 32 bytes further inside the swizzle atom
+            umma_bf16(dt, ah + o, bh + o, idesc, (ci > 0 || kk > 0) ? 1u : 0u);
+            umma_bf16(dt, ah + o, bl + o, idesc, 1u);
+            umma_bf16(dt, al + o, bh + o, idesc, 1u);
+          }
+          umma_commit(smem_u32(&tail->empty[s]));
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      if (lane == 0) umma_commit(smem_u32(&tail->acc_full[b]));
+      __syncwarp();
+      ++unit;
+    }
+  } else {
+    // ---------------- epilogue warps 6-9 (TMEM lane quarter warp % 4); exits agreed by a vote
+    const int q4 = warp & 3, row = 32 * q4 + lane;
+    uint32_t unit = 0;
+    while (up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
+      const int b = unit & 1;
+      const bool okw = up_wait(&tail->acc_full[b], (unit >> 1) & 1, tail, P.st);
+      if (!bar_and(1, 128, okw)) break;
+      tc_fence_after();
+      const uint32_t ta = tbase + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * 256);
+      float* yd = P.yd + ((int64_t)p * T + tok0) * F.ws.max_d_in + 128 * go + row;
+      for (int cb = 0; cb < ntok; cb += 16) {
+        uint32_t r[16];
+        tmem_ld16(ta + cb, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int jj = 0; jj < 16; ++jj)
+          if (cb + jj < ntok) yd[(int64_t)(cb + jj) * F.ws.max_d_in] = __uint_as_float(r[jj]);
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&tail->acc_empty[b]);
+      ++unit;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
 // Debug unpacker: the integer codes back out of the packed layout with the extraction helpers
 // the serving kernels use.  One thread per (V: tile, block, half, lane) or (U: o-tile16, lane).
 // ---------------------------------------------------------------------------------------------
@@ -2226,6 +2683,13 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     F.order[i] = ord[i];
     F.tile_prefix[i + 1] = F.tile_prefix[i] + lins[ord[i]].d_out / 128;
   }
+  // long segments take the tensor-core delta path when the batch is large enough
+  F.pf = (flags & DC_DELTA) && !(flags & DC_DECODE_ONLY) && T >= 2 * DC_PF_MIN;
+  if (F.pf) {
+    dc_status st0 = encode_bf16_map(&F.tmap, (const uint8_t*)ws + F.ws.thl, F.ws.tcols, (int64_t)2 * n_lin * T,
+                                    F.ws.tcols, 256);
+    if (st0) return st0;
+  }
   cudaStream_t s = (cudaStream_t)stream;
   dc_status st;
   if (!(flags & DC_REUSE_ROUTING)) {
@@ -2287,6 +2751,26 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "delta output kernel");
     if (st) return st;
+    if (F.pf) {
+      prof_before(s, 3);
+      k_thl<<<dim3(T, n_lin), 256, 0, s>>>(F, (uint8_t*)ws);
+      prof_after(s);
+      st = dc_cuda_check(cudaGetLastError(), "t planes kernel");
+      if (st) return st;
+      const size_t psmem = 1024 + (size_t)UP_STAGES * UP_STAGE_BYTES + 2 * UP_BLK_BYTES + sizeof(UpTail);
+      static size_t pset = 0;
+      if (psmem > pset) {
+        st = dc_cuda_check(cudaFuncSetAttribute(k_upre, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem),
+                           "smem attr");
+        if (st) return st;
+        pset = psmem;
+      }
+      prof_before(s, 3);
+      k_upre<<<n_sm, UP_THREADS, psmem, s>>>(F, (uint8_t*)ws);
+      prof_after(s);
+      st = dc_cuda_check(cudaGetLastError(), "prefill delta output kernel");
+      if (st) return st;
+    }
   }
   if (use_tc) {
     F.bt_ntb = (T + F.ws.bt_nb - 1) / F.ws.bt_nb;
