@@ -172,7 +172,9 @@ struct DcFwd {
   int64_t bt_total;            // total chunks
   int32_t bt_ntb, bt_ns, bt_grid, bt_pad;  // token blocks, pipeline stages, CTAs
   CUtensorMap tmap;            // prefill path: bf16 t planes [2 n_lin T rows x tcols], box 64 x 256
+  CUtensorMap xpf[3];          // prefill path: tenant-sorted activations, box 64 x pf_box tokens
   int32_t pf;                  // segments of >= DC_PF_MIN tokens take the prefill delta path
+  int32_t pf_box;              // min(256, T)
   DcWs ws;
 };
 
@@ -342,6 +344,7 @@ __device__ void build_records_for(const DcFwd& F, const WsPtr& P, int p, int s) 
   if (p == 0)
     for (int k = 0; k < len; ++k) P.tseg[st + k] = s;
   if (!R.valid || !(F.flags & DC_DELTA)) return;
+  if (F.pf && len >= DC_PF_MIN) return;  // k_vpre computes t for this segment
   const int passes = (len + DC_V_TOKS - 1) / DC_V_TOKS;
   int per_pass = 0;
   for (int b = 0; b < L.n_bands; ++b) per_pass += (L.band[b].v_tiles + L.band[b].v_group - 1) / L.band[b].v_group;
@@ -1812,38 +1815,14 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
 // ---------------------------------------------------------------------------------------------
 // Prefill delta path (segments of at least DC_PF_MIN tokens), tcgen05 tensor cores.
 //
-// k_thl: t of every token of such a segment as two bf16 planes, t = hi + lo to ~16 bits, in the
-// layout the U-side kernel loads with TMA: [plane][linear][token][tcols], band b of the tenant
-// starting at column sum_{b' < b} align(rank_b', 64) (zeros in the padding).
+// k_vpre computes t and also writes it as two bf16 planes, t = hi + lo to ~16 bits, in the layout
+// k_upre loads with TMA: [plane][linear][token][tcols], band b of the tenant starting at column
+// sum_{b' < b} align(rank_b', 64), zeros in the padding.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ int pf_band_col(const DcURec& R, int b) {
   int c = 0;
   for (int i = 0; i < b; ++i) c += (R.band[i].rank + 63) & ~63;
   return c;
-}
-
-__global__ void __launch_bounds__(256) k_thl(const __grid_constant__ DcFwd F, uint8_t* ws) {
-  WsPtr P = ws_ptr(F.ws, ws);
-  const int T = F.ws.T;
-  const int p = blockIdx.y, tok = blockIdx.x;
-  if (p >= F.n_lin || tok >= T) return;
-  const int sg = P.tseg[tok];
-  const DcURec& R = P.urecs[(int64_t)p * T + sg];
-  if (!R.valid || R.len < DC_PF_MIN) return;
-  const float* tr = P.tws + ((int64_t)p * T + tok) * F.ws.r_stride;
-  __nv_bfloat16* hi = P.thl + ((int64_t)p * T + tok) * F.ws.tcols;
-  __nv_bfloat16* lo = hi + (int64_t)F.n_lin * T * F.ws.tcols;
-  int col = 0;
-  for (int b = 0; b < R.n_bands; ++b) {
-    const int rb = R.band[b].rank, padded = (rb + 63) & ~63;
-    for (int i = threadIdx.x; i < padded; i += blockDim.x) {
-      const float v = i < rb ? tr[R.band[b].r0 + i] : 0.f;
-      const __nv_bfloat16 h = __float2bfloat16_rn(v);
-      hi[col + i] = h;
-      lo[col + i] = __float2bfloat16_rn(v - __bfloat162float(h));
-    }
-    col += padded;
-  }
 }
 
 // One 16-byte chunk (8 consecutive K columns) of a 128-byte-swizzled K-major bf16 tile row.
@@ -2250,6 +2229,393 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
   tc_fence_before();
   __syncthreads();
   if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc(tbase, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// k_vpre: t = S * (V_hat^T x) for segments of at least DC_PF_MIN tokens, on tcgen05.
+// Unit = (linear p, long segment, V group of the tenant: up to 8 tiles of 16 ranks of one band);
+// the segment's tokens in tiles of up to 256 (the MMA N).  K = d_in in chunks of 64 columns.
+//   warp 0      TMA: per chunk the activation tile (256 tenant-sorted tokens x 64); per 512-column
+//               block the group's V block (codes + meta of its tiles) into a two-slot ring
+//   warps 1-8   expansion: (c - z) * scale of the chunk's 128 ranks x 64 columns as bf16 hi/lo
+//   warp 9      TMEM owner and MMA issuer: D[rank][token] += Vhi x + Vlo x (M 128, K 16)
+//   warps 10-13 epilogue: t = S * D into the fp32 t rows and the bf16 t planes
+// ---------------------------------------------------------------------------------------------
+#define VP_THREADS 448
+#define VP_A_BYTES 16384  // 128 ranks x 64 bf16
+#define VP_B_BYTES 32768  // 256 tokens x 64 bf16
+#define VP_STAGE_BYTES (2 * VP_A_BYTES + VP_B_BYTES)
+#define VP_STAGES 2
+#define VP_BLK_BYTES 18432  // largest V group block (2-bit: 8 tiles x 2304 bytes)
+#define VP_MAX_PJ 512
+
+struct VpTail {
+  uint64_t full_b[VP_STAGES], full_a[VP_STAGES], empty[VP_STAGES];
+  uint64_t blk_full[2], blk_empty[2];
+  uint64_t acc_full[2], acc_empty[2];
+  uint32_t tmem_base;
+  int abort;
+  int nlong, npj, box;
+  int lseg[UP_MAX_LONG];
+  int pref[VP_MAX_PJ + 1];  // units (V groups) before each (linear slot, long segment) pair
+};
+
+// Codes of lane `ln` of half h of one (tile, block) region A, group grp: c[s][hh] holds the codes of
+// columns 32 t + 8 s + 4 hh + b (byte b), t = ln % 4.  The same extraction as the decode V kernel.
+__device__ __forceinline__ void vp_lane_codes(const uint8_t* A, int bits, int rows, int ngrp, int h, int ln, int grp,
+                                              uint32_t (&c)[4][2]) {
+  const int nh = h == 0 ? min(rows, 8) : rows - 8;
+#pragma unroll
+  for (int s = 0; s < 4; ++s) c[s][0] = c[s][1] = 0u;
+  if ((ln >> 2) >= nh) return;
+  const uint8_t* hb = A + dc_v_half_off(bits, rows, ngrp, h);
+  const int p0 = dc_v_plane0_bytes(bits, ngrp);
+  if (bits == 2 && ngrp == 4) {
+    const uint4 w0 = *reinterpret_cast<const uint4*>(hb + ln * 32);
+    const uint4 w1 = *reinterpret_cast<const uint4*>(hb + ln * 32 + 16);
+    const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) c[s][hh] = (w[2 * s + hh] >> (2 * grp)) & 0x03030303u;
+  } else if (bits == 8) {
+    const uint4 q0 = *reinterpret_cast<const uint4*>(hb + ln * p0 + 32 * grp);
+    const uint4 q1 = *reinterpret_cast<const uint4*>(hb + ln * p0 + 32 * grp + 16);
+    const uint32_t w[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) c[s][hh] = w[2 * s + hh];
+  } else {
+    const uint2 w2 = *reinterpret_cast<const uint2*>(hb + ln * p0 + 8 * grp);
+    uint32_t w1 = 0;
+    if (bits == 3) w1 = *reinterpret_cast<const uint32_t*>(hb + 4 * nh * p0 + ln * (4 * ngrp) + 4 * grp);
+#pragma unroll
+    for (int s = 0; s < 4; ++s)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t r = reg_shift2((s >> 1) ? w2.y : w2.x, 2 * (s & 1) + hh);
+        if (bits == 3) r |= v_reg_hi3(w1, s, hh);
+        c[s][hh] = r;
+      }
+  }
+}
+
+__device__ __forceinline__ bool vp_aborted(VpTail* tail) { return *reinterpret_cast<volatile int*>(&tail->abort) != 0; }
+__device__ __forceinline__ bool vp_wait(uint64_t* bar, uint32_t parity, VpTail* tail, int* st) {
+  if (vp_aborted(tail)) return false;
+  if (mbar_wait(bar, parity)) return true;
+  tail->abort = 1;
+  set_status(st, DC_ERR_CUDA);
+  return false;
+}
+
+// A V group: band b, group index inside the band, its tiles and first rank.
+struct VpGroup {
+  int b, grp, t0, ntiles, rows_left, r0;  // first tile, tiles, ranks from the first tile on, first rank
+};
+
+struct VpUnit {
+  int p, j, go;  // linear, long segment index, V group index across the tenant's bands
+  DcLayout L;
+  VpGroup G;
+  const DcURec* R;
+};
+
+// Unit u of this batch -> its linear, segment and V group (false past the last unit).
+__device__ __forceinline__ bool vp_unit(const DcFwd& F, const WsPtr& P, const VpTail* tail, int u, VpUnit& U) {
+  if (u >= tail->pref[tail->npj]) return false;
+  int pj = 0;
+  while (tail->pref[pj + 1] <= u) ++pj;
+  const int slot = pj / tail->nlong;
+  U.j = pj % tail->nlong;
+  U.p = F.order[slot];
+  U.go = u - tail->pref[pj];
+  U.R = P.urecs + (int64_t)U.p * F.ws.T + tail->lseg[U.j];
+  const dc_delta_handle* h = F.lin[U.p].tenants + U.R->tenant;
+  U.L = dc_layout(h->desc);
+  U.L.dev_base = (int64_t)h->dev_base;
+  int gi = U.go;
+  for (int b = 0; b < U.L.n_bands; ++b) {
+    const DcBand& B = U.L.band[b];
+    const int ng = (B.v_tiles + B.v_group - 1) / B.v_group;
+    if (gi < ng) {
+      U.G.b = b;
+      U.G.grp = gi;
+      U.G.t0 = gi * B.v_group;
+      U.G.ntiles = dc_v_group_ntiles(B, gi);
+      U.G.rows_left = B.rank - 16 * U.G.t0;
+      U.G.r0 = B.r0 + 16 * U.G.t0;
+      return true;
+    }
+    gi -= ng;
+  }
+  return false;
+}
+
+__global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ DcFwd F, uint8_t* ws) {
+  extern __shared__ __align__(1024) uint8_t vp_raw[];
+  uint8_t* sm = vp_raw + ((1024 - (smem_u32(vp_raw) & 1023)) & 1023);
+  uint8_t* blkring = sm + VP_STAGES * VP_STAGE_BYTES;
+  VpTail* tail = reinterpret_cast<VpTail*>(blkring + 2 * VP_BLK_BYTES);
+  WsPtr P = ws_ptr(F.ws, ws);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int T = F.ws.T;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < VP_STAGES; ++s) {
+      mbar_init(&tail->full_b[s], 1);
+      mbar_init(&tail->full_a[s], 8);
+      mbar_init(&tail->empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&tail->blk_full[b], 1);
+      mbar_init(&tail->blk_empty[b], 8);
+      mbar_init(&tail->acc_full[b], 1);
+      mbar_init(&tail->acc_empty[b], 4);
+    }
+    tail->abort = 0;
+    const int nseg = P.st[DC_WS_NSEG];
+    int n = 0;
+    for (int sg = 0; sg < nseg && n < UP_MAX_LONG; ++sg)
+      if (P.segs[3 * sg] >= 0 && P.segs[3 * sg + 2] >= DC_PF_MIN) tail->lseg[n++] = sg;
+    tail->nlong = n;
+    tail->npj = min(VP_MAX_PJ, F.n_lin * n);
+    fence_mbar_init();
+  }
+  __syncthreads();
+  if (warp == 0) {  // V groups per (linear slot, long segment): the unit prefix table
+    for (int pj = lane; pj < tail->npj; pj += 32) {
+      const int p = F.order[pj / tail->nlong];
+      const DcURec& R = P.urecs[(int64_t)p * T + tail->lseg[pj % tail->nlong]];
+      int cnt = 0;
+      if (R.valid) {
+        const DcLayout L = dc_layout(F.lin[p].tenants[R.tenant].desc);
+        for (int b = 0; b < L.n_bands; ++b) cnt += (L.band[b].v_tiles + L.band[b].v_group - 1) / L.band[b].v_group;
+      }
+      tail->pref[pj + 1] = cnt;
+    }
+    __syncwarp();
+    if (lane == 0) {
+      tail->pref[0] = 0;
+      for (int pj = 0; pj < tail->npj; ++pj) tail->pref[pj + 1] += tail->pref[pj];
+    }
+  } else if (warp == 9) {
+    tmem_alloc(smem_u32(&tail->tmem_base), 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = tail->tmem_base;
+  const int box = F.pf_box;
+  VpUnit U;
+  if (warp == 0) {
+    // ---------------- TMA producer
+    uint32_t seq = 0, bseq = 0;
+    for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+      const DcBand& B = U.L.band[U.G.b];
+      const int m = F.lin[U.p].input;
+      for (int tok0 = U.R->st; tok0 < U.R->st + U.R->len && !vp_aborted(tail); tok0 += 256) {
+        for (int kb = 0; kb < U.L.nkb; ++kb) {
+          const int ngrp = kb == U.L.nkb - 1 ? U.L.tail_groups : 4;
+          const int bs = bseq & 1;
+          if (bseq >= 2 && !vp_wait(&tail->blk_empty[bs], ((bseq >> 1) - 1) & 1, tail, P.st)) break;
+          const int bytes = (int)dc_v_group_block_bytes(B, U.G.grp, ngrp);
+          if (lane == 0) {
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(U.L.dev_base) + B.v_off +
+                                 dc_v_group_block_off(B, U.L, U.G.grp, kb);
+            mbar_arrive_expect_tx(&tail->blk_full[bs], (uint32_t)bytes);
+            bulk_g2s(blkring + bs * VP_BLK_BYTES, src, (uint32_t)bytes, &tail->blk_full[bs]);
+          }
+          __syncwarp();
+          ++bseq;
+          for (int ch = 0; ch < 2 * ngrp; ++ch, ++seq) {
+            const int s = seq % VP_STAGES;
+            if (seq >= VP_STAGES && !vp_wait(&tail->empty[s], ((seq / VP_STAGES) - 1) & 1, tail, P.st)) break;
+            if (lane == 0) {
+              uint8_t* st = sm + (size_t)s * VP_STAGE_BYTES + 2 * VP_A_BYTES;
+              mbar_arrive_expect_tx(&tail->full_b[s], (uint32_t)(box * 128));
+              tma_load_2d(st, &F.xpf[m], 512 * kb + 64 * ch, tok0, &tail->full_b[s]);
+            }
+            __syncwarp();
+          }
+        }
+      }
+    }
+  } else if (warp <= 8) {
+    // ---------------- expansion warps: thread e -> rank row e % 128, column half e / 128 of a chunk
+    const int e = threadIdx.x - 32;
+    const int row = e & 127, part = e >> 7;
+    const int tile = row >> 4, h = (row >> 3) & 1, g = row & 7;
+    uint32_t seq = 0, bseq = 0;
+    for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+      const DcBand& B = U.L.band[U.G.b];
+      const int rows_t = tile < U.G.ntiles ? min(16, U.G.rows_left - 16 * tile) : 0;
+      bool ok = true;
+      for (int tok0 = U.R->st; ok && tok0 < U.R->st + U.R->len; tok0 += 256) {
+        for (int kb = 0; ok && kb < U.L.nkb; ++kb) {
+          const int ngrp = kb == U.L.nkb - 1 ? U.L.tail_groups : 4;
+          const int bs = bseq & 1;
+          if (!vp_wait(&tail->blk_full[bs], (bseq >> 1) & 1, tail, P.st)) {
+            ok = false;
+            break;
+          }
+          ++bseq;
+          const uint8_t* A = blkring + bs * VP_BLK_BYTES + tile * dc_v_block_bytes(B.bits, 16, ngrp);
+          for (int ch = 0; ch < 2 * ngrp; ++ch, ++seq) {
+            const int s = seq % VP_STAGES;
+            if (seq >= VP_STAGES && !vp_wait(&tail->empty[s], ((seq / VP_STAGES) - 1) & 1, tail, P.st)) {
+              ok = false;
+              break;
+            }
+            const int grp = ch >> 1, hc = ch & 1;
+            uint32_t c[4][2];
+            float sc[8], zz[8];
+            if (rows_t > 0) {
+              vp_lane_codes(A, B.bits, rows_t, ngrp, h, 4 * g + 2 * hc + part, grp, c);
+              float s0 = 0.f, z0 = 0.f;
+              if (8 * h + g < rows_t) {
+                const __half2 mz = *reinterpret_cast<const __half2*>(
+                    A + dc_v_block_code_bytes(B.bits, rows_t, ngrp) + 4 * (grp * 16 + g * 2 + h));
+                s0 = __low2float(mz);
+                z0 = __high2float(mz);
+              }
+#pragma unroll
+              for (int k = 0; k < 8; ++k) sc[k] = s0, zz[k] = z0;
+            } else {
+#pragma unroll
+              for (int k = 0; k < 4; ++k) c[k][0] = c[k][1] = 0u;
+#pragma unroll
+              for (int k = 0; k < 8; ++k) sc[k] = zz[k] = 0.f;
+            }
+            uint8_t* ahi = sm + (size_t)s * VP_STAGE_BYTES;
+#pragma unroll
+            for (int sidx = 0; sidx < 4; ++sidx) {
+              uint4 hv, lv;
+              pf_dequant8(c[sidx][0], c[sidx][1], sc, zz, hv, lv);
+              sw128_store(ahi, row, 4 * part + sidx, hv);
+              sw128_store(ahi + VP_A_BYTES, row, 4 * part + sidx, lv);
+            }
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&tail->full_a[s]);
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&tail->blk_empty[bs]);
+        }
+      }
+      if (!ok) break;
+    }
+  } else if (warp == 9) {
+    // ---------------- MMA issuer
+    uint32_t seq = 0, unit = 0;
+    for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+      bool ok = true;
+      for (int tok0 = U.R->st; ok && tok0 < U.R->st + U.R->len; tok0 += 256, ++unit) {
+        const int ntok = min(256, U.R->st + U.R->len - tok0);
+        const uint32_t idesc = umma_idesc_bf16(128, (ntok + 15) & ~15);
+        const int b = unit & 1;
+        if (unit >= 2 && !vp_wait(&tail->acc_empty[b], ((unit >> 1) - 1) & 1, tail, P.st)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t dt = tbase + (uint32_t)(b * 256);
+        int ci = 0;
+        for (int kb = 0; ok && kb < U.L.nkb; ++kb) {
+          const int ngrp = kb == U.L.nkb - 1 ? U.L.tail_groups : 4;
+          for (int ch = 0; ch < 2 * ngrp; ++ch, ++seq, ++ci) {
+            const int s = seq % VP_STAGES;
+            const uint32_t ph = (seq / VP_STAGES) & 1;
+            if (!vp_wait(&tail->full_b[s], ph, tail, P.st) || !vp_wait(&tail->full_a[s], ph, tail, P.st)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            if (lane == 0) {
+              const uint32_t a0 = smem_u32(sm + (size_t)s * VP_STAGE_BYTES);
+              const uint64_t ah = umma_desc_sw128(a0), al = umma_desc_sw128(a0 + VP_A_BYTES);
+              const uint64_t bx = umma_desc_sw128(a0 + 2 * VP_A_BYTES);
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk) {
+                const uint64_t o = (uint64_t)(2 * kk);
+                umma_bf16(dt, ah + o, bx + o, idesc, (ci > 0 || kk > 0) ? 1u : 0u);
+                umma_bf16(dt, al + o, bx + o, idesc, 1u);
+              }
+              umma_commit(smem_u32(&tail->empty[s]));
+            }
+            __syncwarp();
+          }
+        }
+        if (!ok) break;
+        if (lane == 0) umma_commit(smem_u32(&tail->acc_full[b]));
+        __syncwarp();
+      }
+      if (!ok) break;
+    }
+  } else {
+    // ---------------- epilogue warps 10-13 (TMEM lane quarter warp % 4); exits agreed by a vote
+    const int q4 = warp & 3, row = 32 * q4 + lane;
+    uint32_t unit = 0;
+    bool go_on = true;
+    for (int u = blockIdx.x; go_on && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+      const DcBand& B = U.L.band[U.G.b];
+      const int nvalid = min(16 * U.G.ntiles, U.G.rows_left);
+      const int rank = U.G.r0 + row;
+      const float Sv = row < nvalid ? reinterpret_cast<const float*>(U.L.dev_base + U.L.s_off)[rank] : 0.f;
+      int bandcol = 0;
+      for (int bb = 0; bb < U.G.b; ++bb) bandcol += (U.L.band[bb].rank + 63) & ~63;
+      const int col = bandcol + (rank - B.r0);
+      const bool padrow = row >= nvalid && rank - B.r0 >= B.rank && rank - B.r0 < ((B.rank + 63) & ~63);
+      for (int tok0 = U.R->st; tok0 < U.R->st + U.R->len; tok0 += 256, ++unit) {
+        const int ntok = min(256, U.R->st + U.R->len - tok0);
+        const int b = unit & 1;
+        const bool okw = vp_wait(&tail->acc_full[b], (unit >> 1) & 1, tail, P.st);
+        if (!bar_and(1, 128, okw)) {
+          go_on = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t ta = tbase + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * 256);
+        const int64_t trow0 = (int64_t)U.p * T + tok0;
+        for (int cb = 0; cb < ntok; cb += 16) {
+          uint32_t r[16];
+          tmem_ld16(ta + cb, r);
+          tmem_ld_wait();
+          if (row < nvalid) {
+#pragma unroll
+            for (int jj = 0; jj < 16; ++jj) {
+              if (cb + jj < ntok) {
+                const float t = Sv * __uint_as_float(r[jj]);
+                const int64_t tr = trow0 + cb + jj;
+                P.tws[tr * F.ws.r_stride + rank] = t;
+                const __nv_bfloat16 hb = __float2bfloat16_rn(t);
+                P.thl[tr * F.ws.tcols + col] = hb;
+                P.thl[((int64_t)F.n_lin * T + tr) * F.ws.tcols + col] = __float2bfloat16_rn(t - __bfloat162float(hb));
+              }
+            }
+          } else if (padrow) {  // zero the band's padding columns of the t planes (read by k_upre)
+            for (int jj = 0; jj < 16; ++jj) {
+              if (cb + jj < ntok) {
+                const int64_t tr = trow0 + cb + jj;
+                P.thl[tr * F.ws.tcols + col] = __float2bfloat16_rn(0.f);
+                P.thl[((int64_t)F.n_lin * T + tr) * F.ws.tcols + col] = __float2bfloat16_rn(0.f);
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&tail->acc_empty[b]);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -2686,9 +3052,16 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   // long segments take the tensor-core delta path when the batch is large enough
   F.pf = (flags & DC_DELTA) && !(flags & DC_DECODE_ONLY) && T >= 2 * DC_PF_MIN;
   if (F.pf) {
+    if (dtype_in != DC_DTYPE_BF16) return dc_fail(DC_ERR_UNSUPPORTED, "the prefill path needs bf16 activations");
     dc_status st0 = encode_bf16_map(&F.tmap, (const uint8_t*)ws + F.ws.thl, F.ws.tcols, (int64_t)2 * n_lin * T,
                                     F.ws.tcols, 256);
     if (st0) return st0;
+    F.pf_box = std::min(256, T);
+    for (int m = 0; m < n_in; ++m) {
+      const uint8_t* xb = (const uint8_t*)ws + F.ws.xsort + (int64_t)m * T * F.ws.max_d_in * 2;
+      st0 = encode_bf16_map(&F.xpf[m], xb, dxs[m], T, F.ws.max_d_in, F.pf_box);
+      if (st0) return st0;
+    }
   }
   cudaStream_t s = (cudaStream_t)stream;
   dc_status st;
@@ -2735,6 +3108,21 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "rank-reduction kernel");
     if (st) return st;
+    if (F.pf) {
+      const size_t qsmem = 1024 + (size_t)VP_STAGES * VP_STAGE_BYTES + 2 * VP_BLK_BYTES + sizeof(VpTail);
+      static size_t qset = 0;
+      if (qsmem > qset) {
+        st = dc_cuda_check(cudaFuncSetAttribute(k_vpre, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsmem),
+                           "smem attr");
+        if (st) return st;
+        qset = qsmem;
+      }
+      prof_before(s, 2);
+      k_vpre<<<n_sm, VP_THREADS, qsmem, s>>>(F, (uint8_t*)ws);
+      prof_after(s);
+      st = dc_cuda_check(cudaGetLastError(), "prefill rank-reduction kernel");
+      if (st) return st;
+    }
   }
   if (flags & DC_DELTA) {
     const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_BBUF + U_BCONST + sizeof(USmemTail);
@@ -2752,11 +3140,6 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     st = dc_cuda_check(cudaGetLastError(), "delta output kernel");
     if (st) return st;
     if (F.pf) {
-      prof_before(s, 3);
-      k_thl<<<dim3(T, n_lin), 256, 0, s>>>(F, (uint8_t*)ws);
-      prof_after(s);
-      st = dc_cuda_check(cudaGetLastError(), "t planes kernel");
-      if (st) return st;
       const size_t psmem = 1024 + (size_t)UP_STAGES * UP_STAGE_BYTES + 2 * UP_BLK_BYTES + sizeof(UpTail);
       static size_t pset = 0;
       if (psmem > pset) {
