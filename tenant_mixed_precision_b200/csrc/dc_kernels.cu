@@ -1859,14 +1859,14 @@ __device__ __forceinline__ void pf_dequant8(uint32_t r0, uint32_t r1, const floa
 // tiles of up to 256 (the MMA N).  K = the tenant's ranks, band by band, in chunks of 64.
 //   warp 0     TMA: per chunk the t planes (hi, lo: 256 tokens x 64 ranks each); per U block the
 //              block's bytes (codes of the eight 16-row tiles + meta) into a two-slot ring
-//   warps 1-4  expansion: (c - z) * scale of the chunk's 128 x 64 codes as bf16 hi and lo
-//              (128-byte-swizzled K-major tiles), from the staged block
-//   warp 5     TMEM owner and MMA issuer: D[row][token] += Uhi thi + Uhi tlo + Ulo thi
+//   warps 1-8  expansion (one 16-row tile each): (c - z) * scale of the chunk's 128 x 64 codes
+//              as bf16 hi and lo (128-byte-swizzled K-major tiles), from the staged block
+//   warp 9     TMEM owner and MMA issuer: D[row][token] += Uhi thi + Uhi tlo + Ulo thi
 //              (M 128, N tokens, K 16 per instruction), two accumulators
-//   warps 6-9  epilogue: TMEM lane = output row, writes ydelta
+//   warps 10-13 epilogue: TMEM lane = output row, writes ydelta
 // Units are dealt to the persistent CTAs round robin; every wait is bounded.
 // ---------------------------------------------------------------------------------------------
-#define UP_THREADS 320
+#define UP_THREADS 448
 #define UP_A_BYTES 16384                  // 128 rows x 64 bf16
 #define UP_B_BYTES 32768                  // 256 tokens x 64 bf16
 #define UP_STAGE_BYTES (2 * UP_A_BYTES + 2 * UP_B_BYTES)
@@ -1882,6 +1882,7 @@ struct UpTail {
   int abort;
   int nlong;
   int lseg[UP_MAX_LONG];
+  DcURec rec[UP_THREADS / 32];  // each warp's copy of its current unit's record
 };
 
 struct UpChunk {
@@ -2017,14 +2018,22 @@ __device__ __forceinline__ bool up_wait(uint64_t* bar, uint32_t parity, UpTail* 
 struct UpIter {
   int u, tt;  // current unit (-1 before the first) and token tile
 };
-__device__ __forceinline__ bool up_next(const DcFwd& F, const WsPtr& P, const UpTail* tail, UpIter& it, int& p,
+// The unit's record is copied into the calling warp's slot in shared memory (R points there).
+__device__ __forceinline__ void up_load_rec(const DcURec* src, DcURec* dst) {
+  constexpr int NV = sizeof(DcURec) / 16;
+  const int lane = threadIdx.x & 31;
+  __syncwarp();
+  if (lane < NV) reinterpret_cast<uint4*>(dst)[lane] = ldg128(reinterpret_cast<const uint8_t*>(src) + 16 * lane);
+  __syncwarp();
+}
+
+__device__ __forceinline__ bool up_next(const DcFwd& F, const WsPtr& P, UpTail* tail, UpIter& it, int& p,
                                         int& go, const DcURec*& R, int& tok0, int& ntok) {
   const int T = F.ws.T;
+  DcURec* mine = &tail->rec[threadIdx.x >> 5];
   for (;;) {
     if (it.u >= 0) {
-      int j;
-      if (!up_unit(F, tail->nlong, it.u, p, j, go)) return false;
-      R = P.urecs + (int64_t)p * T + tail->lseg[j];
+      R = mine;  // still the current unit's record
       if (R->valid && 256 * (it.tt + 1) < R->len) {
         ++it.tt;
         tok0 = R->st + 256 * it.tt;
@@ -2038,7 +2047,8 @@ __device__ __forceinline__ bool up_next(const DcFwd& F, const WsPtr& P, const Up
     it.tt = 0;
     int j;
     if (!up_unit(F, tail->nlong, it.u, p, j, go)) return false;
-    R = P.urecs + (int64_t)p * T + tail->lseg[j];
+    up_load_rec(P.urecs + (int64_t)p * T + tail->lseg[j], mine);
+    R = mine;
     if (!R->valid) {
       it.tt = 1 << 20;  // skip: the next call moves to the next unit
       continue;
@@ -2060,12 +2070,12 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
   if (threadIdx.x == 0) {
     for (int s = 0; s < UP_STAGES; ++s) {
       mbar_init(&tail->full_b[s], 1);
-      mbar_init(&tail->full_a[s], 4);
+      mbar_init(&tail->full_a[s], 8);
       mbar_init(&tail->empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tail->blk_full[b], 1);
-      mbar_init(&tail->blk_empty[b], 4);
+      mbar_init(&tail->blk_empty[b], 8);
       mbar_init(&tail->acc_full[b], 1);
       mbar_init(&tail->acc_empty[b], 4);
     }
@@ -2077,7 +2087,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
     tail->nlong = n;
     fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     tmem_alloc(smem_u32(&tail->tmem_base), 512);
     tmem_relinquish();
   }
@@ -2123,8 +2133,8 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
         __syncwarp();
       }
     }
-  } else if (warp <= 4) {
-    // ---------------- expansion warps: tiles 2 (warp - 1) and 2 (warp - 1) + 1
+  } else if (warp <= 8) {
+    // ---------------- expansion warps: warp w expands the 16-row tile w - 1
     const int e = warp - 1;
     uint32_t seq = 0, bseq = 0;
     while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
@@ -2152,7 +2162,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
         uint8_t* ahi = sm + (size_t)s * UP_STAGE_BYTES;
         const uint8_t* blk = blkring + ((bseq - 1) & 1) * UP_BLK_BYTES;
         const DcUBand UB = R->band[C.b];
-        for (int tl = 0; tl < 2; ++tl) up_expand_tile(blk, UB, C.k, C.c0, 2 * e + tl, lane, ahi, ahi + UP_A_BYTES);
+        up_expand_tile(blk, UB, C.k, C.c0, e, lane, ahi, ahi + UP_A_BYTES);
         fence_proxy_async();  // generic-proxy writes -> tensor-core (async proxy) reads
         __syncwarp();
         if (lane == 0) mbar_arrive(&tail->full_a[s]);
@@ -2161,7 +2171,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
       __syncwarp();
       if (lb >= 0 && lane == 0) mbar_arrive(&tail->blk_empty[(bseq - 1) & 1]);
     }
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ---------------- MMA issuer
     uint32_t seq = 0, unit = 0;
     while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
@@ -2202,7 +2212,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
       ++unit;
     }
   } else {
-    // ---------------- epilogue warps 6-9 (TMEM lane quarter warp % 4); exits agreed by a vote
+    // ---------------- epilogue warps 10-13 (TMEM lane quarter warp % 4); exits agreed by a vote
     const int q4 = warp & 3, row = 32 * q4 + lane;
     uint32_t unit = 0;
     while (up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
@@ -2228,7 +2238,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
@@ -2318,11 +2328,12 @@ struct VpGroup {
   int b, grp, t0, ntiles, rows_left, r0;  // first tile, tiles, ranks from the first tile on, first rank
 };
 
-struct VpUnit {
-  int p, j, go;  // linear, long segment index, V group index across the tenant's bands
-  DcLayout L;
+struct VpUnit {  // compact: kept in registers by every role
+  int p, j;            // linear, long segment index
+  int64_t base, s_off; // blob address, offset of S
+  DcBand B;            // the group's band
+  int nkb, tail_groups, bandcol, st, len;
   VpGroup G;
-  const DcURec* R;
 };
 
 // Unit u of this batch -> its linear, segment and V group (false past the last unit).
@@ -2333,16 +2344,22 @@ __device__ __forceinline__ bool vp_unit(const DcFwd& F, const WsPtr& P, const Vp
   const int slot = pj / tail->nlong;
   U.j = pj % tail->nlong;
   U.p = F.order[slot];
-  U.go = u - tail->pref[pj];
-  U.R = P.urecs + (int64_t)U.p * F.ws.T + tail->lseg[U.j];
-  const dc_delta_handle* h = F.lin[U.p].tenants + U.R->tenant;
-  U.L = dc_layout(h->desc);
-  U.L.dev_base = (int64_t)h->dev_base;
-  int gi = U.go;
-  for (int b = 0; b < U.L.n_bands; ++b) {
-    const DcBand& B = U.L.band[b];
+  const DcURec& R = P.urecs[(int64_t)U.p * F.ws.T + tail->lseg[U.j]];
+  U.st = R.st;
+  U.len = R.len;
+  const dc_delta_handle* h = F.lin[U.p].tenants + R.tenant;
+  const DcLayout L = dc_layout(h->desc);
+  U.base = (int64_t)h->dev_base;
+  U.s_off = L.s_off;
+  U.nkb = L.nkb;
+  U.tail_groups = L.tail_groups;
+  int gi = u - tail->pref[pj];
+  U.bandcol = 0;
+  for (int b = 0; b < L.n_bands; ++b) {
+    const DcBand& B = L.band[b];
     const int ng = (B.v_tiles + B.v_group - 1) / B.v_group;
     if (gi < ng) {
+      U.B = B;
       U.G.b = b;
       U.G.grp = gi;
       U.G.t0 = gi * B.v_group;
@@ -2352,6 +2369,7 @@ __device__ __forceinline__ bool vp_unit(const DcFwd& F, const WsPtr& P, const Vp
       return true;
     }
     gi -= ng;
+    U.bandcol += (B.rank + 63) & ~63;
   }
   return false;
 }
@@ -2416,17 +2434,18 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
     // ---------------- TMA producer
     uint32_t seq = 0, bseq = 0;
     for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
-      const DcBand& B = U.L.band[U.G.b];
+      const DcBand& B = U.B;
       const int m = F.lin[U.p].input;
-      for (int tok0 = U.R->st; tok0 < U.R->st + U.R->len && !vp_aborted(tail); tok0 += 256) {
-        for (int kb = 0; kb < U.L.nkb; ++kb) {
-          const int ngrp = kb == U.L.nkb - 1 ? U.L.tail_groups : 4;
+      for (int tok0 = U.st; tok0 < U.st + U.len && !vp_aborted(tail); tok0 += 256) {
+        for (int kb = 0; kb < U.nkb; ++kb) {
+          const int ngrp = kb == U.nkb - 1 ? U.tail_groups : 4;
           const int bs = bseq & 1;
           if (bseq >= 2 && !vp_wait(&tail->blk_empty[bs], ((bseq >> 1) - 1) & 1, tail, P.st)) break;
           const int bytes = (int)dc_v_group_block_bytes(B, U.G.grp, ngrp);
           if (lane == 0) {
-            const uint8_t* src = reinterpret_cast<const uint8_t*>(U.L.dev_base) + B.v_off +
-                                 dc_v_group_block_off(B, U.L, U.G.grp, kb);
+            const uint8_t* src = reinterpret_cast<const uint8_t*>(U.base) + B.v_off +
+                                 (int64_t)U.G.grp * B.v_group * B.v_tile_bytes +
+                                 (int64_t)kb * dc_v_group_block_bytes(B, U.G.grp, 4);
             mbar_arrive_expect_tx(&tail->blk_full[bs], (uint32_t)bytes);
             bulk_g2s(blkring + bs * VP_BLK_BYTES, src, (uint32_t)bytes, &tail->blk_full[bs]);
           }
@@ -2452,12 +2471,12 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
     const int tile = row >> 4, h = (row >> 3) & 1, g = row & 7;
     uint32_t seq = 0, bseq = 0;
     for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
-      const DcBand& B = U.L.band[U.G.b];
+      const DcBand& B = U.B;
       const int rows_t = tile < U.G.ntiles ? min(16, U.G.rows_left - 16 * tile) : 0;
       bool ok = true;
-      for (int tok0 = U.R->st; ok && tok0 < U.R->st + U.R->len; tok0 += 256) {
-        for (int kb = 0; ok && kb < U.L.nkb; ++kb) {
-          const int ngrp = kb == U.L.nkb - 1 ? U.L.tail_groups : 4;
+      for (int tok0 = U.st; ok && tok0 < U.st + U.len; tok0 += 256) {
+        for (int kb = 0; ok && kb < U.nkb; ++kb) {
+          const int ngrp = kb == U.nkb - 1 ? U.tail_groups : 4;
           const int bs = bseq & 1;
           if (!vp_wait(&tail->blk_full[bs], (bseq >> 1) & 1, tail, P.st)) {
             ok = false;
@@ -2514,8 +2533,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
     uint32_t seq = 0, unit = 0;
     for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
       bool ok = true;
-      for (int tok0 = U.R->st; ok && tok0 < U.R->st + U.R->len; tok0 += 256, ++unit) {
-        const int ntok = min(256, U.R->st + U.R->len - tok0);
+      for (int tok0 = U.st; ok && tok0 < U.st + U.len; tok0 += 256, ++unit) {
+        const int ntok = min(256, U.st + U.len - tok0);
         const uint32_t idesc = umma_idesc_bf16(128, (ntok + 15) & ~15);
         const int b = unit & 1;
         if (unit >= 2 && !vp_wait(&tail->acc_empty[b], ((unit >> 1) - 1) & 1, tail, P.st)) {
@@ -2525,8 +2544,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
         tc_fence_after();
         const uint32_t dt = tbase + (uint32_t)(b * 256);
         int ci = 0;
-        for (int kb = 0; ok && kb < U.L.nkb; ++kb) {
-          const int ngrp = kb == U.L.nkb - 1 ? U.L.tail_groups : 4;
+        for (int kb = 0; ok && kb < U.nkb; ++kb) {
+          const int ngrp = kb == U.nkb - 1 ? U.tail_groups : 4;
           for (int ch = 0; ch < 2 * ngrp; ++ch, ++seq, ++ci) {
             const int s = seq % VP_STAGES;
             const uint32_t ph = (seq / VP_STAGES) & 1;
@@ -2562,16 +2581,14 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
     uint32_t unit = 0;
     bool go_on = true;
     for (int u = blockIdx.x; go_on && vp_unit(F, P, tail, u, U); u += gridDim.x) {
-      const DcBand& B = U.L.band[U.G.b];
+      const DcBand& B = U.B;
       const int nvalid = min(16 * U.G.ntiles, U.G.rows_left);
       const int rank = U.G.r0 + row;
-      const float Sv = row < nvalid ? reinterpret_cast<const float*>(U.L.dev_base + U.L.s_off)[rank] : 0.f;
-      int bandcol = 0;
-      for (int bb = 0; bb < U.G.b; ++bb) bandcol += (U.L.band[bb].rank + 63) & ~63;
-      const int col = bandcol + (rank - B.r0);
+      const float Sv = row < nvalid ? reinterpret_cast<const float*>(U.base + U.s_off)[rank] : 0.f;
+      const int col = U.bandcol + (rank - B.r0);
       const bool padrow = row >= nvalid && rank - B.r0 >= B.rank && rank - B.r0 < ((B.rank + 63) & ~63);
-      for (int tok0 = U.R->st; tok0 < U.R->st + U.R->len; tok0 += 256, ++unit) {
-        const int ntok = min(256, U.R->st + U.R->len - tok0);
+      for (int tok0 = U.st; tok0 < U.st + U.len; tok0 += 256, ++unit) {
+        const int ntok = min(256, U.st + U.len - tok0);
         const int b = unit & 1;
         const bool okw = vp_wait(&tail->acc_full[b], (unit >> 1) & 1, tail, P.st);
         if (!bar_and(1, 128, okw)) {
