@@ -922,10 +922,9 @@ __device__ __forceinline__ void ud_mma(const uint8_t* blk, int bits, int nq, int
   // codes' row sums), column 7 a row of zeros; both constant rows sit after the two limb matrices
   const uint8_t* brow = (g < 6 ? bsm + g * U_BROW : bconst + (g - 6) * U_BROW) + 8 * t;
   const int pstride = g < 6 ? 6 * U_BROW : 0;
-  if (ns == 0) {  // 2-bit block: one or two quads in straight-line code
+  if (nq == 2 && ns == 0) {  // full 2-bit block: two quads in straight-line code
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
-      if (q >= nq) break;
       const uint4 wq = *reinterpret_cast<const uint4*>(ub + 512 * q + 16 * lane);
       uint2 bq[NPAIR][4];
 #pragma unroll
@@ -1534,14 +1533,15 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ D
 // whatever the tile count.  Per CTA: warp 0 loads each chunk's W slice (128 x 64) and activation
 // slice (NB x 64) with 2-D TMA into a ring of stages; warp 1 owns two NB-column fp32
 // accumulators in Tensor Memory and, from one thread, issues 4 MMAs (M 128, N NB, K 16) per
-// chunk, releasing the stage with a commit; warps 2-5 (one TMEM lane quarter each, lane = output
-// row) drain a finished accumulator.  A unit shared by several CTAs leaves fp32 partial tiles;
+// chunk, releasing the stage with a commit; warps 2-9 (two warpgroups, one TMEM lane quarter per
+// warp, lane = output row) drain a finished accumulator.  A unit shared by several CTAs leaves fp32 partial tiles;
 // the last contributor to arrive (a counter per unit) adds them in k order, so the result does
 // not depend on timing.  The epilogue adds the delta and writes y in the tokens' original order.
 // ---------------------------------------------------------------------------------------------
-#define BT_THREADS 192
+#define BT_THREADS 320
 #define BT_MAX_STAGES 8
 #define BT_A_BYTES 16384  // 128 rows x 64 bf16
+#define BT_MAX_SEGS 64
 
 struct BtTail {
   uint64_t full[BT_MAX_STAGES];
@@ -1553,6 +1553,8 @@ struct BtTail {
   int last_flag;
   int perm[256];    // epilogue: original position of each token of the unit's block (-1: none)
   uint8_t dfl[256]; // epilogue: the token has a delta
+  int nseg;         // segments of this CTA's chunk range (-1: more than BT_MAX_SEGS)
+  int64_t sg[BT_MAX_SEGS];  // their first chunks, in processing order
 };
 
 __device__ __forceinline__ int64_t bt_g0(const DcFwd& F, int c) { return (int64_t)c * F.bt_total / F.bt_grid; }
@@ -1627,9 +1629,28 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tail->acc_full[b], 1);
-      mbar_init(&tail->acc_empty[b], 4);
+      mbar_init(&tail->acc_empty[b], 8);
     }
     tail->abort = 0;
+    // Segment order: the range's last segment, then its first, then the rest.  Both ends are
+    // usually units shared with the neighbouring CTAs; doing them first lets the last contributor
+    // finish those units while streaming continues, instead of in the range's tail.
+    int n = 0;
+    for (int64_t g = g0; g < g1; ++n) {
+      if (n < BT_MAX_SEGS) tail->sg[n] = g;
+      const BtSeg S = bt_seg_at(F, g, g1);
+      g = S.ustart + S.k1;
+    }
+    if (n <= BT_MAX_SEGS) {
+      if (n >= 2) {
+        const int64_t last = tail->sg[n - 1];
+        for (int i = n - 1; i > 0; --i) tail->sg[i] = tail->sg[i - 1];
+        tail->sg[0] = last;
+      }
+      tail->nseg = n;
+    } else {
+      tail->nseg = -1;  // natural order
+    }
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -1643,8 +1664,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
   if (warp == 0) {
     // ---------------- TMA producer
     uint32_t seq = 0;
-    for (int64_t g = g0; g < g1 && !bt_aborted(tail);) {
-      const BtSeg S = bt_seg_at(F, g, g1);
+    const int nseg = tail->nseg;
+    int64_t g = g0;
+    for (int si = 0; (nseg >= 0 ? si < nseg : g < g1) && !bt_aborted(tail); ++si) {
+      const BtSeg S = bt_seg_at(F, nseg >= 0 ? tail->sg[si] : g, g1);
       const int p = F.order[S.slot];
       const int m = F.lin[p].input;
       for (int k = S.k0; k < S.k1; ++k, ++seq) {
@@ -1664,8 +1687,10 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
     // ---------------- MMA issuer (one thread)
     const uint32_t idesc = umma_idesc_bf16(128, NB);
     uint32_t seq = 0, segi = 0;
-    for (int64_t g = g0; g < g1 && !bt_aborted(tail); ++segi) {
-      const BtSeg S = bt_seg_at(F, g, g1);
+    const int nseg = tail->nseg;
+    int64_t g = g0;
+    for (int si = 0; (nseg >= 0 ? si < nseg : g < g1) && !bt_aborted(tail); ++si, ++segi) {
+      const BtSeg S = bt_seg_at(F, nseg >= 0 ? tail->sg[si] : g, g1);
       const int b = segi & 1;
       if (segi >= 2 && !bt_wait(&tail->acc_empty[b], ((segi >> 1) - 1) & 1, tail, P.st)) break;
       tc_fence_after();
@@ -1694,20 +1719,23 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
       g = S.ustart + S.k1;
     }
   } else {
-    // ---------------- epilogue warpgroup (warps 2-5): TMEM lane quarter warp % 4
-    const int q4 = warp & 3;
+    // ---------------- epilogue: two warpgroups (warps 2-5, 6-9), TMEM lane quarter warp % 4;
+    // warpgroup wg drains the 16-column blocks 2 i + wg of the accumulator
+    const int q4 = warp & 3, wg = (warp - 2) >> 2;
     const int row = 32 * q4 + lane;  // output row inside the tile
     const bool delta = (F.flags & DC_DELTA) != 0;
     float* part_base = reinterpret_cast<float*>(ws + F.ws.bt_part);
     int* cnt = reinterpret_cast<int*>(ws + F.ws.bt_cnt);
     uint32_t segi = 0;
-    // The four warps leave the loop together: the outcome of every wait is agreed through a
+    // The eight warps leave the loop together: the outcome of every wait is agreed through a
     // reducing named barrier, so no warp is left waiting at a barrier the others skipped.
-    for (int64_t g = g0; g < g1; ++segi) {
-      const BtSeg S = bt_seg_at(F, g, g1);
+    const int nseg = tail->nseg;
+    int64_t g = g0;
+    for (int si = 0; nseg >= 0 ? si < nseg : g < g1; ++si, ++segi) {
+      const BtSeg S = bt_seg_at(F, nseg >= 0 ? tail->sg[si] : g, g1);
       const int b = segi & 1;
       const bool okw = bt_wait(&tail->acc_full[b], (segi >> 1) & 1, tail, P.st);
-      if (!bar_and(1, 128, okw)) break;
+      if (!bar_and(1, 256, okw)) break;
       tc_fence_after();
       const int p = F.order[S.slot];
       const DcLinDev& lin = F.lin[p];
@@ -1716,16 +1744,16 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
       float* mypart = part_base + ((int64_t)(2 * c + my_slot) * NB) * 128;
       const uint32_t ta = tbase + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * NB);
       const int orow = S.ot * 128 + row;
-      const int et = threadIdx.x - 64;  // 0..127
+      const int et = threadIdx.x - 64;  // 0..255
       // destinations of the block's tokens, staged once per unit
-      for (int col = et; col < NB; col += 128) {
+      for (int col = et; col < NB; col += 256) {
         const int ts = S.tb * NB + col;
         tail->perm[col] = ts < T ? P.perm[ts] : -1;
         tail->dfl[col] = (delta && ts < T) ? P.dflag[(int64_t)p * T + ts] : 0;
       }
-      named_bar(1, 128);
+      named_bar(1, 256);
       const float* ydp = P.yd + (int64_t)p * T * F.ws.max_d_in + orow;
-      for (int cb = 0; cb < NB; cb += 16) {
+      for (int cb = 16 * wg; cb < NB; cb += 32) {
         uint32_t r[16];
         tmem_ld16(ta + cb, r);
         tmem_ld_wait();
@@ -1759,16 +1787,16 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
       if (!whole) {
         // hand the partial over; the last contributor of the unit finishes it
         __threadfence();
-        named_bar(1, 128);
+        named_bar(1, 256);
         const int c0 = bt_cta_of(F, S.ustart), c1 = bt_cta_of(F, S.ustart + S.K - 1);
         if (et == 0) {
           const int old = atomicAdd(cnt + S.u, 1);
           tail->last_flag = old == c1 - c0;
           __threadfence();
         }
-        named_bar(1, 128);
+        named_bar(1, 256);
         if (tail->last_flag) {
-          for (int cb = 0; cb < NB; cb += 16) {
+          for (int cb = 16 * wg; cb < NB; cb += 32) {
             float yv[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) yv[j] = 0.f;
