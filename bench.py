@@ -488,6 +488,77 @@ def run_prefill(args):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# Stress sweep (7B shapes, 100 tenants, Zipf(1.1)): tokens/s against T for three budgets
+# ------------------------------------------------------------------------------------------------
+SWEEP_METRIC = "tokens/s and % of HBM roofline, 100-tenant Zipf(1.1) 7B decode sweep"
+
+
+def run_sweep(args):
+    import numpy as np
+    import torch
+
+    import tenant_mixed_precision_b200 as dc
+    from tenant_mixed_precision_b200 import plans, synth
+    from tenant_mixed_precision_b200.stack import DeltaStack
+    from tenant_mixed_precision_b200.synth_stack import populate
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    layers = args.layers or 32
+    n_ten = args.tenants or 100
+    Ts = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+    budgets = [("1/16", 1 / 16, plans.MIXED_1_16), ("1/32", 1 / 32, plans.MIXED_1_32),
+               ("all-3-bit", 1 / 16, plans.ALL_3BIT)]
+    peak, peak_kind = _peaks()
+    for name, ratio, widths in budgets:
+        def plan_fn(l, p, d_out, d_in, t, ratio=ratio, widths=widths):
+            return plans.budget_plan(d_out, d_in, ratio, widths)
+
+        stack = DeltaStack(4096, 11008, layers, n_ten, max(Ts), plan_fn, out_dtype=torch.bfloat16)
+        populate(stack, 20245)
+        stream = torch.cuda.Stream()
+        for T in Ts:
+            ids = synth.zipf_tenants(np.random.default_rng(5000 + T), T, n_ten)
+            ids_dev = torch.from_numpy(ids).cuda()
+            with torch.cuda.stream(stream):
+                stack.forward(ids_dev, T)
+            stream.synchronize()
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph, stream=stream):
+                stack.forward(ids_dev, T)
+            for _ in range(args.warmup):
+                graph.replay()
+            torch.cuda.synchronize()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                e0.record(stream)
+                for _ in range(args.steps):
+                    graph.replay()
+                e1.record(stream)
+            e1.synchronize()
+            ms = e0.elapsed_time(e1) / args.steps
+            status = dc.dc_read_device_status(stack.ws, stream)
+            ab = stack.algorithmic_bytes(ids)
+            gbs = ab["total"] / (ms * 1e-3) / 1e9
+            print(json.dumps({
+                "metric": SWEEP_METRIC, "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+                "scaling": "weak", "vs_baseline": None, "dtype": "u8xs8->s32 delta, bf16xbf16->f32 backbone",
+                "data": "synthetic",
+                "config": {"workload": f"llama2-7b linear stack, {n_ten} resident tenants, Zipf(1.1), budget {name}",
+                           "layers": layers, "T": T, "budget": name, "distinct_tenants": ab["distinct_tenants"],
+                           "cuda_graph": True},
+                "step_hbm": {"algorithmic_bytes": ab["total"], "achieved_gbs": gbs, "peak_gbs": peak,
+                             "frac": gbs / peak, "peak_source": peak_kind},
+                "device_status": status}), flush=True)
+            del graph
+        del stack
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -498,8 +569,9 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=0, help="smaller stack for profiling captures (default: 32)")
     ap.add_argument("--tenants", type=int, default=0, help="fewer resident tenants (default: 50)")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill"],
-                    help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill pass")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep"],
+                    help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill "
+                         "pass; sweep: 100 Zipf tenants, T = 1..256, three budgets (one line per point)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -507,6 +579,8 @@ def main():
         return run_reference(args)
     if args.workload == "prefill":
         return run_prefill(args)
+    if args.workload == "sweep":
+        return run_sweep(args)
     return run_gpu(args)
 
 
