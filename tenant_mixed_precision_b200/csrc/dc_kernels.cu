@@ -984,6 +984,67 @@ __device__ __forceinline__ void ud_mma(const uint8_t* blk, int bits, int nq, int
   }
 }
 
+// One stage of the delta-output consumers for a pass of NTOK tokens: for every block of the batch,
+// the limb matrix of scale * t (one rank per thread), a barrier, then the MMAs of this warp's tile;
+// 8-bit blocks take the scalar path.
+template <int NTOK>
+__device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, uint8_t* bsm, const uint8_t* bconst,
+                                         uint32_t& nmma, int (&C)[2][4][4], float (&zc)[DC_V_TOKS], float (&s8)[2],
+                                         int tid, int warp, int lane) {
+      const float* tw = reinterpret_cast<const float*>(stage + d.code_bytes);
+      const int tfl = d.tfl;
+      float pe[DC_V_TOKS];
+#pragma unroll
+      for (int q = 0; q < DC_V_TOKS; ++q) pe[q] = d.pe[q];
+      int off = 0, ro = d.t_shift;
+      for (int i = 0; i < d.nsub; ++i) {
+        const int p0 = d.sub[i][0], p1 = d.sub[i][1];
+        const int bits = p0 & 15, nq = (p0 >> 4) & 15, ns = (p0 >> 8) & 255, last = p0 >> 16;
+        const int nr = p1 & 0xffff, tile_bytes = p1 >> 16;
+        const int code_bytes = bits == 8 ? (int)dc_align((int64_t)128 * nr, 16) : 8 * tile_bytes;
+        const uint8_t* blk = stage + off;
+        const uint8_t* meta = blk + code_bytes;
+        if (bits != 8) {
+          // ---- limbs of scale * t * 2^e for rank tid of the block, every pass token
+          uint8_t* bb = bsm + (nmma & 1) * U_BBUF;
+          if (tid < nr) {
+            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * tid);
+            const float sc = __low2float(mz), zs = sc * __high2float(mz);
+#pragma unroll
+            for (int q = 0; q < NTOK; ++q) {
+              {
+                const float tq = tw[q * tfl + ro + tid];
+                const uint32_t v = __float_as_uint(fmaf(sc, tq * pe[q], U_MAGIC));
+                uint8_t* col = bb + (6 * (q >> 1) + (q & 1)) * U_BROW + tid;
+                col[0] = (uint8_t)v;
+                col[2 * U_BROW] = (uint8_t)(v >> 8);
+                col[4 * U_BROW] = (uint8_t)(v >> 16);
+                zc[q] = fmaf(zs, tq, zc[q]);
+              }
+            }
+          }
+          named_bar(1, 32 * U_CONSUMERS);
+          ud_mma<(NTOK + 1) / 2>(blk, bits, nq, ns, last, tile_bytes, bb, bconst, C, warp, lane);
+          ++nmma;
+        } else {
+          // ---- 8-bit band: scalar fp32, lane = (row lane & 15, tokens 2 (lane >> 4) + {0, 1})
+          const int row = lane & 15, th = lane >> 4;
+          const uint8_t* cr = blk + (16 * warp + row) * nr;
+          for (int k = 0; k < nr; ++k) {
+            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
+            const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const int q = 2 * th + h;
+              if (q < NTOK) s8[h] = fmaf(f, tw[q * tfl + ro + k], s8[h]);
+            }
+          }
+        }
+        off += code_bytes + (int)dc_align((int64_t)4 * nr, 16);
+        ro += nr;
+      }
+    }
+
 __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __grid_constant__ DcFwd F, uint8_t* ws) {
   extern __shared__ __align__(128) uint8_t usm[];
   uint8_t* bsm = usm + U_STAGES * U_STAGE_BYTES;  // two limb matrices, then the constant rows
@@ -1177,60 +1238,11 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       s8[0] = s8[1] = 0.f;
     }
     if (!d.error) {
-      const float* tw = reinterpret_cast<const float*>(stage + d.code_bytes);
-      const int tfl = d.tfl;
-      float pe[DC_V_TOKS];
-#pragma unroll
-      for (int q = 0; q < DC_V_TOKS; ++q) pe[q] = d.pe[q];
-      int off = 0, ro = d.t_shift;
-      for (int i = 0; i < d.nsub; ++i) {
-        const int p0 = d.sub[i][0], p1 = d.sub[i][1];
-        const int bits = p0 & 15, nq = (p0 >> 4) & 15, ns = (p0 >> 8) & 255, last = p0 >> 16;
-        const int nr = p1 & 0xffff, tile_bytes = p1 >> 16;
-        const int code_bytes = bits == 8 ? (int)dc_align((int64_t)128 * nr, 16) : 8 * tile_bytes;
-        const uint8_t* blk = stage + off;
-        const uint8_t* meta = blk + code_bytes;
-        if (bits != 8) {
-          // ---- limbs of scale * t * 2^e for rank tid of the block, every pass token
-          uint8_t* bb = bsm + (nmma & 1) * U_BBUF;
-          if (tid < nr) {
-            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * tid);
-            const float sc = __low2float(mz), zs = sc * __high2float(mz);
-#pragma unroll
-            for (int q = 0; q < DC_V_TOKS; ++q) {
-              if (q < ntok) {
-                const float tq = tw[q * tfl + ro + tid];
-                const uint32_t v = __float_as_uint(fmaf(sc, tq * pe[q], U_MAGIC));
-                uint8_t* col = bb + (6 * (q >> 1) + (q & 1)) * U_BROW + tid;
-                col[0] = (uint8_t)v;
-                col[2 * U_BROW] = (uint8_t)(v >> 8);
-                col[4 * U_BROW] = (uint8_t)(v >> 16);
-                zc[q] = fmaf(zs, tq, zc[q]);
-              }
-            }
-          }
-          named_bar(1, 32 * U_CONSUMERS);
-          if (ntok > 2)
-            ud_mma<2>(blk, bits, nq, ns, last, tile_bytes, bb, bconst, C, warp, lane);
-          else
-            ud_mma<1>(blk, bits, nq, ns, last, tile_bytes, bb, bconst, C, warp, lane);
-          ++nmma;
-        } else {
-          // ---- 8-bit band: scalar fp32, lane = (row lane & 15, tokens 2 (lane >> 4) + {0, 1})
-          const int row = lane & 15, th = lane >> 4;
-          const uint8_t* cr = blk + (16 * warp + row) * nr;
-          for (int k = 0; k < nr; ++k) {
-            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
-            const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int q = 2 * th + h;
-              if (q < ntok) s8[h] = fmaf(f, tw[q * tfl + ro + k], s8[h]);
-            }
-          }
-        }
-        off += code_bytes + (int)dc_align((int64_t)4 * nr, 16);
-        ro += nr;
+      switch (ntok) {
+        case 1: ud_stage<1>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
+        case 2: ud_stage<2>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
+        case 3: ud_stage<3>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
+        default: ud_stage<4>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
       }
     }
     const bool ulast = d.ulast;
