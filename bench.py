@@ -193,6 +193,25 @@ def run_reference(args):
 
 
 # ------------------------------------------------------------------------------------------------
+# Replica aggregation (one process per GPU, no data-path collective)
+# ------------------------------------------------------------------------------------------------
+def replica_throughput(ms_local: float, tokens_per_rank: int, dist=None, device: str = "cuda"):
+    """Whole-job throughput of N independent replicas: the step time is the max over ranks of the
+    device-timed region, and the job processed every rank's tokens in that time.
+    Returns (ms_max, tokens_per_s)."""
+    import torch
+
+    world = 1
+    ms_max = float(ms_local)
+    if dist is not None and dist.is_initialized():
+        world = dist.get_world_size()
+        t = torch.tensor([float(ms_local)], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms_max = float(t.item())
+    return ms_max, tokens_per_rank * world / (ms_max / 1e3)
+
+
+# ------------------------------------------------------------------------------------------------
 # GPU arm
 # ------------------------------------------------------------------------------------------------
 def run_gpu(args):
@@ -262,12 +281,7 @@ def run_gpu(args):
     if dist:
         dist.barrier()
     ms = ev0.elapsed_time(ev1)
-    ms_t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-    if dist:
-        dist.all_reduce(ms_t, op=dist.ReduceOp.MAX)
-    ms_max = float(ms_t.item())
-    tokens = T * args.steps * world
-    value = tokens / (ms_max / 1e3)
+    ms_max, value = replica_throughput(ms, T * args.steps, dist)
     ms_per_step = ms_max / args.steps
     status = dc.dc_read_device_status(stack.ws, stream)
 
@@ -293,10 +307,7 @@ def run_gpu(args):
         e1.record(stream)
     e1.synchronize()
     e2e_ms = e0.elapsed_time(e1)
-    e_t = torch.tensor([e2e_ms], dtype=torch.float64, device="cuda")
-    if dist:
-        dist.all_reduce(e_t, op=dist.ReduceOp.MAX)
-    e2e_value = tokens / (float(e_t.item()) / 1e3)
+    _, e2e_value = replica_throughput(e2e_ms, T * args.steps, dist)
 
     # ---- per-kernel durations (eager calls with CUDA events around every launch on its stream)
     n_prof = max(3, min(args.steps, 10))
