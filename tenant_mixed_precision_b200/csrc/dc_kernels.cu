@@ -537,14 +537,13 @@ __device__ __forceinline__ void v_block(int rows, int ngrp_rt, const uint8_t* A,
   uint4 wm0a = make_uint4(0, 0, 0, 0), wm0b = wm0a, wm1a = wm0a, wm1b = wm0a;
   if (BITS == 2 && FULL) {
     if (ok0) {
-      const uint8_t* pp = A + lane * 32;
-      wm0a = *reinterpret_cast<const uint4*>(pp);
-      wm0b = *reinterpret_cast<const uint4*>(pp + 16);
+      wm0a = *reinterpret_cast<const uint4*>(A + dc_v_mask_off(4 * nh0, lane, 0));
+      wm0b = *reinterpret_cast<const uint4*>(A + dc_v_mask_off(4 * nh0, lane, 1));
     }
     if (ok1) {
-      const uint8_t* pp = A + dc_v_half_off(2, rows, 4, 1) + lane * 32;
-      wm1a = *reinterpret_cast<const uint4*>(pp);
-      wm1b = *reinterpret_cast<const uint4*>(pp + 16);
+      const uint8_t* h1 = A + dc_v_half_off(2, rows, 4, 1);
+      wm1a = *reinterpret_cast<const uint4*>(h1 + dc_v_mask_off(4 * nh1, lane, 0));
+      wm1b = *reinterpret_cast<const uint4*>(h1 + dc_v_mask_off(4 * nh1, lane, 1));
     }
   }
 #pragma unroll
@@ -869,8 +868,8 @@ struct USmemTail {
   int bfirst[U_MAXBLK + 1];      // producer: batches of the current pass (first block of each)
   int nbatch;
   float zpart[U_CONSUMERS][DC_V_TOKS];     // per-warp zero-point sums of a unit
-  float s8[U_CONSUMERS][16][DC_V_TOKS];    // 8-bit band partials of a unit
-  int cbuf[U_CONSUMERS][2][16][8];         // combined integer MMA results of a unit: [warp][pair][row][col]
+  float s8[128][DC_V_TOKS + 1];            // 8-bit band partials of a unit: [row][token] (padded: no bank conflicts)
+  int cbuf[2][128][9];                     // combined integer MMA results of a unit: [pair][row][col] (padded)
   float uie[DC_V_TOKS];                    // 2^-e of the unit's tokens
 };
 
@@ -1280,9 +1279,9 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       if (warp == 0) tail->uie[lane] = e;
     }
     {
-      const int row = lane & 15, th = lane >> 4;
-      tail->s8[warp][row][2 * th] = s8[0];
-      tail->s8[warp][row][2 * th + 1] = s8[1];
+      const int row = 16 * warp + (lane & 15), th = lane >> 4;
+      tail->s8[row][2 * th] = s8[0];
+      tail->s8[row][2 * th + 1] = s8[1];
     }
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
@@ -1291,20 +1290,24 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
 #pragma unroll
       for (int r = 0; r < 4; ++r)
         Ct[r] = C[pr][0][r] + (C[pr][1][r] >> 2) + (C[pr][2][r] >> 4) + (C[pr][3][r] >> 6);
-      *reinterpret_cast<int2*>(&tail->cbuf[warp][pr][g][2 * t]) = make_int2(Ct[0], Ct[1]);
-      *reinterpret_cast<int2*>(&tail->cbuf[warp][pr][g + 8][2 * t]) = make_int2(Ct[2], Ct[3]);
+      int* c0 = tail->cbuf[pr][16 * warp + g];
+      int* c1 = tail->cbuf[pr][16 * warp + g + 8];
+      c0[2 * t] = Ct[0];
+      c0[2 * t + 1] = Ct[1];
+      c1[2 * t] = Ct[2];
+      c1[2 * t + 1] = Ct[3];
     }
     named_bar(2, 32 * U_CONSUMERS);
     // cbuf columns: 2 limb + token-in-pair for limbs 0..2, column 6 = the codes' row sum
     for (int idx = tid; idx < 128 * ntok; idx += 32 * U_CONSUMERS) {
       const int row = idx & 127, q = idx >> 7;
-      const int w = row >> 4, rr = row & 15, pr = q >> 1, tk = q & 1;
-      const int* cr = tail->cbuf[w][pr][rr];
+      const int pr = q >> 1, tk = q & 1;
+      const int* cr = tail->cbuf[pr][row];
       const float v = (float)(cr[4 + tk] - 64 * cr[6]) * 65536.f + (float)cr[2 + tk] * 256.f + (float)cr[tk];
       float zs = 0.f;
 #pragma unroll
       for (int ww = 0; ww < U_CONSUMERS; ++ww) zs += tail->zpart[ww][q];
-      const float y = fmaf(v, tail->uie[q], -zs) + tail->s8[w][rr][q];
+      const float y = fmaf(v, tail->uie[q], -zs) + tail->s8[row][q];
       P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + row] = y;
     }
     ++unit;
@@ -2324,8 +2327,8 @@ __device__ __forceinline__ void vp_lane_codes(const uint8_t* A, int bits, int ro
   const uint8_t* hb = A + dc_v_half_off(bits, rows, ngrp, h);
   const int p0 = dc_v_plane0_bytes(bits, ngrp);
   if (bits == 2 && ngrp == 4) {
-    const uint4 w0 = *reinterpret_cast<const uint4*>(hb + ln * 32);
-    const uint4 w1 = *reinterpret_cast<const uint4*>(hb + ln * 32 + 16);
+    const uint4 w0 = *reinterpret_cast<const uint4*>(hb + dc_v_mask_off(4 * nh, ln, 0));
+    const uint4 w1 = *reinterpret_cast<const uint4*>(hb + dc_v_mask_off(4 * nh, ln, 1));
     const uint32_t w[8] = {w0.x, w0.y, w0.z, w0.w, w1.x, w1.y, w1.z, w1.w};
 #pragma unroll
     for (int s = 0; s < 4; ++s)
@@ -2703,7 +2706,7 @@ __global__ void k_unpack_v(const uint8_t* blob, DcLayout L, int bi, uint8_t* out
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t r;
         if (B.bits == 2 && ngrp == 4) {
-          const uint4 q = ldg128(blk + lane * 32 + 16 * (s >> 1));
+          const uint4 q = ldg128(blk + dc_v_mask_off(4 * nh, lane, s >> 1));
           r = v_reg_mask2(wsel(q, 2 * (s & 1) + hh), grp) >> (2 * grp);
         } else if (B.bits == 8) {
           r = ldg32(blk + lane * p0 + 32 * grp + 4 * (2 * s + hh));

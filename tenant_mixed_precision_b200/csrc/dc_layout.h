@@ -25,7 +25,8 @@
 // valid rows (4 per row) present:
 //   2-bit, full block : 8 words per lane; word 2s+hh, bits [8b+2p, 8b+2p+2) hold the code of
 //                       group p (p = 0..3) -- a register is extracted with one AND and carries
-//                       the weight 4^p, removed in the fp32 epilogue ("mask" layout);
+//                       the weight 4^p, removed in the fp32 epilogue ("mask" layout); words 0-3
+//                       of every lane come first, then words 4-7 of every lane (dc_v_mask_off);
 //   2-bit, tail block : 2 words per group; word s/2, bits [8b+2q, 8b+2q+2), q = 2(s%2)+hh
 //                       ("shift" layout);
 //   3-bit             : the 2-bit plane in the shift layout plus a 1-bit plane of one word per
@@ -134,6 +135,10 @@ DC_HD int64_t dc_v_half_off(int32_t bits, int32_t rows, int32_t ngrp, int32_t h)
   int32_t n0 = rows < 8 ? rows : 8;
   return h == 0 ? 0 : (int64_t)4 * n0 * dc_v_lane_group_bytes(bits) * ngrp;
 }
+// 2-bit full blocks (mask layout): byte offset, inside a half of nl lanes, of lane `lane`'s words
+// 4 hi .. 4 hi + 3 -- the first 16 bytes of every lane, then the second 16 bytes of every lane, so
+// that consecutive lanes' 16-byte loads fall on different shared-memory banks.
+DC_HD int32_t dc_v_mask_off(int32_t nl, int32_t lane, int32_t hi) { return 16 * nl * hi + 16 * lane; }
 // bytes of one U shift-layout step holding nl lanes (both planes, each padded to 16)
 DC_HD int64_t dc_u_step_bytes(int32_t bits, int32_t nl) {
   return dc_align((int64_t)nl * 4, 16) + (bits == 3 ? dc_align((int64_t)nl * 2, 16) : 0);

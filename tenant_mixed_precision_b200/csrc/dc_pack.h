@@ -64,7 +64,13 @@ DC_HD uint32_t dc_pack_v_word(const DcLayout& L, const DcBand& B, int64_t off, c
   const int32_t nl = 4 * nh;
   const int32_t p0 = dc_v_plane0_bytes(bits, ngrp);
   int32_t plane, lane, wi;
-  if (in_half < (int64_t)nl * p0) {
+  if (bits == 2 && ngrp == 4) {  // mask layout: words 0-3 of every lane, then words 4-7
+    plane = 0;
+    const int32_t hi = (int32_t)(in_half / (16 * nl));
+    const int32_t within = (int32_t)(in_half % (16 * nl));
+    lane = within / 16;
+    wi = 4 * hi + (within % 16) / 4;
+  } else if (in_half < (int64_t)nl * p0) {
     plane = 0;
     lane = (int32_t)(in_half / p0);
     wi = (int32_t)((in_half % p0) / 4);
