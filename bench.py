@@ -88,10 +88,20 @@ class ClockSampler:
                 "reasons": reasons, "samples": len(rows)}
 
 
-def _kernel_source_sha() -> str:
-    h = hashlib.sha256()
-    with open(os.path.join(ROOT, "tenant_mixed_precision_b200", "csrc", "dc_kernels.cu"), "rb") as f:
-        h.update(f.read())
+def _kernel_source_sha(kernel: str) -> str:
+    """Hash of what decides `kernel`'s DRAM traffic: its section of dc_kernels.cu (from its
+    "// <name>:" header to the next section) and the layout headers."""
+    csrc = os.path.join(ROOT, "tenant_mixed_precision_b200", "csrc")
+    with open(os.path.join(csrc, "dc_kernels.cu")) as f:
+        text = f.read()
+    sep = "// " + "-" * 93 + "\n"
+    start = text.find("\n// " + kernel + ":")
+    end = text.find(sep + "// ", start + 1) if start >= 0 else -1
+    section = text[start:end] if start >= 0 else text
+    h = hashlib.sha256(section.encode())
+    for name in ("dc_layout.h", "dc_internal.h", "dc_pack.h"):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(f.read())
     return h.hexdigest()[:16]
 
 
@@ -100,7 +110,7 @@ def _ncu_traffic(kernel: str):
     path = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(path):
         return None
-    sha = _kernel_source_sha()
+    sha = _kernel_source_sha(kernel)
     with open(path) as f:
         for line in f:
             kv = dict(p.split("=", 1) for p in line.split() if "=" in p)
@@ -332,7 +342,7 @@ def run_gpu(args):
     }
     peak, peak_kind = _peaks()
     achieved = per_launch_bytes.get(dom, 0.0) / (dom_avg_ms * 1e-3) / 1e9
-    kname = {"backbone_output": "k_base", "delta_output": "k_udelta", "rank_reduction": "k_vstage", "prep": "k_prep",
+    kname = {"backbone_output": "k_base_tc", "delta_output": "k_udelta", "rank_reduction": "k_vstage", "prep": "k_prep",
              "routing": "k_segments"}[dom]
     step_gbs = ab["total"] / (ms_per_step * 1e-3) / 1e9
 
