@@ -1,0 +1,129 @@
+"""GPU parity on the remaining workload shapes and edge cases.
+
+* one Llama-2-7B-shaped layer in bf16 (q/k/v/o 4096x4096, gate/up 11008x4096, down 4096x11008),
+  8 tenants at the 1/16 budget, a decode batch of 8 tokens with one token per tenant: every
+  output of three projections (q, gate, down: the three shapes) against the oracle;
+* the 13B-shaped prefill layer (2048 tokens in segments of 32-256, 16 tenants): sampled outputs
+  against the oracle, on the tensor-core prefill path;
+* edge cases: a batch of backbone-only tokens, tenants without a delta, one token.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import tenant_mixed_precision_b200 as dc
+from tenant_mixed_precision_b200 import plans, synth
+from tenant_mixed_precision_b200.synth_stack import host_activations, host_factors
+
+from dc_testlib import TenantDeltas, assert_close, gaussian_factors, oracle_y
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+if not torch.cuda.is_available():  # pragma: no cover
+    pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def _stack(hidden, ffn, n_ten, T, seed, s0):
+    from tenant_mixed_precision_b200.stack import DeltaStack
+    from tenant_mixed_precision_b200.synth_stack import populate
+
+    def plan_fn(l, p, d_out, d_in, t):
+        return plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+
+    st = DeltaStack(hidden, ffn, 1, n_ten, T, plan_fn, out_dtype=torch.float32)
+    populate(st, seed, s0=s0)
+    return st
+
+
+def _run(st, ids, flags):
+    ids_d = torch.from_numpy(ids).cuda()
+    st.forward(ids_d, len(ids), flags=flags)
+    torch.cuda.synchronize()
+    assert dc.dc_read_device_status(st.ws) == 0
+    return [y.cpu().numpy().astype(np.float64) for y in st.y[0]]
+
+
+def _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, flags):
+    plan = plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+    r = sum(x for _, x in plan)
+    _, xv = host_activations(seed, 0, synth.PROJ_INPUT[proj], T, d_in)
+    arts = {}
+    for k in toks:
+        t = int(ids[k])
+        if t >= 0 and t not in arts:
+            f = host_factors(seed, 0, proj, t, d_out, d_in, r, s0=s0)
+            arts[t] = oracle.compress_factors(f.U, f.S, f.Vt, plan)
+    x = xv[toks].astype(np.float64)
+    if flags & dc.DC_BASE:
+        _, wv = synth.stream_base_weight(seed, 0, proj, d_out, d_in, rows=rows)
+        return oracle.delta_linear(wv.astype(np.float64), arts, x, ids[toks], rows=rows)
+    return oracle.delta_only(arts, x, ids[toks], rows=rows)
+
+
+def test_one_7b_layer_8_tenants_one_token_each():
+    seed, s0, T = 20242, 0.02 * np.sqrt(4096.0), 8
+    st = _stack(4096, 11008, 8, T, seed, s0)
+    ids = np.arange(8, dtype=np.int32)
+    full = _run(st, ids, dc.DC_BASE | dc.DC_DELTA)
+    delta = _run(st, ids, dc.DC_DELTA)
+    toks = np.arange(T)
+    for proj in (0, 4, 6):  # q (4096x4096), gate (11008x4096), down (4096x11008)
+        d_out, d_in = st.shapes[proj]
+        rows = np.arange(d_out)
+        ref = _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, dc.DC_BASE | dc.DC_DELTA)
+        assert_close(full[proj], ref, f"7B layer proj {proj}")
+        ref_d = _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, dc.DC_DELTA)
+        assert_close(delta[proj], ref_d, f"7B layer proj {proj} delta")
+    for y in full + delta:
+        assert np.isfinite(y).all()
+
+
+def test_13b_prefill_layer_sampled_against_oracle():
+    seed, s0, T = 20244, 0.02 * np.sqrt(5120.0), 2048
+    st = _stack(5120, 13824, 16, T, seed, s0)
+    ids = synth.prefill_segments(np.random.default_rng(4), T, 16)
+    full = _run(st, ids, dc.DC_BASE | dc.DC_DELTA)
+    delta = _run(st, ids, dc.DC_DELTA)
+    rng = np.random.default_rng(7)
+    toks = np.sort(rng.choice(T, size=4, replace=False))
+    for proj in (0, 6):  # q (5120x5120) and down (5120x13824)
+        d_out, d_in = st.shapes[proj]
+        rows = np.concatenate([np.arange(128) + 128 * int(rng.integers(0, d_out // 128)) for _ in range(2)])
+        ref = _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, dc.DC_BASE | dc.DC_DELTA)
+        assert_close(full[proj][toks][:, rows], ref, f"13B prefill proj {proj}")
+        ref_d = _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, dc.DC_DELTA)
+        assert_close(delta[proj][toks][:, rows], ref_d, f"13B prefill proj {proj} delta")
+
+
+@pytest.mark.parametrize("case", ["all_backbone", "tenants_without_delta", "one_token"])
+def test_edge_cases(case):
+    rng = np.random.default_rng(11)
+    d_out, d_in = 640, 384
+    plan = [(8, 2), (3, 20), (2, 90)]
+    if case == "tenants_without_delta":
+        factors = [gaussian_factors(rng, d_out, d_in, 112), None, gaussian_factors(rng, d_out, d_in, 112), None]
+        ids = np.array([1, 0, 3, 2, 1, -1, 0, 3, 3, 1], dtype=np.int32)
+    else:
+        factors = [gaussian_factors(rng, d_out, d_in, 112) for _ in range(3)]
+        ids = np.full(9, -1, dtype=np.int32) if case == "all_backbone" else np.array([2], dtype=np.int32)
+    plans_ = [plan if f is not None else None for f in factors]
+    td = TenantDeltas(torch, d_out, d_in, factors, plans_)
+    T = len(ids)
+    wb, wv = synth.bf16_round((0.02 * rng.standard_normal((d_out, d_in))).astype(np.float32))
+    xb, xv = synth.bf16_round(rng.standard_normal((T, d_in)).astype(np.float32))
+    W = torch.from_numpy(wb.view(np.int16)).cuda().view(torch.bfloat16)
+    x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
+    lin = td.linear(W)
+    ws = torch.zeros(dc.dc_workspace_size(T, max(td.max_rank, 1), max(d_in, d_out), 1, len(factors)), dtype=torch.uint8,
+                     device="cuda")
+    for flags in (dc.DC_DELTA, dc.DC_BASE | dc.DC_DELTA):
+        y = torch.full((T, d_out), float("nan"), dtype=torch.float32, device="cuda")
+        dc.dc_delta_linear_segmented(lin, x, y, torch.from_numpy(ids).cuda(), T, flags, ws)
+        torch.cuda.synchronize()
+        assert dc.dc_read_device_status(ws) == 0
+        got = y.cpu().numpy().astype(np.float64)
+        want = oracle_y(wv.astype(np.float64), td, xv.astype(np.float64), ids, flags)
+        if not (flags & dc.DC_BASE) and not np.any(want):
+            assert np.array_equal(got, want), case  # no delta anywhere: exactly zero
+        else:
+            assert_close(got, want, f"{case} flags={flags}")
