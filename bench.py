@@ -370,7 +370,7 @@ def run_gpu(args):
         "config": {"workload": W["name"], "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
                    "tenants_resident": W["n_tenants"], "T": T, "distinct_tenants": ab["distinct_tenants"],
                    "budget": "1/16: 8-bit x2, 3-bit x32, 2-bit remainder", "output_dtype": "bf16",
-                   "l2": "inputs larger than L2 (~46 GB read per step); no flush", "cuda_graph": True,
+                   "l2": f"inputs larger than L2 (~{ab['total'] / 1e9:.1f} GB read per step); no flush", "cuda_graph": True,
                    "parallelism": f"replicas x{world}"},
         "step_hbm": {"algorithmic_bytes": ab["total"], "achieved_gbs": step_gbs, "peak_gbs": peak,
                      "frac": step_gbs / peak, "peak_source": peak_kind},
@@ -381,7 +381,8 @@ def run_gpu(args):
         "kernel_ms_per_step": {k: v / n_prof for k, v in tot.items()},
         "kernel_gbs": {k: per_launch_bytes[k] / (statistics.mean(per[k]) * 1e-3) / 1e9 for k in per_launch_bytes if k in per},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                "what": "per step: tenant ids and layer-0 activations in from pinned host memory, layer-31 outputs out"},
+                "what": "per step: tenant ids and layer-0 activations in from pinned host memory, "
+                        f"layer-{W['layers'] - 1} outputs out"},
         "gpu_launches": (1 + 4 * W["layers"]) * args.steps,
         "cpu_baseline": cpu,
         "clocks": ck,
