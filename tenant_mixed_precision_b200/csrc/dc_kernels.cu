@@ -834,9 +834,8 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
 #define U_MAXSUB 8           // blocks per batch
 #define U_MAXBLK 64          // blocks per (linear, tenant) U run of one group
 #define U_CHUNK 4            // 128-row output groups per chunk of work
-#define U_BROW 288           // row stride of the staged limb matrix (rows g and g+4 on different banks)
-#define U_BBUF (12 * U_BROW) // one limb matrix: 2 token pairs x (3 limbs x 2 tokens)
-#define U_BCONST (2 * U_BROW) // B columns 6 and 7 of every step: a row of ones and a row of zeros
+#define U_LROW 544           // row stride of a limb matrix = rank slots per stage (rows 8 banks apart)
+#define U_LBUF (16 * U_LROW) // one limb matrix: rows 6 pr + 2 limb + token-in-pair, then constant rows
 #define U_CONSUMERS 8
 #define U_THREADS (32 * (U_CONSUMERS + 1))
 #define U_MAGIC 12582912.0f  // 1.5 * 2^23
@@ -850,7 +849,9 @@ struct UDesc {
   int t_shift;           // position of the batch's first rank inside the t window
   int ufirst, ulast;     // the batch opens / closes its (group, pass) unit
   int error;
-  int sub[U_MAXSUB][2];  // per block: bits | nq << 4 | ns << 8 | last << 16, and nr | tile_bytes << 16
+  alignas(16) int sub[U_MAXSUB][4];  // per block: bits | nq << 4 | ns << 8 | last << 16; nr | tile_bytes << 16;
+                         // stage offset of the codes | limb slot << 16; stage offset of the meta |
+                         // offset of the first rank in the t windows << 16
   float pe[DC_V_TOKS];   // 2^e per pass token
   float ie[DC_V_TOKS];   // 2^-e
 };
@@ -863,14 +864,14 @@ struct USmemTail {
   UDesc desc[U_STAGES];
   uint64_t full[U_STAGES];
   uint64_t empty[U_STAGES];
-  DcURec rec;                    // producer: record of the current chunk
+  alignas(16) DcURec rec;        // producer: record of the current chunk
   UBlkE tbl[U_MAXBLK];           // producer: blocks of the current chunk's runs
-  int bfirst[U_MAXBLK + 1];      // producer: batches of the current pass (first block of each)
+  alignas(16) int bsub[U_MAXBLK][4];  // producer: per block of the pass, its UDesc.sub entry
+  int4 bat[U_MAXBLK];                 // producer: per batch, first block | blocks << 8 | t shift << 16,
+                                      // code bytes, t window floats, first t column
   int nbatch;
-  float zpart[U_CONSUMERS][DC_V_TOKS];     // per-warp zero-point sums of a unit
-  float s8[128][DC_V_TOKS + 1];            // 8-bit band partials of a unit: [row][token] (padded: no bank conflicts)
-  int cbuf[2][128][9];                     // combined integer MMA results of a unit: [pair][row][col] (padded)
-  float uie[DC_V_TOKS];                    // 2^-e of the unit's tokens
+  alignas(16) float zpart[2][DC_V_TOKS][U_CONSUMERS];  // per-warp zero-point sums of a unit (two units in flight)
+  float s8[128][DC_V_TOKS + 1];            // 8-bit band sums of a unit: [row][token] (padded: no bank conflicts)
 };
 
 // D += A(u8, 16x32, row) * B(u8, 32x8, col), int32 accumulate.
@@ -910,17 +911,71 @@ __device__ __forceinline__ int ud_exponent(float umax, int tmax_bits) {
   return max(-120, min(120, 21 - E));
 }
 
-// MMA over one block for this warp's 16-row tile.  C[pair][position][reg].
+// Limb-matrix row of B column g (0..7) for token pair pr: columns 0..5 are the limbs of the pair's
+// tokens (rows 6 pr + g), column 6 a row of ones (the codes' row sums), column 7 a row of zeros.
+// The constant rows are 14/15 for pair 0 and 12/13 for pair 1: with rows 8 banks apart, the rows
+// one 16-lane half of a warp reads lie on four different groups of 8 banks.
+__device__ __forceinline__ int ud_brow(int g, int pr) { return g < 6 ? 6 * pr + g : (pr ? 12 : 14) + (g - 6); }
+
+// Shift-layout steps of one 16-row tile, the first of them being MMA step k0 of the block.  Every
+// step but a partial last one stores all 32 lanes: lane l's 2-bit word at 4 l, its 3-bit high
+// plane at 128 + 2 l.  A partial last step stores nl = 8 ceil(last / 8) lanes, row g's words
+// at g * nl / 8 + t.
+template <int BITS, int NPAIR>
+__device__ __forceinline__ void ud_steps(const uint8_t* sb, int k0, int ns, int last, const uint8_t* brow,
+                                         int pstride, int (&C)[2][4][4], int lane) {
+  constexpr int SB = BITS == 3 ? 192 : 128;  // bytes of a full step (both planes)
+  const int g = lane >> 2, t = lane & 3;
+  const int nfull = last == 32 ? ns : ns - 1;
+#pragma unroll 2
+  for (int si = 0; si < nfull; ++si) {
+    const uint8_t* p = sb + si * SB;
+    const uint32_t wv = reinterpret_cast<const uint32_t*>(p)[lane];
+    uint32_t hv = 0;
+    if (BITS == 3) hv = reinterpret_cast<const uint16_t*>(p + 128)[lane];
+    uint32_t a[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a[j] = reg_shift2(wv, j);
+      if (BITS == 3) a[j] |= u_reg_hi3(hv, j);
+    }
+#pragma unroll
+    for (int pr = 0; pr < NPAIR; ++pr) {
+      const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * (k0 + si));
+      mma_u8u8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
+    }
+  }
+  if (nfull == ns) return;
+  const uint8_t* p = sb + nfull * SB;
+  const int nl = dc_u_step_lanes(last);
+  const int ntv = nl / 8;
+  uint32_t wv = 0, hv = 0;
+  if (t < ntv) {
+    wv = *reinterpret_cast<const uint32_t*>(p + 4 * (g * ntv + t));
+    if (BITS == 3) hv = *reinterpret_cast<const uint16_t*>(p + 4 * nl + 2 * (g * ntv + t));
+  }
+  uint32_t a[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    a[j] = reg_shift2(wv, j);
+    if (BITS == 3) a[j] |= u_reg_hi3(hv, j);
+  }
+#pragma unroll
+  for (int pr = 0; pr < NPAIR; ++pr) {
+    const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * (k0 + nfull));
+    mma_u8u8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
+  }
+}
+
+// MMA over one block for this warp's 16-row tile.  `lb` is the block's slot in the limb matrix.
+// C[pair][position][reg].
 template <int NPAIR>
 __device__ __forceinline__ void ud_mma(const uint8_t* blk, int bits, int nq, int ns, int last, int tile_bytes,
-                                       const uint8_t* bsm, const uint8_t* bconst, int (&C)[2][4][4], int warp,
-                                       int lane) {
+                                       const uint8_t* lb, int (&C)[2][4][4], int warp, int lane) {
   const int g = lane >> 2, t = lane & 3;
   const uint8_t* ub = blk + warp * tile_bytes;
-  // B column g: limb rows 0..5 of pair 0 (pair 1 six rows further), column 6 a row of ones (the
-  // codes' row sums), column 7 a row of zeros; both constant rows sit after the two limb matrices
-  const uint8_t* brow = (g < 6 ? bsm + g * U_BROW : bconst + (g - 6) * U_BROW) + 8 * t;
-  const int pstride = g < 6 ? 6 * U_BROW : 0;
+  const uint8_t* brow = lb + ud_brow(g, 0) * U_LROW + 8 * t;
+  const int pstride = (ud_brow(g, 1) - ud_brow(g, 0)) * U_LROW;
   if (nq == 2 && ns == 0) {  // full 2-bit block: two quads in straight-line code
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
@@ -956,99 +1011,84 @@ __device__ __forceinline__ void ud_mma(const uint8_t* blk, int bits, int nq, int
       }
     }
   }
-  const uint8_t* sb = ub + 512 * nq;
-#pragma unroll 1
-  for (int si = 0; si < ns; ++si) {
-    const int valid = (si == ns - 1) ? last : 32;
-    const int nl = dc_u_step_lanes(valid);
-    const int ntv = nl / 8;
-    uint32_t wv = 0, hv = 0;
-    if (t < ntv) {
-      wv = *reinterpret_cast<const uint32_t*>(sb + 4 * (g * ntv + t));
-      if (bits == 3) hv = *reinterpret_cast<const uint16_t*>(sb + dc_align((int64_t)nl * 4, 16) + 2 * (g * ntv + t));
-    }
-    uint32_t a[4];
+  if (ns == 0) return;
+  if (bits == 3)
+    ud_steps<3, NPAIR>(ub + 512 * nq, 4 * nq, ns, last, brow, pstride, C, lane);
+  else
+    ud_steps<2, NPAIR>(ub + 512 * nq, 4 * nq, ns, last, brow, pstride, C, lane);
+}
+
+// fields read with 16-byte vector loads
+static_assert(offsetof(USmemTail, zpart) % 16 == 0 && offsetof(USmemTail, rec) % 16 == 0 &&
+                  offsetof(USmemTail, bsub) % 16 == 0 && offsetof(USmemTail, bat) % 16 == 0 &&
+                  offsetof(UDesc, sub) % 16 == 0 && sizeof(UDesc) % 16 == 0 && (U_STAGES * U_STAGE_BYTES) % 16 == 0 &&
+                  U_LBUF % 16 == 0,
+              "delta-output shared-memory alignment");
+// two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
+static_assert(U_STAGES * U_STAGE_BYTES + 2 * U_LBUF + sizeof(USmemTail) + 1024 <= 233472 / U_CTAS_PER_SM,
+              "delta-output shared memory exceeds the per-CTA share");
+
+// One stage of the delta-output consumers for a pass of ntok <= NTOK tokens (limb columns of tokens
+// ntok .. NTOK - 1 keep stale bytes; their outputs are never formed).  Phase A: the limb matrix of
+// scale * t for every 2/3-bit block of the batch (one rank per thread, each block in its own slot).
+// One barrier.  Phase B: this warp's MMAs over every block; 8-bit blocks take a scalar fp32 path
+// whose lanes split rows (lane & 15) and ranks (lane >> 4).  `lb` is this stage's limb matrix.
+template <int NTOK>
+__device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, uint8_t* lb, int (&C)[2][4][4],
+                                         float (&zc)[DC_V_TOKS], float (&s8)[DC_V_TOKS], int ntok, int tid,
+                                         int warp, int lane) {
+  const float* tw = reinterpret_cast<const float*>(stage + d.code_bytes);
+  const int tfl = d.tfl, nsub = d.nsub;
+  float pe[NTOK];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      a[j] = reg_shift2(wv, j);
-      if (bits == 3) a[j] |= u_reg_hi3(hv, j);
-    }
-    const int step = 4 * nq + si;
+  for (int q = 0; q < NTOK; ++q) pe[q] = d.pe[q];
+  for (int i = 0; i < nsub; ++i) {
+    const int4 sd = *reinterpret_cast<const int4*>(d.sub[i]);
+    const int nr = sd.y & 0xffff;
+    if ((sd.x & 15) == 8 || tid >= nr) continue;
+    const int slot = sd.z >> 16, moff = sd.w & 0xffff, ro = sd.w >> 16;
+    const __half2 mz = *reinterpret_cast<const __half2*>(stage + moff + 4 * tid);
+    const float sc = __low2float(mz), zs = sc * __high2float(mz);
+    uint8_t* col = lb + slot + tid;
 #pragma unroll
-    for (int pr = 0; pr < NPAIR; ++pr) {
-      const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * step);
-      mma_u8u8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
+    for (int q = 0; q < NTOK; ++q) {
+      if (q >= ntok) break;
+      const float tq = tw[q * tfl + ro + tid];
+      const uint32_t v = __float_as_uint(fmaf(sc, tq * pe[q], U_MAGIC));
+      uint8_t* c = col + (6 * (q >> 1) + (q & 1)) * U_LROW;
+      c[0] = (uint8_t)v;
+      c[2 * U_LROW] = (uint8_t)(v >> 8);
+      c[4 * U_LROW] = (uint8_t)(v >> 16);
+      zc[q] = fmaf(zs, tq, zc[q]);
     }
-    sb += dc_u_step_bytes(bits, nl);
+  }
+  named_bar(1, 32 * U_CONSUMERS);
+  for (int i = 0; i < nsub; ++i) {
+    const int4 sd = *reinterpret_cast<const int4*>(d.sub[i]);
+    const int bits = sd.x & 15, nr = sd.y & 0xffff;
+    const uint8_t* blk = stage + (sd.z & 0xffff);
+    if (bits != 8) {
+      const int nq = (sd.x >> 4) & 15, ns = (sd.x >> 8) & 255, last = sd.x >> 16;
+      ud_mma<(NTOK + 1) / 2>(blk, bits, nq, ns, last, sd.y >> 16, lb + (sd.z >> 16), C, warp, lane);
+    } else {
+      const uint8_t* meta = stage + (sd.w & 0xffff);
+      const float* tr = tw + (sd.w >> 16);
+      const uint8_t* cr = blk + (16 * warp + (lane & 15)) * nr;
+      for (int k = lane >> 4; k < nr; k += 2) {
+        const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
+        const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
+#pragma unroll
+        for (int q = 0; q < NTOK; ++q)
+          if (q < ntok) s8[q] = fmaf(f, tr[q * tfl + k], s8[q]);
+      }
+    }
   }
 }
 
-// One stage of the delta-output consumers for a pass of NTOK tokens: for every block of the batch,
-// the limb matrix of scale * t (one rank per thread), a barrier, then the MMAs of this warp's tile;
-// 8-bit blocks take the scalar path.
-template <int NTOK>
-__device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, uint8_t* bsm, const uint8_t* bconst,
-                                         uint32_t& nmma, int (&C)[2][4][4], float (&zc)[DC_V_TOKS], float (&s8)[2],
-                                         int tid, int warp, int lane) {
-      const float* tw = reinterpret_cast<const float*>(stage + d.code_bytes);
-      const int tfl = d.tfl;
-      float pe[DC_V_TOKS];
-#pragma unroll
-      for (int q = 0; q < DC_V_TOKS; ++q) pe[q] = d.pe[q];
-      int off = 0, ro = d.t_shift;
-      for (int i = 0; i < d.nsub; ++i) {
-        const int p0 = d.sub[i][0], p1 = d.sub[i][1];
-        const int bits = p0 & 15, nq = (p0 >> 4) & 15, ns = (p0 >> 8) & 255, last = p0 >> 16;
-        const int nr = p1 & 0xffff, tile_bytes = p1 >> 16;
-        const int code_bytes = bits == 8 ? (int)dc_align((int64_t)128 * nr, 16) : 8 * tile_bytes;
-        const uint8_t* blk = stage + off;
-        const uint8_t* meta = blk + code_bytes;
-        if (bits != 8) {
-          // ---- limbs of scale * t * 2^e for rank tid of the block, every pass token
-          uint8_t* bb = bsm + (nmma & 1) * U_BBUF;
-          if (tid < nr) {
-            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * tid);
-            const float sc = __low2float(mz), zs = sc * __high2float(mz);
-#pragma unroll
-            for (int q = 0; q < NTOK; ++q) {
-              {
-                const float tq = tw[q * tfl + ro + tid];
-                const uint32_t v = __float_as_uint(fmaf(sc, tq * pe[q], U_MAGIC));
-                uint8_t* col = bb + (6 * (q >> 1) + (q & 1)) * U_BROW + tid;
-                col[0] = (uint8_t)v;
-                col[2 * U_BROW] = (uint8_t)(v >> 8);
-                col[4 * U_BROW] = (uint8_t)(v >> 16);
-                zc[q] = fmaf(zs, tq, zc[q]);
-              }
-            }
-          }
-          named_bar(1, 32 * U_CONSUMERS);
-          ud_mma<(NTOK + 1) / 2>(blk, bits, nq, ns, last, tile_bytes, bb, bconst, C, warp, lane);
-          ++nmma;
-        } else {
-          // ---- 8-bit band: scalar fp32, lane = (row lane & 15, tokens 2 (lane >> 4) + {0, 1})
-          const int row = lane & 15, th = lane >> 4;
-          const uint8_t* cr = blk + (16 * warp + row) * nr;
-          for (int k = 0; k < nr; ++k) {
-            const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
-            const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const int q = 2 * th + h;
-              if (q < NTOK) s8[h] = fmaf(f, tw[q * tfl + ro + k], s8[h]);
-            }
-          }
-        }
-        off += code_bytes + (int)dc_align((int64_t)4 * nr, 16);
-        ro += nr;
-      }
-    }
-
 __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __grid_constant__ DcFwd F, uint8_t* ws) {
   extern __shared__ __align__(128) uint8_t usm[];
-  uint8_t* bsm = usm + U_STAGES * U_STAGE_BYTES;  // two limb matrices, then the constant rows
-  uint8_t* bconst = bsm + 2 * U_BBUF;
-  USmemTail* tail = reinterpret_cast<USmemTail*>(bconst + U_BCONST);
+  uint8_t* lbuf = usm + U_STAGES * U_STAGE_BYTES;  // two limb matrices
+  USmemTail* tail = reinterpret_cast<USmemTail*>(lbuf + 2 * U_LBUF);
   WsPtr P = ws_ptr(F.ws, ws);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = F.ws.T;
@@ -1059,8 +1099,10 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     }
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < U_BCONST / 4; i += blockDim.x)
-    reinterpret_cast<uint32_t*>(bconst)[i] = i < U_BROW / 4 ? 0x01010101u : 0u;
+  for (int i = threadIdx.x; i < 2 * U_LROW; i += blockDim.x) {  // constant rows 12..15 of both matrices
+    const int b = i / U_LROW, w = i % U_LROW, row = 12 + w / (U_LROW / 4);
+    reinterpret_cast<uint32_t*>(lbuf + b * U_LBUF + 12 * U_LROW)[w] = (row == 12 || row == 14) ? 0x01010101u : 0u;
+  }
   __syncthreads();
   if (warp == U_CONSUMERS) {
     // ---------------- producer warp
@@ -1130,40 +1172,46 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
           if (pt0 != R.st) ctm = lane < ntok ? P.tmax[cp * T + pt0 + lane] : 0;
           const int e = ud_exponent(R.umax, ctm);  // lane q: token q
           const float pe = ldexpf(1.f, e), ie = ldexpf(1.f, -e);
-          if (lane == 0) {  // batches of consecutive blocks that fit a stage with this pass's t windows
+          if (lane == 0) {
+            // batches of consecutive blocks that fit a stage with this pass's t windows and the
+            // limb matrix; per block, its stage offsets, limb slot and t offset (the same for every
+            // group of the chunk)
             int nbt = 0, i = 0;
             while (i < NB) {
-              tail->bfirst[nbt++] = i;
-              int cb = 0, j = i;
+              const UBlkE& Ei = tail->tbl[i];
+              const int w0 = Ei.r0 & ~3;
+              int cb = 0, sl = 0, tfl = 0, j = i;
               while (j < NB && j - i < U_MAXSUB) {
-                const int w0 = tail->tbl[i].r0 & ~3;
-                const int tfl = (int)dc_align(tail->tbl[j].r0 + tail->tbl[j].nr, 4) - w0;
-                if (j > i && cb + tail->tbl[j].bytes + ntok * 4 * tfl > U_STAGE_BYTES) break;
-                cb += tail->tbl[j].bytes;
+                const UBlkE& Ej = tail->tbl[j];
+                const int tj = (int)dc_align(Ej.r0 + Ej.nr, 4) - w0;
+                const int sj = (Ej.p0 & 15) == 8 ? 0 : (int)dc_align(Ej.nr, 32);
+                if (j > i && (cb + Ej.bytes + ntok * 4 * tj > U_STAGE_BYTES || sl + sj > U_LROW)) break;
+                const int off = Ej.off - Ei.off;
+                *reinterpret_cast<int4*>(tail->bsub[j]) =
+                    make_int4(Ej.p0, Ej.p1, off | (sl << 16),
+                              (off + Ej.bytes - (int)dc_align((int64_t)4 * Ej.nr, 16)) | ((Ej.r0 - w0) << 16));
+                cb = off + Ej.bytes;
+                sl += sj;
+                tfl = tj;
                 ++j;
               }
+              tail->bat[nbt++] = make_int4(i | ((j - i) << 8) | ((Ei.r0 - w0) << 16), cb, tfl, w0);
               i = j;
             }
-            tail->bfirst[nbt] = NB;
             tail->nbatch = nbt;
           }
           __syncwarp();
           const int nbatch = tail->nbatch;
           for (int go = cgo0; go < cgo0 + cngo; ++go) {
             for (int j = 0; j < nbatch; ++j) {
-              const int f = tail->bfirst[j], nsub = tail->bfirst[j + 1] - f;
-              const UBlkE& E0 = tail->tbl[f];
-              const UBlkE& E1 = tail->tbl[f + nsub - 1];
-              const int code_bytes = E1.off + E1.bytes - E0.off;
-              const int w0 = E0.r0 & ~3;
-              const int tfl = (int)dc_align(E1.r0 + E1.nr, 4) - w0;
+              const int4 B = tail->bat[j];
+              const int f = B.x & 0xff, nsub = (B.x >> 8) & 0xff, code_bytes = B.y, tfl = B.z, w0 = B.w;
               const bool fits = code_bytes + ntok * 4 * tfl <= U_STAGE_BYTES;
               int s;
               if (!acquire(s)) return;
               uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
               UDesc& d = tail->desc[s];
-              if (lane < 2 * nsub) d.sub[lane >> 1][lane & 1] = (lane & 1) ? tail->tbl[f + (lane >> 1)].p1
-                                                                            : tail->tbl[f + (lane >> 1)].p0;
+              if (lane < 4 * nsub) d.sub[lane >> 2][lane & 3] = tail->bsub[f + (lane >> 2)][lane & 3];
               if (lane < DC_V_TOKS) {
                 d.pe[lane] = pe;
                 d.ie[lane] = ie;
@@ -1171,7 +1219,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
               if (lane == 0) {
                 d.kind = 1;
                 d.p = cp, d.go = go, d.tok0 = pt0, d.ntok = ntok;
-                d.nsub = nsub, d.code_bytes = code_bytes, d.tfl = tfl, d.t_shift = E0.r0 - w0;
+                d.nsub = nsub, d.code_bytes = code_bytes, d.tfl = tfl, d.t_shift = B.x >> 16;
                 d.ufirst = j == 0, d.ulast = j == nbatch - 1;
                 d.error = fits ? 0 : 1;
                 if (fits) {
@@ -1184,7 +1232,8 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
               __syncwarp();
               if (fits) {
                 if (lane == 0) {
-                  bulk_g2s(stage, runs + (int64_t)go * R.u_unit + E0.off, (uint32_t)code_bytes, &tail->full[s]);
+                  bulk_g2s(stage, runs + (int64_t)go * R.u_unit + tail->tbl[f].off, (uint32_t)code_bytes,
+                           &tail->full[s]);
                 } else if (lane <= ntok) {
                   const int q = lane - 1;
                   const float* src = P.tws + ((int64_t)cp * T + pt0 + q) * F.ws.r_stride + w0;
@@ -1210,15 +1259,18 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
   }
   // ---------------- consumer warps
   const int tid = threadIdx.x;  // 0..255
-  const int g = lane >> 2, t = lane & 3;
+  const int t = lane & 3;
   int C[2][4][4];
   float zc[DC_V_TOKS];
-  float s8[2];
-  uint32_t seq = 0, nmma = 0, unit = 0;
+  float s8[DC_V_TOKS];
+  uint32_t seq = 0, unit = 0;
   for (;;) {
     const int s = seq % U_STAGES;
-    if (!mbar_wait(&tail->full[s], (seq / U_STAGES) & 1)) {
-      set_status(P.st, DC_ERR_CUDA);
+    // every consumer warp waits for the stage itself; the vote makes all of them leave together
+    // when any wait ran out, so none is left at a named barrier of the stage
+    const bool okw = mbar_wait(&tail->full[s], (seq / U_STAGES) & 1);
+    if (!bar_and(3, 32 * U_CONSUMERS, okw)) {
+      if (!okw) set_status(P.st, DC_ERR_CUDA);
       return;
     }
     const UDesc& d = tail->desc[s];
@@ -1233,82 +1285,95 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
 #pragma unroll
           for (int q = 0; q < 4; ++q) C[a][b][q] = 0;
 #pragma unroll
-      for (int q = 0; q < DC_V_TOKS; ++q) zc[q] = 0.f;
-      s8[0] = s8[1] = 0.f;
+      for (int q = 0; q < DC_V_TOKS; ++q) zc[q] = s8[q] = 0.f;
     }
+    // the limb matrices alternate by stage: a warp writes matrix (seq & 1) only after every warp
+    // has passed the previous stage's barrier, i.e. finished its MMAs on the matrix of two stages ago
+    uint8_t* lb = lbuf + (seq & 1) * U_LBUF;
     if (!d.error) {
-      switch (ntok) {
-        case 1: ud_stage<1>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
-        case 2: ud_stage<2>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
-        case 3: ud_stage<3>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
-        default: ud_stage<4>(d, stage, bsm, bconst, nmma, C, zc, s8, tid, warp, lane); break;
-      }
+      // two code copies (one or two token pairs) keep the loop body small
+      if (ntok <= 2)
+        ud_stage<2>(d, stage, lb, C, zc, s8, ntok, tid, warp, lane);
+      else
+        ud_stage<4>(d, stage, lb, C, zc, s8, ntok, tid, warp, lane);
+    } else {
+      named_bar(1, 32 * U_CONSUMERS);  // keep the stage's barrier count uniform
     }
     const bool ulast = d.ulast;
-    const int p = d.p, go = d.go, tok0 = d.tok0;
-    float ie[DC_V_TOKS];
+    int p = 0, go = 0, tok0 = 0;
+    float ie[DC_V_TOKS] = {0.f, 0.f, 0.f, 0.f};
+    if (ulast) {  // read before the stage (and its descriptor) is handed back
+      p = d.p, go = d.go, tok0 = d.tok0;
 #pragma unroll
-    for (int q = 0; q < DC_V_TOKS; ++q) ie[q] = d.ie[q];
+      for (int q = 0; q < DC_V_TOKS; ++q) ie[q] = d.ie[q];
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(&tail->empty[s]);
     ++seq;
     if (!ulast) continue;
-    // ---- epilogue of the (group, pass) unit.  Phase 1: per-warp zero-point sums, 8-bit partials
-    // and the integer MMA results (positions combined) go to shared memory; phase 2: every
-    // thread finishes (row, token) outputs.  Sums run in a fixed order (deterministic).
-    float zw[DC_V_TOKS];
+    // ---- epilogue of the (group, pass) unit.  The zero-point sums are per token (the same for
+    // every row of the group): each warp's share goes to shared memory, one barrier, and every warp
+    // then finishes its own 16 rows.  Sums run in a fixed order (deterministic).
+    const int ub = unit & 1;
+    {  // warp sums of the zero-point terms, reduced and scattered: lane 8 q ends with token q's sum
+      const bool hi = lane & 16, b3 = lane & 8;
+      float k0 = hi ? zc[2] : zc[0], k1 = hi ? zc[3] : zc[1];
+      k0 += __shfl_xor_sync(FULLMASK, hi ? zc[0] : zc[2], 16);
+      k1 += __shfl_xor_sync(FULLMASK, hi ? zc[1] : zc[3], 16);
+      float v = b3 ? k1 : k0;
+      v += __shfl_xor_sync(FULLMASK, b3 ? k0 : k1, 8);
 #pragma unroll
-    for (int q = 0; q < DC_V_TOKS; ++q) {
-      float v = 0.f;
-      if (q < ntok) {
-        v = zc[q];
-#pragma unroll
-        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
-      }
-      zw[q] = v;
+      for (int o = 4; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
+      if ((lane & 7) == 0) tail->zpart[ub][lane >> 3][warp] = v;
     }
-    named_bar(2, 32 * U_CONSUMERS);  // the previous unit's phase 2 is over
-    if (lane < DC_V_TOKS) {
-      float v = zw[0], e = ie[0];
-#pragma unroll
-      for (int q = 1; q < DC_V_TOKS; ++q) {
-        v = lane == q ? zw[q] : v;
-        e = lane == q ? ie[q] : e;
-      }
-      tail->zpart[warp][lane] = v;
-      if (warp == 0) tail->uie[lane] = e;
-    }
-    {
+    {  // 8-bit sums: add the two rank halves of each row; half th keeps tokens 2 th, 2 th + 1
       const int row = 16 * warp + (lane & 15), th = lane >> 4;
-      tail->s8[row][2 * th] = s8[0];
-      tail->s8[row][2 * th + 1] = s8[1];
+      const float k0 = (th ? s8[2] : s8[0]) + __shfl_xor_sync(FULLMASK, th ? s8[0] : s8[2], 16);
+      const float k1 = (th ? s8[3] : s8[1]) + __shfl_xor_sync(FULLMASK, th ? s8[1] : s8[3], 16);
+      tail->s8[row][2 * th] = k0;
+      tail->s8[row][2 * th + 1] = k1;
     }
+    named_bar(2, 32 * U_CONSUMERS);
+    // lane t of quad g holds columns 2t, 2t+1 of rows g and g+8 (regs 0, 1 and 2, 3).  Column 7 is
+    // zero: lane 3 replaces it by column 6 (the row sum), then a 4x4 transpose inside the quad
+    // leaves lane t with register t of every lane of its quad, i.e. output (row g + 8 (t >> 1),
+    // token-in-pair t & 1): w[0] limb 0, w[1] limb 1, w[2] limb 2, w[3] the row sum.
+    const int orow = 16 * warp + (lane >> 2) + 8 * (t >> 1);
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
       if (2 * pr >= ntok) continue;
-      int Ct[4];
+      int w[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r)
-        Ct[r] = C[pr][0][r] + (C[pr][1][r] >> 2) + (C[pr][2][r] >> 4) + (C[pr][3][r] >> 6);
-      int* c0 = tail->cbuf[pr][16 * warp + g];
-      int* c1 = tail->cbuf[pr][16 * warp + g + 8];
-      c0[2 * t] = Ct[0];
-      c0[2 * t + 1] = Ct[1];
-      c1[2 * t] = Ct[2];
-      c1[2 * t + 1] = Ct[3];
-    }
-    named_bar(2, 32 * U_CONSUMERS);
-    // cbuf columns: 2 limb + token-in-pair for limbs 0..2, column 6 = the codes' row sum
-    for (int idx = tid; idx < 128 * ntok; idx += 32 * U_CONSUMERS) {
-      const int row = idx & 127, q = idx >> 7;
-      const int pr = q >> 1, tk = q & 1;
-      const int* cr = tail->cbuf[pr][row];
-      const float v = (float)(cr[4 + tk] - 64 * cr[6]) * 65536.f + (float)cr[2 + tk] * 256.f + (float)cr[tk];
-      float zs = 0.f;
-#pragma unroll
-      for (int ww = 0; ww < U_CONSUMERS; ++ww) zs += tail->zpart[ww][q];
-      const float y = fmaf(v, tail->uie[q], -zs) + tail->s8[row][q];
-      P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + row] = y;
+        w[r] = C[pr][0][r] + (C[pr][1][r] >> 2) + (C[pr][2][r] >> 4) + (C[pr][3][r] >> 6);
+      if (t == 3) {
+        w[1] = w[0];
+        w[3] = w[2];
+      }
+      // transpose: round 1 swaps with lane t ^ 1 the registers whose bit 0 differs from t's,
+      // round 2 with lane t ^ 2 those whose bit 1 differs
+      {
+        const bool o = t & 1;
+        const int a = __shfl_xor_sync(FULLMASK, o ? w[0] : w[1], 1);
+        const int b = __shfl_xor_sync(FULLMASK, o ? w[2] : w[3], 1);
+        if (o) { w[0] = a; w[2] = b; } else { w[1] = a; w[3] = b; }
+      }
+      {
+        const bool o = (t >> 1) & 1;
+        const int a = __shfl_xor_sync(FULLMASK, o ? w[0] : w[2], 2);
+        const int b = __shfl_xor_sync(FULLMASK, o ? w[1] : w[3], 2);
+        if (o) { w[0] = a; w[1] = b; } else { w[2] = a; w[3] = b; }
+      }
+      const int q = 2 * pr + (t & 1);
+      const float ieq = (t & 1) ? ie[2 * pr + 1] : ie[2 * pr];
+      if (q < ntok) {
+        const float4 z0 = *reinterpret_cast<const float4*>(&tail->zpart[ub][q][0]);
+        const float4 z1 = *reinterpret_cast<const float4*>(&tail->zpart[ub][q][4]);
+        const float zs = ((z0.x + z0.y) + (z0.z + z0.w)) + ((z1.x + z1.y) + (z1.z + z1.w));
+        const float v = (float)(w[2] - 64 * w[3]) * 65536.f + (float)w[1] * 256.f + (float)w[0];
+        const float y = fmaf(v, ieq, -zs) + tail->s8[orow][q];
+        P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + orow] = y;
+      }
     }
     ++unit;
   }
@@ -1605,16 +1670,6 @@ __device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1
 }
 
 __device__ __forceinline__ bool bt_aborted(BtTail* tail) { return *reinterpret_cast<volatile int*>(&tail->abort) != 0; }
-
-// AND of `ok` over the `count` threads of named barrier `id` (all of them take part).
-__device__ __forceinline__ bool bar_and(int id, int count, bool ok) {
-  uint32_t r;
-  asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
-               : "=r"(r)
-               : "r"((uint32_t)ok), "r"(id), "r"(count)
-               : "memory");
-  return r != 0;
-}
 
 __device__ __forceinline__ bool bt_wait(uint64_t* bar, uint32_t parity, BtTail* tail, int* st) {
   if (bt_aborted(tail)) return false;
@@ -3185,7 +3240,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     }
   }
   if (flags & DC_DELTA) {
-    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_BBUF + U_BCONST + sizeof(USmemTail);
+    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_LBUF + sizeof(USmemTail);
     if (usmem > 227 * 1024)
       return dc_fail(DC_ERR_UNSUPPORTED, "max_rank %d needs %zu bytes of shared memory", max_rank, usmem);
     static size_t usmem_set = 0;

@@ -88,3 +88,13 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const void* tmap, int x, 
 __device__ __forceinline__ void named_bar(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
+
+// AND of `ok` over the `count` threads of named barrier `id` (all of them take part).
+__device__ __forceinline__ bool bar_and(int id, int count, bool ok) {
+  uint32_t r;
+  asm volatile("{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.and.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+               : "=r"(r)
+               : "r"((uint32_t)ok), "r"(id), "r"(count)
+               : "memory");
+  return r != 0;
+}
