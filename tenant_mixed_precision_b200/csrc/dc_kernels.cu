@@ -499,25 +499,22 @@ struct VSmemTail {
   DcVItem rec[2];  // producer: current and next item
 };
 
-// acc[q] += s_row * (C[q] - z_row * xs_tok) for the C fragment entries that hold a valid token.
-// C entries: q = 0 (row g, pair token 0), 1 (row g, token 1), 2 (row g+8, token 0), 3 (row g+8, token 1).
-template <bool TOK1>
+// acc[q] += s_row * (C[q] - z_row * xs_tok).  C entries: q = 0 (row g, pair token 0), 1 (row g,
+// token 1), 2 (row g+8, token 0), 3 (row g+8, token 1).  Tokens past the pass have zero limbs and
+// zero limb sums, so their entries stay zero.
 __device__ __forceinline__ void v_epi(float (&acc)[4], const int (&C)[4], float sA, float zA, float sB, float zB,
                                       float x0, float x1) {
   acc[0] = fmaf(sA, fmaf(-zA, x0, (float)C[0]), acc[0]);
   acc[2] = fmaf(sB, fmaf(-zB, x0, (float)C[2]), acc[2]);
-  if (TOK1) {
-    acc[1] = fmaf(sA, fmaf(-zA, x1, (float)C[1]), acc[1]);
-    acc[3] = fmaf(sB, fmaf(-zB, x1, (float)C[3]), acc[3]);
-  }
+  acc[1] = fmaf(sA, fmaf(-zA, x1, (float)C[1]), acc[1]);
+  acc[3] = fmaf(sB, fmaf(-zB, x1, (float)C[3]), acc[3]);
 }
 
-// One 512-column block of one 16-rank tile, NTOK tokens (1..4), all loops unrolled.
+// One 512-column block of one 16-rank tile for ntok <= 2 NPAIR tokens, all loops unrolled.
 // FULL: the block holds 4 groups (2-bit codes then use the mask layout); otherwise ngrp < 4.
-template <int BITS, int NTOK, bool FULL>
-__device__ __forceinline__ void v_block(int rows, int ngrp_rt, const uint8_t* A, const uint8_t* X,
+template <int BITS, int NPAIR, bool FULL>
+__device__ __forceinline__ void v_block(int ntok, int rows, int ngrp_rt, const uint8_t* A, const uint8_t* X,
                                         float (&acc)[2][4], int lane) {
-  constexpr int NPAIR = (NTOK + 1) / 2;
   const int ngrp = FULL ? 4 : ngrp_rt;
   const int g = lane >> 2, t = lane & 3;
   const int nh0 = min(rows, 8), nh1 = max(0, rows - 8);
@@ -530,7 +527,7 @@ __device__ __forceinline__ void v_block(int rows, int ngrp_rt, const uint8_t* A,
 #pragma unroll
   for (int pr = 0; pr < NPAIR; ++pr) {
     const int tk = 2 * pr + (g & 1);
-    xval[pr] = (g < 6) && (tk < NTOK);
+    xval[pr] = (g < 6) && (tk < ntok);
     xrow[pr] = X + (xval[pr] ? tk * V_XTOK + 512 * limb : 0) + 32 * t;
   }
   const float* xsum = reinterpret_cast<const float*>(X + 1536 + 4 * (t < 3 ? t : 0));
@@ -561,9 +558,9 @@ __device__ __forceinline__ void v_block(int rows, int ngrp_rt, const uint8_t* A,
       bw[pr][0] = q0.x, bw[pr][1] = q0.y, bw[pr][2] = q0.z, bw[pr][3] = q0.w;
       bw[pr][4] = q1.x, bw[pr][5] = q1.y, bw[pr][6] = q1.z, bw[pr][7] = q1.w;
     }
-    float xs[NTOK];
+    float xs[2 * NPAIR];
 #pragma unroll
-    for (int k = 0; k < NTOK; ++k) xs[k] = t < 3 ? xsum[k * (V_XTOK / 4) + grp * 4] : 0.f;
+    for (int k = 0; k < 2 * NPAIR; ++k) xs[k] = (t < 3 && k < ntok) ? xsum[k * (V_XTOK / 4) + grp * 4] : 0.f;
     const uint2 mt = *reinterpret_cast<const uint2*>(meta + (grp * 8 + g) * 8);
     uint32_t a[4][4];  // [step][reg]
     if (BITS == 2 && FULL) {
@@ -618,30 +615,30 @@ __device__ __forceinline__ void v_block(int rows, int ngrp_rt, const uint8_t* A,
     const __half2 m1 = *reinterpret_cast<const __half2*>(&mt.y);
     const float sA = __low2float(m0) * (1.f / w), zA = __high2float(m0) * w;
     const float sB = __low2float(m1) * (1.f / w), zB = __high2float(m1) * w;
-    v_epi<(NTOK > 1)>(acc[0], C[0], sA, zA, sB, zB, xs[0], NTOK > 1 ? xs[NTOK > 1 ? 1 : 0] : 0.f);
-    if (NPAIR > 1)
-      v_epi<(NTOK > 3)>(acc[1], C[NPAIR - 1], sA, zA, sB, zB, xs[NTOK > 2 ? 2 : 0], NTOK > 3 ? xs[NTOK > 3 ? 3 : 0] : 0.f);
+    v_epi(acc[0], C[0], sA, zA, sB, zB, xs[0], xs[1]);
+    if (NPAIR > 1) v_epi(acc[1], C[NPAIR - 1], sA, zA, sB, zB, xs[2 * NPAIR - 2], xs[2 * NPAIR - 1]);
   }
 }
 
-template <int BITS, int NTOK>
-__device__ __forceinline__ void v_block_dispatch_ngrp(bool full, int rows, int ngrp, const uint8_t* A,
+// Code copies: per bit width one or two token pairs; only 2-bit codes have a separate layout for
+// full blocks (3/8-bit blocks take the group count at run time).  Few copies keep the consumer
+// loop small in the instruction cache.
+template <int BITS, int NPAIR>
+__device__ __forceinline__ void v_block_dispatch_ngrp(int ntok, bool full, int rows, int ngrp, const uint8_t* A,
                                                       const uint8_t* X, float (&acc)[2][4], int lane) {
-  if (full)
-    v_block<BITS, NTOK, true>(rows, 4, A, X, acc, lane);
+  if (BITS == 2 && full)
+    v_block<BITS, NPAIR, true>(ntok, rows, 4, A, X, acc, lane);
   else
-    v_block<BITS, NTOK, false>(rows, ngrp, A, X, acc, lane);
+    v_block<BITS, NPAIR, false>(ntok, rows, ngrp, A, X, acc, lane);
 }
 
 template <int BITS>
 __device__ __forceinline__ void v_block_dispatch(int ntok, bool full, int rows, int ngrp, const uint8_t* A,
                                                  const uint8_t* X, float (&acc)[2][4], int lane) {
-  switch (ntok) {
-    case 1: v_block_dispatch_ngrp<BITS, 1>(full, rows, ngrp, A, X, acc, lane); break;
-    case 2: v_block_dispatch_ngrp<BITS, 2>(full, rows, ngrp, A, X, acc, lane); break;
-    case 3: v_block_dispatch_ngrp<BITS, 3>(full, rows, ngrp, A, X, acc, lane); break;
-    default: v_block_dispatch_ngrp<BITS, 4>(full, rows, ngrp, A, X, acc, lane); break;
-  }
+  if (ntok <= 2)
+    v_block_dispatch_ngrp<BITS, 1>(ntok, full, rows, ngrp, A, X, acc, lane);
+  else
+    v_block_dispatch_ngrp<BITS, 2>(ntok, full, rows, ngrp, A, X, acc, lane);
 }
 
 __device__ __forceinline__ uint4 ldg128_item(const DcVItem* it, int lane) {
