@@ -133,12 +133,14 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.xe = take((int64_t)W.n_in * T * 4);
   W.tws = take((int64_t)n_lin * T * W.r_stride * 4);
   W.yd = take((int64_t)n_lin * T * W.max_d_in * 4);
-  W.dflag = take((int64_t)n_lin * T);
-  W.tmax = take((int64_t)n_lin * T * 4);
+  // per-call state reset by one memset: delta flags, output bounds, backbone unit counters
   W.bt_nb = T <= 256 ? (int32_t)dc_align(T > 0 ? T : 1, 16) : 256;
   W.bt_units = n_lin * (W.max_d_in / 128) * (int32_t)((T + W.bt_nb - 1) / W.bt_nb);
-  W.bt_part = take((int64_t)2 * DC_BT_MAX_CTAS * 128 * W.bt_nb * 4);
+  W.dflag = take((int64_t)n_lin * T);
+  W.tmax = take((int64_t)n_lin * T * 4);
   W.bt_cnt = take((int64_t)W.bt_units * 4);
+  W.reset_bytes = off - W.dflag;
+  W.bt_part = take((int64_t)2 * DC_BT_MAX_CTAS * 128 * W.bt_nb * 4);
   W.tseg = take((int64_t)T * 4);
   W.tcols = (int32_t)dc_align(max_rank > 0 ? max_rank : 1, 64) + 64 * (DC_MAX_BANDS - 1);
   W.thl = T >= DC_PF_MIN ? take((int64_t)2 * n_lin * T * W.tcols * 2) : take(0);
@@ -3191,9 +3193,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   // work counters (item count, work cursors) and per-token delta flags start from zero on every call
   st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * 4, s), "counter reset");
   if (st) return st;
-  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.dflag, 0, (size_t)n_lin * T, s), "flag reset");
-  if (st) return st;
-  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.tmax, 0, (size_t)n_lin * T * 4, s), "bound reset");
+  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.dflag, 0, (size_t)F.ws.reset_bytes, s), "flag reset");
   if (st) return st;
   const int nb_items = (T + 255) / 256;
   k_prep<<<dim3(T + nb_items, std::max(n_in, n_lin)), 256, 0, s>>>(F, (uint8_t*)ws);
@@ -3286,9 +3286,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
       if (st) return st;
       tset = tsmem;
     }
-    st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.bt_cnt, 0, (size_t)F.ws.bt_units * 4, s), "unit counters");
-    if (st) return st;
-    prof_before(s, 4);
+    prof_before(s, 4);  // the unit counters were zeroed with the call's other per-call state
     k_base_tc<<<F.bt_grid, BT_THREADS, tsmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
     return dc_cuda_check(cudaGetLastError(), "tensor-core output kernel");
