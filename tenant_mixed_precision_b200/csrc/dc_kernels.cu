@@ -1029,9 +1029,9 @@ static_assert(U_STAGES * U_STAGE_BYTES + 2 * U_LBUF + sizeof(USmemTail) + 1024 <
 
 // One stage of the delta-output consumers for a pass of ntok <= NTOK tokens (limb columns of tokens
 // ntok .. NTOK - 1 keep stale bytes; their outputs are never formed).  Phase A: the limb matrix of
-// scale * t for every 2/3-bit block of the batch (one rank per thread, each block in its own slot).
-// One barrier.  Phase B: this warp's MMAs over every block; 8-bit blocks take a scalar fp32 path
-// whose lanes split rows (lane & 15) and ranks (lane >> 4).  `lb` is this stage's limb matrix.
+// scale * t for every 2/3-bit block of the batch (one rank per thread, each block in its own slot);
+// 8-bit blocks are summed in fp32 by threads 128..255, one output row each.  One barrier.
+// Phase B: this warp's MMAs over every 2/3-bit block.  `lb` is this stage's limb matrix.
 template <int NTOK>
 __device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, uint8_t* lb, int (&C)[2][4][4],
                                          float (&zc)[DC_V_TOKS], float (&s8)[DC_V_TOKS], int ntok, int tid,
@@ -1044,7 +1044,23 @@ __device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, u
   for (int i = 0; i < nsub; ++i) {
     const int4 sd = *reinterpret_cast<const int4*>(d.sub[i]);
     const int nr = sd.y & 0xffff;
-    if ((sd.x & 15) == 8 || tid >= nr) continue;
+    if ((sd.x & 15) == 8) {  // row tid - 128: sum over the block's ranks of (c - z) * s * t
+      const int row = tid - 128;
+      if (row >= 0) {
+        const uint8_t* cr = stage + (sd.z & 0xffff) + row * nr;
+        const uint8_t* meta = stage + (sd.w & 0xffff);
+        const float* tr = tw + (sd.w >> 16);
+        for (int k = 0; k < nr; ++k) {
+          const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
+          const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
+#pragma unroll
+          for (int q = 0; q < NTOK; ++q)
+            if (q < ntok) s8[q] = fmaf(f, tr[q * tfl + k], s8[q]);
+        }
+      }
+      continue;
+    }
+    if (tid >= nr) continue;
     const int slot = sd.z >> 16, moff = sd.w & 0xffff, ro = sd.w >> 16;
     const __half2 mz = *reinterpret_cast<const __half2*>(stage + moff + 4 * tid);
     const float sc = __low2float(mz), zs = sc * __high2float(mz);
@@ -1064,23 +1080,11 @@ __device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, u
   named_bar(1, 32 * U_CONSUMERS);
   for (int i = 0; i < nsub; ++i) {
     const int4 sd = *reinterpret_cast<const int4*>(d.sub[i]);
-    const int bits = sd.x & 15, nr = sd.y & 0xffff;
-    const uint8_t* blk = stage + (sd.z & 0xffff);
-    if (bits != 8) {
-      const int nq = (sd.x >> 4) & 15, ns = (sd.x >> 8) & 255, last = sd.x >> 16;
-      ud_mma<(NTOK + 1) / 2>(blk, bits, nq, ns, last, sd.y >> 16, lb + (sd.z >> 16), C, warp, lane);
-    } else {
-      const uint8_t* meta = stage + (sd.w & 0xffff);
-      const float* tr = tw + (sd.w >> 16);
-      const uint8_t* cr = blk + (16 * warp + (lane & 15)) * nr;
-      for (int k = lane >> 4; k < nr; k += 2) {
-        const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * k);
-        const float f = ((float)cr[k] - __high2float(mz)) * __low2float(mz);
-#pragma unroll
-        for (int q = 0; q < NTOK; ++q)
-          if (q < ntok) s8[q] = fmaf(f, tr[q * tfl + k], s8[q]);
-      }
-    }
+    const int bits = sd.x & 15;
+    if (bits == 8) continue;
+    const int nq = (sd.x >> 4) & 15, ns = (sd.x >> 8) & 255, last = sd.x >> 16;
+    ud_mma<(NTOK + 1) / 2>(stage + (sd.z & 0xffff), bits, nq, ns, last, sd.y >> 16, lb + (sd.z >> 16), C, warp,
+                           lane);
   }
 }
 
@@ -1325,12 +1329,9 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       for (int o = 4; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
       if ((lane & 7) == 0) tail->zpart[ub][lane >> 3][warp] = v;
     }
-    {  // 8-bit sums: add the two rank halves of each row; half th keeps tokens 2 th, 2 th + 1
-      const int row = 16 * warp + (lane & 15), th = lane >> 4;
-      const float k0 = (th ? s8[2] : s8[0]) + __shfl_xor_sync(FULLMASK, th ? s8[0] : s8[2], 16);
-      const float k1 = (th ? s8[3] : s8[1]) + __shfl_xor_sync(FULLMASK, th ? s8[1] : s8[3], 16);
-      tail->s8[row][2 * th] = k0;
-      tail->s8[row][2 * th + 1] = k1;
+    if (tid >= 128) {  // 8-bit sums of row tid - 128
+#pragma unroll
+      for (int q = 0; q < DC_V_TOKS; ++q) tail->s8[tid - 128][q] = s8[q];
     }
     named_bar(2, 32 * U_CONSUMERS);
     // lane t of quad g holds columns 2t, 2t+1 of rows g and g+8 (regs 0, 1 and 2, 3).  Column 7 is
