@@ -827,23 +827,26 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
 // the codes' row sums, which remove the 2^22 bias.  The zero points are removed in fp32
 // (sum over ranks of zero * scale * t), then the exponent.  8-bit bands use a scalar fp32 path.
 // ---------------------------------------------------------------------------------------------
+#define U_GSTAGE 2           // 128-row output groups per stage (same tenant, linear and pass)
 #define U_STAGES 4
-#define U_STAGE_BYTES 22528  // a batch of blocks (codes + meta) and the t windows of its tokens
-#define U_CTAS_PER_SM 2      // two CTAs per SM: their producers' and consumers' stalls overlap
+#define U_STAGE_BYTES 45056  // a batch of blocks (codes + meta) for each group, then the t windows
+#define U_CTAS_PER_SM 1
 #define U_MAXSUB 8           // blocks per batch
 #define U_MAXBLK 64          // blocks per (linear, tenant) U run of one group
 #define U_CHUNK 4            // 128-row output groups per chunk of work
 #define U_LROW 544           // row stride of a limb matrix = rank slots per stage (rows 8 banks apart)
 #define U_LBUF (16 * U_LROW) // one limb matrix: rows 6 pr + 2 limb + token-in-pair, then constant rows
-#define U_CONSUMERS 8
+#define U_CONSUMERS 16       // 8 warps per group of the stage: warp w owns rows 16 (w % 8) .. + 15
 #define U_THREADS (32 * (U_CONSUMERS + 1))
 #define U_MAGIC 12582912.0f  // 1.5 * 2^23
 
 struct UDesc {
   int kind;              // 1 batch, 2 end
   int p, go, tok0, ntok;
+  int ng;                // groups go, go + 1, ... in the stage (1 .. U_GSTAGE)
   int nsub;              // blocks in the batch
-  int code_bytes;        // bytes of the batch's blocks (the t windows follow)
+  int code_bytes;        // bytes of the batch's blocks of one group (group g at g * code_bytes; the t
+                         // windows at U_GSTAGE * code_bytes)
   int tfl;               // floats per token t window
   int t_shift;           // position of the batch's first rank inside the t window
   int ufirst, ulast;     // the batch opens / closes its (group, pass) unit
@@ -869,8 +872,8 @@ struct USmemTail {
   int4 bat[U_MAXBLK];                 // producer: per batch, first block | blocks << 8 | t shift << 16,
                                       // code bytes, t window floats, first t column
   int nbatch;
-  alignas(16) float zpart[2][DC_V_TOKS][U_CONSUMERS];  // per-warp zero-point sums of a unit (two units in flight)
-  float s8[128][DC_V_TOKS + 1];            // 8-bit band sums of a unit: [row][token] (padded: no bank conflicts)
+  alignas(16) float zpart[2][U_GSTAGE][DC_V_TOKS][8];  // per-warp zero-point sums of a stage's units (two in flight)
+  float s8[U_GSTAGE][128][DC_V_TOKS + 1];  // 8-bit band sums of a unit: [row][token] (padded: no bank conflicts)
 };
 
 // D += A(u8, 16x32, row) * B(u8, 32x8, col), int32 accumulate.
@@ -1024,20 +1027,23 @@ static_assert(offsetof(USmemTail, zpart) % 16 == 0 && offsetof(USmemTail, rec) %
                   U_LBUF % 16 == 0,
               "delta-output shared-memory alignment");
 // two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA
-static_assert(U_STAGES * U_STAGE_BYTES + 2 * U_LBUF + sizeof(USmemTail) + 1024 <= 233472 / U_CTAS_PER_SM,
+static_assert(U_STAGES * U_STAGE_BYTES + 2 * U_GSTAGE * U_LBUF + sizeof(USmemTail) + 1024 <= 233472 / U_CTAS_PER_SM &&
+                  U_STAGES * U_STAGE_BYTES + 2 * U_GSTAGE * U_LBUF + sizeof(USmemTail) <= 232448,
               "delta-output shared memory exceeds the per-CTA share");
 
-// One stage of the delta-output consumers for a pass of ntok <= NTOK tokens (limb columns of tokens
-// ntok .. NTOK - 1 keep stale bytes; their outputs are never formed).  Phase A: the limb matrix of
-// scale * t for every 2/3-bit block of the batch (one rank per thread, each block in its own slot);
-// 8-bit blocks are summed in fp32 by threads 128..255, one output row each.  One barrier.
-// Phase B: this warp's MMAs over every 2/3-bit block.  `lb` is this stage's limb matrix.
+// One group of one stage of the delta-output consumers for a pass of ntok <= NTOK tokens (limb
+// columns of tokens ntok .. NTOK - 1 keep stale bytes; their outputs are never formed).  The group's
+// 256 threads (tid) and 8 warps (warp) work on its blocks at `stage`; `tw` are the t windows both
+// groups share.  Phase A: the limb matrix of scale * t for every 2/3-bit block of the batch (one rank
+// per thread, each block in its own slot); 8-bit blocks are summed in fp32 by threads 128..255, one
+// output row each.  One barrier of all consumer warps.  Phase B: this warp's MMAs over every
+// 2/3-bit block.  `lb` is the group's limb matrix of this stage.  A group slot the stage does not
+// use (active false) only takes part in the barrier.
 template <int NTOK>
-__device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, uint8_t* lb, int (&C)[2][4][4],
-                                         float (&zc)[DC_V_TOKS], float (&s8)[DC_V_TOKS], int ntok, int tid,
-                                         int warp, int lane) {
-  const float* tw = reinterpret_cast<const float*>(stage + d.code_bytes);
-  const int tfl = d.tfl, nsub = d.nsub;
+__device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, const float* tw, bool active,
+                                         uint8_t* lb, int (&C)[2][4][4], float (&zc)[DC_V_TOKS],
+                                         float (&s8)[DC_V_TOKS], int ntok, int tid, int warp, int lane) {
+  const int tfl = d.tfl, nsub = active ? d.nsub : 0;
   float pe[NTOK];
 #pragma unroll
   for (int q = 0; q < NTOK; ++q) pe[q] = d.pe[q];
@@ -1090,8 +1096,8 @@ __device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, u
 
 __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __grid_constant__ DcFwd F, uint8_t* ws) {
   extern __shared__ __align__(128) uint8_t usm[];
-  uint8_t* lbuf = usm + U_STAGES * U_STAGE_BYTES;  // two limb matrices
-  USmemTail* tail = reinterpret_cast<USmemTail*>(lbuf + 2 * U_LBUF);
+  uint8_t* lbuf = usm + U_STAGES * U_STAGE_BYTES;  // limb matrices [stage parity][group of the stage]
+  USmemTail* tail = reinterpret_cast<USmemTail*>(lbuf + 2 * U_GSTAGE * U_LBUF);
   WsPtr P = ws_ptr(F.ws, ws);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = F.ws.T;
@@ -1102,7 +1108,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     }
     fence_mbar_init();
   }
-  for (int i = threadIdx.x; i < 2 * U_LROW; i += blockDim.x) {  // constant rows 12..15 of both matrices
+  for (int i = threadIdx.x; i < 2 * U_GSTAGE * U_LROW; i += blockDim.x) {  // constant rows 12..15 of every matrix
     const int b = i / U_LROW, w = i % U_LROW, row = 12 + w / (U_LROW / 4);
     reinterpret_cast<uint32_t*>(lbuf + b * U_LBUF + 12 * U_LROW)[w] = (row == 12 || row == 14) ? 0x01010101u : 0u;
   }
@@ -1188,7 +1194,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
                 const UBlkE& Ej = tail->tbl[j];
                 const int tj = (int)dc_align(Ej.r0 + Ej.nr, 4) - w0;
                 const int sj = (Ej.p0 & 15) == 8 ? 0 : (int)dc_align(Ej.nr, 32);
-                if (j > i && (cb + Ej.bytes + ntok * 4 * tj > U_STAGE_BYTES || sl + sj > U_LROW)) break;
+                if (j > i && (U_GSTAGE * (cb + Ej.bytes) + ntok * 4 * tj > U_STAGE_BYTES || sl + sj > U_LROW)) break;
                 const int off = Ej.off - Ei.off;
                 *reinterpret_cast<int4*>(tail->bsub[j]) =
                     make_int4(Ej.p0, Ej.p1, off | (sl << 16),
@@ -1205,11 +1211,12 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
           }
           __syncwarp();
           const int nbatch = tail->nbatch;
-          for (int go = cgo0; go < cgo0 + cngo; ++go) {
+          for (int go = cgo0; go < cgo0 + cngo; go += U_GSTAGE) {
+            const int ng = min(U_GSTAGE, cgo0 + cngo - go);  // groups of this stage
             for (int j = 0; j < nbatch; ++j) {
               const int4 B = tail->bat[j];
               const int f = B.x & 0xff, nsub = (B.x >> 8) & 0xff, code_bytes = B.y, tfl = B.z, w0 = B.w;
-              const bool fits = code_bytes + ntok * 4 * tfl <= U_STAGE_BYTES;
+              const bool fits = U_GSTAGE * code_bytes + ntok * 4 * tfl <= U_STAGE_BYTES;
               int s;
               if (!acquire(s)) return;
               uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
@@ -1221,12 +1228,12 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
               }
               if (lane == 0) {
                 d.kind = 1;
-                d.p = cp, d.go = go, d.tok0 = pt0, d.ntok = ntok;
+                d.p = cp, d.go = go, d.tok0 = pt0, d.ntok = ntok, d.ng = ng;
                 d.nsub = nsub, d.code_bytes = code_bytes, d.tfl = tfl, d.t_shift = B.x >> 16;
                 d.ufirst = j == 0, d.ulast = j == nbatch - 1;
                 d.error = fits ? 0 : 1;
                 if (fits) {
-                  mbar_arrive_expect_tx(&tail->full[s], (uint32_t)(code_bytes + ntok * 4 * tfl));
+                  mbar_arrive_expect_tx(&tail->full[s], (uint32_t)(ng * code_bytes + ntok * 4 * tfl));
                 } else {
                   set_status(P.st, DC_ERR_UNSUPPORTED);
                   mbar_arrive(&tail->full[s]);
@@ -1234,13 +1241,13 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
               }
               __syncwarp();
               if (fits) {
-                if (lane == 0) {
-                  bulk_g2s(stage, runs + (int64_t)go * R.u_unit + tail->tbl[f].off, (uint32_t)code_bytes,
-                           &tail->full[s]);
-                } else if (lane <= ntok) {
-                  const int q = lane - 1;
+                if (lane < ng) {  // group go + lane's blocks
+                  bulk_g2s(stage + lane * code_bytes, runs + (int64_t)(go + lane) * R.u_unit + tail->tbl[f].off,
+                           (uint32_t)code_bytes, &tail->full[s]);
+                } else if (lane >= U_GSTAGE && lane < U_GSTAGE + ntok) {
+                  const int q = lane - U_GSTAGE;
                   const float* src = P.tws + ((int64_t)cp * T + pt0 + q) * F.ws.r_stride + w0;
-                  bulk_g2s(stage + code_bytes + q * 4 * tfl, src, (uint32_t)(4 * tfl), &tail->full[s]);
+                  bulk_g2s(stage + U_GSTAGE * code_bytes + q * 4 * tfl, src, (uint32_t)(4 * tfl), &tail->full[s]);
                 }
               }
               __syncwarp();
@@ -1261,7 +1268,8 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     return;
   }
   // ---------------- consumer warps
-  const int tid = threadIdx.x;  // 0..255
+  const int gs = warp >> 3, w8 = warp & 7;  // group slot of the stage, tile of the group
+  const int tid = threadIdx.x & 255;        // thread of the group slot
   const int t = lane & 3;
   int C[2][4][4];
   float zc[DC_V_TOKS];
@@ -1280,6 +1288,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     if (d.kind == 2) return;
     const uint8_t* stage = usm + (size_t)s * U_STAGE_BYTES;
     const int ntok = d.ntok;
+    const bool active = gs < d.ng;  // this slot's group is part of the stage
     if (d.ufirst) {
 #pragma unroll
       for (int a = 0; a < 2; ++a)
@@ -1292,13 +1301,15 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     }
     // the limb matrices alternate by stage: a warp writes matrix (seq & 1) only after every warp
     // has passed the previous stage's barrier, i.e. finished its MMAs on the matrix of two stages ago
-    uint8_t* lb = lbuf + (seq & 1) * U_LBUF;
+    uint8_t* lb = lbuf + ((seq & 1) * U_GSTAGE + gs) * U_LBUF;
     if (!d.error) {
+      const uint8_t* blocks = stage + gs * d.code_bytes;
+      const float* tw = reinterpret_cast<const float*>(stage + U_GSTAGE * d.code_bytes);
       // two code copies (one or two token pairs) keep the loop body small
       if (ntok <= 2)
-        ud_stage<2>(d, stage, lb, C, zc, s8, ntok, tid, warp, lane);
+        ud_stage<2>(d, blocks, tw, active, lb, C, zc, s8, ntok, tid, w8, lane);
       else
-        ud_stage<4>(d, stage, lb, C, zc, s8, ntok, tid, warp, lane);
+        ud_stage<4>(d, blocks, tw, active, lb, C, zc, s8, ntok, tid, w8, lane);
     } else {
       named_bar(1, 32 * U_CONSUMERS);  // keep the stage's barrier count uniform
     }
@@ -1306,7 +1317,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     int p = 0, go = 0, tok0 = 0;
     float ie[DC_V_TOKS] = {0.f, 0.f, 0.f, 0.f};
     if (ulast) {  // read before the stage (and its descriptor) is handed back
-      p = d.p, go = d.go, tok0 = d.tok0;
+      p = d.p, go = d.go + gs, tok0 = d.tok0;
 #pragma unroll
       for (int q = 0; q < DC_V_TOKS; ++q) ie[q] = d.ie[q];
     }
@@ -1314,9 +1325,10 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
     if (lane == 0) mbar_arrive(&tail->empty[s]);
     ++seq;
     if (!ulast) continue;
-    // ---- epilogue of the (group, pass) unit.  The zero-point sums are per token (the same for
-    // every row of the group): each warp's share goes to shared memory, one barrier, and every warp
-    // then finishes its own 16 rows.  Sums run in a fixed order (deterministic).
+    // ---- epilogue of the stage's (group, pass) units.  The zero-point sums are per token (the same
+    // for every row of a group): each warp's share goes to shared memory, one barrier, and every
+    // warp then finishes its own 16 rows.  Sums run in a fixed order (deterministic).  A slot whose
+    // group the stage did not hold writes nothing.
     const int ub = unit & 1;
     {  // warp sums of the zero-point terms, reduced and scattered: lane 8 q ends with token q's sum
       const bool hi = lane & 16, b3 = lane & 8;
@@ -1327,21 +1339,21 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       v += __shfl_xor_sync(FULLMASK, b3 ? k0 : k1, 8);
 #pragma unroll
       for (int o = 4; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
-      if ((lane & 7) == 0) tail->zpart[ub][lane >> 3][warp] = v;
+      if ((lane & 7) == 0) tail->zpart[ub][gs][lane >> 3][w8] = v;
     }
     if (tid >= 128) {  // 8-bit sums of row tid - 128
 #pragma unroll
-      for (int q = 0; q < DC_V_TOKS; ++q) tail->s8[tid - 128][q] = s8[q];
+      for (int q = 0; q < DC_V_TOKS; ++q) tail->s8[gs][tid - 128][q] = s8[q];
     }
     named_bar(2, 32 * U_CONSUMERS);
     // lane t of quad g holds columns 2t, 2t+1 of rows g and g+8 (regs 0, 1 and 2, 3).  Column 7 is
     // zero: lane 3 replaces it by column 6 (the row sum), then a 4x4 transpose inside the quad
     // leaves lane t with register t of every lane of its quad, i.e. output (row g + 8 (t >> 1),
     // token-in-pair t & 1): w[0] limb 0, w[1] limb 1, w[2] limb 2, w[3] the row sum.
-    const int orow = 16 * warp + (lane >> 2) + 8 * (t >> 1);
+    const int orow = 16 * w8 + (lane >> 2) + 8 * (t >> 1);
 #pragma unroll
     for (int pr = 0; pr < 2; ++pr) {
-      if (2 * pr >= ntok) continue;
+      if (2 * pr >= ntok || !active) continue;
       int w[4];
 #pragma unroll
       for (int r = 0; r < 4; ++r)
@@ -1367,11 +1379,11 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       const int q = 2 * pr + (t & 1);
       const float ieq = (t & 1) ? ie[2 * pr + 1] : ie[2 * pr];
       if (q < ntok) {
-        const float4 z0 = *reinterpret_cast<const float4*>(&tail->zpart[ub][q][0]);
-        const float4 z1 = *reinterpret_cast<const float4*>(&tail->zpart[ub][q][4]);
+        const float4 z0 = *reinterpret_cast<const float4*>(&tail->zpart[ub][gs][q][0]);
+        const float4 z1 = *reinterpret_cast<const float4*>(&tail->zpart[ub][gs][q][4]);
         const float zs = ((z0.x + z0.y) + (z0.z + z0.w)) + ((z1.x + z1.y) + (z1.z + z1.w));
         const float v = (float)(w[2] - 64 * w[3]) * 65536.f + (float)w[1] * 256.f + (float)w[0];
-        const float y = fmaf(v, ieq, -zs) + tail->s8[orow][q];
+        const float y = fmaf(v, ieq, -zs) + tail->s8[gs][orow][q];
         P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + orow] = y;
       }
     }
@@ -1450,7 +1462,9 @@ __device__ void b_base_f32(const DcFwd& F, const DcLinDev& lin, const int* perm,
   }
 }
 
-__global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ DcFwd F, uint8_t* ws) {
+#define KB_CONSUMERS 8  // consumer warps of k_base (warp w: rows 16 w .. 16 w + 15 of the tile)
+#define KB_THREADS (32 * (KB_CONSUMERS + 1))
+__global__ void __launch_bounds__(KB_THREADS, 1) k_base(const __grid_constant__ DcFwd F, uint8_t* ws) {
   extern __shared__ __align__(1024) uint8_t bsm_raw[];
   uint8_t* sm = bsm_raw + ((1024 - (smem_u32(bsm_raw) & 1023)) & 1023);  // 1024-aligned for swizzled tiles
   BSmemTail* tail = reinterpret_cast<BSmemTail*>(sm + B_STAGES * B_STAGE_BYTES);
@@ -1461,12 +1475,12 @@ __global__ void __launch_bounds__(U_THREADS, 1) k_base(const __grid_constant__ D
   if (threadIdx.x == 0) {
     for (int s = 0; s < B_STAGES; ++s) {
       mbar_init(&tail->full[s], 1);
-      mbar_init(&tail->empty[s], U_CONSUMERS);
+      mbar_init(&tail->empty[s], KB_CONSUMERS);
     }
     fence_mbar_init();
   }
   __syncthreads();
-  if (warp == U_CONSUMERS) {
+  if (warp == KB_CONSUMERS) {
     // ---------------- producer warp
     const int n_units = F.tile_prefix[F.n_lin] * nTB;
     uint32_t seq = 0;
@@ -3238,7 +3252,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     }
   }
   if (flags & DC_DELTA) {
-    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_LBUF + sizeof(USmemTail);
+    const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_GSTAGE * U_LBUF + sizeof(USmemTail);
     if (usmem > 227 * 1024)
       return dc_fail(DC_ERR_UNSUPPORTED, "max_rank %d needs %zu bytes of shared memory", max_rank, usmem);
     static size_t usmem_set = 0;
@@ -3301,7 +3315,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   }
   const int n_units = F.tile_prefix[n_lin] * ((T + DC_TOK_BLOCK - 1) / DC_TOK_BLOCK);
   prof_before(s, 4);
-  k_base<<<std::min(n_sm, n_units), U_THREADS, bsmem, s>>>(F, (uint8_t*)ws);
+  k_base<<<std::min(n_sm, n_units), KB_THREADS, bsmem, s>>>(F, (uint8_t*)ws);
   prof_after(s);
   return dc_cuda_check(cudaGetLastError(), "output kernel");
 }
