@@ -1621,8 +1621,9 @@ __global__ void __launch_bounds__(KB_THREADS, 1) k_base(const __grid_constant__ 
 
 // ---------------------------------------------------------------------------------------------
 // k_base_tc: y = W_base x (+ ydelta) on the tcgen05 tensor cores, for bf16 backbones.
-// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens); its K is cut
-// into 64-column chunks.  The units' chunks, largest-K linears first, form one sequence that is
+// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens), token block
+// outer and tile inner within a linear; its K is cut into 64-column chunks.  The units' chunks,
+// largest-K linears first, form one sequence that is
 // split evenly over the persistent CTAs (stream-K), so every CTA moves the same number of bytes
 // whatever the tile count.  Per CTA: warp 0 loads each chunk's W slice (128 x 64) and activation
 // slice (NB x 64) with 2-D TMA into a ring of stages; warp 1 owns two NB-column fp32
@@ -1674,9 +1675,13 @@ __device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1
   S.slot = slot;
   S.K = F.lin[F.order[slot]].d_in / 64;
   const int64_t local = (g - F.bt_chunk_prefix[slot]) / S.K;
+  // token block outer, row tile inner: the CTAs that run side by side (their chunk ranges start
+  // one token block apart) read the same weight tile at about the same time, so a tile comes from
+  // DRAM once per batch and from L2 for its other token blocks
+  const int ntiles = F.lin[F.order[slot]].d_out / 128;
   S.u = (int)(F.tile_prefix[slot] * (int64_t)F.bt_ntb + local);
-  S.ot = (int)(local / F.bt_ntb);
-  S.tb = (int)(local % F.bt_ntb);
+  S.ot = (int)(local % ntiles);
+  S.tb = (int)(local / ntiles);
   S.ustart = F.bt_chunk_prefix[slot] + local * S.K;
   S.k0 = (int)(g - S.ustart);
   S.k1 = (int)min((int64_t)S.K, g1 - S.ustart);
