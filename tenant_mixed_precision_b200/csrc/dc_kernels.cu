@@ -173,6 +173,7 @@ struct DcFwd {
   int64_t bt_chunk_prefix[8];  // tensor-core backbone: cumulative 64-column chunks of all units, same order
   int64_t bt_total;            // total chunks
   int32_t bt_ntb, bt_ns, bt_grid, bt_pad;  // token blocks, pipeline stages, CTAs
+  int32_t bt_gtiles[8];        // per linear (same order): row tiles per group of the unit order
   CUtensorMap tmap;            // prefill path: bf16 t planes [2 n_lin T rows x tcols], box 64 x 256
   CUtensorMap xpf[3];          // prefill path: tenant-sorted activations, box 64 x pf_box tokens
   int32_t pf;                  // segments of >= DC_PF_MIN tokens take the prefill delta path
@@ -1621,9 +1622,9 @@ __global__ void __launch_bounds__(KB_THREADS, 1) k_base(const __grid_constant__ 
 
 // ---------------------------------------------------------------------------------------------
 // k_base_tc: y = W_base x (+ ydelta) on the tcgen05 tensor cores, for bf16 backbones.
-// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens), token block
-// outer and tile inner within a linear; its K is cut into 64-column chunks.  The units' chunks,
-// largest-K linears first, form one sequence that is
+// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens), ordered inside
+// a linear by group of tiles, token block, tile; its K is cut into 64-column chunks.  The units'
+// chunks, largest-K linears first, form one sequence that is
 // split evenly over the persistent CTAs (stream-K), so every CTA moves the same number of bytes
 // whatever the tile count.  Per CTA: warp 0 loads each chunk's W slice (128 x 64) and activation
 // slice (NB x 64) with 2-D TMA into a ring of stages; warp 1 owns two NB-column fp32
@@ -1675,13 +1676,17 @@ __device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1
   S.slot = slot;
   S.K = F.lin[F.order[slot]].d_in / 64;
   const int64_t local = (g - F.bt_chunk_prefix[slot]) / S.K;
-  // token block outer, row tile inner: the CTAs that run side by side (their chunk ranges start
-  // one token block apart) read the same weight tile at about the same time, so a tile comes from
-  // DRAM once per batch and from L2 for its other token blocks
-  const int ntiles = F.lin[F.order[slot]].d_out / 128;
-  S.u = (int)(F.tile_prefix[slot] * (int64_t)F.bt_ntb + local);
-  S.ot = (int)(local % ntiles);
-  S.tb = (int)(local / ntiles);
+  // unit order inside a linear: groups of G row tiles (about one CTA's share of chunks), then the
+  // token block, then the tile inside the group.  The CTAs working on one group for different
+  // token blocks start within about one tile of each other and walk the same tiles in step, so a
+  // weight tile comes from DRAM once and from L2 for its other token blocks.
+  const int ntiles = F.lin[F.order[slot]].d_out / 128, ntb = F.bt_ntb, G = F.bt_gtiles[slot];
+  const int grp = (int)(local / ((int64_t)G * ntb));
+  const int gl = min(G, ntiles - grp * G);  // tiles of this group (the last may be short)
+  const int rem = (int)(local - (int64_t)grp * G * ntb);
+  S.u = (int)(F.tile_prefix[slot] * (int64_t)ntb + local);
+  S.ot = grp * G + rem % gl;
+  S.tb = rem / gl;
   S.ustart = F.bt_chunk_prefix[slot] + local * S.K;
   S.k0 = (int)(g - S.ustart);
   S.k1 = (int)min((int64_t)S.K, g1 - S.ustart);
@@ -3298,6 +3303,11 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     const int stage_bytes = BT_A_BYTES + F.ws.bt_nb * 128;
     F.bt_ns = std::min(BT_MAX_STAGES, (int)((200 * 1024) / stage_bytes));
     F.bt_grid = (int)std::min<int64_t>(std::min(n_sm, DC_BT_MAX_CTAS), F.bt_total);
+    for (int i = 0; i < n_lin; ++i) {  // tile groups of about one CTA's share of chunks
+      const dc_linear& l = lins[ord[i]];
+      const int64_t share = (F.bt_total + F.bt_grid - 1) / F.bt_grid;
+      F.bt_gtiles[i] = (int)std::max<int64_t>(1, std::min<int64_t>(l.d_out / 128, share / (l.d_in / 64)));
+    }
     const size_t tsmem = 1024 + (size_t)F.bt_ns * stage_bytes + sizeof(BtTail);
     static size_t tset = 0;
     if (tsmem > tset) {
