@@ -485,7 +485,8 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
 #define V_A_BYTES 18432   // one block of the item's tiles: 8 x 2304 (2-bit), 5 x 3328 (3-bit), 2 x 8448 (8-bit)
 #define V_XTOK DC_XBLK    // one token's limb block in shared memory (1616: offsets tokens by 20 banks)
 #define V_X_BYTES (4 * V_XTOK)
-#define V_STAGE_BYTES (V_A_BYTES + V_X_BYTES)
+#define V_S_BYTES 512     // the item's S (at most 128 ranks), staged with its last block
+#define V_STAGE_BYTES (V_A_BYTES + V_X_BYTES + V_S_BYTES)
 #define V_CONSUMERS 8
 #define V_THREADS (32 * (V_CONSUMERS + 1))
 
@@ -493,6 +494,7 @@ struct VDesc {
   int kind;  // 0 block, 1 end
   int bits, rows_left, ntiles, tok0, ntok, m, p, kb, ngrp, first, last, rank0, pad;
   int64_t sbase;
+  int e[DC_V_TOKS];  // activation exponents of the pass tokens (set with the item's last block)
 };
 
 struct VSmemTail {
@@ -501,6 +503,10 @@ struct VSmemTail {
   uint64_t empty[V_STAGES];
   DcVItem rec[2];  // producer: current and next item
 };
+// two CTAs per SM: 228 KB of shared memory per SM, 1 KB of it reserved per CTA; 16-byte staged rows
+static_assert(V_STAGES * V_STAGE_BYTES + sizeof(VSmemTail) + 1024 <= 233472 / V_CTAS_PER_SM &&
+                  (V_A_BYTES + V_X_BYTES) % 16 == 0 && V_STAGE_BYTES % 16 == 0,
+              "rank-reduction shared memory");
 
 // acc[q] += s_row * (C[q] - z_row * xs_tok).  C entries: q = 0 (row g, pair token 0), 1 (row g,
 // token 1), 2 (row g+8, token 0), 3 (row g+8, token 1).  Tokens past the pass have zero limbs and
@@ -685,6 +691,18 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
       }
       const DcVItem& I = tail->rec[0];
       const int nkb = end ? 1 : I.nkb;
+      // the epilogue's operands, fetched now and staged with the item's last block: S of the item's
+      // ranks (lane l: ranks 4 l .. 4 l + 3) and the pass tokens' activation exponents
+      float sv[4] = {0.f, 0.f, 0.f, 0.f};
+      int ev = 0;
+      if (!end) {
+        const float* S = reinterpret_cast<const float*>(I.sbase);
+        const int nr = min(16 * I.ntiles, I.rows_left);
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          if (4 * lane + j < nr) sv[j] = S[4 * lane + j];
+        if (lane < I.ntok) ev = P.xe[I.m * T + I.tok0 + lane];
+      }
       for (int kb = 0; kb < nkb; ++kb) {
         const int s = seq % V_STAGES;
         if (seq >= V_STAGES && !mbar_wait(&tail->empty[s], ((seq / V_STAGES) - 1) & 1)) {
@@ -705,6 +723,11 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
         const uint32_t code_bytes = (uint32_t)((I.ntiles - 1) * dc_v_block_bytes(I.bits, 16, ngrp) +
                                                dc_v_block_bytes(I.bits, last_rows, ngrp));
         const uint32_t total = code_bytes + (uint32_t)(I.ntok * DC_XBLK);
+        if (kb == I.nkb - 1) {  // ordered before the stage's arrive by the warp barrier below
+          *reinterpret_cast<float4*>(stage + V_A_BYTES + V_X_BYTES + 16 * lane) = make_float4(sv[0], sv[1], sv[2], sv[3]);
+          if (lane < DC_V_TOKS) tail->desc[s].e[lane] = ev;
+        }
+        __syncwarp();
         if (lane == 0) {
           VDesc& d = tail->desc[s];
           d.kind = 0;
@@ -749,7 +772,7 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
       set_status(P.st, DC_ERR_CUDA);
       return;
     }
-    const VDesc d = tail->desc[s];
+    const VDesc& d = tail->desc[s];  // read only before the stage is handed back
     if (d.kind == 1) return;
     const uint8_t* stage = vsm + (size_t)s * V_STAGE_BYTES;
     if (warp < d.ntiles) {
@@ -772,7 +795,7 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
       if (d.last) {
         // combine the three limbs (lane t holds limb t), scale by 2^-e and S, store t
         const float lw = (float)(1 << (8 * min(t, 2)));
-        const float* S = reinterpret_cast<const float*>(d.sbase);
+        const float* S = reinterpret_cast<const float*>(stage + V_A_BYTES + V_X_BYTES);  // staged S
         float tmx[DC_V_TOKS] = {0.f, 0.f, 0.f, 0.f};  // max |t| per pass token over this warp's rows
 #pragma unroll
         for (int pr = 0; pr < 2; ++pr)
@@ -786,8 +809,7 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
             if (t == 0 && row < rows && tk < d.ntok) {
               const int rl = 16 * warp + row;  // row within the item
               const int tok = d.tok0 + tk;
-              const int e = P.xe[d.m * T + tok];
-              const float tv = ldexpf(v, -e) * S[rl];
+              const float tv = ldexpf(v, -d.e[tk]) * S[rl];
               P.tws[((int64_t)d.p * T + tok) * F.ws.r_stride + d.rank0 + rl] = tv;
               tmx[tk] = fmaxf(tmx[tk], fabsf(tv));
             }
