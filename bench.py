@@ -90,7 +90,8 @@ class ClockSampler:
 
 def _kernel_source_sha(kernel: str) -> str:
     """Hash of what decides `kernel`'s DRAM traffic: its section of dc_kernels.cu (from its
-    "// <name>:" header to the next section) and the layout headers."""
+    "// <name>:" header to the next section) and the layout headers, with comments and blank lines
+    left out so that editing a comment keeps the committed traffic figure."""
     csrc = os.path.join(ROOT, "tenant_mixed_precision_b200", "csrc")
     with open(os.path.join(csrc, "dc_kernels.cu")) as f:
         text = f.read()
@@ -98,10 +99,19 @@ def _kernel_source_sha(kernel: str) -> str:
     start = text.find("\n// " + kernel + ":")
     end = text.find(sep + "// ", start + 1) if start >= 0 else -1
     section = text[start:end] if start >= 0 else text
-    h = hashlib.sha256(section.encode())
+
+    def code_only(src: str) -> str:
+        out = []
+        for line in src.splitlines():
+            line = line.split("//", 1)[0].rstrip()
+            if line:
+                out.append(line)
+        return "\n".join(out)
+
+    h = hashlib.sha256(code_only(section).encode())
     for name in ("dc_layout.h", "dc_internal.h", "dc_pack.h"):
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

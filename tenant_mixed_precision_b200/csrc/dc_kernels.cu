@@ -478,7 +478,8 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
 // producer takes one work item at a time (prefetching the next item's record), and streams the
 // item's 512-column blocks -- codes and meta of every tile, the activation limbs and limb sums of
 // the pass's tokens -- into a ring of shared-memory stages with bulk copies; consumer warp w
-// decodes tile w from shared memory into u8 MMA operands.
+// decodes tile w from shared memory into u8 MMA operands.  With the item's last block the producer
+// also stages S of the item's ranks and the tokens' activation exponents for the epilogue.
 // ---------------------------------------------------------------------------------------------
 #define V_STAGES 4
 #define V_CTAS_PER_SM 2  // two CTAs per SM: twice the warps to hide the consumers' latencies
@@ -836,11 +837,12 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
 // ---------------------------------------------------------------------------------------------
 // k_udelta: ydelta[token, row] = (U_hat (scale * t))[row] for every token of every segment with a
 // delta.  Work is taken from a global counter in chunks of (linear, segment, up to U_CHUNK
-// consecutive 128-row output groups).  For each pass of <= 4 tokens and each group of the chunk
-// the producer warp streams the group's U blocks in batches of consecutive blocks (codes of the
-// eight 16-row tiles and the meta of the blocks' ranks: one bulk copy) together with the pass's
-// t values of the batch's ranks (one copy per token) through a ring of shared-memory stages.
-// Consumer warp w owns rows 16w..16w+15 of the group.
+// consecutive 128-row output groups).  For each pass of <= 4 tokens and each pair of groups of
+// the chunk the producer warp streams the groups' U blocks in batches of consecutive blocks
+// (codes of the eight 16-row tiles and the meta of the blocks' ranks: one bulk copy per group),
+// together with the pass's t values of the batch's ranks (one copy per token, shared by the two
+// groups), through a ring of shared-memory stages.  One CTA per SM: consumer warp w works on
+// group w / 8 of the stage and owns its rows 16 (w % 8) .. 16 (w % 8) + 15.
 //
 // Arithmetic of a (group, pass) unit: B = scale * t is written, per token, as the fixed-point
 // integer rint(B * 2^e) with e fixed by the bound umax * max|t| (so |B * 2^e| < 2^21): one fp32
@@ -848,7 +850,8 @@ __global__ void __launch_bounds__(V_THREADS, V_CTAS_PER_SM) k_vstage(const __gri
 // whose three low bytes are the unsigned limbs of the operand.  The tensor cores multiply the u8
 // codes by those u8 limbs exactly (mma m16n8k32 u8.u8 -> s32); B column 6 is all ones, giving
 // the codes' row sums, which remove the 2^22 bias.  The zero points are removed in fp32
-// (sum over ranks of zero * scale * t), then the exponent.  8-bit bands use a scalar fp32 path.
+// (sum over ranks of zero * scale * t), then the exponent.  8-bit bands are summed in fp32
+// during the limb phase, one output row per thread.
 // ---------------------------------------------------------------------------------------------
 #define U_GSTAGE 2           // 128-row output groups per stage (same tenant, linear and pass)
 #define U_STAGES 4
