@@ -75,7 +75,6 @@ struct DcWs {
   int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, bt_part, bt_cnt;
   int64_t tseg;      // per tenant-sorted token: its segment
   int64_t thl;       // bf16 t, high and low parts: [2][n_lin][T][tcols]
-  int64_t reset_bytes;  // dflag .. end of bt_cnt: zeroed at the start of every call
   int64_t total;
 };
 

@@ -133,13 +133,13 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.xe = take((int64_t)W.n_in * T * 4);
   W.tws = take((int64_t)n_lin * T * W.r_stride * 4);
   W.yd = take((int64_t)n_lin * T * W.max_d_in * 4);
-  // per-call state reset by one memset: delta flags, output bounds, backbone unit counters
+  // per-call state: delta flags (written for every token by k_prep), output bounds and backbone
+  // unit counters (zeroed by k_prep)
   W.bt_nb = T <= 256 ? (int32_t)dc_align(T > 0 ? T : 1, 16) : 256;
   W.bt_units = n_lin * (W.max_d_in / 128) * (int32_t)((T + W.bt_nb - 1) / W.bt_nb);
   W.dflag = take((int64_t)n_lin * T);
   W.tmax = take((int64_t)n_lin * T * 4);
   W.bt_cnt = take((int64_t)W.bt_units * 4);
-  W.reset_bytes = off - W.dflag;
   W.bt_part = take((int64_t)2 * DC_BT_MAX_CTAS * 128 * W.bt_nb * 4);
   W.tseg = take((int64_t)T * 4);
   W.tcols = (int32_t)dc_align(max_rank > 0 ? max_rank : 1, 64) + 64 * (DC_MAX_BANDS - 1);
@@ -394,6 +394,11 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
     for (int s = (blockIdx.x - W.T) * blockDim.x + threadIdx.x; s < nseg; s += (gridDim.x - W.T) * blockDim.x)
       build_records_for(F, P, p, s);
     return;
+  }
+  if (blockIdx.y == 0) {  // this call's output bounds and backbone unit counters start from zero
+    int* cnt = reinterpret_cast<int*>(ws + W.bt_cnt);
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < W.n_lin * W.T; i += W.T * blockDim.x) P.tmax[i] = 0;
+    for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < W.bt_units; i += W.T * blockDim.x) cnt[i] = 0;
   }
   if (blockIdx.y >= (unsigned)W.n_in) return;
   const int j = blockIdx.x, m = blockIdx.y;
@@ -3243,8 +3248,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   // work counters (item count, work cursors) and per-token delta flags start from zero on every call
   st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * 4, s), "counter reset");
   if (st) return st;
-  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.dflag, 0, (size_t)F.ws.reset_bytes, s), "flag reset");
-  if (st) return st;
+  // the delta flags are written for every token by k_prep's record blocks (every token is in a
+  // segment); its limb blocks zero the output bounds and the backbone unit counters
   const int nb_items = (T + 255) / 256;
   k_prep<<<dim3(T + nb_items, std::max(n_in, n_lin)), 256, 0, s>>>(F, (uint8_t*)ws);
   prof_after(s);
