@@ -1073,7 +1073,8 @@ static_assert(U_STAGES * U_STAGE_BYTES + 2 * U_GSTAGE * U_LBUF + sizeof(USmemTai
 template <int NTOK>
 __device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, const float* tw, bool active,
                                          uint8_t* lb, int (&C)[2][4][4], float (&zc)[DC_V_TOKS],
-                                         float (&s8)[DC_V_TOKS], int ntok, int tid, int warp, int lane) {
+                                         float (&s8)[DC_V_TOKS], int ntok, int tid, int warp, int lane,
+                                         int bar) {
   const int tfl = d.tfl, nsub = active ? d.nsub : 0;
   float pe[NTOK];
 #pragma unroll
@@ -1114,7 +1115,7 @@ __device__ __forceinline__ void ud_stage(const UDesc& d, const uint8_t* stage, c
       zc[q] = fmaf(zs, tq, zc[q]);
     }
   }
-  named_bar(1, 32 * U_CONSUMERS);
+  named_bar(bar, 256);
   for (int i = 0; i < nsub; ++i) {
     const int4 sd = *reinterpret_cast<const int4*>(d.sub[i]);
     const int bits = sd.x & 15;
@@ -1308,10 +1309,11 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
   uint32_t seq = 0, unit = 0;
   for (;;) {
     const int s = seq % U_STAGES;
-    // every consumer warp waits for the stage itself; the vote makes all of them leave together
-    // when any wait ran out, so none is left at a named barrier of the stage
+    // every consumer warp waits for the stage itself; the vote makes the warps of a group slot
+    // leave together when any of their waits ran out, so none is left at a named barrier.  The two
+    // slots have their own barriers (a slot may run up to the ring's depth ahead of the other)
     const bool okw = mbar_wait(&tail->full[s], (seq / U_STAGES) & 1);
-    if (!bar_and(3, 32 * U_CONSUMERS, okw)) {
+    if (!bar_and(3 + gs, 256, okw)) {
       if (!okw) set_status(P.st, DC_ERR_CUDA);
       return;
     }
@@ -1338,11 +1340,11 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       const float* tw = reinterpret_cast<const float*>(stage + U_GSTAGE * d.code_bytes);
       // two code copies (one or two token pairs) keep the loop body small
       if (ntok <= 2)
-        ud_stage<2>(d, blocks, tw, active, lb, C, zc, s8, ntok, tid, w8, lane);
+        ud_stage<2>(d, blocks, tw, active, lb, C, zc, s8, ntok, tid, w8, lane, 1 + gs);
       else
-        ud_stage<4>(d, blocks, tw, active, lb, C, zc, s8, ntok, tid, w8, lane);
+        ud_stage<4>(d, blocks, tw, active, lb, C, zc, s8, ntok, tid, w8, lane, 1 + gs);
     } else {
-      named_bar(1, 32 * U_CONSUMERS);  // keep the stage's barrier count uniform
+      named_bar(1 + gs, 256);  // keep the stage's barrier count uniform
     }
     const bool ulast = d.ulast;
     int p = 0, go = 0, tok0 = 0;
@@ -1376,7 +1378,7 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
 #pragma unroll
       for (int q = 0; q < DC_V_TOKS; ++q) tail->s8[gs][tid - 128][q] = s8[q];
     }
-    named_bar(2, 32 * U_CONSUMERS);
+    named_bar(5 + gs, 256);
     // lane t of quad g holds columns 2t, 2t+1 of rows g and g+8 (regs 0, 1 and 2, 3).  Column 7 is
     // zero: lane 3 replaces it by column 6 (the row sum), then a 4x4 transpose inside the quad
     // leaves lane t with register t of every lane of its quad, i.e. output (row g + 8 (t >> 1),
