@@ -502,7 +502,9 @@ def run_prefill(args):
     line = {
         "metric": PREFILL_METRIC, "value": T / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 backbone, u8xs8->s32 delta", "data": "synthetic",
+        "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16xbf16->f32 backbone, f16xf16->f32 delta (segments >= 64 tokens), u8xs8->s32 delta (shorter)",
+        "data": "synthetic",
         "config": {"workload": W["name"], "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
                    "tenants_resident": W["n_tenants"], "T": T,
                    "segments": int(1 + np.count_nonzero(np.diff(ids))), "distinct_tenants": len(set(ids.tolist())),

@@ -70,11 +70,12 @@ struct DcWs {
   int32_t T, max_rank, max_d_in, n_lin, n_in, r_stride, max_items, max_tenants, nkb, pad;
   int32_t bt_nb;     // token block of the tensor-core backbone (multiple of 16, <= 256)
   int32_t bt_units;  // upper bound on its (linear, 128-row tile, token block) units
-  int32_t tcols;     // columns of the bf16 t planes: every band starts on a multiple of 64
+  int32_t tcols;     // columns of the fp16 t plane: every band starts on a multiple of 64
   int32_t pad2;
   int64_t status, perm, inv, segs, items, urecs, xl, xsort, xe, tws, yd, dflag, tmax, bt_part, bt_cnt;
   int64_t tseg;      // per tenant-sorted token: its segment
-  int64_t thl;       // bf16 t, high and low parts: [2][n_lin][T][tcols]
+  int64_t t16;       // fp16 t / 2^E(token): [n_lin][T][tcols] (prefill path)
+  int64_t xs16;      // fp16 x * 2^(14 - E(token)), tenant-sorted: [n_in][T][max_d_in] (prefill path)
   int64_t total;
 };
 

@@ -143,7 +143,8 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.bt_part = take((int64_t)2 * DC_BT_MAX_CTAS * 128 * W.bt_nb * 4);
   W.tseg = take((int64_t)T * 4);
   W.tcols = (int32_t)dc_align(max_rank > 0 ? max_rank : 1, 64) + 64 * (DC_MAX_BANDS - 1);
-  W.thl = T >= DC_PF_MIN ? take((int64_t)2 * n_lin * T * W.tcols * 2) : take(0);
+  W.t16 = T >= DC_PF_MIN ? take((int64_t)n_lin * T * W.tcols * 2) : take(0);
+  W.xs16 = T >= DC_PF_MIN ? take((int64_t)W.n_in * T * W.max_d_in * 2) : take(0);
   W.total = off;
   return W;
 }
@@ -174,8 +175,8 @@ struct DcFwd {
   int64_t bt_total;            // total chunks
   int32_t bt_ntb, bt_ns, bt_grid, bt_pad;  // token blocks, pipeline stages, CTAs
   int32_t bt_gtiles[8];        // per linear (same order): row tiles per group of the unit order
-  CUtensorMap tmap;            // prefill path: bf16 t planes [2 n_lin T rows x tcols], box 64 x 256
-  CUtensorMap xpf[3];          // prefill path: tenant-sorted activations, box 64 x pf_box tokens
+  CUtensorMap tmap;            // prefill path: fp16 t plane [n_lin T rows x tcols], box 64 x 256
+  CUtensorMap xpf[3];          // prefill path: fp16 scaled tenant-sorted activations, box 64 x pf_box
   int32_t pf;                  // segments of >= DC_PF_MIN tokens take the prefill delta path
   int32_t pf_box;              // min(256, T)
   DcWs ws;
@@ -196,7 +197,8 @@ struct WsPtr {
   uint8_t* dflag;
   int* tmax;  // per (linear, sorted token): max |t| over the 2/3-bit ranks, as fp32 bits
   int* tseg;  // per sorted token: its segment
-  __nv_bfloat16* thl;  // t as bf16 high and low parts (prefill path)
+  __half* t16;    // prefill path: t / 2^E per token as fp16
+  __half* xs16;   // prefill path: x * 2^(14 - E) per token as fp16
 };
 __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   WsPtr p;
@@ -214,7 +216,8 @@ __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   p.dflag = ws + W.dflag;
   p.tmax = (int*)(ws + W.tmax);
   p.tseg = (int*)(ws + W.tseg);
-  p.thl = (__nv_bfloat16*)(ws + W.thl);
+  p.t16 = (__half*)(ws + W.t16);
+  p.xs16 = (__half*)(ws + W.xs16);
   return p;
 }
 
@@ -438,12 +441,21 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
     e = 22 - E;      // |x| * 2^e < 2^22
   }
   uint8_t* xcol = P.xl + ((int64_t)m * W.nkb * T + j) * DC_XBLK;  // block kb at + kb * T * DC_XBLK
+  // prefill operand: x * 2^(e - 8) = x * 2^(14 - E), below 2^14 in magnitude; a bf16 value
+  // (8 significant bits) is exact in fp16 unless it is below 2^-31 max|x|
+  const float sx16 = ldexpf(1.f, e - 8);
   for (int k = tid * 4; k < d; k += 1024) {
     float v[4];
     load4(k, v);
     if (F.dtype_in == DC_DTYPE_BF16)  // tenant-sorted copy for the backbone tiles
       *reinterpret_cast<uint2*>(P.xsort + ((int64_t)(m * T + j) * maxd + k) * 2) =
           *reinterpret_cast<const uint2*>((const __nv_bfloat16*)F.x[m] + (int64_t)i * d + k);
+    if (F.pf) {
+      const __half2 h01 = __floats2half2_rn(v[0] * sx16, v[1] * sx16);
+      const __half2 h23 = __floats2half2_rn(v[2] * sx16, v[3] * sx16);
+      *reinterpret_cast<uint2*>(P.xs16 + (int64_t)(m * T + j) * maxd + k) =
+          make_uint2(*reinterpret_cast<const uint32_t*>(&h01), *reinterpret_cast<const uint32_t*>(&h23));
+    }
     uint32_t w0 = 0, w1 = 0, w2 = 0;
     int s0 = 0, s1 = 0, s2 = 0;
 #pragma unroll
@@ -1834,7 +1846,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
           const uint64_t ad = umma_desc_sw128(a0), bd = umma_desc_sw128(a0 + BT_A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)  // K = 16 per MMA: 32 bytes further inside the swizzle atom
-            umma_bf16(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (k > S.k0 || kk > 0) ? 1u : 0u);
+            umma_f16(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (k > S.k0 || kk > 0) ? 1u : 0u);
           umma_commit(smem_u32(&tail->empty[s]));  // the stage is free once these MMAs have read it
         }
         __syncwarp();
@@ -1984,47 +1996,48 @@ __device__ __forceinline__ void sw128_store(uint8_t* tile, int row, int chunk, u
   *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = v;
 }
 
-// bf16 high and low parts of (c - z) * s for 8 codes (4 bytes of r0, then 4 of r1).
-__device__ __forceinline__ void pf_dequant8(uint32_t r0, uint32_t r1, const float (&s)[8], const float (&z)[8],
-                                            uint4& hv, uint4& lv) {
-  uint32_t h[4], l[4];
+// fp16 (c - z) * s for 8 codes (4 bytes of r0, then 4 of r1); pair k covers codes 2k and 2k + 1,
+// zb[k] holds 1024 + z and s[k] the scale of each.  A byte c placed under the fp16 exponent of 1024
+// reads as 1024 + c, so one subtraction of 1024 + z gives c - z exactly (z is an integer code, both
+// terms are integers below 2048); the product is then the one rounding, to nearest even.
+__device__ __forceinline__ uint4 pf_deq16(uint32_t r0, uint32_t r1, const __half2 (&s)[4], const __half2 (&zb)[4]) {
+  const uint32_t c[4] = {__byte_perm(r0, 0x64646464u, 0x5140), __byte_perm(r0, 0x64646464u, 0x7362),
+                         __byte_perm(r1, 0x64646464u, 0x5140), __byte_perm(r1, 0x64646464u, 0x7362)};
+  uint32_t h[4];
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
-    float v[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int idx = 2 * k + e;
-      const uint32_t c = ((idx < 4 ? r0 : r1) >> (8 * (idx & 3))) & 0xffu;
-      v[e] = ((float)c - z[idx]) * s[idx];
-    }
-    const __nv_bfloat162 hb = __floats2bfloat162_rn(v[0], v[1]);
-    const float2 hf = __bfloat1622float2(hb);
-    const __nv_bfloat162 lb = __floats2bfloat162_rn(v[0] - hf.x, v[1] - hf.y);
-    h[k] = *reinterpret_cast<const uint32_t*>(&hb);
-    l[k] = *reinterpret_cast<const uint32_t*>(&lb);
+    const __half2 v = __hmul2(__hsub2(*reinterpret_cast<const __half2*>(&c[k]), zb[k]), s[k]);
+    h[k] = *reinterpret_cast<const uint32_t*>(&v);
   }
-  hv = make_uint4(h[0], h[1], h[2], h[3]);
-  lv = make_uint4(l[0], l[1], l[2], l[3]);
+  return make_uint4(h[0], h[1], h[2], h[3]);
+}
+
+// (1024 + z, scale) of a stored (scale, zero) pair, both halves of each result the same.
+__device__ __forceinline__ void pf_meta_bcast(__half2 mz, __half2& s2, __half2& zb2) {
+  s2 = __low2half2(mz);
+  zb2 = __hadd2(__high2half2(mz), __float2half2_rn(1024.f));
 }
 
 // ---------------------------------------------------------------------------------------------
 // k_upre: ydelta = U_hat t for segments of at least DC_PF_MIN tokens, on tcgen05.
 // Unit = (linear p, long segment, 128-row output group go); the segment's tokens are taken in
 // tiles of up to 256 (the MMA N).  K = the tenant's ranks, band by band, in chunks of 64.
-//   warp 0     TMA: per chunk the t planes (hi, lo: 256 tokens x 64 ranks each); per U block the
-//              block's bytes (codes of the eight 16-row tiles + meta) into a two-slot ring
+// Both operands are fp16: U_hat as the fp16 rounding of (c - z) * scale, and t scaled per token
+// by 2^-E (2^E > max |x| of the token), which the epilogue undoes.
+//   warp 0     TMA: per chunk the t plane tile (256 tokens x 64 ranks); per U block the block's
+//              bytes (codes of the eight 16-row tiles + meta) into a two-slot ring
 //   warps 1-8  expansion (one 16-row tile each): (c - z) * scale of the chunk's 128 x 64 codes
-//              as bf16 hi and lo (128-byte-swizzled K-major tiles), from the staged block
-//   warp 9     TMEM owner and MMA issuer: D[row][token] += Uhi thi + Uhi tlo + Ulo thi
-//              (M 128, N tokens, K 16 per instruction), two accumulators
-//   warps 10-13 epilogue: TMEM lane = output row, writes ydelta
+//              as fp16 (a 128-byte-swizzled K-major tile), from the staged block
+//   warp 9     TMEM owner and MMA issuer: D[row][token] += U_hat t (M 128, N tokens, K 16 per
+//              instruction), two accumulators
+//   warps 10-13 epilogue: TMEM lane = output row, writes ydelta = D * 2^E
 // Units are dealt to the persistent CTAs round robin; every wait is bounded.
 // ---------------------------------------------------------------------------------------------
 #define UP_THREADS 448
-#define UP_A_BYTES 16384                  // 128 rows x 64 bf16
-#define UP_B_BYTES 32768                  // 256 tokens x 64 bf16
-#define UP_STAGE_BYTES (2 * UP_A_BYTES + 2 * UP_B_BYTES)
-#define UP_STAGES 2
+#define UP_A_BYTES 16384                  // 128 rows x 64 fp16
+#define UP_B_BYTES 32768                  // 256 tokens x 64 fp16
+#define UP_STAGE_BYTES (UP_A_BYTES + UP_B_BYTES)
+#define UP_STAGES 4
 #define UP_BLK_BYTES 13312                // largest U block (3-bit, 8 steps, with meta)
 #define UP_MAX_LONG 256
 
@@ -2038,6 +2051,9 @@ struct UpTail {
   int lseg[UP_MAX_LONG];
   DcURec rec[UP_THREADS / 32];  // each warp's copy of its current unit's record
 };
+
+static_assert(1024 + UP_STAGES * UP_STAGE_BYTES + 2 * UP_BLK_BYTES + sizeof(UpTail) <= 232448,
+              "k_upre shared memory exceeds the 227 KB a block may use");
 
 struct UpChunk {
   int b, c0;   // band, first band-relative rank of the chunk
@@ -2090,9 +2106,9 @@ __device__ __forceinline__ bool up_unit(const DcFwd& F, int nlong, int u, int& p
 }
 
 // Expand ranks [c0, c0 + 64) of band UB for the 16-row tile `tile` of the staged block `blk`
-// (block k of the band) into the bf16 tiles ahi / alo (rows 16 tile + g and + g + 8).
+// (block k of the band) into the fp16 tile `at` (rows 16 tile + g and + g + 8).
 __device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand& UB, int k, int c0, int tile,
-                                               int lane, uint8_t* ahi, uint8_t* alo) {
+                                               int lane, uint8_t* at) {
   const int g = lane >> 2, t = lane & 3;
   const DcBand B = up_band(UB);
   const DcUBlk K = dc_u_block(B, k);
@@ -2100,9 +2116,9 @@ __device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand
   for (int s = 0; s < 2; ++s) {
     const int rs = c0 + 32 * s;  // first band-relative rank of the step
     uint32_t a[4] = {0u, 0u, 0u, 0u};
-    float sc[8], zz[8];
+    __half2 mz[8];  // (scale, zero) of ranks rs + 8 t + e; zero for ranks past the band
 #pragma unroll
-    for (int e = 0; e < 8; ++e) sc[e] = zz[e] = 0.f;
+    for (int e = 0; e < 8; ++e) mz[e] = __float2half2_rn(0.f);
     if (rs < UB.rank) {
       if (UB.bits == 8) {
 #pragma unroll
@@ -2141,20 +2157,17 @@ __device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
         const int i = rs + 8 * t + e;
-        if (i < UB.rank) {
-          const __half2 mz = *reinterpret_cast<const __half2*>(meta + 4 * (i - K.rr0));
-          sc[e] = __low2float(mz);
-          zz[e] = __high2float(mz);
-        }
+        if (i < UB.rank) mz[e] = *reinterpret_cast<const __half2*>(meta + 4 * (i - K.rr0));
       }
     }
-    uint4 hv, lv;
-    pf_dequant8(a[0], a[2], sc, zz, hv, lv);  // row g: ranks 8t .. 8t + 7
-    sw128_store(ahi, 16 * tile + g, 4 * s + t, hv);
-    sw128_store(alo, 16 * tile + g, 4 * s + t, lv);
-    pf_dequant8(a[1], a[3], sc, zz, hv, lv);  // row g + 8
-    sw128_store(ahi, 16 * tile + g + 8, 4 * s + t, hv);
-    sw128_store(alo, 16 * tile + g + 8, 4 * s + t, lv);
+    __half2 s2[4], zb2[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      s2[q] = __lows2half2(mz[2 * q], mz[2 * q + 1]);
+      zb2[q] = __hadd2(__highs2half2(mz[2 * q], mz[2 * q + 1]), __float2half2_rn(1024.f));
+    }
+    sw128_store(at, 16 * tile + g, 4 * s + t, pf_deq16(a[0], a[2], s2, zb2));      // row g: ranks 8t .. 8t + 7
+    sw128_store(at, 16 * tile + g + 8, 4 * s + t, pf_deq16(a[1], a[3], s2, zb2));  // row g + 8
   }
 }
 
@@ -2253,7 +2266,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
   int p = 0, go = 0, tok0 = 0, ntok = 0;
   const DcURec* R = nullptr;
   if (warp == 0) {
-    // ---------------- TMA producer: t planes per chunk, U blocks into the ring
+    // ---------------- TMA producer: t plane tiles per chunk, U blocks into the ring
     uint32_t seq = 0, bseq = 0;
     while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
       const uint8_t* run = reinterpret_cast<const uint8_t*>(R->blob) + R->u_off + (int64_t)go * R->u_unit;
@@ -2277,12 +2290,10 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
         const int s = seq % UP_STAGES;
         if (seq >= UP_STAGES && !up_wait(&tail->empty[s], ((seq / UP_STAGES) - 1) & 1, tail, P.st)) break;
         if (lane == 0) {
-          uint8_t* st = sm + (size_t)s * UP_STAGE_BYTES + 2 * UP_A_BYTES;
+          uint8_t* st = sm + (size_t)s * UP_STAGE_BYTES + UP_A_BYTES;
           const int col = pf_band_col(*R, C.b) + C.c0;
-          const int row = p * T + tok0;
-          mbar_arrive_expect_tx(&tail->full_b[s], (uint32_t)(2 * UP_B_BYTES));
-          tma_load_2d(st, &F.tmap, col, row, &tail->full_b[s]);
-          tma_load_2d(st + UP_B_BYTES, &F.tmap, col, F.n_lin * T + row, &tail->full_b[s]);
+          mbar_arrive_expect_tx(&tail->full_b[s], (uint32_t)UP_B_BYTES);
+          tma_load_2d(st, &F.tmap, col, p * T + tok0, &tail->full_b[s]);
         }
         __syncwarp();
       }
@@ -2313,10 +2324,9 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
           ok = false;
           break;
         }
-        uint8_t* ahi = sm + (size_t)s * UP_STAGE_BYTES;
         const uint8_t* blk = blkring + ((bseq - 1) & 1) * UP_BLK_BYTES;
         const DcUBand UB = R->band[C.b];
-        up_expand_tile(blk, UB, C.k, C.c0, e, lane, ahi, ahi + UP_A_BYTES);
+        up_expand_tile(blk, UB, C.k, C.c0, e, lane, sm + (size_t)s * UP_STAGE_BYTES);
         fence_proxy_async();  // generic-proxy writes -> tensor-core (async proxy) reads
         __syncwarp();
         if (lane == 0) mbar_arrive(&tail->full_a[s]);
@@ -2330,7 +2340,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
     uint32_t seq = 0, unit = 0;
     while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
       const int N = (ntok + 15) & ~15;
-      const uint32_t idesc = umma_idesc_bf16(128, N);
+      const uint32_t idesc = umma_idesc_f16(128, N);
       const int b = unit & 1;
       if (unit >= 2 && !up_wait(&tail->acc_empty[b], ((unit >> 1) - 1) & 1, tail, P.st)) break;
       tc_fence_after();
@@ -2347,14 +2357,11 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
         tc_fence_after();
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sm + (size_t)s * UP_STAGE_BYTES);
-          const uint64_t ah = umma_desc_sw128(a0), al = umma_desc_sw128(a0 + UP_A_BYTES);
-          const uint64_t bh = umma_desc_sw128(a0 + 2 * UP_A_BYTES), bl = umma_desc_sw128(a0 + 2 * UP_A_BYTES + UP_B_BYTES);
+          const uint64_t ad = umma_desc_sw128(a0), bd = umma_desc_sw128(a0 + UP_A_BYTES);
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk) {
             const uint64_t o = (uint64_t)(2 * kk);  // 32 bytes further inside the swizzle atom
-            umma_bf16(dt, ah + o, bh + o, idesc, (ci > 0 || kk > 0) ? 1u : 0u);
-            umma_bf16(dt, ah + o, bl + o, idesc, 1u);
-            umma_bf16(dt, al + o, bh + o, idesc, 1u);
+            umma_f16(dt, ad + o, bd + o, idesc, (ci > 0 || kk > 0) ? 1u : 0u);
           }
           umma_commit(smem_u32(&tail->empty[s]));
         }
@@ -2376,13 +2383,18 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
       tc_fence_after();
       const uint32_t ta = tbase + ((uint32_t)(32 * q4) << 16) + (uint32_t)(b * 256);
       float* yd = P.yd + ((int64_t)p * T + tok0) * F.ws.max_d_in + 128 * go + row;
+      const int* xe = P.xe + F.lin[p].input * T + tok0;  // e = 22 - E per token
       for (int cb = 0; cb < ntok; cb += 16) {
         uint32_t r[16];
         tmem_ld16(ta + cb, r);
+        // lane l < 16 holds 2^E of token cb + l
+        const float pe = (lane < 16 && cb + lane < ntok) ? ldexpf(1.f, 22 - xe[cb + lane]) : 0.f;
         tmem_ld_wait();
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj)
-          if (cb + jj < ntok) yd[(int64_t)(cb + jj) * F.ws.max_d_in] = __uint_as_float(r[jj]);
+        for (int jj = 0; jj < 16; ++jj) {
+          const float sc = __shfl_sync(FULLMASK, pe, jj);
+          if (cb + jj < ntok) yd[(int64_t)(cb + jj) * F.ws.max_d_in] = __uint_as_float(r[jj]) * sc;
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -2402,17 +2414,19 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
 // k_vpre: t = S * (V_hat^T x) for segments of at least DC_PF_MIN tokens, on tcgen05.
 // Unit = (linear p, long segment, V group of the tenant: up to 8 tiles of 16 ranks of one band);
 // the segment's tokens in tiles of up to 256 (the MMA N).  K = d_in in chunks of 64 columns.
+// Both operands are fp16: V_hat as the fp16 rounding of (c - z) * scale, and the token's x scaled
+// by 2^(14 - E) (2^E > max |x|), written by the prep kernel and exact for bf16 inputs.
 //   warp 0      TMA: per chunk the activation tile (256 tenant-sorted tokens x 64); per 512-column
 //               block the group's V block (codes + meta of its tiles) into a two-slot ring
-//   warps 1-8   expansion: (c - z) * scale of the chunk's 128 ranks x 64 columns as bf16 hi/lo
-//   warp 9      TMEM owner and MMA issuer: D[rank][token] += Vhi x + Vlo x (M 128, K 16)
-//   warps 10-13 epilogue: t = S * D into the fp32 t rows and the bf16 t planes
+//   warps 1-8   expansion: (c - z) * scale of the chunk's 128 ranks x 64 columns as fp16
+//   warp 9      TMEM owner and MMA issuer: D[rank][token] += V_hat x (M 128, K 16)
+//   warps 10-13 epilogue: the fp16 t plane, S * D * 2^-14 = t / 2^E, read by k_upre
 // ---------------------------------------------------------------------------------------------
 #define VP_THREADS 448
-#define VP_A_BYTES 16384  // 128 ranks x 64 bf16
-#define VP_B_BYTES 32768  // 256 tokens x 64 bf16
-#define VP_STAGE_BYTES (2 * VP_A_BYTES + VP_B_BYTES)
-#define VP_STAGES 2
+#define VP_A_BYTES 16384  // 128 ranks x 64 fp16
+#define VP_B_BYTES 32768  // 256 tokens x 64 fp16
+#define VP_STAGE_BYTES (VP_A_BYTES + VP_B_BYTES)
+#define VP_STAGES 3
 #define VP_BLK_BYTES 18432  // largest V group block (2-bit: 8 tiles x 2304 bytes)
 #define VP_MAX_PJ 512
 
@@ -2426,6 +2440,9 @@ struct VpTail {
   int lseg[UP_MAX_LONG];
   int pref[VP_MAX_PJ + 1];  // units (V groups) before each (linear slot, long segment) pair
 };
+
+static_assert(1024 + VP_STAGES * VP_STAGE_BYTES + 2 * VP_BLK_BYTES + sizeof(VpTail) <= 232448,
+              "k_vpre shared memory exceeds the 227 KB a block may use");
 
 // Codes of lane `ln` of half h of one (tile, block) region A, group grp: c[s][hh] holds the codes of
 // columns 32 t + 8 s + 4 hh + b (byte b), t = ln % 4.  The same extraction as the decode V kernel.
@@ -2609,7 +2626,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
             const int s = seq % VP_STAGES;
             if (seq >= VP_STAGES && !vp_wait(&tail->empty[s], ((seq / VP_STAGES) - 1) & 1, tail, P.st)) break;
             if (lane == 0) {
-              uint8_t* st = sm + (size_t)s * VP_STAGE_BYTES + 2 * VP_A_BYTES;
+              uint8_t* st = sm + (size_t)s * VP_STAGE_BYTES + VP_A_BYTES;
               mbar_arrive_expect_tx(&tail->full_b[s], (uint32_t)(box * 128));
               tma_load_2d(st, &F.xpf[m], 512 * kb + 64 * ch, tok0, &tail->full_b[s]);
             }
@@ -2646,32 +2663,23 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
             }
             const int grp = ch >> 1, hc = ch & 1;
             uint32_t c[4][2];
-            float sc[8], zz[8];
+            __half2 mz = __float2half2_rn(0.f);  // (scale, zero) of this row's group; zero: no row
             if (rows_t > 0) {
               vp_lane_codes(A, B.bits, rows_t, ngrp, h, 4 * g + 2 * hc + part, grp, c);
-              float s0 = 0.f, z0 = 0.f;
-              if (8 * h + g < rows_t) {
-                const __half2 mz = *reinterpret_cast<const __half2*>(
-                    A + dc_v_block_code_bytes(B.bits, rows_t, ngrp) + 4 * (grp * 16 + g * 2 + h));
-                s0 = __low2float(mz);
-                z0 = __high2float(mz);
-              }
-#pragma unroll
-              for (int k = 0; k < 8; ++k) sc[k] = s0, zz[k] = z0;
+              if (8 * h + g < rows_t)
+                mz = *reinterpret_cast<const __half2*>(A + dc_v_block_code_bytes(B.bits, rows_t, ngrp) +
+                                                       4 * (grp * 16 + g * 2 + h));
             } else {
 #pragma unroll
               for (int k = 0; k < 4; ++k) c[k][0] = c[k][1] = 0u;
-#pragma unroll
-              for (int k = 0; k < 8; ++k) sc[k] = zz[k] = 0.f;
             }
-            uint8_t* ahi = sm + (size_t)s * VP_STAGE_BYTES;
+            __half2 s2[4], zb2[4];
+            pf_meta_bcast(mz, s2[0], zb2[0]);
 #pragma unroll
-            for (int sidx = 0; sidx < 4; ++sidx) {
-              uint4 hv, lv;
-              pf_dequant8(c[sidx][0], c[sidx][1], sc, zz, hv, lv);
-              sw128_store(ahi, row, 4 * part + sidx, hv);
-              sw128_store(ahi + VP_A_BYTES, row, 4 * part + sidx, lv);
-            }
+            for (int k = 1; k < 4; ++k) s2[k] = s2[0], zb2[k] = zb2[0];
+            uint8_t* at = sm + (size_t)s * VP_STAGE_BYTES;
+#pragma unroll
+            for (int sidx = 0; sidx < 4; ++sidx) sw128_store(at, row, 4 * part + sidx, pf_deq16(c[sidx][0], c[sidx][1], s2, zb2));
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) mbar_arrive(&tail->full_a[s]);
@@ -2689,7 +2697,7 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
       bool ok = true;
       for (int tok0 = U.st; ok && tok0 < U.st + U.len; tok0 += 256, ++unit) {
         const int ntok = min(256, U.st + U.len - tok0);
-        const uint32_t idesc = umma_idesc_bf16(128, (ntok + 15) & ~15);
+        const uint32_t idesc = umma_idesc_f16(128, (ntok + 15) & ~15);
         const int b = unit & 1;
         if (unit >= 2 && !vp_wait(&tail->acc_empty[b], ((unit >> 1) - 1) & 1, tail, P.st)) {
           ok = false;
@@ -2710,13 +2718,11 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
             tc_fence_after();
             if (lane == 0) {
               const uint32_t a0 = smem_u32(sm + (size_t)s * VP_STAGE_BYTES);
-              const uint64_t ah = umma_desc_sw128(a0), al = umma_desc_sw128(a0 + VP_A_BYTES);
-              const uint64_t bx = umma_desc_sw128(a0 + 2 * VP_A_BYTES);
+              const uint64_t ad = umma_desc_sw128(a0), bx = umma_desc_sw128(a0 + VP_A_BYTES);
 #pragma unroll
               for (int kk = 0; kk < 4; ++kk) {
                 const uint64_t o = (uint64_t)(2 * kk);
-                umma_bf16(dt, ah + o, bx + o, idesc, (ci > 0 || kk > 0) ? 1u : 0u);
-                umma_bf16(dt, al + o, bx + o, idesc, 1u);
+                umma_f16(dt, ad + o, bx + o, idesc, (ci > 0 || kk > 0) ? 1u : 0u);
               }
               umma_commit(smem_u32(&tail->empty[s]));
             }
@@ -2738,7 +2744,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
       const DcBand& B = U.B;
       const int nvalid = min(16 * U.G.ntiles, U.G.rows_left);
       const int rank = U.G.r0 + row;
-      const float Sv = row < nvalid ? reinterpret_cast<const float*>(U.base + U.s_off)[rank] : 0.f;
+      // S * 2^-14: D carries x * 2^(14 - E), so S * D * 2^-14 = t / 2^E (scaling by 2^-14 is exact)
+      const float Sv = row < nvalid ? reinterpret_cast<const float*>(U.base + U.s_off)[rank] * 0x1p-14f : 0.f;
       const int col = U.bandcol + (rank - B.r0);
       const bool padrow = row >= nvalid && rank - B.r0 >= B.rank && rank - B.r0 < ((B.rank + 63) & ~63);
       for (int tok0 = U.st; tok0 < U.st + U.len; tok0 += 256, ++unit) {
@@ -2758,24 +2765,11 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
           tmem_ld_wait();
           if (row < nvalid) {
 #pragma unroll
-            for (int jj = 0; jj < 16; ++jj) {
-              if (cb + jj < ntok) {
-                const float t = Sv * __uint_as_float(r[jj]);
-                const int64_t tr = trow0 + cb + jj;
-                P.tws[tr * F.ws.r_stride + rank] = t;
-                const __nv_bfloat16 hb = __float2bfloat16_rn(t);
-                P.thl[tr * F.ws.tcols + col] = hb;
-                P.thl[((int64_t)F.n_lin * T + tr) * F.ws.tcols + col] = __float2bfloat16_rn(t - __bfloat162float(hb));
-              }
-            }
-          } else if (padrow) {  // zero the band's padding columns of the t planes (read by k_upre)
-            for (int jj = 0; jj < 16; ++jj) {
-              if (cb + jj < ntok) {
-                const int64_t tr = trow0 + cb + jj;
-                P.thl[tr * F.ws.tcols + col] = __float2bfloat16_rn(0.f);
-                P.thl[((int64_t)F.n_lin * T + tr) * F.ws.tcols + col] = __float2bfloat16_rn(0.f);
-              }
-            }
+            for (int jj = 0; jj < 16; ++jj)
+              if (cb + jj < ntok) P.t16[(trow0 + cb + jj) * F.ws.tcols + col] = __float2half_rn(Sv * __uint_as_float(r[jj]));
+          } else if (padrow) {  // zero the band's padding columns of the t plane (read by k_upre)
+            for (int jj = 0; jj < 16; ++jj)
+              if (cb + jj < ntok) P.t16[(trow0 + cb + jj) * F.ws.tcols + col] = __float2half_rn(0.f);
           }
         }
         tc_fence_before();
@@ -3121,17 +3115,17 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   return fn;
 }
 
-// 2-D bf16 tensor map: `rows` x `cols` (row pitch `pitch` elements), box 64 columns x box_rows rows,
-// 128-byte swizzle.
-static dc_status encode_bf16_map(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t pitch,
-                                 int box_rows) {
+// 2-D tensor map of 16-bit elements (bf16 unless `dtype` says fp16): `rows` x `cols` (row pitch
+// `pitch` elements), box 64 columns x box_rows rows, 128-byte swizzle.
+static dc_status encode_map16(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t pitch,
+                                 int box_rows, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return dc_fail(DC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)pitch * 2};
   const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
-  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+  const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return dc_fail(DC_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
@@ -3201,13 +3195,13 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   if (flags & DC_BASE) {
     for (int p = 0; p < n_lin; ++p)
       if (lins[p].w_dtype == DC_DTYPE_BF16) {
-        dc_status st0 = encode_bf16_map(&F.wmap[p], lins[p].W_base, lins[p].d_in, lins[p].d_out, lins[p].d_in, 128);
+        dc_status st0 = encode_map16(&F.wmap[p], lins[p].W_base, lins[p].d_in, lins[p].d_out, lins[p].d_in, 128);
         if (st0) return st0;
       }
     if (dtype_in == DC_DTYPE_BF16)
       for (int m = 0; m < n_in; ++m) {
         const uint8_t* xb = (const uint8_t*)ws + F.ws.xsort + (int64_t)m * T * F.ws.max_d_in * 2;
-        dc_status st0 = encode_bf16_map(&F.xmap[m], xb, dxs[m], T, F.ws.max_d_in, use_tc ? F.ws.bt_nb : std::min(64, T));
+        dc_status st0 = encode_map16(&F.xmap[m], xb, dxs[m], T, F.ws.max_d_in, use_tc ? F.ws.bt_nb : std::min(64, T));
         if (st0) return st0;
       }
   }
@@ -3224,13 +3218,13 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   F.pf = (flags & DC_DELTA) && !(flags & DC_DECODE_ONLY) && T >= 2 * DC_PF_MIN;
   if (F.pf) {
     if (dtype_in != DC_DTYPE_BF16) return dc_fail(DC_ERR_UNSUPPORTED, "the prefill path needs bf16 activations");
-    dc_status st0 = encode_bf16_map(&F.tmap, (const uint8_t*)ws + F.ws.thl, F.ws.tcols, (int64_t)2 * n_lin * T,
-                                    F.ws.tcols, 256);
+    dc_status st0 = encode_map16(&F.tmap, (const uint8_t*)ws + F.ws.t16, F.ws.tcols, (int64_t)n_lin * T,
+                                    F.ws.tcols, 256, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (st0) return st0;
     F.pf_box = std::min(256, T);
     for (int m = 0; m < n_in; ++m) {
-      const uint8_t* xb = (const uint8_t*)ws + F.ws.xsort + (int64_t)m * T * F.ws.max_d_in * 2;
-      st0 = encode_bf16_map(&F.xpf[m], xb, dxs[m], T, F.ws.max_d_in, F.pf_box);
+      const uint8_t* xb = (const uint8_t*)ws + F.ws.xs16 + (int64_t)m * T * F.ws.max_d_in * 2;
+      st0 = encode_map16(&F.xpf[m], xb, dxs[m], T, F.ws.max_d_in, F.pf_box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
       if (st0) return st0;
     }
   }

@@ -1,9 +1,9 @@
 // Fifth-generation tensor cores (tcgen05) on sm_100a: shared-memory matrix descriptors, the
-// instruction descriptor of a dense bf16 MMA, Tensor Memory (TMEM) allocation, MMA issue,
+// instruction descriptors of dense bf16 and fp16 MMAs, Tensor Memory (TMEM) allocation, MMA issue,
 // completion tracking through mbarriers, and TMEM -> register loads.
 //
-// Conventions used here: both operands are K-major tiles written by a TMA load with the
-// 128-byte swizzle (rows of 64 bf16 = 128 bytes, 8-row swizzle atoms of 1024 bytes, tile base
+// Conventions used here: both operands are K-major tiles in the 128-byte swizzle (rows of 64
+// 16-bit elements = 128 bytes, 8-row swizzle atoms of 1024 bytes, tile base
 // 1024-byte aligned).  The accumulator is fp32 in TMEM: lane = row of A (M = 128), column =
 // row of B (N).  No instruction here uses cluster multicast.
 #pragma once
@@ -30,6 +30,10 @@ __device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
 __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// The same with fp16 A and B (a_format = b_format = 0).
+__host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 
 // TMEM allocation of `ncols` columns (a power of two >= 32) by one whole warp; the base address
 // is written to shared memory at `dst_saddr`.
@@ -47,8 +51,9 @@ __device__ __forceinline__ void tmem_dealloc(uint32_t taddr, uint32_t ncols) {
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 
-// D[tmem] (+)= A * B^T for one K = 16 slice; issued by one thread.  accumulate = 0 overwrites D.
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+// D[tmem] (+)= A * B^T for one K = 16 slice of kind::f16 (both operands bf16 or both fp16, as the
+// instruction descriptor says); issued by one thread.  accumulate = 0 overwrites D.
+__device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                           uint32_t accumulate) {
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"

@@ -2,6 +2,11 @@
 tokens take the tensor-core kernels.  Checked against the fp64 oracle (full output and delta
 alone) and against the same batch forced through the decode kernels (DC_DECODE_ONLY), whose
 parity is established by test_gpu_parity.py.
+
+The prefill kernels multiply fp16 operands: U_hat and V_hat rounded to fp16 as the method's own
+fp16 dequantisation does, and t rounded to fp16.  Each rounding adds about 1.5-2e-4 relative L2
+error to the delta, about 3e-4 together (the decode kernels are exact up to fp32), so the delta
+alone is held to the parity bound 1e-3 and the full output, where the delta is 1-2 %, to 1e-4.
 """
 import numpy as np
 import pytest
@@ -16,6 +21,11 @@ pytestmark = pytest.mark.gpu
 
 if not torch.cuda.is_available():  # pragma: no cover
     pytest.skip("no CUDA device", allow_module_level=True)
+
+
+def _tol(flags):
+    """Bound on the prefill path vs the decode path (fp16 operands, see the module docstring)."""
+    return 1e-3 if not (flags & dc.DC_BASE) else 1e-4
 
 
 def _segments(lengths_tenants):
@@ -65,7 +75,7 @@ def test_prefill_path_against_oracle_and_decode_path(case, flags):
     assert np.isfinite(outs[0]).all()
     want = oracle_y(wv.astype(np.float64), td, xv.astype(np.float64), ids, flags)
     assert_close(outs[0], want, "prefill path vs oracle")
-    assert rel_l2(outs[0], outs[dc.DC_DECODE_ONLY]) <= 1e-4, "prefill path vs decode path"
+    assert rel_l2(outs[0], outs[dc.DC_DECODE_ONLY]) <= _tol(flags), "prefill path vs decode path"
 
 
 def test_prefill_13b_layer_against_decode_path():
@@ -96,4 +106,4 @@ def test_prefill_13b_layer_against_decode_path():
             a = res[(0, flags)][p].cpu().numpy().astype(np.float64)
             b = res[(dc.DC_DECODE_ONLY, flags)][p].cpu().numpy().astype(np.float64)
             assert np.isfinite(a).all()
-            assert rel_l2(a, b) <= 1e-4, (flags, p, rel_l2(a, b))
+            assert rel_l2(a, b) <= _tol(flags), (flags, p, rel_l2(a, b))
