@@ -2026,14 +2026,17 @@ __device__ __forceinline__ void pf_meta_bcast(__half2 mz, __half2& s2, __half2& 
 // by 2^-E (2^E > max |x| of the token), which the epilogue undoes.
 //   warp 0     TMA: per chunk the t plane tile (256 tokens x 64 ranks); per U block the block's
 //              bytes (codes of the eight 16-row tiles + meta) into a two-slot ring
-//   warps 1-8  expansion (one 16-row tile each): (c - z) * scale of the chunk's 128 x 64 codes
-//              as fp16 (a 128-byte-swizzled K-major tile), from the staged block
-//   warp 9     TMEM owner and MMA issuer: D[row][token] += U_hat t (M 128, N tokens, K 16 per
+//   warps 1-16 expansion, two sets of eight taking alternate chunks (one 16-row tile per warp):
+//              (c - z) * scale of the chunk's 128 x 64 codes as fp16 (a 128-byte-swizzled
+//              K-major tile), from the staged block
+//   warp 17    TMEM owner and MMA issuer: D[row][token] += U_hat t (M 128, N tokens, K 16 per
 //              instruction), two accumulators
-//   warps 10-13 epilogue: TMEM lane = output row, writes ydelta = D * 2^E
+//   warps 18-21 epilogue: TMEM lane quarter = warp % 4, writes ydelta = D * 2^E
 // Units are dealt to the persistent CTAs round robin; every wait is bounded.
 // ---------------------------------------------------------------------------------------------
-#define UP_THREADS 448
+#define UP_EXP_WARPS 16
+#define UP_MMA_WARP (1 + UP_EXP_WARPS)
+#define UP_THREADS (32 * (UP_MMA_WARP + 5))
 #define UP_A_BYTES 16384                  // 128 rows x 64 fp16
 #define UP_B_BYTES 32768                  // 256 tokens x 64 fp16
 #define UP_STAGE_BYTES (UP_A_BYTES + UP_B_BYTES)
@@ -2106,40 +2109,46 @@ __device__ __forceinline__ bool up_unit(const DcFwd& F, int nlong, int u, int& p
 }
 
 // Expand ranks [c0, c0 + 64) of band UB for the 16-row tile `tile` of the staged block `blk`
-// (block k of the band) into the fp16 tile `at` (rows 16 tile + g and + g + 8).
-__device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand& UB, int k, int c0, int tile,
-                                               int lane, uint8_t* at) {
+// (geometry K) into the fp16 tile `at` (rows 16 tile + g and + g + 8).  Only the band's last shift
+// step can be short, and it is the last step of its block, so every step of a block before it
+// starts a whole step's bytes after the previous one.
+__device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand& UB, const DcUBlk& K, int c0,
+                                               int tile, int lane, uint8_t* at) {
   const int g = lane >> 2, t = lane & 3;
-  const DcBand B = up_band(UB);
-  const DcUBlk K = dc_u_block(B, k);
+  const uint8_t* tb = blk + tile * K.tile_bytes;
+  const uint8_t* meta = blk + K.code_bytes;
+  uint32_t a[2][4];
 #pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int rs = c0 + 32 * s;  // first band-relative rank of the step
-    uint32_t a[4] = {0u, 0u, 0u, 0u};
-    __half2 mz[8];  // (scale, zero) of ranks rs + 8 t + e; zero for ranks past the band
+  for (int s = 0; s < 2; ++s)
 #pragma unroll
-    for (int e = 0; e < 8; ++e) mz[e] = __float2half2_rn(0.f);
-    if (rs < UB.rank) {
-      if (UB.bits == 8) {
+    for (int jj = 0; jj < 4; ++jj) a[s][jj] = 0u;
+  if (UB.bits == 2 && c0 < 128 * UB.quads) {  // both steps in one mask-layout quad
+    const uint4 wq = *reinterpret_cast<const uint4*>(tb + 512 * (c0 / 128 - K.q0) + 16 * lane);
+    const int ps = (c0 & 127) >> 5;  // 0 or 2
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj)
+    for (int s = 0; s < 2; ++s)
 #pragma unroll
-          for (int b = 0; b < 4; ++b) {
-            const int i = rs + 8 * t + 4 * (jj >> 1) + b;
-            const int row = 16 * tile + g + 8 * (jj & 1);
-            const uint32_t c = i < UB.rank ? blk[row * K.nr + (i - K.rr0)] : 0u;
-            a[jj] |= c << (8 * b);
-          }
-      } else if (UB.bits == 2 && rs < 128 * UB.quads) {
-        const int qb = rs / 128 - K.q0, ps = (rs % 128) / 32;
-        const uint4 wq = *reinterpret_cast<const uint4*>(blk + tile * K.tile_bytes + 512 * qb + 16 * lane);
+      for (int jj = 0; jj < 4; ++jj) a[s][jj] = (wsel(wq, jj) >> (2 * (ps + s))) & 0x03030303u;
+  } else if (UB.bits == 8) {
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) a[jj] = (wsel(wq, jj) >> (2 * ps)) & 0x03030303u;
-      } else {
-        const int si = (rs - 128 * UB.quads) / 32;  // shift-layout step of the band
-        const uint8_t* sb = blk + tile * K.tile_bytes + 512 * K.nq;
-        for (int s2 = K.s0; s2 < si; ++s2)
-          sb += dc_u_step_bytes(UB.bits, dc_u_step_lanes(s2 == UB.steps - 1 ? UB.last : 32));
+    for (int s = 0; s < 2; ++s)
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+        for (int b = 0; b < 4; ++b) {
+          const int i = c0 + 32 * s + 8 * t + 4 * (jj >> 1) + b;
+          const int row = 16 * tile + g + 8 * (jj & 1);
+          const uint32_t c = i < UB.rank ? blk[row * K.nr + (i - K.rr0)] : 0u;
+          a[s][jj] |= c << (8 * b);
+        }
+  } else {  // shift-layout steps
+    const int full_step = (int)dc_u_step_bytes(UB.bits, 32);
+#pragma unroll
+    for (int s = 0; s < 2; ++s) {
+      const int rs = c0 + 32 * s;
+      if (rs < UB.rank) {
+        const int si = (rs - 128 * UB.quads) >> 5;  // shift-layout step of the band
+        const uint8_t* sb = tb + 512 * K.nq + (si - K.s0) * full_step;
         const int valid = si == UB.steps - 1 ? UB.last : 32;
         const int nl = dc_u_step_lanes(valid), ntv = nl / 8;
         uint32_t wv = 0, hv = 0;
@@ -2149,25 +2158,34 @@ __device__ __forceinline__ void up_expand_tile(const uint8_t* blk, const DcUBand
         }
 #pragma unroll
         for (int jj = 0; jj < 4; ++jj) {
-          a[jj] = reg_shift2(wv, jj);
-          if (UB.bits == 3) a[jj] |= u_reg_hi3(hv, jj);
+          a[s][jj] = reg_shift2(wv, jj);
+          if (UB.bits == 3) a[s][jj] |= u_reg_hi3(hv, jj);
         }
       }
-      const uint8_t* meta = blk + K.code_bytes;
+    }
+  }
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const int i = rs + 8 * t + e;
-        if (i < UB.rank) mz[e] = *reinterpret_cast<const __half2*>(meta + 4 * (i - K.rr0));
-      }
+  for (int s = 0; s < 2; ++s) {
+    const int r8 = c0 + 32 * s + 8 * t;  // band-relative rank of this lane's first column
+    uint32_t mw[8];  // (scale, zero) of ranks r8 .. r8 + 7; zero past the band
+    if (r8 + 8 <= UB.rank) {
+      const uint4 m0 = *reinterpret_cast<const uint4*>(meta + 4 * (r8 - K.rr0));
+      const uint4 m1 = *reinterpret_cast<const uint4*>(meta + 4 * (r8 - K.rr0) + 16);
+      mw[0] = m0.x, mw[1] = m0.y, mw[2] = m0.z, mw[3] = m0.w, mw[4] = m1.x, mw[5] = m1.y, mw[6] = m1.z, mw[7] = m1.w;
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mw[e] = r8 + e < UB.rank ? *reinterpret_cast<const uint32_t*>(meta + 4 * (r8 + e - K.rr0)) : 0u;
     }
     __half2 s2[4], zb2[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      s2[q] = __lows2half2(mz[2 * q], mz[2 * q + 1]);
-      zb2[q] = __hadd2(__highs2half2(mz[2 * q], mz[2 * q + 1]), __float2half2_rn(1024.f));
+      const uint32_t sp = __byte_perm(mw[2 * q], mw[2 * q + 1], 0x5410);  // the two scales
+      const uint32_t zp = __byte_perm(mw[2 * q], mw[2 * q + 1], 0x7632);  // the two zeros
+      s2[q] = *reinterpret_cast<const __half2*>(&sp);
+      zb2[q] = __hadd2(*reinterpret_cast<const __half2*>(&zp), __float2half2_rn(1024.f));
     }
-    sw128_store(at, 16 * tile + g, 4 * s + t, pf_deq16(a[0], a[2], s2, zb2));      // row g: ranks 8t .. 8t + 7
-    sw128_store(at, 16 * tile + g + 8, 4 * s + t, pf_deq16(a[1], a[3], s2, zb2));  // row g + 8
+    sw128_store(at, 16 * tile + g, 4 * s + t, pf_deq16(a[s][0], a[s][2], s2, zb2));      // row g: ranks 8t .. 8t + 7
+    sw128_store(at, 16 * tile + g + 8, 4 * s + t, pf_deq16(a[s][1], a[s][3], s2, zb2));  // row g + 8
   }
 }
 
@@ -2242,7 +2260,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&tail->blk_full[b], 1);
-      mbar_init(&tail->blk_empty[b], 8);
+      mbar_init(&tail->blk_empty[b], UP_EXP_WARPS);
       mbar_init(&tail->acc_full[b], 1);
       mbar_init(&tail->acc_empty[b], 4);
     }
@@ -2254,7 +2272,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
     tail->nlong = n;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == UP_MMA_WARP) {
     tmem_alloc(smem_u32(&tail->tmem_base), 512);
     tmem_relinquish();
   }
@@ -2298,13 +2316,15 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
         __syncwarp();
       }
     }
-  } else if (warp <= 8) {
-    // ---------------- expansion warps: warp w expands the 16-row tile w - 1
-    const int e = warp - 1;
+  } else if (warp <= UP_EXP_WARPS) {
+    // ---------------- expansion warps: warp w expands the 16-row tile (w - 1) % 8 of the chunks
+    // whose sequence number has the parity (w - 1) / 8; every warp takes every block
+    const int e = (warp - 1) & 7, set = (warp - 1) >> 3;
     uint32_t seq = 0, bseq = 0;
     while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
       int lb = -1, lk = -1;
       UpChunk C;
+      DcUBlk K;
       bool ok = true;
       for (int ci = 0; up_chunk(*R, ci, C); ++ci, ++seq) {
         if (C.b != lb || C.k != lk) {
@@ -2313,20 +2333,21 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
             if (lane == 0) mbar_arrive(&tail->blk_empty[(bseq - 1) & 1]);
           }
           lb = C.b, lk = C.k;
+          K = dc_u_block(up_band(R->band[C.b]), C.k);
           if (!up_wait(&tail->blk_full[bseq & 1], (bseq >> 1) & 1, tail, P.st)) {
             ok = false;
             break;
           }
           ++bseq;
         }
+        if ((int)(seq & 1) != set) continue;  // the other set expands this chunk
         const int s = seq % UP_STAGES;
         if (seq >= UP_STAGES && !up_wait(&tail->empty[s], ((seq / UP_STAGES) - 1) & 1, tail, P.st)) {
           ok = false;
           break;
         }
         const uint8_t* blk = blkring + ((bseq - 1) & 1) * UP_BLK_BYTES;
-        const DcUBand UB = R->band[C.b];
-        up_expand_tile(blk, UB, C.k, C.c0, e, lane, sm + (size_t)s * UP_STAGE_BYTES);
+        up_expand_tile(blk, R->band[C.b], K, C.c0, e, lane, sm + (size_t)s * UP_STAGE_BYTES);
         fence_proxy_async();  // generic-proxy writes -> tensor-core (async proxy) reads
         __syncwarp();
         if (lane == 0) mbar_arrive(&tail->full_a[s]);
@@ -2335,7 +2356,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
       __syncwarp();
       if (lb >= 0 && lane == 0) mbar_arrive(&tail->blk_empty[(bseq - 1) & 1]);
     }
-  } else if (warp == 9) {
+  } else if (warp == UP_MMA_WARP) {
     // ---------------- MMA issuer
     uint32_t seq = 0, unit = 0;
     while (!up_aborted(tail) && up_next(F, P, tail, it, p, go, R, tok0, ntok)) {
@@ -2404,7 +2425,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == UP_MMA_WARP) {
     tc_fence_after();
     tmem_dealloc(tbase, 512);
   }
