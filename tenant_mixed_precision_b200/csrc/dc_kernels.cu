@@ -2450,11 +2450,16 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
 #define VP_STAGES 3
 #define VP_BLK_BYTES 18432  // largest V group block (2-bit: 8 tiles x 2304 bytes)
 #define VP_MAX_PJ 512
+#define VP_UQ 4                                // slots of the unit ring
+#define VP_COUNTER_SLOT 6                      // status word: next unit to claim (zeroed per call)
+#define VP_TAKERS (VP_THREADS / 32 - 1)        // warps that read the unit ring
 
 struct VpTail {
   uint64_t full_b[VP_STAGES], full_a[VP_STAGES], empty[VP_STAGES];
   uint64_t blk_full[2], blk_empty[2];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t uq_full[VP_UQ], uq_empty[VP_UQ];
+  int uq[VP_UQ];  // units claimed by the producer, in order
   uint32_t tmem_base;
   int abort;
   int nlong, npj, box;
@@ -2513,6 +2518,31 @@ __device__ __forceinline__ bool vp_wait(uint64_t* bar, uint32_t parity, VpTail* 
   tail->abort = 1;
   set_status(st, DC_ERR_CUDA);
   return false;
+}
+
+// Units are claimed dynamically, largest first (linears by d_in, longest first): the producer warp
+// takes the next unit index from a global counter and posts it in a ring; the other warps take
+// the same sequence from the ring.  A failed wait returns an index past the last unit.
+__device__ __forceinline__ int vp_claim(VpTail* tail, const WsPtr& P, uint32_t& k) {
+  const int slot = k % VP_UQ;
+  if (k >= VP_UQ && !vp_wait(&tail->uq_empty[slot], ((k / VP_UQ) - 1) & 1, tail, P.st)) return 1 << 30;
+  int u = 0;
+  if ((threadIdx.x & 31) == 0) {
+    u = atomicAdd(P.st + VP_COUNTER_SLOT, 1);
+    tail->uq[slot] = u;
+    mbar_arrive(&tail->uq_full[slot]);
+  }
+  ++k;
+  return __shfl_sync(FULLMASK, u, 0);
+}
+__device__ __forceinline__ int vp_take(VpTail* tail, const WsPtr& P, uint32_t& k) {
+  const int slot = k % VP_UQ;
+  if (!vp_wait(&tail->uq_full[slot], (k / VP_UQ) & 1, tail, P.st)) return 1 << 30;
+  const int u = *reinterpret_cast<volatile int*>(&tail->uq[slot]);
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(&tail->uq_empty[slot]);
+  ++k;
+  return u;
 }
 
 // A V group: band b, group index inside the band, its tiles and first rank.
@@ -2586,6 +2616,10 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
       mbar_init(&tail->acc_full[b], 1);
       mbar_init(&tail->acc_empty[b], 4);
     }
+    for (int q = 0; q < VP_UQ; ++q) {
+      mbar_init(&tail->uq_full[q], 1);
+      mbar_init(&tail->uq_empty[q], VP_TAKERS);
+    }
     tail->abort = 0;
     const int nseg = P.st[DC_WS_NSEG];
     int n = 0;
@@ -2624,8 +2658,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
   VpUnit U;
   if (warp == 0) {
     // ---------------- TMA producer
-    uint32_t seq = 0, bseq = 0;
-    for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+    uint32_t seq = 0, bseq = 0, kq = 0;
+    for (int u = vp_claim(tail, P, kq); !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u = vp_claim(tail, P, kq)) {
       const DcBand& B = U.B;
       const int m = F.lin[U.p].input;
       for (int tok0 = U.st; tok0 < U.st + U.len && !vp_aborted(tail); tok0 += 256) {
@@ -2661,8 +2695,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
     const int e = threadIdx.x - 32;
     const int row = e & 127, part = e >> 7;
     const int tile = row >> 4, h = (row >> 3) & 1, g = row & 7;
-    uint32_t seq = 0, bseq = 0;
-    for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+    uint32_t seq = 0, bseq = 0, kq = 0;
+    for (int u = vp_take(tail, P, kq); !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u = vp_take(tail, P, kq)) {
       const DcBand& B = U.B;
       const int rows_t = tile < U.G.ntiles ? min(16, U.G.rows_left - 16 * tile) : 0;
       bool ok = true;
@@ -2713,8 +2747,8 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
     }
   } else if (warp == 9) {
     // ---------------- MMA issuer
-    uint32_t seq = 0, unit = 0;
-    for (int u = blockIdx.x; !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+    uint32_t seq = 0, unit = 0, kq = 0;
+    for (int u = vp_take(tail, P, kq); !vp_aborted(tail) && vp_unit(F, P, tail, u, U); u = vp_take(tail, P, kq)) {
       bool ok = true;
       for (int tok0 = U.st; ok && tok0 < U.st + U.len; tok0 += 256, ++unit) {
         const int ntok = min(256, U.st + U.len - tok0);
@@ -2759,9 +2793,9 @@ __global__ void __launch_bounds__(VP_THREADS, 1) k_vpre(const __grid_constant__ 
   } else {
     // ---------------- epilogue warps 10-13 (TMEM lane quarter warp % 4); exits agreed by a vote
     const int q4 = warp & 3, row = 32 * q4 + lane;
-    uint32_t unit = 0;
+    uint32_t unit = 0, kq = 0;
     bool go_on = true;
-    for (int u = blockIdx.x; go_on && vp_unit(F, P, tail, u, U); u += gridDim.x) {
+    for (int u = vp_take(tail, P, kq); go_on && vp_unit(F, P, tail, u, U); u = vp_take(tail, P, kq)) {
       const DcBand& B = U.B;
       const int nvalid = min(16 * U.G.ntiles, U.G.rows_left);
       const int rank = U.G.r0 + row;
@@ -3263,7 +3297,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   }
   prof_before(s, 1);
   // work counters (item count, work cursors) and per-token delta flags start from zero on every call
-  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * 4, s), "counter reset");
+  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * (VP_COUNTER_SLOT - DC_WS_VCOUNTER + 1), s),
+                     "counter reset");
   if (st) return st;
   // the delta flags are written for every token by k_prep's record blocks (every token is in a
   // segment); its limb blocks zero the output bounds and the backbone unit counters
