@@ -153,7 +153,8 @@ dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int32_t n, void
  * most max_tenants tenants (n_linears = 1 or 7).  The workspace holds the routing result, the
  * per-token activation limbs, the rank-reduction results and the device status word.  The same
  * arguments must be passed to the calls that use the workspace (through dc_linear.max_rank and
- * the batch size); a workspace smaller than this gives DC_ERR_WORKSPACE. */
+ * the batch size); a workspace smaller than this gives DC_ERR_WORKSPACE.  For T >= 64 it also
+ * holds the prefill path's fp16 activation and t planes. */
 size_t dc_workspace_size(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_linears,
                          int32_t max_tenants);
 
@@ -175,7 +176,14 @@ dc_status dc_read_segments(const void* ws, int32_t T, int32_t* perm_dev, int32_t
 
 /* y[T, d_out] = (flags & DC_BASE ? W_base x : 0) + (flags & DC_DELTA ? U_hat (S * V_hat^T x) : 0)
  * for every token with its own tenant.  x: device [T, d_in] of dtype_in; y: device [T, d_out]
- * of dtype_out (F32 or BF16).  Runs dc_build_segments itself.  T >= 0 (T = 0 is a no-op). */
+ * of dtype_out (F32 or BF16).  Runs dc_build_segments itself.  T >= 0 (T = 0 is a no-op).
+ * Arithmetic of the delta: a tenant with 64 or more tokens in a batch of at least 128 tokens
+ * takes the tensor-core prefill path, which needs BF16 activations.  It multiplies fp16
+ * operands: U_hat and V_hat rounded to fp16, x and t scaled per token by a power of two, t
+ * rounded to fp16.  That is about 3e-4 relative L2 error on the delta.  Every other token (and
+ * every token with DC_DECODE_ONLY) is exact up to fp32: integer tensor-core products of the
+ * codes, scales and zeros applied in fp32.  The backbone multiplies bf16 operands (or fp32 for
+ * an F32 W_base) with fp32 accumulation. */
 dc_status dc_delta_linear_segmented(const dc_linear* lin, const void* x, void* y,
                                     const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
                                     int32_t dtype_out, int32_t flags, void* ws, size_t ws_bytes,
