@@ -2044,10 +2044,16 @@ __device__ __forceinline__ void pf_meta_bcast(__half2 mz, __half2& s2, __half2& 
 #define UP_BLK_BYTES 13312                // largest U block (3-bit, 8 steps, with meta)
 #define UP_MAX_LONG 256
 
+#define UP_UQ 4                          // slots of the unit ring
+#define UP_COUNTER_SLOT 7                // status word: next unit to claim (zeroed per call)
+#define UP_TAKERS (UP_THREADS / 32 - 1)  // warps that read the unit ring
+
 struct UpTail {
   uint64_t full_b[UP_STAGES], full_a[UP_STAGES], empty[UP_STAGES];
   uint64_t blk_full[2], blk_empty[2];
   uint64_t acc_full[2], acc_empty[2];
+  uint64_t uq_full[UP_UQ], uq_empty[UP_UQ];
+  int uq[UP_UQ];  // units claimed by the producer, in order
   uint32_t tmem_base;
   int abort;
   int nlong;
@@ -2201,7 +2207,8 @@ __device__ __forceinline__ bool up_wait(uint64_t* bar, uint32_t parity, UpTail* 
 
 // Next (unit, token tile) of this CTA's sequence; the same for every role.
 struct UpIter {
-  int u, tt;  // current unit (-1 before the first) and token tile
+  int u, tt;    // current unit (-1 before the first) and token tile
+  uint32_t kq;  // units taken from the ring so far
 };
 // The unit's record is copied into the calling warp's slot in shared memory (R points there).
 __device__ __forceinline__ void up_load_rec(const DcURec* src, DcURec* dst) {
@@ -2210,6 +2217,30 @@ __device__ __forceinline__ void up_load_rec(const DcURec* src, DcURec* dst) {
   __syncwarp();
   if (lane < NV) reinterpret_cast<uint4*>(dst)[lane] = ldg128(reinterpret_cast<const uint8_t*>(src) + 16 * lane);
   __syncwarp();
+}
+
+// Units are claimed dynamically: the producer warp takes the next unit index from a global counter
+// and posts it in a ring; the other warps take the same sequence from the ring.  A failed wait
+// gives an index past the last unit.
+__device__ __forceinline__ int up_unit_index(const WsPtr& P, UpTail* tail, uint32_t& k) {
+  const int slot = k % UP_UQ;
+  int u = 1 << 30;
+  if (threadIdx.x < 32) {  // producer warp: claim
+    if (k >= UP_UQ && !up_wait(&tail->uq_empty[slot], ((k / UP_UQ) - 1) & 1, tail, P.st)) return u;
+    if (threadIdx.x == 0) {
+      u = atomicAdd(P.st + UP_COUNTER_SLOT, 1);
+      tail->uq[slot] = u;
+      mbar_arrive(&tail->uq_full[slot]);
+    }
+    u = __shfl_sync(FULLMASK, u, 0);
+  } else {
+    if (!up_wait(&tail->uq_full[slot], (k / UP_UQ) & 1, tail, P.st)) return u;
+    u = *reinterpret_cast<volatile int*>(&tail->uq[slot]);
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&tail->uq_empty[slot]);
+  }
+  ++k;
+  return u;
 }
 
 __device__ __forceinline__ bool up_next(const DcFwd& F, const WsPtr& P, UpTail* tail, UpIter& it, int& p,
@@ -2225,10 +2256,8 @@ __device__ __forceinline__ bool up_next(const DcFwd& F, const WsPtr& P, UpTail* 
         ntok = min(256, R->st + R->len - tok0);
         return true;
       }
-      it.u += gridDim.x;
-    } else {
-      it.u = blockIdx.x;
     }
+    it.u = up_unit_index(P, tail, it.kq);
     it.tt = 0;
     int j;
     if (!up_unit(F, tail->nlong, it.u, p, j, go)) return false;
@@ -2264,6 +2293,10 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
       mbar_init(&tail->acc_full[b], 1);
       mbar_init(&tail->acc_empty[b], 4);
     }
+    for (int q = 0; q < UP_UQ; ++q) {
+      mbar_init(&tail->uq_full[q], 1);
+      mbar_init(&tail->uq_empty[q], UP_TAKERS);
+    }
     tail->abort = 0;
     const int nseg = P.st[DC_WS_NSEG];  // long segments, in segment order
     int n = 0;
@@ -2280,7 +2313,7 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = tail->tmem_base;
-  UpIter it{-1, 0};
+  UpIter it{-1, 0, 0u};
   int p = 0, go = 0, tok0 = 0, ntok = 0;
   const DcURec* R = nullptr;
   if (warp == 0) {
@@ -3297,7 +3330,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   }
   prof_before(s, 1);
   // work counters (item count, work cursors) and per-token delta flags start from zero on every call
-  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * (VP_COUNTER_SLOT - DC_WS_VCOUNTER + 1), s),
+  static_assert(VP_COUNTER_SLOT < UP_COUNTER_SLOT && UP_COUNTER_SLOT < DC_WS_SLOTS, "status words");
+  st = dc_cuda_check(cudaMemsetAsync((uint8_t*)ws + F.ws.status + 4 * DC_WS_VCOUNTER, 0, 4 * (UP_COUNTER_SLOT - DC_WS_VCOUNTER + 1), s),
                      "counter reset");
   if (st) return st;
   // the delta flags are written for every token by k_prep's record blocks (every token is in a
