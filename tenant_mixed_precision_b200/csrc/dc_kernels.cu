@@ -2032,7 +2032,8 @@ __device__ __forceinline__ void pf_meta_bcast(__half2 mz, __half2& s2, __half2& 
 //   warp 17    TMEM owner and MMA issuer: D[row][token] += U_hat t (M 128, N tokens, K 16 per
 //              instruction), two accumulators
 //   warps 18-21 epilogue: TMEM lane quarter = warp % 4, writes ydelta = D * 2^E
-// Units are dealt to the persistent CTAs round robin; every wait is bounded.
+// Units are claimed dynamically (a global counter, posted to every warp through a shared-memory
+// ring); every wait is bounded.
 // ---------------------------------------------------------------------------------------------
 #define UP_EXP_WARPS 16
 #define UP_MMA_WARP (1 + UP_EXP_WARPS)
@@ -2475,6 +2476,8 @@ __global__ void __launch_bounds__(UP_THREADS, 1) k_upre(const __grid_constant__ 
 //   warps 1-8   expansion: (c - z) * scale of the chunk's 128 ranks x 64 columns as fp16
 //   warp 9      TMEM owner and MMA issuer: D[rank][token] += V_hat x (M 128, K 16)
 //   warps 10-13 epilogue: the fp16 t plane, S * D * 2^-14 = t / 2^E, read by k_upre
+// Units are claimed dynamically in their order, linears of the largest d_in first (a global
+// counter, posted to every warp through a shared-memory ring); every wait is bounded.
 // ---------------------------------------------------------------------------------------------
 #define VP_THREADS 448
 #define VP_A_BYTES 16384  // 128 ranks x 64 fp16
