@@ -131,6 +131,20 @@ def test_workspace_size_rules():
     assert dc.dc_workspace_size(64, 1470, 11008, 3, 50) == 0  # n_linears must be 1 or 7
 
 
+def test_workspace_holds_the_prefill_planes_from_64_tokens():
+    """From T = 64 on the workspace also holds the prefill path's fp16 t plane [n_lin][T][tcols]
+    (tcols: the ranks rounded up to 64, plus 64 per further band) and the fp16 scaled activations
+    [n_in][T][max_d_in]; below 64 tokens it holds neither."""
+    max_rank, max_d_in, n_lin, n_in = 1470, 11008, 7, 3
+    tcols = (max_rank + 63) // 64 * 64 + 64 * (dc.DC_MAX_BANDS - 1)
+    planes = n_lin * 64 * tcols * 2 + n_in * 64 * max_d_in * 2
+    ws = {T: dc.dc_workspace_size(T, max_rank, max_d_in, n_lin, 50) for T in (62, 63, 64)}
+    per_token = ws[63] - ws[62]
+    assert per_token < planes // 8
+    assert ws[64] - ws[63] >= planes
+    assert ws[64] - ws[63] <= planes + 2 * per_token + 256 * 32  # token-sized regions and alignment
+
+
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     import importlib
     monkeypatch.setattr(dc, "LIB_PATH", str(tmp_path / "nope.so"))
