@@ -1981,9 +1981,9 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
 // ---------------------------------------------------------------------------------------------
 // Prefill delta path (segments of at least DC_PF_MIN tokens), tcgen05 tensor cores.
 //
-// k_vpre computes t and also writes it as two bf16 planes, t = hi + lo to ~16 bits, in the layout
-// k_upre loads with TMA: [plane][linear][token][tcols], band b of the tenant starting at column
-// sum_{b' < b} align(rank_b', 64), zeros in the padding.
+// k_vpre computes t and writes it as one fp16 plane, t / 2^E per token (2^E > max |x| of the
+// token), in the layout k_upre loads with TMA: [linear][token][tcols], band b of the tenant
+// starting at column sum_{b' < b} align(rank_b', 64), zeros in the padding.
 // ---------------------------------------------------------------------------------------------
 __device__ __forceinline__ int pf_band_col(const DcURec& R, int b) {
   int c = 0;
@@ -1991,7 +1991,7 @@ __device__ __forceinline__ int pf_band_col(const DcURec& R, int b) {
   return c;
 }
 
-// One 16-byte chunk (8 consecutive K columns) of a 128-byte-swizzled K-major bf16 tile row.
+// One 16-byte chunk (8 consecutive K columns) of a 128-byte-swizzled K-major 16-bit tile row.
 __device__ __forceinline__ void sw128_store(uint8_t* tile, int row, int chunk, uint4 v) {
   *reinterpret_cast<uint4*>(tile + row * 128 + ((chunk ^ (row & 7)) << 4)) = v;
 }
