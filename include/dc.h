@@ -100,19 +100,29 @@ typedef struct {
   const dc_delta_handle* tenants_dev;  /* device array [n_tenants] (dc_tenant_table_upload)   */
 } dc_linear;
 
-/* Text of the last error raised on the calling thread ("" if none). */
+/* Text of the last error raised on the calling thread ("" if none).
+ * Passage: none (error reporting of this library; no counterpart in the pages). */
 const char* dc_last_error(void);
 
-/* Library version string. */
+/* Library version string.  Passage: none (no counterpart in the pages). */
 const char* dc_version(void);
 
-/* Size in bytes of the packed blob of one tenant's linear.  Returns 0 for an invalid descriptor
+/* Passage: "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language
+ * Models", section "Approach" (singular vectors kept at 8/3/2 bits by singular-value
+ * rank, the smallest dropped at 0 bits); the byte layout itself is this library's.
+ * Size in bytes of the packed blob of one tenant's linear.  Returns 0 for an invalid descriptor
  * (and sets dc_last_error).  The blob holds: S as fp32 [r]; V_hat^T codes as bit planes in
  * 16-rank tiles; U_hat codes as bit planes in 16-row tiles; fp16 scale and zero per group of
  * 128 for every kept singular vector. */
 size_t dc_packed_size(const dc_factor_desc* desc);
 
-/* Host round-to-nearest quantiser (deterministic, fp64 arithmetic), one rule for every group
+/* Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的技术原理"
+ * (mixed-precision quantisation of the singular vectors: higher precision for larger singular
+ * values); "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language
+ * Models", section "Approach" (8/3/2-bit groups).  The
+ * grid (round to nearest, groups of 128, fp16 scale and zero) is this library's reading of a point
+ * the pages leave open.
+ * Host round-to-nearest quantiser (deterministic, fp64 arithmetic), one rule for every group
  * of 128 elements of every kept singular vector:
  *   lo = min(0, min g), hi = max(0, max g), qmax = 2^b - 1,
  *   scale = fp16_rne((hi - lo) / qmax) (1 if it is 0), zero = clamp(rint(-lo / scale), 0, qmax),
@@ -126,14 +136,20 @@ size_t dc_packed_size(const dc_factor_desc* desc);
 dc_status dc_quantize_rtn(const dc_factor_desc* desc, const float* U, const float* Vt,
                           uint8_t* codes_u, uint8_t* codes_v, uint16_t* sz_u, uint16_t* sz_v);
 
-/* Pack host codes into the serving layout and copy them to dev_dst (caller-owned, at least
+/* Passage: "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language
+ * Models", section "Approach" (the compressed delta of one
+ * tenant); the serving layout is this library's.
+ * Pack host codes into the serving layout and copy them to dev_dst (caller-owned, at least
  * dc_packed_size bytes, 256-byte aligned).  S: host fp32 [r].  Synchronises the stream before
  * returning so the host buffers may be freed.  Fills *out. */
 dc_status dc_pack_upload(const dc_factor_desc* desc, const uint8_t* codes_u, const uint8_t* codes_v,
                          const uint16_t* sz_u, const uint16_t* sz_v, const float* S,
                          void* dev_dst, size_t dev_bytes, void* stream, dc_delta_handle* out);
 
-/* Device quantiser + packer: the same rule as dc_quantize_rtn, run on the GPU from device fp32
+/* Passage: as dc_quantize_rtn ("Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法",
+ * "Delta-CoMe的技术原理"; "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large
+ * Language Models", "Approach").
+ * Device quantiser + packer: the same rule as dc_quantize_rtn, run on the GPU from device fp32
  * factors (U column-major [d_out, r], Vt row-major [r, d_in], S [r]) straight into the serving
  * layout at dev_dst.  Produces bit-identical codes to dc_quantize_rtn.  Asynchronous.
  * scratch: caller device buffer of dc_quantize_scratch_size(desc) bytes; its first int32 is a
@@ -143,12 +159,15 @@ dc_status dc_quantize_pack_device(const dc_factor_desc* desc, const float* U_dev
                                   const float* S_dev, void* dev_dst, size_t dev_bytes, void* scratch,
                                   size_t scratch_bytes, void* stream, dc_delta_handle* out);
 
-/* Copy n handles into a caller-owned device array (n * sizeof(dc_delta_handle) bytes).
+/* Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的应用场景" (multi-tenant
+ * serving: one backbone, a compressed delta per customer).
+ * Copy n handles into a caller-owned device array (n * sizeof(dc_delta_handle) bytes).
  * Asynchronous; the host array must stay alive until the stream reaches the copy. */
 dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int32_t n, void* dev_dst,
                                  size_t dev_bytes, void* stream);
 
-/* Bytes of workspace needed by dc_delta_linear_segmented / dc_layer_forward for a batch of at
+/* Passage: none (sizing of this library's scratch memory; no counterpart in the pages).
+ * Bytes of workspace needed by dc_delta_linear_segmented / dc_layer_forward for a batch of at
  * most T tokens whose linears have ranks up to max_rank, d_in and d_out up to max_d_in and at
  * most max_tenants tenants (n_linears = 1 or 7).  The workspace holds the routing result, the
  * per-token activation limbs, the rank-reduction results and the device status word.  The same
@@ -158,23 +177,34 @@ dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int32_t n, void
 size_t dc_workspace_size(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_linears,
                          int32_t max_tenants);
 
-/* Quantise on the device needs plain codes as scratch: bytes of scratch for one descriptor. */
+/* Passage: none (scratch sizing; no counterpart in the pages).
+ * Quantise on the device needs plain codes as scratch: bytes of scratch for one descriptor. */
 size_t dc_quantize_scratch_size(const dc_factor_desc* desc);
 
-/* Token routing: stable counting sort of tenant ids (device int32 [T], -1 = backbone only, -1
+/* Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的应用场景" (multi-tenant
+ * serving); "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language
+ * Models", section "Problem" (serving many fine-tuned models
+ * cheaply).  Every token of a batch goes to its own tenant's delta.
+ * Token routing: stable counting sort of tenant ids (device int32 [T], -1 = backbone only, -1
  * first) into the workspace: permutation, inverse permutation and the segment list
  * {tenant, start, length} in ascending tenant order.  Resets the device status word.  Ids out
  * of range set DC_ERR_TENANT in the status word and are routed as -1. */
 dc_status dc_build_segments(const int32_t* tenant_ids_dev, int32_t T, int32_t n_tenants,
                             void* ws, size_t ws_bytes, void* stream);
 
-/* Copy the routing result out of the workspace (debug/test helper; device -> caller device
+/* Passage: none (a check helper; no counterpart in the pages).
+ * Copy the routing result out of the workspace (debug/test helper; device -> caller device
  * buffers): perm int32 [T], inv_perm int32 [T], segments int32 [T, 3] (first n_segments rows
  * valid), n_segments int32 [1]. */
 dc_status dc_read_segments(const void* ws, int32_t T, int32_t* perm_dev, int32_t* inv_perm_dev,
                            int32_t* segments_dev, int32_t* n_segments_dev, void* stream);
 
-/* y[T, d_out] = (flags & DC_BASE ? W_base x : 0) + (flags & DC_DELTA ? U_hat (S * V_hat^T x) : 0)
+/* Passage: "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for Large Language
+ * Models", sections "Problem" and "Approach" (backbone plus
+ * compressed delta per fine-tuned model); "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法",
+ * sections "Delta-CoMe的技术原理" (low-rank decomposition of the delta) and "Delta-CoMe的应用场景"
+ * (multi-tenant serving).
+ * y[T, d_out] = (flags & DC_BASE ? W_base x : 0) + (flags & DC_DELTA ? U_hat (S * V_hat^T x) : 0)
  * for every token with its own tenant.  x: device [T, d_in] of dtype_in; y: device [T, d_out]
  * of dtype_out (F32 or BF16).  Runs dc_build_segments itself.  T >= 0 (T = 0 is a no-op).
  * Arithmetic of the delta: a tenant with 64 or more tokens in a batch of at least 128 tokens
@@ -214,14 +244,17 @@ dc_status dc_delta_linear_segmented(const dc_linear* lin, const void* x, void* y
  *   device that can overlap (different streams, or different threads without ordering) race on
  *   it and give wrong results.  Serialise the calls on a device.
  * - host_status: NULL, or where to store the device status word of this call (then the call
- *   waits for the stream and clears the word, like dc_read_device_status). */
+ *   waits for the stream and clears the word, like dc_read_device_status).  With T = 0 nothing
+ *   is launched and *host_status is set to 0. */
 #define DC_STATIC_WORKSPACE_BYTES ((size_t)16 << 20)
 dc_status dc_delta_linear_segmented_static(const dc_linear* lin, const void* x, void* y,
                                            const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
                                            int32_t dtype_out, int32_t flags, void* stream,
                                            int32_t* host_status);
 
-/* The seven projections of one Llama-style decoder layer in one call, sharing one routing:
+/* Passage: as dc_delta_linear_segmented; the layer shapes are those of the Llama-2 backbones
+ * that "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的技术原理", names.
+ * The seven projections of one Llama-style decoder layer in one call, sharing one routing:
  * lin[0..6] = q, k, v, o, gate, up, down.  q, k, v, gate and up read x_h [T, hidden]; o reads
  * x_o [T, hidden]; down reads x_f [T, ffn].  y[p] receives [T, lin[p].d_out]. */
 dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* x_o, const void* x_f,
@@ -229,14 +262,16 @@ dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* 
                            int32_t dtype_in, int32_t dtype_out, int32_t flags, void* ws,
                            size_t ws_bytes, void* stream);
 
-/* Decode the integer codes of one tenant's linear back out of the packed layout, with the same
+/* Passage: none (a check helper; no counterpart in the pages).
+ * Decode the integer codes of one tenant's linear back out of the packed layout, with the same
  * device decode functions the serving kernels use.  which = 0: U codes as uint8 [r, d_out]
  * (row i = codes of u_i); which = 1: V codes as uint8 [r, d_in].  out_dev: caller device
  * buffer. */
 dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t which, uint8_t* out_dev,
                                 void* stream);
 
-/* Per-kernel timing: after dc_profile_begin(capacity) every kernel launched by the serving entry
+/* Passage: none (profiling; no counterpart in the pages).
+ * Per-kernel timing: after dc_profile_begin(capacity) every kernel launched by the serving entry
  * points on this thread is bracketed by two CUDA events recorded on its stream (at most
  * `capacity` launches).  dc_profile_end synchronises those events, writes each launch's duration
  * in milliseconds and its kernel kind (0 routing, 1 activation prep, 2 rank reduction, 3 delta
@@ -247,7 +282,8 @@ dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t which, uint8_t
 dc_status dc_profile_begin(int32_t capacity);
 int32_t dc_profile_end(float* ms_out, int32_t* kind_out, int32_t capacity);
 
-/* Read (and then clear) the device status word of a workspace; synchronises the stream. */
+/* Passage: none (error reporting; no counterpart in the pages).
+ * Read (and then clear) the device status word of a workspace; synchronises the stream. */
 dc_status dc_read_device_status(void* ws, void* stream, int32_t* host_status);
 
 #ifdef __cplusplus

@@ -21,7 +21,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 LIBS = {
     "libdc.so": {
         "sources": ["dc_host.cpp", "dc_kernels.cu"],
-        "headers": ["dc_layout.h", "dc_pack.h", "dc_internal.h", "dc_tma.h", "dc_umma.h"],
+        "headers": ["dc_layout.h", "dc_pack.h", "dc_internal.h", "dc_tma.h", "dc_umma.h", "dc_devstate.h"],
         "link": ["-lcudart"],
     },
     "libdc_synth.so": {
@@ -54,10 +54,8 @@ def build(force: bool = False, verbose: bool = False) -> list[str]:
             os.makedirs(os.path.dirname(obj), exist_ok=True)
             cmd = [NVCC, "-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC, *ARCH,
                    "-c", src, "-o", obj]
-            if src.endswith(".cu"):
-                cmd[1:1] = ["-Xptxas", "-v"] if verbose else []
-            else:
-                cmd[1:1] = ["-x", "cu"] if False else []
+            if src.endswith(".cu") and verbose:
+                cmd[1:1] = ["-Xptxas", "-v"]
             r = subprocess.run(cmd, capture_output=True, text=True)
             if r.returncode != 0:
                 raise RuntimeError(f"nvcc failed for {src}:\n{r.stdout}\n{r.stderr}")

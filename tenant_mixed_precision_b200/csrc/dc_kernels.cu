@@ -28,6 +28,7 @@
 #include <mutex>
 
 #include "dc.h"
+#include "dc_devstate.h"
 #include "dc_internal.h"
 #include "dc_layout.h"
 #include "dc_pack.h"
@@ -3159,6 +3160,33 @@ extern "C" dc_status dc_quantize_pack_device(const dc_factor_desc* desc, const f
   return DC_OK;
 }
 
+// Per-device launch state (SM count, dynamic shared-memory limits set per kernel): these belong to
+// each device's context, so they are keyed by the current device under one mutex.
+static DcDevState g_devstate;
+
+static int current_device() {
+  int d = 0;
+  if (cudaGetDevice(&d) != cudaSuccess) d = 0;
+  return d;
+}
+
+static int device_sm_count(int dev) {
+  return g_devstate.sm_count(dev, [](int d) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, d) != cudaSuccess) return 0;
+    return n;
+  });
+}
+
+// Allow kernel `fn` (id `kid`) `need` bytes of dynamic shared memory on device `dev`.
+static dc_status allow_smem(int dev, int kid, const void* fn, size_t need) {
+  const int e = g_devstate.ensure_smem(dev, kid, need, [&](size_t n) {
+    return (int)cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)n);
+  });
+  if (e == -1) return dc_fail(DC_ERR_UNSUPPORTED, "device index %d is beyond this build's table", dev);
+  return e ? dc_cuda_check((cudaError_t)e, "shared-memory attribute") : DC_OK;
+}
+
 extern "C" dc_status dc_build_segments(const int32_t* tenant_ids_dev, int32_t T, int32_t n_tenants, void* ws,
                                        size_t ws_bytes, void* stream) {
   dc_clear_error();
@@ -3169,8 +3197,10 @@ extern "C" dc_status dc_build_segments(const int32_t* tenant_ids_dev, int32_t T,
   const DcWs W = dc_ws_layout(T, 0, 0, 1, 0);
   if (ws_bytes < (size_t)W.total) return dc_fail(DC_ERR_WORKSPACE, "workspace too small for routing");
   const size_t smem = (size_t)2 * (n_tenants + 1) * 4;
-  if (smem > 48 * 1024)
-    cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (smem > 48 * 1024) {
+    const dc_status st = allow_smem(current_device(), DC_K_SEGMENTS, (const void*)k_segments, smem);
+    if (st) return st;
+  }
   k_segments<<<1, 256, smem, (cudaStream_t)stream>>>(tenant_ids_dev, T, n_tenants, (uint8_t*)ws, W);
   return dc_cuda_check(cudaGetLastError(), "routing kernel");
 }
@@ -3194,15 +3224,16 @@ extern "C" dc_status dc_read_segments(const void* ws, int32_t T, int32_t* perm_d
 }
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no link-time libcuda dependency).
+// The driver entry point is process-wide; the first call looks it up (thread-safe static init).
 static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  if (!fn) {
+  static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
         q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-  }
+      return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    return nullptr;
+  }();
   return fn;
 }
 
@@ -3320,11 +3351,15 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     }
   }
   cudaStream_t s = (cudaStream_t)stream;
+  const int dev = current_device();
   dc_status st;
   if (!(flags & DC_REUSE_ROUTING)) {
     if (max_ten > DC_MAX_TENANTS) return dc_fail(DC_ERR_UNSUPPORTED, "too many tenants");
     const size_t smem = (size_t)2 * (max_ten + 1) * 4;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(k_segments, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (smem > 48 * 1024) {
+      st = allow_smem(dev, DC_K_SEGMENTS, (const void*)k_segments, smem);
+      if (st) return st;
+    }
     prof_before(s, 0);
     k_segments<<<1, 256, smem, s>>>(ids, T, max_ten, (uint8_t*)ws, F.ws);
     prof_after(s);
@@ -3344,21 +3379,11 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   prof_after(s);
   st = dc_cuda_check(cudaGetLastError(), "prep kernel");
   if (st) return st;
-  static int n_sm = 0;
-  if (!n_sm) {
-    int dev = 0;
-    cudaGetDevice(&dev);
-    cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev);
-    if (n_sm <= 0) n_sm = 148;
-  }
+  const int n_sm = device_sm_count(dev);
   if (flags & DC_DELTA) {
     const size_t vsmem = (size_t)V_STAGES * V_STAGE_BYTES + sizeof(VSmemTail);
-    static bool vset = false;
-    if (!vset) {
-      st = dc_cuda_check(cudaFuncSetAttribute(k_vstage, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vsmem), "smem attr");
-      if (st) return st;
-      vset = true;
-    }
+    st = allow_smem(dev, DC_K_VSTAGE, (const void*)k_vstage, vsmem);
+    if (st) return st;
     prof_before(s, 2);
     k_vstage<<<V_CTAS_PER_SM * n_sm, V_THREADS, vsmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
@@ -3366,13 +3391,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (st) return st;
     if (F.pf) {
       const size_t qsmem = 1024 + (size_t)VP_STAGES * VP_STAGE_BYTES + 2 * VP_BLK_BYTES + sizeof(VpTail);
-      static size_t qset = 0;
-      if (qsmem > qset) {
-        st = dc_cuda_check(cudaFuncSetAttribute(k_vpre, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsmem),
-                           "smem attr");
-        if (st) return st;
-        qset = qsmem;
-      }
+      st = allow_smem(dev, DC_K_VPRE, (const void*)k_vpre, qsmem);
+      if (st) return st;
       prof_before(s, 2);
       k_vpre<<<n_sm, VP_THREADS, qsmem, s>>>(F, (uint8_t*)ws);
       prof_after(s);
@@ -3384,12 +3404,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_GSTAGE * U_LBUF + sizeof(USmemTail);
     if (usmem > 227 * 1024)
       return dc_fail(DC_ERR_UNSUPPORTED, "max_rank %d needs %zu bytes of shared memory", max_rank, usmem);
-    static size_t usmem_set = 0;
-    if (usmem > usmem_set) {
-      st = dc_cuda_check(cudaFuncSetAttribute(k_udelta, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usmem), "smem attr");
-      if (st) return st;
-      usmem_set = usmem;
-    }
+    st = allow_smem(dev, DC_K_UDELTA, (const void*)k_udelta, usmem);
+    if (st) return st;
     prof_before(s, 3);
     k_udelta<<<U_CTAS_PER_SM * n_sm, U_THREADS, usmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
@@ -3397,13 +3413,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     if (st) return st;
     if (F.pf) {
       const size_t psmem = 1024 + (size_t)UP_STAGES * UP_STAGE_BYTES + 2 * UP_BLK_BYTES + sizeof(UpTail);
-      static size_t pset = 0;
-      if (psmem > pset) {
-        st = dc_cuda_check(cudaFuncSetAttribute(k_upre, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)psmem),
-                           "smem attr");
-        if (st) return st;
-        pset = psmem;
-      }
+      st = allow_smem(dev, DC_K_UPRE, (const void*)k_upre, psmem);
+      if (st) return st;
       prof_before(s, 3);
       k_upre<<<n_sm, UP_THREADS, psmem, s>>>(F, (uint8_t*)ws);
       prof_after(s);
@@ -3428,25 +3439,16 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
       F.bt_gtiles[i] = (int)std::max<int64_t>(1, std::min<int64_t>(l.d_out / 128, share / (l.d_in / 64)));
     }
     const size_t tsmem = 1024 + (size_t)F.bt_ns * stage_bytes + sizeof(BtTail);
-    static size_t tset = 0;
-    if (tsmem > tset) {
-      st = dc_cuda_check(cudaFuncSetAttribute(k_base_tc, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tsmem),
-                         "smem attr");
-      if (st) return st;
-      tset = tsmem;
-    }
+    st = allow_smem(dev, DC_K_BASE_TC, (const void*)k_base_tc, tsmem);
+    if (st) return st;
     prof_before(s, 4);  // the unit counters were zeroed with the call's other per-call state
     k_base_tc<<<F.bt_grid, BT_THREADS, tsmem, s>>>(F, (uint8_t*)ws);
     prof_after(s);
     return dc_cuda_check(cudaGetLastError(), "tensor-core output kernel");
   }
   const size_t bsmem = 1024 + (size_t)B_STAGES * B_STAGE_BYTES + sizeof(BSmemTail);
-  static bool bset = false;
-  if (!bset) {
-    st = dc_cuda_check(cudaFuncSetAttribute(k_base, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bsmem), "smem attr");
-    if (st) return st;
-    bset = true;
-  }
+  st = allow_smem(dev, DC_K_BASE, (const void*)k_base, bsmem);
+  if (st) return st;
   const int n_units = F.tile_prefix[n_lin] * ((T + DC_TOK_BLOCK - 1) / DC_TOK_BLOCK);
   prof_before(s, 4);
   k_base<<<std::min(n_sm, n_units), KB_THREADS, bsmem, s>>>(F, (uint8_t*)ws);
@@ -3521,9 +3523,8 @@ extern "C" dc_status dc_read_device_status(void* ws, void* stream, int32_t* host
 static __device__ __align__(256) uint8_t dc_static_ws[DC_STATIC_WORKSPACE_BYTES];
 
 namespace {
-constexpr int kStaticMaxDevices = 64;
 std::mutex g_static_mu;
-void* g_static_ptr[kStaticMaxDevices];  // device address of dc_static_ws per device, once looked up
+void* g_static_ptr[DC_MAX_DEVICES];  // device address of dc_static_ws per device, once looked up
 }  // namespace
 
 extern "C" dc_status dc_delta_linear_segmented_static(const dc_linear* lin, const void* x, void* y,
@@ -3535,7 +3536,10 @@ extern "C" dc_status dc_delta_linear_segmented_static(const dc_linear* lin, cons
   if (flags & DC_REUSE_ROUTING)
     return dc_fail(DC_ERR_INVALID_ARG, "the static workspace rebuilds the routing on every call (no DC_REUSE_ROUTING)");
   if (T < 0) return dc_fail(DC_ERR_INVALID_ARG, "negative T");
-  if (T == 0) return DC_OK;
+  if (T == 0) {  // nothing launched: report a clean status
+    if (host_status) *host_status = 0;
+    return DC_OK;
+  }
   const size_t need =
       dc_workspace_size(T, lin->max_rank, std::max(lin->d_in, lin->d_out), 1, lin->n_tenants);
   if (need == 0) return dc_fail(DC_ERR_INVALID_ARG, "invalid sizes in the linear");
@@ -3547,7 +3551,7 @@ extern "C" dc_status dc_delta_linear_segmented_static(const dc_linear* lin, cons
   int dev = 0;
   dc_status st = dc_cuda_check(cudaGetDevice(&dev), "cudaGetDevice");
   if (st) return st;
-  if (dev < 0 || dev >= kStaticMaxDevices) return dc_fail(DC_ERR_UNSUPPORTED, "device index %d", dev);
+  if (dev < 0 || dev >= DC_MAX_DEVICES) return dc_fail(DC_ERR_UNSUPPORTED, "device index %d", dev);
   void* ws = nullptr;
   {
     std::lock_guard<std::mutex> lock(g_static_mu);

@@ -4,7 +4,8 @@
   8 tenants at the 1/16 budget, a decode batch of 8 tokens with one token per tenant: every
   output of three projections (q, gate, down: the three shapes) against the oracle;
 * the 13B-shaped prefill layer (2048 tokens in segments of 32-256, 16 tenants): sampled outputs
-  against the oracle, on the tensor-core prefill path;
+  of q, gate and down against the oracle, with sampled tokens taken both from tenants with 64+
+  tokens (the tensor-core prefill path) and from a tenant with fewer (the decode kernels);
 * edge cases: a batch of backbone-only tokens, tenants without a delta, one token.
 """
 import numpy as np
@@ -78,6 +79,9 @@ def test_one_7b_layer_8_tenants_one_token_each():
         assert np.isfinite(y).all()
 
 
+PF_MIN = 64  # a tenant with this many tokens in a batch of 128+ takes the prefill path (include/dc.h)
+
+
 def test_13b_prefill_layer_sampled_against_oracle():
     seed, s0, T = 20244, 0.02 * np.sqrt(5120.0), 2048
     st = _stack(5120, 13824, 16, T, seed, s0)
@@ -85,8 +89,16 @@ def test_13b_prefill_layer_sampled_against_oracle():
     full = _run(st, ids, dc.DC_BASE | dc.DC_DELTA)
     delta = _run(st, ids, dc.DC_DELTA)
     rng = np.random.default_rng(7)
-    toks = np.sort(rng.choice(T, size=4, replace=False))
-    for proj in (0, 6):  # q (5120x5120) and down (5120x13824)
+    # two tokens of tenants with 64+ tokens in the batch (the tensor-core prefill path), one of the
+    # tenant with fewer (the decode kernels), and one at random
+    counts = np.bincount(ids, minlength=16)
+    long_t = [k for k in range(T) if counts[ids[k]] >= PF_MIN]
+    short_t = [k for k in range(T) if 0 < counts[ids[k]] < PF_MIN]
+    assert long_t and short_t, "the prefill draw should hold both kinds of segment"
+    picks = [long_t[0], long_t[-1], short_t[len(short_t) // 2], int(rng.integers(0, T))]
+    toks = np.array(sorted(set(int(k) for k in picks)))
+    assert counts[ids[toks]].max() >= PF_MIN and counts[ids[toks]].min() < PF_MIN
+    for proj in (0, 4, 6):  # q (5120x5120), gate (13824x5120) and down (5120x13824)
         d_out, d_in = st.shapes[proj]
         rows = np.concatenate([np.arange(128) + 128 * int(rng.integers(0, d_out // 128)) for _ in range(2)])
         ref = _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, dc.DC_BASE | dc.DC_DELTA)

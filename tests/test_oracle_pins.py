@@ -99,6 +99,29 @@ def test_rtn_codes_in_range_and_error_bound(bits):
     assert np.all(q.zeros == np.round(q.zeros)) and q.zeros.min() >= 0 and q.zeros.max() <= qmax
 
 
+@pytest.mark.parametrize("bits", [2, 3, 8])
+@pytest.mark.parametrize("sign", [1.0, -1.0])
+def test_rtn_one_sign_group_stays_on_the_grid(bits, sign):
+    # A group whose values all have one sign: 0 is forced into the range (lo = min(0, min g),
+    # hi = max(0, max g)), so the grid runs from 0 to the far end of the group and no element is
+    # clipped by more than the fp16 rounding of the scale can move the grid's end:
+    # |v - v_hat| <= scale / 2 + qmax * |scale - (hi - lo) / qmax|.
+    rng = np.random.default_rng(300 + bits)
+    qmax = (1 << bits) - 1
+    for _ in range(40):
+        g = sign * (np.abs(rng.standard_normal(128)) * rng.uniform(1e-4, 2.0) + rng.uniform(0, 0.5))
+        c, s, z = oracle.rtn_quantize_group(g, bits)
+        lo, hi = min(0.0, g.min()), max(0.0, g.max())
+        assert z == (0.0 if sign > 0 else float(qmax)) or abs(z - (-lo / s)) <= 0.5 + 1e-12
+        assert c.min() >= 0 and c.max() <= qmax
+        slack = qmax * abs(s - (hi - lo) / qmax)
+        err = np.abs(g - (c - z) * s)
+        assert np.all(err <= s / 2 + slack + 1e-15)
+        # the element farthest from 0 lands on the grid's far end (or one step in)
+        far = int(np.argmax(np.abs(g)))
+        assert c[far] in ((qmax, qmax - 1) if sign > 0 else (0, 1))
+
+
 def test_rtn_vectorised_rows_match_group_loop():
     rng = np.random.default_rng(3)
     M = rng.standard_normal((5, 384)) * 0.05
@@ -337,6 +360,30 @@ def test_activation_error_small_and_ordered():
     e_full = oracle.activation_error(D, oracle.compress_factors(f32(U), f32(s), f32(Vt), [(16, 512)]), x)
     assert e_full < e_more < e_mixed < 1.0
     assert e_full < 1e-2   # 16-bit grids have fp16-subnormal scales (see the test above)
+
+
+def test_activation_error_equals_frobenius_error_of_the_explicit_matrix():
+    # With X = I the activation error is ||Delta - Delta_hat||_F / ||Delta||_F, Delta_hat formed
+    # explicitly as sum_i S_i u_hat_i v_hat_i^T; an orthogonal X or a scaled X leaves it unchanged
+    # (the Frobenius norm is invariant under rotations, the ratio under scaling).  The shape is
+    # not square, so a transposed evaluation fails.
+    rng = np.random.default_rng(31)
+    d_out, d_in = 256, 384
+    Q1, _ = np.linalg.qr(rng.standard_normal((d_out, d_out)))
+    Q2, _ = np.linalg.qr(rng.standard_normal((d_in, d_out)))
+    D = Q1 @ np.diag(0.05 / np.arange(1, d_out + 1)) @ Q2.T
+    a = oracle.compress_delta(D, [(8, 2), (3, 16), (2, 48)])
+    Uh, S, Vt = oracle.dequantized_factors(a)
+    M = np.zeros((d_out, d_in))
+    for i in range(S.shape[0]):
+        for o in range(d_out):
+            M[o] += S[i] * Uh[o, i] * Vt[i]
+    want = np.linalg.norm(D - M) / np.linalg.norm(D)
+    assert 1e-3 < want < 1.0
+    assert abs(oracle.activation_error(D, a, np.eye(d_in)) - want) <= 1e-12 * want
+    R, _ = np.linalg.qr(rng.standard_normal((d_in, d_in)))
+    assert abs(oracle.activation_error(D, a, R) - want) <= 1e-10 * want
+    assert abs(oracle.activation_error(D, a, 3.0 * R) - want) <= 1e-10 * want
 
 
 def test_long_tail_mixed_precision_beats_single_precision_same_size():
