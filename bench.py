@@ -658,6 +658,111 @@ def run_sweep(args):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# Tenant paging (7B shapes, 100 Zipf(1.1) tenants, fewer device slots than tenants)
+# ------------------------------------------------------------------------------------------------
+PAGING_METRIC = "tokens/s and hit rate, 100-tenant Zipf(1.1) 7B decode with on-demand tenant paging"
+
+
+def run_paging(args):
+    import numpy as np
+    import torch
+
+    import tenant_mixed_precision_b200 as dc
+    from tenant_mixed_precision_b200 import plans, synth
+    from tenant_mixed_precision_b200.stack import DeltaStack, PagedStack
+    from tenant_mixed_precision_b200.synth_stack import populate
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    layers = args.layers or 4
+    n_ten = args.tenants or 100
+    n_slots = args.slots or 32
+    T = 64
+
+    def plan_fn(l, p, d_out, d_in, t):
+        return plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+
+    t_setup = time.time()
+    ref = DeltaStack(4096, 11008, layers, n_ten, T, plan_fn, out_dtype=torch.bfloat16)
+    populate(ref, 20245)
+    paged = PagedStack(ref, n_slots, keep_ref_arena=False)
+    torch.cuda.empty_cache()
+    setup_s = time.time() - t_setup
+    compute, copy = torch.cuda.Stream(), torch.cuda.Stream()
+    n_batches = args.warmup + args.steps
+    batches = [synth.zipf_tenants(np.random.default_rng(7000 + i), T, n_ten) for i in range(n_batches)]
+    ids_host = [torch.from_numpy(b).pin_memory() for b in batches]
+    ids_dev = torch.zeros(T, dtype=torch.int32, device="cuda")
+
+    def layers_fwd():
+        for l in range(layers):
+            f = dc.DC_BASE | dc.DC_DELTA | (dc.DC_REUSE_ROUTING if l > 0 else 0)
+            xh, xo, xf = ref.x[l]
+            dc.dc_layer_forward(paged.lins[l], xh, xo, xf, ref.y[l], ids_dev, T, f, ref.ws, stream=compute)
+
+    # eager pass on the first batch (sets kernel attributes), then capture the layers as a graph
+    paged.pager.prepare(batches[0], copy, compute)
+    with torch.cuda.stream(compute):
+        ids_dev.copy_(ids_host[0], non_blocking=True)
+        layers_fwd()
+    paged.pager.commit(compute)
+    compute.synchronize()
+    assert dc.dc_read_device_status(ref.ws, compute) == 0
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=compute):
+        layers_fwd()
+
+    def step(i):
+        paged.pager.prepare(batches[i], copy, compute)
+        with torch.cuda.stream(compute):
+            ids_dev.copy_(ids_host[i], non_blocking=True)
+            graph.replay()
+        paged.pager.commit(compute)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    s0 = paged.pager.stats()
+    clocks = ClockSampler(int(os.environ.get("LOCAL_RANK", "0")))
+    clocks.start()
+    time.sleep(0.3)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(compute)
+    for i in range(args.warmup, n_batches):
+        step(i)
+    e1.record(compute)
+    e1.synchronize()
+    ck = clocks.stop()
+    ms = e0.elapsed_time(e1) / args.steps
+    s1 = paged.pager.stats()
+    status = dc.dc_read_device_status(ref.ws, compute)
+    d = {k: s1[k] - s0[k] for k in s1}
+    lookups = d["hits"] + d["misses"]
+    distinct = statistics.mean(len(set(b.tolist())) for b in batches[args.warmup:])
+    per_tenant = statistics.mean(paged.image_bytes(t) for t in range(n_ten))
+    line = {
+        "metric": PAGING_METRIC, "value": T / (ms * 1e-3), "unit": "tokens/s", "n_gpus": 1, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "u8xs8->s32 delta, bf16xbf16->f32 backbone", "data": "synthetic",
+        "config": {"workload": f"llama2-7b linear stack ({layers} layers) decode, {n_ten} tenants with Zipf(1.1) "
+                               f"popularity, {n_slots} resident slots, the rest paged from pinned host memory",
+                   "layers": layers, "T": T, "tenants": n_ten, "slots": n_slots, "budget": "1/16",
+                   "mean_distinct_tenants_per_batch": distinct, "tenant_image_bytes": per_tenant,
+                   "cuda_graph": True, "copies": "one cudaMemcpyAsync per missing tenant on a copy stream"},
+        "paging": {"hit_rate": d["hits"] / lookups if lookups else None, "hits": d["hits"], "misses": d["misses"],
+                   "evictions": d["evictions"], "bytes_loaded_per_step": d["bytes_loaded"] / args.steps,
+                   "h2d_gbs": d["bytes_loaded"] / (ms * 1e-3 * args.steps) / 1e9},
+        "gpu_launches": (1 + 4 * layers) * args.steps + d["batches"],
+        "clocks": ck, "device_status": status, "setup_s": setup_s,
+    }
+    print(json.dumps(line), flush=True)
+    del graph
+    paged.pager.close()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -668,9 +773,11 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     ap.add_argument("--layers", type=int, default=0, help="smaller stack for profiling captures (default: 32)")
     ap.add_argument("--tenants", type=int, default=0, help="fewer resident tenants (default: 50)")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep"],
+    ap.add_argument("--slots", type=int, default=0, help="paging workload: resident tenant slots (default: 32)")
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep", "paging"],
                     help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill "
-                         "pass; sweep: 100 Zipf tenants, T = 1..256, three budgets (one line per point)")
+                         "pass; sweep: 100 Zipf tenants, T = 1..256, three budgets (one line per point); paging: "
+                         "100 Zipf tenants served from fewer device slots with on-demand host->device loads")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -680,6 +787,8 @@ def main():
         return run_prefill(args)
     if args.workload == "sweep":
         return run_sweep(args)
+    if args.workload == "paging":
+        return run_paging(args)
     return run_gpu(args)
 
 

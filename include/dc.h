@@ -262,6 +262,117 @@ dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* 
                            int32_t dtype_in, int32_t dtype_out, int32_t flags, void* ws,
                            size_t ws_bytes, void* stream);
 
+/* ---- Device compressor: the SVD step.
+ * Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的技术原理"
+ * (SVD of the parameter delta); "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for
+ * Large Language Models", section "Approach".
+ *
+ * Top-r singular triplets of Delta = W_ft - W_base on the GPU, for dc_quantize_pack_device: a
+ * randomized range finder (Gaussian test matrix of r + oversample columns from `seed`, power_iters
+ * power iterations, each basis made orthonormal by one-sided Jacobi) and a one-sided Jacobi SVD of
+ * the projected matrix, in fp32 with fp64 Jacobi sums.  W_ft, W_base: device, row-major
+ * [d_out, d_in], dtype DC_DTYPE_F32 or DC_DTYPE_BF16.  Outputs (device, caller-owned):
+ * U_out [r, d_out] (row i = u_i), S_out [r] (descending), Vt_out [r, d_in] (row i = v_i), each pair
+ * signed so that the largest-magnitude entry of v_i is positive (the lowest index on ties).  The
+ * truncation error approaches the Eckart-Young optimum sqrt(sum_{i>r} sigma_i^2) as oversample and
+ * power_iters grow (e.g. oversample = r/10 + 16, power_iters = 2).  ws: caller device memory of
+ * dc_svd_workspace_size bytes (256-byte aligned).  Synchronises the stream (once per Jacobi sweep,
+ * to test convergence) and returns after the outputs are written; *sweeps_out (if not NULL)
+ * receives the number of Jacobi sweeps run. */
+size_t dc_svd_workspace_size(int32_t d_out, int32_t d_in, int32_t r, int32_t oversample);
+dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t dtype, int32_t d_out, int32_t d_in, int32_t r,
+                        int32_t oversample, int32_t power_iters, uint64_t seed, float* U_out, float* S_out,
+                        float* Vt_out, void* ws, size_t ws_bytes, void* stream, int32_t* sweeps_out);
+
+/* ---- PrinMix allocation variants (offline, host, fp64).
+ * Passage: "Enhancing Delta Compression in LLMs via SVD-based Quantization Error Minimization",
+ * sections 2.1 (eq. 5: the output error of quantising row i of V on calibration activations X is
+ * about Sigma_ii^2 dV_i X X^T dV_i^T), 2.2 (bit allocation as a 0/1 integer linear program: one
+ * width per row, a bit budget, candidate widths, at most K distinct widths) and 2.3
+ * (reconstruction-target correction: U refit to the quantised V before U is quantised).
+ * Widths are from {0, 2, 3, 8}; a width b costs b (d_out + d_in) code bits per rank; the budget is
+ * ratio * 16 * d_out * d_in code bits.  X: host fp32 [n, d_in] calibration tokens (rows).  All host
+ * arrays are caller-owned; nothing is allocated on the device.
+ *
+ * dc_prinmix_scores: scores[i * n_widths + j] = S_i^2 |dV_i(widths[j]) X^T|^2, dV_i = v_i minus its
+ *   round-to-nearest image at that width (the dc_quantize_rtn rule), v_i itself for 0 bits.
+ *   Vt: [r, d_in] rows v_i.
+ * dc_prinmix_allocate: the exact optimum of the ILP over those scores (widths must include 0; a
+ *   dynamic program over the budget per allowed set of nonzero widths); width_out[r]; *objective =
+ *   the summed error of the optimum.
+ * dc_prinmix_rtc: U_out = U M with M = H G^-1, G = A A^T, H = B A^T, A = Sigma V_hat X^T,
+ *   B = Sigma V X^T (the least-squares refit), by a Cholesky factorisation of G in fp64 (with a
+ *   1e-12 relative ridge).  U, U_out: column-major [d_out, k] (row i of the buffer = u_i); Vt_hat:
+ *   the dequantised V rows [k, d_in].  DC_ERR_INVALID_ARG if G is not positive definite.
+ * dc_prinmix_compress: scores, allocation, then the kept ranks grouped into bands by width, widest
+ *   first (8, 3, 2), singular-value order inside a band: desc_out (the plan), perm_out[r] (source
+ *   rank of kept rank i; -1 past the kept ones), U_out [k, d_out] / S_out [k] / Vt_out [k, d_in] of
+ *   the kept ranks in that order, U refit by RTC when rtc != 0.  Quantise and pack the outputs with
+ *   dc_quantize_rtn and dc_pack_upload (or dc_quantize_pack_device). */
+dc_status dc_prinmix_scores(const float* Vt, const float* S, int32_t r, int32_t d_in, const float* X, int32_t n,
+                            const int32_t* widths, int32_t n_widths, double* scores);
+dc_status dc_prinmix_allocate(const double* scores, int32_t r, const int32_t* widths, int32_t n_widths, int32_t d_out,
+                              int32_t d_in, double ratio, int32_t max_kinds, int32_t* width_out, double* objective);
+dc_status dc_prinmix_rtc(const float* U, const float* S, const float* Vt, const float* Vt_hat, int32_t k,
+                         int32_t d_out, int32_t d_in, const float* X, int32_t n, float* U_out);
+dc_status dc_prinmix_compress(const float* U, const float* S, const float* Vt, int32_t r, int32_t d_out, int32_t d_in,
+                              const float* X, int32_t n, double ratio, const int32_t* widths, int32_t n_widths,
+                              int32_t max_kinds, int32_t rtc, dc_factor_desc* desc_out, int32_t* perm_out,
+                              float* U_out, float* S_out, float* Vt_out, double* objective);
+
+/* ---- Tenant paging.
+ * Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", FAQ "多模型同机部署最该关注什么？"
+ * (keep the frequently used models resident, load the long-tail ones on demand).
+ *
+ * A pager keeps at most n_slots tenants resident in a caller-owned device arena of n_slots slots of
+ * slot_bytes each.  Every tenant's packed deltas for all of its linears form one host image (pinned
+ * host memory, caller-owned, alive while the pager uses it); blob_offsets[i] is where the blob of
+ * table i lies in the image (256-byte aligned; -1: the tenant has no delta for that linear).  The
+ * pager keeps n_tables device tenant tables (the tenants_dev arrays of the linears, caller-owned,
+ * already filled with every tenant's handles) pointing at the right slots: a handle's dev_base is the
+ * blob's device address while the tenant is resident and 0 otherwise (its tokens then get the
+ * backbone only).  Start with dev_base = 0 for every paged tenant.
+ *
+ * Per batch: dc_pager_prepare(ids) on the host, then enqueue the batch's kernels on compute_stream,
+ * then dc_pager_commit(compute_stream).  prepare picks slots for the batch's missing tenants (least
+ * recently used first, never a tenant of the batch) and, on copy_stream, waits for the last batch
+ * that read each victim slot, copies the images (one cudaMemcpyAsync each) and patches the tables;
+ * compute_stream is made to wait for that work.  Copies for the next batch overlap the kernels of the
+ * current one when prepare is called before those kernels finish.  prepare fails with
+ * DC_ERR_UNSUPPORTED (changing nothing) if a batch holds more distinct tenants than slots, and with
+ * DC_ERR_TENANT on an id >= n_tenants; ids < 0 are backbone-only tokens.  scratch: caller device
+ * memory of dc_pager_scratch_size bytes (16-byte aligned) for the table patches.  The pager
+ * allocates no device memory; it owns CUDA events and host bookkeeping only.  One pager per device
+ * and thread; its calls are not thread-safe. */
+typedef struct dc_pager dc_pager;
+typedef struct {
+  int32_t n_tenants;    /* tenant ids 0 .. n_tenants - 1                          */
+  int32_t n_slots;      /* tenants resident at once                               */
+  uint64_t slot_bytes;  /* bytes of one slot (multiple of 256, >= every image)     */
+  int32_t n_tables;     /* tenant tables kept current (one per linear)            */
+  int32_t reserved;
+} dc_pager_desc;
+typedef struct {
+  int64_t hits;          /* batch tenants found resident                          */
+  int64_t misses;        /* batch tenants loaded                                  */
+  int64_t evictions;     /* loads that displaced a resident tenant                */
+  int64_t bytes_loaded;  /* host -> device image bytes                            */
+  int64_t batches;       /* prepared batches                                      */
+} dc_pager_stats;
+size_t dc_pager_scratch_size(const dc_pager_desc* desc);
+dc_status dc_pager_create(const dc_pager_desc* desc, void* arena_dev, size_t arena_bytes, void* const* tables_dev,
+                          void* scratch_dev, size_t scratch_bytes, dc_pager** out);
+dc_status dc_pager_set_tenant(dc_pager* pager, int32_t tenant, const void* image_host, uint64_t image_bytes,
+                              const int64_t* blob_offsets);
+dc_status dc_pager_prepare(dc_pager* pager, const int32_t* tenant_ids_host, int32_t T, void* copy_stream,
+                           void* compute_stream);
+dc_status dc_pager_commit(dc_pager* pager, void* compute_stream);
+dc_status dc_pager_get_stats(const dc_pager* pager, dc_pager_stats* out);
+/* Slot of a resident tenant, -1 otherwise (a check helper). */
+int32_t dc_pager_slot_of(const dc_pager* pager, int32_t tenant);
+/* Release the pager's events and bookkeeping (after its streams are idle). */
+dc_status dc_pager_destroy(dc_pager* pager);
+
 /* Passage: none (a check helper; no counterpart in the pages).
  * Decode the integer codes of one tenant's linear back out of the packed layout, with the same
  * device decode functions the serving kernels use.  which = 0: U codes as uint8 [r, d_out]

@@ -47,6 +47,16 @@ class dc_delta_handle(C.Structure):
                 ("rank_total", C.c_int32), ("reserved", C.c_int32)]
 
 
+class dc_pager_desc(C.Structure):
+    _fields_ = [("n_tenants", C.c_int32), ("n_slots", C.c_int32), ("slot_bytes", C.c_uint64),
+                ("n_tables", C.c_int32), ("reserved", C.c_int32)]
+
+
+class dc_pager_stats(C.Structure):
+    _fields_ = [("hits", C.c_int64), ("misses", C.c_int64), ("evictions", C.c_int64), ("bytes_loaded", C.c_int64),
+                ("batches", C.c_int64)]
+
+
 class dc_linear(C.Structure):
     _fields_ = [("W_base", C.c_void_p), ("w_dtype", C.c_int32), ("d_out", C.c_int32), ("d_in", C.c_int32),
                 ("n_tenants", C.c_int32), ("max_rank", C.c_int32), ("tenants_dev", C.c_void_p)]
@@ -82,6 +92,21 @@ def _load():
         "dc_read_device_status": (I32, [VP, VP, P(I32)]),
         "dc_profile_begin": (I32, [I32]),
         "dc_profile_end": (I32, [P(C.c_float), P(I32), I32]),
+        "dc_prinmix_scores": (I32, [VP, VP, I32, I32, VP, I32, VP, I32, VP]),
+        "dc_prinmix_allocate": (I32, [VP, I32, VP, I32, I32, I32, C.c_double, I32, VP, P(C.c_double)]),
+        "dc_prinmix_rtc": (I32, [VP, VP, VP, VP, I32, I32, I32, VP, I32, VP]),
+        "dc_prinmix_compress": (I32, [VP, VP, VP, I32, I32, I32, VP, I32, C.c_double, VP, I32, I32, I32,
+                                      P(dc_factor_desc), VP, VP, VP, VP, P(C.c_double)]),
+        "dc_svd_workspace_size": (SZ, [I32, I32, I32, I32]),
+        "dc_svd_device": (I32, [VP, VP, I32, I32, I32, I32, I32, I32, C.c_uint64, VP, VP, VP, VP, SZ, VP, P(I32)]),
+        "dc_pager_scratch_size": (SZ, [P(dc_pager_desc)]),
+        "dc_pager_create": (I32, [P(dc_pager_desc), VP, SZ, P(VP), VP, SZ, P(VP)]),
+        "dc_pager_set_tenant": (I32, [VP, I32, VP, C.c_uint64, P(C.c_int64)]),
+        "dc_pager_prepare": (I32, [VP, P(I32), I32, VP, VP]),
+        "dc_pager_commit": (I32, [VP, VP]),
+        "dc_pager_get_stats": (I32, [VP, P(dc_pager_stats)]),
+        "dc_pager_slot_of": (I32, [VP, I32]),
+        "dc_pager_destroy": (I32, [VP]),
     }
     for name, (res, args) in sig.items():
         f = getattr(lib, name)
@@ -102,7 +127,9 @@ def exported_symbols() -> list[str]:
             "dc_workspace_size", "dc_build_segments", "dc_read_segments", "dc_delta_linear_segmented",
             "dc_delta_linear_segmented_static",
             "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status", "dc_profile_begin",
-            "dc_profile_end"]
+            "dc_profile_end", "dc_prinmix_scores", "dc_prinmix_allocate", "dc_prinmix_rtc", "dc_prinmix_compress",
+            "dc_svd_workspace_size", "dc_svd_device", "dc_pager_scratch_size", "dc_pager_create", "dc_pager_set_tenant", "dc_pager_prepare",
+            "dc_pager_commit", "dc_pager_get_stats", "dc_pager_slot_of", "dc_pager_destroy"]
 
 
 def _check(st: int):
@@ -309,6 +336,138 @@ def dc_profile_end(capacity: int):
     if n < 0:
         raise DcError(DC_ERR_CUDA, "profiling failed: " + dc_last_error())
     return [(KERNEL_KINDS[kinds[i]], float(ms[i])) for i in range(min(n, capacity))]
+
+
+# ------------------------------------------------------------------------------------------
+# PrinMix allocation variants (host)
+# ------------------------------------------------------------------------------------------
+PRINMIX_WIDTHS = (0, 2, 3, 8)
+
+
+def _f32(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float32))
+
+
+def dc_prinmix_scores(Vt, S, X, widths=PRINMIX_WIDTHS) -> np.ndarray:
+    Vt, S, X = _f32(Vt), _f32(S), _f32(X)
+    w = np.ascontiguousarray(widths, dtype=np.int32)
+    out = np.zeros((Vt.shape[0], len(w)), np.float64)
+    _check(_load().dc_prinmix_scores(_ptr(Vt), _ptr(S), Vt.shape[0], Vt.shape[1], _ptr(X), X.shape[0], _ptr(w), len(w),
+                                     _ptr(out)))
+    return out
+
+
+def dc_prinmix_allocate(scores, widths, d_out: int, d_in: int, ratio: float, max_kinds: int):
+    sc = np.ascontiguousarray(scores, dtype=np.float64)
+    w = np.ascontiguousarray(widths, dtype=np.int32)
+    out = np.zeros(sc.shape[0], np.int32)
+    obj = C.c_double(0.0)
+    _check(_load().dc_prinmix_allocate(_ptr(sc), sc.shape[0], _ptr(w), len(w), d_out, d_in, ratio, max_kinds, _ptr(out),
+                                       C.byref(obj)))
+    return out, obj.value
+
+
+def dc_prinmix_rtc(U, S, Vt, Vt_hat, X) -> np.ndarray:
+    """U: [d_out, k] (columns u_i) -> U~ [d_out, k]."""
+    Uc = _f32(np.asarray(U, dtype=np.float32).T)  # rows u_i
+    S, Vt, Vh, X = _f32(S), _f32(Vt), _f32(Vt_hat), _f32(X)
+    k, d_out, d_in = Uc.shape[0], Uc.shape[1], Vt.shape[1]
+    out = np.zeros((k, d_out), np.float32)
+    _check(_load().dc_prinmix_rtc(_ptr(Uc), _ptr(S), _ptr(Vt), _ptr(Vh), k, d_out, d_in, _ptr(X), X.shape[0], _ptr(out)))
+    return out.T
+
+
+def dc_prinmix_compress(U, S, Vt, X, ratio: float, max_kinds: int, widths=PRINMIX_WIDTHS, rtc: bool = True):
+    """U: [d_out, r] (columns u_i), S [r], Vt [r, d_in]; returns (desc, perm, U_out [d_out, k],
+    S_out [k], Vt_out [k, d_in], objective)."""
+    Uc = _f32(np.asarray(U, dtype=np.float32).T)
+    S, Vt, X = _f32(S), _f32(Vt), _f32(X)
+    r, d_out, d_in = Uc.shape[0], Uc.shape[1], Vt.shape[1]
+    w = np.ascontiguousarray(widths, dtype=np.int32)
+    desc = dc_factor_desc()
+    perm = np.zeros(r, np.int32)
+    Uo = np.zeros((r, d_out), np.float32)
+    So = np.zeros(r, np.float32)
+    Vo = np.zeros((r, d_in), np.float32)
+    obj = C.c_double(0.0)
+    _check(_load().dc_prinmix_compress(_ptr(Uc), _ptr(S), _ptr(Vt), r, d_out, d_in, _ptr(X), X.shape[0], ratio, _ptr(w),
+                                       len(w), max_kinds, 1 if rtc else 0, C.byref(desc), _ptr(perm), _ptr(Uo),
+                                       _ptr(So), _ptr(Vo), C.byref(obj)))
+    k = desc_rank(desc)
+    return desc, perm, Uo[:k].T, So[:k], Vo[:k], obj.value
+
+
+# ------------------------------------------------------------------------------------------
+# device compressor (SVD step)
+# ------------------------------------------------------------------------------------------
+def dc_svd_workspace_size(d_out: int, d_in: int, r: int, oversample: int) -> int:
+    return _load().dc_svd_workspace_size(d_out, d_in, r, oversample)
+
+
+def dc_svd_device(W_ft, W_base, r: int, oversample: int, power_iters: int, seed: int, U_out, S_out, Vt_out, ws,
+                  stream=None) -> int:
+    """Top-r SVD of W_ft - W_base on the device into U_out [r, d_out], S_out [r], Vt_out [r, d_in]
+    (float32 device tensors).  Returns the number of Jacobi sweeps run."""
+    d_out, d_in = W_ft.shape
+    sw = C.c_int32(0)
+    _check(_load().dc_svd_device(_ptr(W_ft), _ptr(W_base), _dtype_code(W_ft), d_out, d_in, r, oversample, power_iters,
+                                 seed, _ptr(U_out), _ptr(S_out), _ptr(Vt_out), _ptr(ws), ws.numel() * ws.element_size(),
+                                 _stream(stream), C.byref(sw)))
+    return sw.value
+
+
+# ------------------------------------------------------------------------------------------
+# tenant paging
+# ------------------------------------------------------------------------------------------
+class Pager:
+    """dc_pager_* over caller-owned device memory: `arena` (n_slots * slot_bytes bytes), the device
+    tenant tables `tables` (one per linear) and a patch scratch allocated here as a torch tensor."""
+
+    def __init__(self, n_tenants: int, n_slots: int, slot_bytes: int, arena, tables):
+        import torch
+        self.desc = dc_pager_desc(n_tenants, n_slots, slot_bytes, len(tables), 0)
+        nsc = _load().dc_pager_scratch_size(C.byref(self.desc))
+        self.scratch = torch.empty(max(nsc, 16), dtype=torch.uint8, device=arena.device)
+        self._tables = (C.c_void_p * len(tables))(*[_ptr(t) for t in tables])
+        self._arena = arena
+        h = C.c_void_p()
+        _check(_load().dc_pager_create(C.byref(self.desc), _ptr(arena), arena.numel() * arena.element_size(),
+                                       self._tables, _ptr(self.scratch), nsc, C.byref(h)))
+        self.h = h
+        self._images = {}
+
+    def set_tenant(self, tenant: int, image_host, blob_offsets):
+        """image_host: pinned host uint8 tensor (kept alive here); blob_offsets: per table, -1 = none."""
+        offs = (C.c_int64 * len(blob_offsets))(*[int(o) for o in blob_offsets])
+        _check(_load().dc_pager_set_tenant(self.h, tenant, _ptr(image_host), image_host.numel(), offs))
+        self._images[tenant] = image_host
+
+    def prepare(self, tenant_ids_host: np.ndarray, copy_stream, compute_stream):
+        ids = np.ascontiguousarray(tenant_ids_host, dtype=np.int32)
+        _check(_load().dc_pager_prepare(self.h, ids.ctypes.data_as(C.POINTER(C.c_int32)), len(ids),
+                                        _stream(copy_stream), _stream(compute_stream)))
+
+    def commit(self, compute_stream):
+        _check(_load().dc_pager_commit(self.h, _stream(compute_stream)))
+
+    def stats(self) -> dict:
+        st = dc_pager_stats()
+        _check(_load().dc_pager_get_stats(self.h, C.byref(st)))
+        return {f: getattr(st, f) for f, _ in dc_pager_stats._fields_}
+
+    def slot_of(self, tenant: int) -> int:
+        return _load().dc_pager_slot_of(self.h, tenant)
+
+    def close(self):
+        if self.h:
+            _load().dc_pager_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
 
 
 # ------------------------------------------------------------------------------------------

@@ -102,8 +102,7 @@ double dc_f16_to_f64(uint16_t h) {
 
 // One group of RTN: the rule stated in dc.h.  Returns false on a non-finite value or an fp16
 // scale overflow.
-static bool rtn_group(const float* v, int64_t stride, int n, int bits, uint8_t* codes, int64_t cstride,
-                      uint16_t* sz) {
+bool dc_rtn_group(const float* v, int64_t stride, int n, int bits, uint8_t* codes, int64_t cstride, uint16_t* sz) {
   const double qmax = (double)((1 << bits) - 1);
   double lo = 0.0, hi = 0.0;
   for (int i = 0; i < n; ++i) {
@@ -152,11 +151,11 @@ extern "C" dc_status dc_quantize_rtn(const dc_factor_desc* desc, const float* U,
     for (int i = (int)tid; i < r; i += (int)nth) {
       const int bits = bits_of[i];
       for (int g = 0; g < L.groups_in; ++g)
-        if (!rtn_group(Vt + (int64_t)i * d_in + g * 128, 1, 128, bits, codes_v + (int64_t)i * d_in + g * 128, 1,
+        if (!dc_rtn_group(Vt + (int64_t)i * d_in + g * 128, 1, 128, bits, codes_v + (int64_t)i * d_in + g * 128, 1,
                        sz_v + ((int64_t)i * L.groups_in + g) * 2))
           bad[tid] = i;
       for (int g = 0; g < L.groups_out; ++g)
-        if (!rtn_group(U + (int64_t)i * d_out + g * 128, 1, 128, bits, codes_u + (int64_t)i * d_out + g * 128, 1,
+        if (!dc_rtn_group(U + (int64_t)i * d_out + g * 128, 1, 128, bits, codes_u + (int64_t)i * d_out + g * 128, 1,
                        sz_u + ((int64_t)i * L.groups_out + g) * 2))
           bad[tid] = i;
     }

@@ -13,6 +13,10 @@ dc_status dc_check_desc(const dc_factor_desc* d, DcLayout* L);
 void dc_fill_handle(const dc_factor_desc* desc, const DcLayout& L, void* dev, dc_delta_handle* out);
 uint16_t dc_f64_to_f16(double x);
 double dc_f16_to_f64(uint16_t h);
+// One group of round-to-nearest quantisation (the rule of dc_quantize_rtn): n values at stride
+// `stride` -> codes at stride `cstride`, sz = fp16 bits of (scale, zero).  False on a non-finite
+// value or an fp16 scale overflow.
+bool dc_rtn_group(const float* v, int64_t stride, int n, int bits, uint8_t* codes, int64_t cstride, uint16_t* sz);
 
 // Limits of this build.
 #define DC_MAX_TENANTS 8192     // routing histogram lives in shared memory

@@ -130,3 +130,86 @@ class DeltaStack:
                         u += b["u"]
         return {"backbone": w, "delta_v": v, "delta_u": u, "activations": act, "total": w + v + u + act,
                 "distinct_tenants": len(distinct)}
+
+
+class PagedStack:
+    """The tenants of a populated DeltaStack served from fewer device slots through the library's
+    pager (dc_pager_*): frequently used tenants stay resident, long-tail ones are copied in from
+    pinned host memory when a batch needs them.
+
+    Each tenant's packed blobs for all (layer, projection) form one host image (256-byte aligned
+    pieces); the stack owns the slot arena and its own device tenant tables, whose handles start
+    with dev_base = 0 and are kept current by the pager.  Backbone weights, inputs, outputs and the
+    workspace are those of `ref`.
+    """
+
+    def __init__(self, ref: DeltaStack, n_slots: int, keep_ref_arena: bool = True):
+        from . import Pager, make_linear as _ml
+        self.ref = ref
+        self.n_slots = n_slots
+        n_tab = ref.layers * 7
+        self.images, self.blob_offsets = {}, {}
+        sizes = []
+        for t in range(ref.n_tenants):
+            offs, size = [], 0
+            for l in range(ref.layers):
+                for p in range(7):
+                    if (l, p, t) in ref.descs:
+                        offs.append(size)
+                        size += _align(dc_packed_size(ref.descs[(l, p, t)]))
+                    else:
+                        offs.append(-1)
+            self.blob_offsets[t] = offs
+            sizes.append(size)
+        self.slot_bytes = _align(max(sizes + [256]))
+        for t in range(ref.n_tenants):
+            img = torch.empty(max(sizes[t], 256), dtype=torch.uint8, pin_memory=True)
+            for l in range(ref.layers):
+                for p in range(7):
+                    o = self.blob_offsets[t][7 * l + p]
+                    if o < 0:
+                        continue
+                    n = dc_packed_size(ref.descs[(l, p, t)])
+                    src = ref.offsets[(l, p, t)]
+                    img[o:o + n].copy_(ref.arena[src:src + n])
+            self.images[t] = img
+        torch.cuda.synchronize()
+        self.arena = torch.empty(n_slots * self.slot_bytes, dtype=torch.uint8, device=ref.device)
+        self.tables = torch.zeros_like(ref.tables)
+        keep = []
+        self.lins = []
+        for l in range(ref.layers):
+            lins = []
+            for p, (d_out, d_in) in enumerate(ref.shapes):
+                hs = []
+                for t in range(ref.n_tenants):
+                    h = ref.handles.get((l, p, t))
+                    h2 = dc_delta_handle.from_buffer_copy(h) if h is not None else dc_delta_handle()
+                    h2.dev_base = 0
+                    hs.append(h2)
+                if ref.n_tenants:
+                    keep.append(dc_tenant_table_upload(hs, self.tables[l, p]))
+                lins.append(_ml(ref.W[l][p], d_out, d_in, ref.n_tenants, ref.max_rank[p], self.tables[l, p]))
+            self.lins.append(lins)
+        torch.cuda.synchronize()
+        del keep
+        self.pager = Pager(ref.n_tenants, n_slots, self.slot_bytes, self.arena,
+                           [self.tables[l, p] for l in range(ref.layers) for p in range(7)])
+        for t in range(ref.n_tenants):
+            self.pager.set_tenant(t, self.images[t], self.blob_offsets[t])
+        if not keep_ref_arena:
+            ref.arena = None
+
+    def forward(self, ids_host, ids_dev, T: int, compute_stream, copy_stream, flags: int = DC_BASE | DC_DELTA):
+        """Make the batch's tenants resident (copies on copy_stream), then run every layer on
+        compute_stream, then mark the batch's slots as in use until those kernels finish."""
+        self.pager.prepare(ids_host[:T], copy_stream, compute_stream)
+        r = self.ref
+        for l in range(r.layers):
+            f = flags | (DC_REUSE_ROUTING if l > 0 else 0)
+            xh, xo, xf = r.x[l]
+            dc_layer_forward(self.lins[l], xh, xo, xf, r.y[l], ids_dev, T, f, r.ws, stream=compute_stream)
+        self.pager.commit(compute_stream)
+
+    def image_bytes(self, t: int) -> int:
+        return self.images[t].numel()
