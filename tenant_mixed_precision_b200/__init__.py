@@ -96,7 +96,7 @@ def _load():
         "dc_prinmix_allocate": (I32, [VP, I32, VP, I32, I32, I32, C.c_double, I32, VP, P(C.c_double)]),
         "dc_prinmix_rtc": (I32, [VP, VP, VP, VP, I32, I32, I32, VP, I32, VP]),
         "dc_prinmix_compress": (I32, [VP, VP, VP, I32, I32, I32, VP, I32, C.c_double, VP, I32, I32, I32,
-                                      P(dc_factor_desc), VP, VP, VP, VP, P(C.c_double)]),
+                                      VP, VP, VP, VP, VP, P(C.c_double)]),
         "dc_svd_workspace_size": (SZ, [I32, I32, I32, I32]),
         "dc_svd_device": (I32, [VP, VP, I32, I32, I32, I32, I32, I32, C.c_uint64, VP, VP, VP, VP, SZ, VP, P(I32)]),
         "dc_pager_scratch_size": (SZ, [P(dc_pager_desc)]),
@@ -391,7 +391,7 @@ def dc_prinmix_compress(U, S, Vt, X, ratio: float, max_kinds: int, widths=PRINMI
     Vo = np.zeros((r, d_in), np.float32)
     obj = C.c_double(0.0)
     _check(_load().dc_prinmix_compress(_ptr(Uc), _ptr(S), _ptr(Vt), r, d_out, d_in, _ptr(X), X.shape[0], ratio, _ptr(w),
-                                       len(w), max_kinds, 1 if rtc else 0, C.byref(desc), _ptr(perm), _ptr(Uo),
+                                       len(w), max_kinds, 1 if rtc else 0, C.addressof(desc), _ptr(perm), _ptr(Uo),
                                        _ptr(So), _ptr(Vo), C.byref(obj)))
     k = desc_rank(desc)
     return desc, perm, Uo[:k].T, So[:k], Vo[:k], obj.value
