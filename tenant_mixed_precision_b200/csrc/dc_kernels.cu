@@ -24,7 +24,6 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
-#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -1435,484 +1434,6 @@ __global__ void __launch_bounds__(U_THREADS, U_CTAS_PER_SM) k_udelta(const __gri
       }
     }
     ++unit;
-  }
-}
-
-// ---------------------------------------------------------------------------------------------
-// k_uout: the same product as k_udelta, ydelta[token, row] = (U_hat (scale * t))[row], streamed
-// without a producer warp.  A CTA of 8 warps serves one 128-row output group at a time (warp w owns
-// rows 16 w .. 16 w + 15, i.e. tile w of every U block); CTAs claim chunks of up to UO_CHUNK
-// consecutive groups of one (linear, segment) from a global counter.  Per chunk, warp 0 lists the
-// run's 2/3-bit blocks (offset, tile bytes, first limb slot, quads, shift steps).  The chunk's
-// (pass, group, block) sequence is one stream per warp: the lanes copy the warp's tile of each
-// block (contiguous bytes) with 16-byte cp.async into a private ring of UO_D slots in shared
-// memory, UO_D - 1 blocks ahead of the one being multiplied, across unit boundaries.  Per
-// (group, pass of <= 4 tokens) unit:
-//   - the 256 threads build the limb matrix of B = scale * t for every 2/3-bit rank, four ranks per
-//     thread (one 16-byte meta load, three 32-bit limb stores per token), and the zero-point sums
-//     sum_i zero * scale * t; warps sum their 8-bit ranks in fp32 for their own rows;
-//   - one barrier; then each warp multiplies its tile of every block, one mma.m16n8k32 u8.u8 per
-//     32-rank step and pair of tokens;
-//   - the epilogue combines the integer columns (limbs, row sums) exactly as k_udelta does and
-//     writes the group's outputs.
-// Limb matrices are double-buffered, so a unit takes one CTA barrier per window of UO_LMAX limb
-// slots (every 7B/13B unit fits one window).  Arithmetic is that of k_udelta.
-// ---------------------------------------------------------------------------------------------
-#define UO_THREADS 256
-#define UO_CTAS_PER_SM 2
-#define UO_LMAX 1792             // limb slots per window (a multiple of 256: bands and blocks start on multiples of 256 slots)
-#define UO_LROW (UO_LMAX + 32)   // row stride of a limb matrix: rows 8 banks apart
-#define UO_LBUF (16 * UO_LROW)   // rows as k_udelta's (ud_brow): limbs of two token pairs, then constants
-#define UO_MAXBLK 64             // 2/3-bit blocks of one record
-#define UO_MAXWIN 8
-#define UO_D 4                   // ring depth per warp (blocks)
-#define UO_SLOT 1536             // bytes of a ring slot: the largest tile of a block (3-bit, 8 steps)
-#define UO_CHUNK 4               // 128-row groups per claimed chunk
-
-struct UoBlk {
-  int32_t off;   // offset of the block's tile 0 inside a group's run
-  int32_t tb;    // bytes of one tile (tile w at off + w * tb)
-  int32_t slot;  // limb slot of the block's first step
-  int32_t geo;   // bits | nq << 4 | ns << 8 | last << 16 (valid ranks of the final shift step)
-};
-struct UoBand {  // a 2/3-bit band, for the limb build
-  int32_t rank, r0, slot0, boff, full, code_full, code_last, nblk;
-};
-struct UoTail {
-  UoBlk blk[UO_MAXBLK];
-  UoBand band[DC_MAX_BANDS];
-  int32_t win_blk[UO_MAXWIN + 1];  // first block of each window
-  alignas(16) float zpart[2][8][DC_V_TOKS];
-  int64_t run0;                     // device address of group 0's run
-  int32_t u_unit, st, len, nb, nwin, nblk, ok;
-  float umax;
-  int32_t n8;                       // 8-bit bands
-  int32_t b8[DC_MAX_BANDS][4];      // per 8-bit band: rank, r0, offset in the run, bytes of a full block
-  int32_t next[2];                  // claimed chunks, alternating: read one while the other is claimed
-};
-static_assert(2 * UO_LBUF + 8 * UO_D * UO_SLOT + sizeof(UoTail) + 128 + 1024 <= 233472 / UO_CTAS_PER_SM,
-              "k_uout shared memory");
-
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-// Exponent e of the fixed-point image of scale * t, as ud_exponent (frexpf's exponent read from the
-// bits; bounds below the normal range take the clamp's end), and 2^e / 2^-e built from their bits.
-__device__ __forceinline__ void uo_exponent(float umax, int tmax_bits, float& pe, float& ie) {
-  const float bound = umax * __int_as_float(tmax_bits);
-  int e = 0;
-  if (bound > 0.f) {
-    const int bits = __float_as_int(bound);
-    const int E = bits >= 0x00800000 ? ((bits >> 23) & 0xff) - 126 : -126;
-    e = max(-120, min(120, 21 - E));
-  }
-  pe = __int_as_float((127 + e) << 23);
-  ie = __int_as_float((127 - e) << 23);
-}
-
-// MMAs of this warp's tile of one block (codes at `tile`, a ring slot): `nq` mask-layout quads then
-// `ns` shift-layout steps; `brow` is this lane's B row of pair 0 at the block's first slot.
-template <int NPAIR>
-__device__ __forceinline__ void uo_block(const uint8_t* tile, int geo, const uint8_t* brow, int pstride,
-                                         int (&C)[2][4][4], int lane) {
-  const int bits = geo & 15, nq = (geo >> 4) & 15, ns = (geo >> 8) & 255, last = geo >> 16;
-  if (nq == 2 && ns == 0) {  // full 2-bit block: two quads in straight-line code
-#pragma unroll
-    for (int q = 0; q < 2; ++q) {
-      const uint4 wq = *reinterpret_cast<const uint4*>(tile + 512 * q + 16 * lane);
-#pragma unroll
-      for (int ps = 0; ps < 4; ++ps) {
-        const uint32_t msk = 0x03030303u << (2 * ps);
-#pragma unroll
-        for (int pr = 0; pr < NPAIR; ++pr) {
-          const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * (4 * q + ps));
-          mma_u8u8(C[pr][ps], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bb.x, bb.y);
-        }
-      }
-    }
-    return;
-  }
-  for (int q = 0; q < nq; ++q) {
-    const uint4 wq = *reinterpret_cast<const uint4*>(tile + 512 * q + 16 * lane);
-#pragma unroll
-    for (int ps = 0; ps < 4; ++ps) {
-      const uint32_t msk = 0x03030303u << (2 * ps);
-#pragma unroll
-      for (int pr = 0; pr < NPAIR; ++pr) {
-        const uint2 bb = *reinterpret_cast<const uint2*>(brow + pr * pstride + 32 * (4 * q + ps));
-        mma_u8u8(C[pr][ps], wq.x & msk, wq.y & msk, wq.z & msk, wq.w & msk, bb.x, bb.y);
-      }
-    }
-  }
-  if (ns == 0) return;
-  // shift-layout steps (ud_steps' layout), reading the tile copy in the ring
-  const uint8_t* sb = tile + 512 * nq;
-  const uint8_t* bs = brow + 32 * 4 * nq;
-  const int SB = bits == 3 ? 192 : 128;
-  const int nfull = last == 32 ? ns : ns - 1;
-  for (int si = 0; si < nfull; ++si) {
-    const uint8_t* p = sb + si * SB;
-    const uint32_t wv = reinterpret_cast<const uint32_t*>(p)[lane];
-    uint32_t a[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) a[j] = reg_shift2(wv, j);
-    if (bits == 3) {
-      const uint32_t hv = reinterpret_cast<const uint16_t*>(p + 128)[lane];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) a[j] |= u_reg_hi3(hv, j);
-    }
-#pragma unroll
-    for (int pr = 0; pr < NPAIR; ++pr) {
-      const uint2 bb = *reinterpret_cast<const uint2*>(bs + pr * pstride + 32 * si);
-      mma_u8u8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
-    }
-  }
-  if (nfull == ns) return;
-  const uint8_t* p = sb + nfull * SB;
-  const int nl = dc_u_step_lanes(last), ntv = nl / 8;
-  const int g = lane >> 2, t = lane & 3;
-  uint32_t wv = 0, hv = 0;
-  if (t < ntv) {
-    wv = *reinterpret_cast<const uint32_t*>(p + 4 * (g * ntv + t));
-    if (bits == 3) hv = *reinterpret_cast<const uint16_t*>(p + 4 * nl + 2 * (g * ntv + t));
-  }
-  uint32_t a[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    a[j] = reg_shift2(wv, j);
-    if (bits == 3) a[j] |= u_reg_hi3(hv, j);
-  }
-#pragma unroll
-  for (int pr = 0; pr < NPAIR; ++pr) {
-    const uint2 bb = *reinterpret_cast<const uint2*>(bs + pr * pstride + 32 * nfull);
-    mma_u8u8(C[pr][0], a[0], a[1], a[2], a[3], bb.x, bb.y);
-  }
-}
-
-// Warp 0: record of (linear p, segment sg) -> the chunk's shared tables (tl->ok: work or not).
-__device__ void uo_setup(const DcFwd& F, const WsPtr& P, UoTail* tl, int p, int sg, int lane) {
-  const DcURec& R = P.urecs[(int64_t)p * F.ws.T + sg];
-  const bool ok = R.valid && !(F.pf && R.len >= DC_PF_MIN);
-  if (!ok) {
-    if (lane == 0) tl->ok = 0;
-    return;
-  }
-  // bands: 8-bit on their own; 2/3-bit with limb slots (each band's first slot a multiple of 256, so
-  // that no block -- 256 ranks at most, starting at a multiple of 256 in its band -- straddles a window)
-  int nb = 0, slot = 0, n8 = 0, nblk = 0;
-  for (int b = 0; b < R.n_bands; ++b) {
-    const DcUBand& U = R.band[b];
-    if (U.bits == 8) {
-      if (lane == 0) {
-        tl->b8[n8][0] = U.rank, tl->b8[n8][1] = U.r0, tl->b8[n8][2] = U.boff, tl->b8[n8][3] = U.full;
-      }
-      ++n8;
-      continue;
-    }
-    DcBand B;
-    B.bits = U.bits, B.rank = U.rank, B.r0 = U.r0;
-    B.u_quads = U.quads, B.u_steps = U.steps, B.u_last = U.last;
-    const DcUBlk K0 = dc_u_block(B, 0), KL = dc_u_block(B, U.nblk - 1);
-    if (lane == 0) {
-      UoBand& O = tl->band[nb];
-      O.rank = U.rank, O.r0 = U.r0, O.slot0 = slot, O.boff = U.boff, O.full = U.full;
-      O.code_full = K0.code_bytes, O.code_last = KL.code_bytes, O.nblk = U.nblk;
-    }
-    // the band's blocks, one lane each
-    for (int k = lane; k < U.nblk; k += 32) {
-      const DcUBlk K = dc_u_block(B, k);
-      if (nblk + k < UO_MAXBLK) {
-        UoBlk& o = tl->blk[nblk + k];
-        o.off = U.boff + k * U.full;
-        o.tb = K.tile_bytes;
-        o.slot = slot + (U.bits == 2 ? (K.nq > 0 ? 128 * K.q0 : 128 * U.quads) : 32 * K.s0);
-        o.geo = U.bits | (K.nq << 4) | (K.ns << 8) | (K.last << 16);
-      }
-    }
-    nblk += U.nblk;
-    slot += (int)dc_align(U.rank, 256);
-    ++nb;
-  }
-  __syncwarp();
-  const int nwin = max(1, (slot + UO_LMAX - 1) / UO_LMAX);
-  if (nblk > UO_MAXBLK || nwin > UO_MAXWIN) {
-    if (lane == 0) {
-      set_status(P.st, DC_ERR_UNSUPPORTED);
-      tl->ok = 0;
-    }
-    return;
-  }
-  // first block of each window (blocks are in slot order and none straddles a window; checked here)
-  bool straddle = false;
-  for (int k = lane; k < nblk; k += 32) {
-    const UoBlk& o = tl->blk[k];
-    const int ns = (o.geo >> 8) & 255, nq = (o.geo >> 4) & 15;
-    const int end = o.slot + 128 * nq + 32 * ns - 1;
-    straddle |= (o.slot / UO_LMAX) != (end / UO_LMAX);
-  }
-  if (__any_sync(FULLMASK, straddle)) {
-    if (lane == 0) {
-      set_status(P.st, DC_ERR_UNSUPPORTED);
-      tl->ok = 0;
-    }
-    return;
-  }
-  for (int w = lane; w <= nwin; w += 32) {
-    int lo = 0;
-    if (w == nwin) {
-      lo = nblk;
-    } else {
-      while (lo < nblk && tl->blk[lo].slot < w * UO_LMAX) ++lo;
-    }
-    tl->win_blk[w] = lo;
-  }
-  if (lane == 0) {
-    tl->ok = 1;
-    tl->nb = nb;
-    tl->nwin = nwin;
-    tl->nblk = nblk;
-    tl->run0 = R.blob + R.u_off;
-    tl->u_unit = R.u_unit;
-    tl->st = R.st;
-    tl->len = R.len;
-    tl->umax = R.umax;
-    tl->n8 = n8;
-  }
-}
-
-// Limb matrix of window `wi` of one unit (all 256 threads), the unit's 8-bit sums for this warp's
-// rows (window 0) and, at the last window, the warp partials of the zero-point sums.
-template <int NTOK>
-__device__ __forceinline__ void uo_build(const UoTail* tl, float* zpart, uint8_t* lb, const uint8_t* run,
-                                         const float* tw, int rs, const float (&pe)[NTOK], int ntok, int wi,
-                                         float (&zc)[NTOK], float (&s8)[NTOK], int tid, int warp, int lane) {
-  const int s_lo = wi * UO_LMAX, s_hi = s_lo + UO_LMAX;
-  for (int b = 0; b < tl->nb; ++b) {
-    const UoBand& B = tl->band[b];
-    const int j_lo = max(0, s_lo - B.slot0), j_hi = min(B.rank, s_hi - B.slot0);
-    for (int j = j_lo + 4 * tid; j < j_hi; j += 4 * UO_THREADS) {
-      const int k = j >> 8, within = j & 255;
-      const uint8_t* mp = run + B.boff + (int64_t)k * B.full + (k < B.nblk - 1 ? B.code_full : B.code_last) + 4 * within;
-      const uint4 mz = ldg128(mp);
-      float sc[4], zs[4];
-      const uint32_t mw[4] = {mz.x, mz.y, mz.z, mz.w};
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const __half2 h = *reinterpret_cast<const __half2*>(&mw[r]);
-        sc[r] = j + r < j_hi ? __low2float(h) : 0.f;
-        zs[r] = sc[r] * __high2float(h);
-      }
-      uint8_t* col = lb + (B.slot0 + j - s_lo);
-#pragma unroll
-      for (int q = 0; q < NTOK; ++q) {
-        if (q >= ntok) break;
-        uint32_t v[4];
-#pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float tq = j + r < j_hi ? tw[q * rs + B.r0 + j + r] : 0.f;
-          v[r] = __float_as_uint(fmaf(sc[r], tq * pe[q], U_MAGIC));
-          zc[q] = fmaf(zs[r], tq, zc[q]);
-        }
-        const uint32_t lo = __byte_perm(v[0], v[1], 0x5140), hi = __byte_perm(v[2], v[3], 0x5140);
-        const uint32_t l2 = __byte_perm(__byte_perm(v[0], v[1], 0x0062), __byte_perm(v[2], v[3], 0x0062), 0x5410);
-        uint8_t* c = col + (6 * (q >> 1) + (q & 1)) * UO_LROW;
-        *reinterpret_cast<uint32_t*>(c) = __byte_perm(lo, hi, 0x5410);
-        *reinterpret_cast<uint32_t*>(c + 2 * UO_LROW) = __byte_perm(lo, hi, 0x7632);
-        *reinterpret_cast<uint32_t*>(c + 4 * UO_LROW) = l2;
-      }
-    }
-  }
-  // 8-bit ranks in fp32 for this warp's rows: lane l takes row 16 warp + (l & 15), ranks of parity l >> 4
-  for (int b8 = 0; wi == 0 && b8 < tl->n8; ++b8) {
-    const int rank8 = tl->b8[b8][0], r08 = tl->b8[b8][1], boff8 = tl->b8[b8][2], full8 = tl->b8[b8][3];
-    const int row = 16 * warp + (lane & 15);
-    for (int k = 0; 64 * k < rank8; ++k) {
-      const int nr = min(64, rank8 - 64 * k);
-      const uint8_t* blk = run + boff8 + (int64_t)k * full8;
-      const uint8_t* meta = blk + dc_align((int64_t)128 * nr, 16);
-      for (int kk = lane >> 4; kk < nr; kk += 2) {
-        const float c = (float)blk[row * nr + kk];
-        const __half2 h = *reinterpret_cast<const __half2*>(meta + 4 * kk);
-        const float f = (c - __high2float(h)) * __low2float(h);
-#pragma unroll
-        for (int q = 0; q < NTOK; ++q)
-          if (q < ntok) s8[q] = fmaf(f, tw[q * rs + r08 + 64 * k + kk], s8[q]);
-      }
-    }
-  }
-  if (wi == tl->nwin - 1) {  // the unit's zero-point sums: warp partials, summed in the epilogue
-#pragma unroll
-    for (int q = 0; q < NTOK; ++q) {
-      float v = zc[q];
-#pragma unroll
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(FULLMASK, v, o);
-      if (lane == 0) zpart[warp * DC_V_TOKS + q] = v;
-    }
-  }
-}
-
-// The stream of one chunk (groups go0 .. go0 + ngo - 1 of the record in `tl`); every unit of the
-// chunk has at most NTOK tokens.
-template <int NTOK>
-__device__ __forceinline__ void uo_chunk(const DcFwd& F, const WsPtr& P, UoTail* tl, uint8_t* lbuf, uint8_t* ring,
-                                         uint32_t& wseq, uint32_t& useq, int p, int go0, int ngo, int tid,
-                                         int warp, int lane) {
-  constexpr int NPAIR = (NTOK + 1) / 2;
-  const int T = F.ws.T, rs = F.ws.r_stride;
-  const int g = lane >> 2, t = lane & 3;
-  const int st = tl->st, len = tl->len, nblk = tl->nblk, nwin = tl->nwin;
-  const int npass = (len + DC_V_TOKS - 1) / DC_V_TOKS;
-  const int nunits = npass * ngo;
-  const uint8_t* run0 = reinterpret_cast<const uint8_t*>(tl->run0);
-  const int64_t u_unit = tl->u_unit;
-  const int pstride = (ud_brow(g, 1) - ud_brow(g, 0)) * UO_LROW;
-  // the copy stream runs UO_D - 1 blocks ahead of the multiplies, across unit boundaries
-  int iss_k = 0, iss_un = nblk > 0 ? 0 : nunits, iss_slot = 0;
-  const uint8_t* iss_run = run0 + (int64_t)go0 * u_unit;
-  auto issue_next = [&]() {
-    if (iss_un < nunits) {
-      const UoBlk b = tl->blk[iss_k];
-      const uint8_t* src = iss_run + b.off + warp * b.tb;
-      uint8_t* dst = ring + iss_slot * UO_SLOT;
-      for (int o = 16 * lane; o < b.tb; o += 512) cp_async16(dst + o, src + o);
-      if (++iss_k == nblk) {
-        iss_k = 0;
-        ++iss_un;
-        iss_run = run0 + (int64_t)(go0 + iss_un % ngo) * u_unit;
-      }
-    }
-    cp_async_commit();
-    if (++iss_slot == UO_D) iss_slot = 0;
-  };
-#pragma unroll 1
-  for (int k = 0; k < UO_D - 1; ++k) issue_next();
-  int cslot = 0;
-  for (int un = 0; un < nunits; ++un) {
-    const int go = go0 + un % ngo, tok0 = st + DC_V_TOKS * (un / ngo);
-    const int ntok = min(DC_V_TOKS, st + len - tok0);
-    const uint8_t* run = run0 + (int64_t)go * u_unit;
-    // exponents: lane q computes token q's, every lane takes them by shuffle
-    float pq = 1.f, iq = 1.f;
-    if (lane < ntok) uo_exponent(tl->umax, P.tmax[p * T + tok0 + lane], pq, iq);
-    float pe[NTOK], ie[NTOK];
-#pragma unroll
-    for (int q = 0; q < NTOK; ++q) {
-      pe[q] = __shfl_sync(FULLMASK, pq, q);
-      ie[q] = __shfl_sync(FULLMASK, iq, q);
-    }
-    const float* tw = P.tws + ((int64_t)p * T + tok0) * rs;
-    int C[2][4][4];
-#pragma unroll
-    for (int a = 0; a < 2; ++a)
-#pragma unroll
-      for (int b = 0; b < 4; ++b)
-#pragma unroll
-        for (int q = 0; q < 4; ++q) C[a][b][q] = 0;
-    float zc[NTOK], s8[NTOK];
-#pragma unroll
-    for (int q = 0; q < NTOK; ++q) zc[q] = s8[q] = 0.f;
-    float* zpart = &tl->zpart[useq & 1][0][0];
-    for (int wi = 0; wi < nwin; ++wi) {
-      uint8_t* lb = lbuf + (wseq & 1) * UO_LBUF;
-      uo_build<NTOK>(tl, zpart, lb, run, tw, rs, pe, ntok, wi, zc, s8, tid, warp, lane);
-      __syncthreads();
-      ++wseq;
-      const uint8_t* brow0 = lb + ud_brow(g, 0) * UO_LROW + 8 * t - wi * UO_LMAX;
-      const int k1 = tl->win_blk[wi + 1];
-#pragma unroll 1
-      for (int k = tl->win_blk[wi]; k < k1; ++k) {
-        issue_next();
-        cp_async_wait<UO_D - 1>();
-        __syncwarp();  // every lane's copies of this block have landed
-        const UoBlk b = tl->blk[k];
-        uo_block<NPAIR>(ring + cslot * UO_SLOT, b.geo, brow0 + b.slot, pstride, C, lane);
-        __syncwarp();  // the slot is read before any lane copies into it again
-        if (++cslot == UO_D) cslot = 0;
-      }
-    }
-    // ---- epilogue (as k_udelta): 8-bit sums to every lane of the row, zero-point sum per token
-#pragma unroll
-    for (int q = 0; q < NTOK; ++q) s8[q] += __shfl_xor_sync(FULLMASK, s8[q], 16);
-    const int orow = 16 * warp + g + 8 * (t >> 1);
-#pragma unroll
-    for (int pr = 0; pr < NPAIR; ++pr) {
-      const float s8a = __shfl_sync(FULLMASK, s8[2 * pr], g + 8 * (t >> 1));
-      const float s8b = __shfl_sync(FULLMASK, s8[2 * pr + 1], g + 8 * (t >> 1));
-      if (2 * pr >= ntok) continue;
-      int w[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) w[r] = C[pr][0][r] + (C[pr][1][r] >> 2) + (C[pr][2][r] >> 4) + (C[pr][3][r] >> 6);
-      if (t == 3) {
-        w[1] = w[0];
-        w[3] = w[2];
-      }
-      {
-        const bool o = t & 1;
-        const int a = __shfl_xor_sync(FULLMASK, o ? w[0] : w[1], 1);
-        const int b = __shfl_xor_sync(FULLMASK, o ? w[2] : w[3], 1);
-        if (o) { w[0] = a; w[2] = b; } else { w[1] = a; w[3] = b; }
-      }
-      {
-        const bool o = (t >> 1) & 1;
-        const int a = __shfl_xor_sync(FULLMASK, o ? w[0] : w[2], 2);
-        const int b = __shfl_xor_sync(FULLMASK, o ? w[1] : w[3], 2);
-        if (o) { w[0] = a; w[1] = b; } else { w[2] = a; w[3] = b; }
-      }
-      const int q = 2 * pr + (t & 1);
-      if (q < ntok) {
-        float zs = 0.f;
-#pragma unroll
-        for (int w8 = 0; w8 < 8; ++w8) zs += zpart[w8 * DC_V_TOKS + q];
-        const float v = (float)(w[2] - 64 * w[3]) * 65536.f + (float)w[1] * 256.f + (float)w[0];
-        const float ieq = (t & 1) ? ie[2 * pr + 1] : ie[2 * pr];
-        const float y = fmaf(v, ieq, -zs) + ((t & 1) ? s8b : s8a);
-        P.yd[((int64_t)p * T + tok0 + q) * F.ws.max_d_in + 128 * go + orow] = y;
-      }
-    }
-    ++useq;
-  }
-  cp_async_wait<0>();
-  __syncwarp();
-}
-
-__global__ void __launch_bounds__(UO_THREADS, UO_CTAS_PER_SM) k_uout(const __grid_constant__ DcFwd F, uint8_t* ws) {
-  extern __shared__ __align__(128) uint8_t uosm[];
-  uint8_t* lbuf = uosm;
-  UoTail* tl = reinterpret_cast<UoTail*>(uosm + 2 * UO_LBUF);
-  uint8_t* rings = uosm + 2 * UO_LBUF + dc_align(sizeof(UoTail), 128);
-  WsPtr P = ws_ptr(F.ws, ws);
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  uint8_t* ring = rings + warp * (UO_D * UO_SLOT);
-  // constant rows 12..15 of both limb matrices: ones (the codes' row sums) in rows 12 and 14, zeros
-  for (int i = tid; i < 2 * UO_LROW; i += UO_THREADS) {
-    const int b = i / UO_LROW, wv = i % UO_LROW, row = 12 + wv / (UO_LROW / 4);
-    reinterpret_cast<uint32_t*>(lbuf + b * UO_LBUF + 12 * UO_LROW)[wv] = (row == 12 || row == 14) ? 0x01010101u : 0u;
-  }
-  const int nseg = P.st[DC_WS_NSEG];
-  if (tid == 0) tl->next[0] = atomicAdd(P.st + DC_WS_UCOUNTER, 1);
-  __syncthreads();
-  uint32_t wseq = 0, useq = 0;
-  for (uint32_t c = 0;; ++c) {
-    const int u = tl->next[c & 1];
-    int p = 0, sg = 0, go0 = 0, ngo = 0;
-    const bool have = nseg > 0 && ud_chunk(F, nseg, u, p, sg, go0, ngo);
-    if (!have) break;
-    if (warp == 0) {
-      uo_setup(F, P, tl, p, sg, lane);
-      if (lane == 0) tl->next[(c + 1) & 1] = atomicAdd(P.st + DC_WS_UCOUNTER, 1);
-    }
-    __syncthreads();
-    if (tl->ok) {
-      if (tl->len <= 2)
-        uo_chunk<2>(F, P, tl, lbuf, ring, wseq, useq, p, go0, ngo, tid, warp, lane);
-      else
-        uo_chunk<4>(F, P, tl, lbuf, ring, wseq, useq, p, go0, ngo, tid, warp, lane);
-    }
-    __syncthreads();  // every warp is done with this chunk's tables
   }
 }
 
@@ -3883,21 +3404,11 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     const size_t usmem = (size_t)U_STAGES * U_STAGE_BYTES + 2 * U_GSTAGE * U_LBUF + sizeof(USmemTail);
     if (usmem > 227 * 1024)
       return dc_fail(DC_ERR_UNSUPPORTED, "max_rank %d needs %zu bytes of shared memory", max_rank, usmem);
-    static const bool stream_u = getenv("DC_U_STREAM") != nullptr;  // experimental streaming U kernel
-    if (!stream_u) {
-      st = allow_smem(dev, DC_K_UDELTA, (const void*)k_udelta, usmem);
-      if (st) return st;
-      prof_before(s, 3);
-      k_udelta<<<U_CTAS_PER_SM * n_sm, U_THREADS, usmem, s>>>(F, (uint8_t*)ws);
-      prof_after(s);
-    } else {
-      const size_t osmem = 2 * (size_t)UO_LBUF + dc_align(sizeof(UoTail), 128) + 8 * UO_D * UO_SLOT;
-      st = allow_smem(dev, DC_K_UDELTA, (const void*)k_uout, osmem);
-      if (st) return st;
-      prof_before(s, 3);
-      k_uout<<<UO_CTAS_PER_SM * n_sm, UO_THREADS, osmem, s>>>(F, (uint8_t*)ws);
-      prof_after(s);
-    }
+    st = allow_smem(dev, DC_K_UDELTA, (const void*)k_udelta, usmem);
+    if (st) return st;
+    prof_before(s, 3);
+    k_udelta<<<U_CTAS_PER_SM * n_sm, U_THREADS, usmem, s>>>(F, (uint8_t*)ws);
+    prof_after(s);
     st = dc_cuda_check(cudaGetLastError(), "delta output kernel");
     if (st) return st;
     if (F.pf) {
