@@ -57,6 +57,7 @@ dc_status dc_check_desc(const dc_factor_desc* d, DcLayout* L) {
 }
 
 extern "C" size_t dc_packed_size(const dc_factor_desc* desc) {
+  DC_NVTX("dc_packed_size");
   DcLayout L;
   if (dc_check_desc(desc, &L) != DC_OK) return 0;
   return (size_t)L.bytes;
@@ -133,6 +134,7 @@ bool dc_rtn_group(const float* v, int64_t stride, int n, int bits, uint8_t* code
 
 extern "C" dc_status dc_quantize_rtn(const dc_factor_desc* desc, const float* U, const float* Vt,
                                      uint8_t* codes_u, uint8_t* codes_v, uint16_t* sz_u, uint16_t* sz_v) {
+  DC_NVTX("dc_quantize_rtn");
   dc_clear_error();
   DcLayout L;
   dc_status st = dc_check_desc(desc, &L);
@@ -199,6 +201,7 @@ void dc_fill_handle(const dc_factor_desc* desc, const DcLayout& L, void* dev, dc
 extern "C" dc_status dc_pack_upload(const dc_factor_desc* desc, const uint8_t* codes_u, const uint8_t* codes_v,
                                     const uint16_t* sz_u, const uint16_t* sz_v, const float* S, void* dev_dst,
                                     size_t dev_bytes, void* stream, dc_delta_handle* out) {
+  DC_NVTX("dc_pack_upload");
   dc_clear_error();
   DcLayout L;
   dc_status st = dc_check_desc(desc, &L);
@@ -230,6 +233,7 @@ extern "C" dc_status dc_pack_upload(const dc_factor_desc* desc, const uint8_t* c
 
 extern "C" dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int32_t n, void* dev_dst,
                                             size_t dev_bytes, void* stream) {
+  DC_NVTX("dc_tenant_table_upload");
   dc_clear_error();
   if (n < 0 || (n > 0 && (!handles || !dev_dst))) return dc_fail(DC_ERR_INVALID_ARG, "bad tenant table arguments");
   if (((uintptr_t)dev_dst) % 16) return dc_fail(DC_ERR_ALIGN, "tenant table must be 16-byte aligned");

@@ -6,6 +6,18 @@
 #include "dc.h"
 #include "dc_layout.h"
 
+#include <nvtx3/nvToolsExt.h>
+
+// An NVTX range named after the entry point for the duration of the call (header-only NVTX v3: a
+// no-op unless a profiler or tracer is attached to the process).
+struct DcNvtxRange {
+  explicit DcNvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~DcNvtxRange() { nvtxRangePop(); }
+  DcNvtxRange(const DcNvtxRange&) = delete;
+  DcNvtxRange& operator=(const DcNvtxRange&) = delete;
+};
+#define DC_NVTX(name) DcNvtxRange dc_nvtx_range_(name)
+
 dc_status dc_fail(dc_status st, const char* fmt, ...);
 dc_status dc_cuda_check(cudaError_t e, const char* what);
 void dc_clear_error();

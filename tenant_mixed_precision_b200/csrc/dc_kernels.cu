@@ -152,6 +152,7 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
 
 extern "C" size_t dc_workspace_size(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_linears,
                                     int32_t max_tenants) {
+  DC_NVTX("dc_workspace_size");
   if (T < 0 || max_rank < 0 || max_d_in < 0 || (n_linears != 1 && n_linears != 7) || max_tenants < 0) return 0;
   return (size_t)dc_ws_layout(T, max_rank, max_d_in, n_linears, max_tenants).total;
 }
@@ -3069,6 +3070,7 @@ static void prof_after(cudaStream_t s) {
 }
 
 extern "C" dc_status dc_profile_begin(int32_t capacity) {
+  DC_NVTX("dc_profile_begin");
   dc_clear_error();
   if (g_prof.ev) return dc_fail(DC_ERR_INVALID_ARG, "profiling already active");
   if (capacity <= 0) return dc_fail(DC_ERR_INVALID_ARG, "capacity must be positive");
@@ -3090,6 +3092,7 @@ extern "C" dc_status dc_profile_begin(int32_t capacity) {
 }
 
 extern "C" int32_t dc_profile_end(float* ms_out, int32_t* kind_out, int32_t capacity) {
+  DC_NVTX("dc_profile_end");
   dc_clear_error();
   if (!g_prof.ev) return -1;
   int32_t n = g_prof.n;
@@ -3114,6 +3117,7 @@ extern "C" int32_t dc_profile_end(float* ms_out, int32_t* kind_out, int32_t capa
 }
 
 extern "C" size_t dc_quantize_scratch_size(const dc_factor_desc* desc) {
+  DC_NVTX("dc_quantize_scratch_size");
   DcLayout L;
   if (dc_check_desc(desc, &L) != DC_OK) return 0;
   return (size_t)(256 + dc_align((int64_t)L.r * L.d_out, 256) + dc_align((int64_t)L.r * L.d_in, 256) +
@@ -3123,6 +3127,7 @@ extern "C" size_t dc_quantize_scratch_size(const dc_factor_desc* desc) {
 extern "C" dc_status dc_quantize_pack_device(const dc_factor_desc* desc, const float* U_dev, const float* Vt_dev,
                                              const float* S_dev, void* dev_dst, size_t dev_bytes, void* scratch,
                                              size_t scratch_bytes, void* stream, dc_delta_handle* out) {
+  DC_NVTX("dc_quantize_pack_device");
   dc_clear_error();
   DcLayout L;
   dc_status st = dc_check_desc(desc, &L);
@@ -3189,6 +3194,7 @@ static dc_status allow_smem(int dev, int kid, const void* fn, size_t need) {
 
 extern "C" dc_status dc_build_segments(const int32_t* tenant_ids_dev, int32_t T, int32_t n_tenants, void* ws,
                                        size_t ws_bytes, void* stream) {
+  DC_NVTX("dc_build_segments");
   dc_clear_error();
   if (T < 0 || n_tenants < 0) return dc_fail(DC_ERR_INVALID_ARG, "negative T or tenant count");
   if (n_tenants > DC_MAX_TENANTS) return dc_fail(DC_ERR_UNSUPPORTED, "at most %d tenants per call", DC_MAX_TENANTS);
@@ -3207,8 +3213,12 @@ extern "C" dc_status dc_build_segments(const int32_t* tenant_ids_dev, int32_t T,
 
 extern "C" dc_status dc_read_segments(const void* ws, int32_t T, int32_t* perm_dev, int32_t* inv_perm_dev,
                                       int32_t* segments_dev, int32_t* n_segments_dev, void* stream) {
+  DC_NVTX("dc_read_segments");
   dc_clear_error();
   if (!ws || T < 0) return dc_fail(DC_ERR_INVALID_ARG, "bad arguments");
+  if (!aligned16(ws) || !aligned16(perm_dev) || !aligned16(inv_perm_dev) || !aligned16(segments_dev) ||
+      !aligned16(n_segments_dev))
+    return dc_fail(DC_ERR_ALIGN, "device pointers must be 16-byte aligned");
   const DcWs W = dc_ws_layout(T, 0, 0, 1, 0);
   cudaStream_t s = (cudaStream_t)stream;
   const uint8_t* b = (const uint8_t*)ws;
@@ -3459,6 +3469,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
 extern "C" dc_status dc_delta_linear_segmented(const dc_linear* lin, const void* x, void* y, const int32_t* tenant_ids_dev,
                                                int32_t T, int32_t dtype_in, int32_t dtype_out, int32_t flags, void* ws,
                                                size_t ws_bytes, void* stream) {
+  DC_NVTX("dc_delta_linear_segmented");
   dc_clear_error();
   if (!lin) return dc_fail(DC_ERR_INVALID_ARG, "null linear");
   const void* xs[1] = {x};
@@ -3470,6 +3481,7 @@ extern "C" dc_status dc_delta_linear_segmented(const dc_linear* lin, const void*
 extern "C" dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* x_o, const void* x_f,
                                       void* const y[7], const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
                                       int32_t dtype_out, int32_t flags, void* ws, size_t ws_bytes, void* stream) {
+  DC_NVTX("dc_layer_forward");
   dc_clear_error();
   if (!lin || !y) return dc_fail(DC_ERR_INVALID_ARG, "null linear array or outputs");
   const void* xs[3] = {x_h, x_o, x_f};
@@ -3478,8 +3490,10 @@ extern "C" dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, c
 }
 
 extern "C" dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t which, uint8_t* out_dev, void* stream) {
+  DC_NVTX("dc_unpack_codes_debug");
   dc_clear_error();
   if (!h || !out_dev || h->dev_base == 0) return dc_fail(DC_ERR_INVALID_ARG, "bad handle or output");
+  if (!aligned16(out_dev) || (h->dev_base & 255) != 0) return dc_fail(DC_ERR_ALIGN, "output or blob misaligned");
   DcLayout L;
   dc_status st = dc_check_desc(&h->desc, &L);
   if (st) return st;
@@ -3503,8 +3517,10 @@ extern "C" dc_status dc_unpack_codes_debug(const dc_delta_handle* h, int32_t whi
 }
 
 extern "C" dc_status dc_read_device_status(void* ws, void* stream, int32_t* host_status) {
+  DC_NVTX("dc_read_device_status");
   dc_clear_error();
   if (!ws || !host_status) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(ws)) return dc_fail(DC_ERR_ALIGN, "workspace must be 16-byte aligned");
   cudaStream_t s = (cudaStream_t)stream;
   int32_t v = 0;
   dc_status st = dc_cuda_check(cudaMemcpyAsync(&v, ws, 4, cudaMemcpyDeviceToHost, s), "status read");
@@ -3531,11 +3547,14 @@ extern "C" dc_status dc_delta_linear_segmented_static(const dc_linear* lin, cons
                                                       const int32_t* tenant_ids_dev, int32_t T, int32_t dtype_in,
                                                       int32_t dtype_out, int32_t flags, void* stream,
                                                       int32_t* host_status) {
+  DC_NVTX("dc_delta_linear_segmented_static");
   dc_clear_error();
   if (!lin) return dc_fail(DC_ERR_INVALID_ARG, "null linear");
   if (flags & DC_REUSE_ROUTING)
     return dc_fail(DC_ERR_INVALID_ARG, "the static workspace rebuilds the routing on every call (no DC_REUSE_ROUTING)");
   if (T < 0) return dc_fail(DC_ERR_INVALID_ARG, "negative T");
+  if (!aligned16(x) || !aligned16(y) || !aligned16(lin->W_base))
+    return dc_fail(DC_ERR_ALIGN, "device pointers must be 16-byte aligned");
   if (T == 0) {  // nothing launched: report a clean status
     if (host_status) *host_status = 0;
     return DC_OK;

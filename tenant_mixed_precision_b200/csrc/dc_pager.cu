@@ -65,6 +65,7 @@ static size_t pager_scratch_recs(const dc_pager_desc* d) {
 }
 
 extern "C" size_t dc_pager_scratch_size(const dc_pager_desc* d) {
+  DC_NVTX("dc_pager_scratch_size");
   if (!d || d->n_slots <= 0 || d->n_tables <= 0) return 0;
   return pager_scratch_recs(d) * sizeof(PatchRec);
 }
@@ -72,6 +73,7 @@ extern "C" size_t dc_pager_scratch_size(const dc_pager_desc* d) {
 extern "C" dc_status dc_pager_create(const dc_pager_desc* d, void* arena_dev, size_t arena_bytes,
                                      void* const* tables_dev, void* scratch_dev, size_t scratch_bytes,
                                      dc_pager** out) {
+  DC_NVTX("dc_pager_create");
   dc_clear_error();
   if (!d || !out || !arena_dev || !tables_dev || !scratch_dev) return dc_fail(DC_ERR_INVALID_ARG, "null argument");
   *out = nullptr;
@@ -108,6 +110,7 @@ extern "C" dc_status dc_pager_create(const dc_pager_desc* d, void* arena_dev, si
 
 extern "C" dc_status dc_pager_set_tenant(dc_pager* P, int32_t tenant, const void* image_host, uint64_t image_bytes,
                                          const int64_t* blob_offsets) {
+  DC_NVTX("dc_pager_set_tenant");
   dc_clear_error();
   if (!P || !image_host || !blob_offsets) return dc_fail(DC_ERR_INVALID_ARG, "null argument");
   if (tenant < 0 || tenant >= P->d.n_tenants) return dc_fail(DC_ERR_TENANT, "tenant %d out of range", tenant);
@@ -130,6 +133,7 @@ extern "C" dc_status dc_pager_set_tenant(dc_pager* P, int32_t tenant, const void
 
 extern "C" dc_status dc_pager_prepare(dc_pager* P, const int32_t* tenant_ids_host, int32_t T, void* copy_stream,
                                       void* compute_stream) {
+  DC_NVTX("dc_pager_prepare");
   dc_clear_error();
   if (!P || (T > 0 && !tenant_ids_host)) return dc_fail(DC_ERR_INVALID_ARG, "null argument");
   if (T < 0) return dc_fail(DC_ERR_INVALID_ARG, "negative T");
@@ -192,6 +196,7 @@ extern "C" dc_status dc_pager_prepare(dc_pager* P, const int32_t* tenant_ids_hos
 }
 
 extern "C" dc_status dc_pager_commit(dc_pager* P, void* compute_stream) {
+  DC_NVTX("dc_pager_commit");
   dc_clear_error();
   if (!P) return dc_fail(DC_ERR_INVALID_ARG, "null pager");
   for (int32_t s : P->batch_slots) {
@@ -204,15 +209,18 @@ extern "C" dc_status dc_pager_commit(dc_pager* P, void* compute_stream) {
 }
 
 extern "C" dc_status dc_pager_get_stats(const dc_pager* P, dc_pager_stats* out) {
+  DC_NVTX("dc_pager_get_stats");
   dc_clear_error();
   if (!P || !out) return dc_fail(DC_ERR_INVALID_ARG, "null argument");
   *out = P->stats;
   return DC_OK;
 }
 
-extern "C" int32_t dc_pager_slot_of(const dc_pager* P, int32_t tenant) { return P ? P->lru.slot_of(tenant) : -1; }
+extern "C" int32_t dc_pager_slot_of(const dc_pager* P, int32_t tenant) {
+  DC_NVTX("dc_pager_slot_of"); return P ? P->lru.slot_of(tenant) : -1; }
 
 extern "C" dc_status dc_pager_destroy(dc_pager* P) {
+  DC_NVTX("dc_pager_destroy");
   dc_clear_error();
   if (!P) return DC_OK;
   if (P->ready) cudaEventDestroy(P->ready);

@@ -64,6 +64,7 @@ bool width_ok(int b) { return b == 0 || b == 2 || b == 3 || b == 8; }
 
 extern "C" dc_status dc_prinmix_scores(const float* Vt, const float* S, int32_t r, int32_t d_in, const float* X,
                                        int32_t n, const int32_t* widths, int32_t n_widths, double* scores) {
+  DC_NVTX("dc_prinmix_scores");
   dc_clear_error();
   if (!Vt || !S || !X || !widths || !scores) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
   if (r <= 0 || d_in <= 0 || d_in % 128 || n <= 0 || n_widths <= 0 || n_widths > 8)
@@ -100,6 +101,7 @@ extern "C" dc_status dc_prinmix_scores(const float* Vt, const float* S, int32_t 
 extern "C" dc_status dc_prinmix_allocate(const double* scores, int32_t r, const int32_t* widths, int32_t n_widths,
                                          int32_t d_out, int32_t d_in, double ratio, int32_t max_kinds,
                                          int32_t* width_out, double* objective) {
+  DC_NVTX("dc_prinmix_allocate");
   dc_clear_error();
   if (!scores || !widths || !width_out) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
   if (r <= 0 || n_widths <= 0 || n_widths > 8 || d_out <= 0 || d_in <= 0 || !(ratio > 0.0) || max_kinds < 1)
@@ -167,6 +169,7 @@ extern "C" dc_status dc_prinmix_allocate(const double* scores, int32_t r, const 
 
 extern "C" dc_status dc_prinmix_rtc(const float* U, const float* S, const float* Vt, const float* Vt_hat, int32_t k,
                                     int32_t d_out, int32_t d_in, const float* X, int32_t n, float* U_out) {
+  DC_NVTX("dc_prinmix_rtc");
   dc_clear_error();
   if (!U || !S || !Vt || !Vt_hat || !X || !U_out) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
   if (k <= 0 || d_out <= 0 || d_in <= 0 || n <= 0) return dc_fail(DC_ERR_SHAPE, "prinmix rtc: bad sizes");
@@ -251,6 +254,7 @@ extern "C" dc_status dc_prinmix_compress(const float* U, const float* S, const f
                                          const int32_t* widths, int32_t n_widths, int32_t max_kinds, int32_t rtc,
                                          dc_factor_desc* desc_out, int32_t* perm_out, float* U_out, float* S_out,
                                          float* Vt_out, double* objective) {
+  DC_NVTX("dc_prinmix_compress");
   dc_clear_error();
   if (!U || !S || !Vt || !X || !widths || !desc_out || !perm_out || !U_out || !S_out || !Vt_out)
     return dc_fail(DC_ERR_INVALID_ARG, "null pointer");

@@ -341,6 +341,7 @@ dc_status jacobi(float* M, int n, int m, float* Jt, float tol, int max_sweeps, i
 }  // namespace
 
 extern "C" size_t dc_svd_workspace_size(int32_t d_out, int32_t d_in, int32_t r, int32_t oversample) {
+  DC_NVTX("dc_svd_workspace_size");
   if (d_out <= 0 || d_in <= 0 || r <= 0 || r > std::min(d_out, d_in) || oversample < 0) return 0;
   return (size_t)svd_ws(d_out, d_in, svd_l(d_out, d_in, r, oversample)).total;
 }
@@ -349,6 +350,7 @@ extern "C" dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t
                                    int32_t r, int32_t oversample, int32_t power_iters, uint64_t seed, float* U_out,
                                    float* S_out, float* Vt_out, void* ws, size_t ws_bytes, void* stream,
                                    int32_t* sweeps_out) {
+  DC_NVTX("dc_svd_device");
   dc_clear_error();
   if (!W_ft || !W_base || !U_out || !S_out || !Vt_out || !ws) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
   if (dtype != DC_DTYPE_F32 && dtype != DC_DTYPE_BF16) return dc_fail(DC_ERR_INVALID_ARG, "dtype");
@@ -356,6 +358,9 @@ extern "C" dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t
     return dc_fail(DC_ERR_SHAPE, "rank %d outside 1..min(d_out, d_in)", r);
   if (oversample < 0 || power_iters < 0 || power_iters > 16) return dc_fail(DC_ERR_INVALID_ARG, "oversample / power_iters");
   if (((uintptr_t)ws & 255) != 0) return dc_fail(DC_ERR_ALIGN, "workspace must be 256-byte aligned");
+  const void* ptrs[5] = {W_ft, W_base, U_out, S_out, Vt_out};
+  for (const void* q : ptrs)
+    if (((uintptr_t)q & 15) != 0) return dc_fail(DC_ERR_ALIGN, "device pointers must be 16-byte aligned");
   const int l = svd_l(d_out, d_in, r, oversample);
   const SvdWs W = svd_ws(d_out, d_in, l);
   if (ws_bytes < (size_t)W.total) return dc_fail(DC_ERR_WORKSPACE, "svd workspace holds %zu bytes, needs %lld", ws_bytes,

@@ -32,6 +32,35 @@ def assert_close(got, ref, what=""):
     assert m <= lim + 1e-30, f"{what}: max abs error {m:.3e} > {lim:.3e}"
 
 
+class Guarded:
+    """A device buffer with guard bytes on both sides -- the stand-in for a memory sanitizer, which
+    is not available on the GPU pool.  The library gets the interior (4096 bytes in, so every
+    alignment rule holds); check() asserts that no byte of either guard changed, i.e. that the
+    kernels wrote nothing outside the buffer they were given."""
+
+    GUARD = 4096
+    PATTERN = 0xA5
+
+    def __init__(self, torch, shape, dtype, fill=None):
+        self.torch = torch
+        n = 1
+        for d in shape:
+            n *= int(d)
+        esz = torch.empty(0, dtype=dtype).element_size()
+        self.nbytes = n * esz
+        self.raw = torch.full((self.nbytes + 2 * self.GUARD,), self.PATTERN, dtype=torch.uint8, device="cuda")
+        self.t = self.raw[self.GUARD:self.GUARD + self.nbytes].view(dtype).view(*shape)
+        if fill is not None:
+            self.t.fill_(fill)
+
+    def check(self, what=""):
+        self.torch.cuda.synchronize()
+        head = self.raw[:self.GUARD]
+        tail = self.raw[self.GUARD + self.nbytes:]
+        bad = int((head != self.PATTERN).sum().item()) + int((tail != self.PATTERN).sum().item())
+        assert bad == 0, f"{what}: {bad} guard bytes around the buffer were overwritten"
+
+
 def gaussian_factors(rng, d_out, d_in, r, s0=1.28, alpha=0.8):
     U = (rng.standard_normal((d_out, r)) / math.sqrt(d_out)).astype(np.float32)
     Vt = (rng.standard_normal((r, d_in)) / math.sqrt(d_in)).astype(np.float32)

@@ -11,7 +11,7 @@ import oracle
 import tenant_mixed_precision_b200 as dc
 from tenant_mixed_precision_b200 import synth
 
-from dc_testlib import TenantDeltas, assert_close, gaussian_factors, oracle_y
+from dc_testlib import Guarded, TenantDeltas, assert_close, gaussian_factors, oracle_y
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -48,13 +48,14 @@ def test_codes_bit_exact_through_unpack(d_out, d_in, plan):
     assert np.array_equal(su[..., 1].view(np.float16).astype(np.float64), a.u_zeros)
     assert np.array_equal(sv[..., 1].view(np.float16).astype(np.float64), a.v_zeros)
     # packed layout decoded by the kernels' own extraction helpers == oracle codes
-    out_u = torch.full((r, d_out), 255, dtype=torch.uint8, device="cuda")
-    out_v = torch.full((r, d_in), 255, dtype=torch.uint8, device="cuda")
-    dc.dc_unpack_codes_debug(td.handles[0], 0, out_u)
-    dc.dc_unpack_codes_debug(td.handles[0], 1, out_v)
-    torch.cuda.synchronize()
-    assert np.array_equal(out_u.cpu().numpy(), a.u_codes.astype(np.uint8))
-    assert np.array_equal(out_v.cpu().numpy(), a.v_codes.astype(np.uint8))
+    gu = Guarded(torch, (r, d_out), torch.uint8, fill=255)
+    gv = Guarded(torch, (r, d_in), torch.uint8, fill=255)
+    dc.dc_unpack_codes_debug(td.handles[0], 0, gu.t)
+    dc.dc_unpack_codes_debug(td.handles[0], 1, gv.t)
+    gu.check("unpack U")
+    gv.check("unpack V")
+    assert np.array_equal(gu.t.cpu().numpy(), a.u_codes.astype(np.uint8))
+    assert np.array_equal(gv.t.cpu().numpy(), a.v_codes.astype(np.uint8))
 
 
 @pytest.mark.parametrize("d_out,d_in,plan", LAYOUT_CASES[:5])
@@ -72,7 +73,8 @@ def test_routing_bit_exact(T, n):
     rng = np.random.default_rng(T + n)
     ids = rng.integers(-1, n, size=T).astype(np.int32)
     ids_d = torch.from_numpy(ids).cuda()
-    ws = torch.zeros(dc.dc_workspace_size(T, 0, 0, 1, n), dtype=torch.uint8, device="cuda")
+    g = Guarded(torch, (dc.dc_workspace_size(T, 0, 0, 1, n),), torch.uint8, fill=0)
+    ws = g.t
     dc.dc_build_segments(ids_d, T, n, ws)
     perm = torch.empty(T, dtype=torch.int32, device="cuda")
     inv = torch.empty(T, dtype=torch.int32, device="cuda")
@@ -87,6 +89,7 @@ def test_routing_bit_exact(T, n):
     assert k == len(s)
     assert [tuple(v) for v in segs.cpu().numpy().reshape(T, 3)[:k].tolist()] == s
     assert dc.dc_read_device_status(ws) == 0
+    g.check("routing workspace")
 
 
 def test_routing_bad_id_sets_status():
@@ -100,14 +103,16 @@ def test_routing_bad_id_sets_status():
 def _run_linear(td, W, x, ids, flags, out_dtype=None):
     T = x.shape[0]
     n_ten = len(td.handles)
-    y = torch.empty((T, td.d_out), dtype=out_dtype or torch.float32, device="cuda")
-    ws = torch.zeros(dc.dc_workspace_size(T, td.max_rank, max(td.d_in, td.d_out), 1, n_ten), dtype=torch.uint8,
-                     device="cuda")
+    gy = Guarded(torch, (T, td.d_out), out_dtype or torch.float32)
+    gw = Guarded(torch, (dc.dc_workspace_size(T, td.max_rank, max(td.d_in, td.d_out), 1, n_ten),), torch.uint8, fill=0)
+    y, ws = gy.t, gw.t
     lin = td.linear(W)
     ids_d = torch.from_numpy(np.asarray(ids, np.int32)).cuda()
     dc.dc_delta_linear_segmented(lin, x, y, ids_d, T, flags, ws)
     torch.cuda.synchronize()
     assert dc.dc_read_device_status(ws) == 0
+    gy.check("output")
+    gw.check("workspace")
     return y
 
 

@@ -14,7 +14,7 @@ import pytest
 import tenant_mixed_precision_b200 as dc
 from tenant_mixed_precision_b200 import synth
 
-from dc_testlib import TenantDeltas, assert_close, gaussian_factors, oracle_y, rel_l2
+from dc_testlib import Guarded, TenantDeltas, assert_close, gaussian_factors, oracle_y, rel_l2
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -63,14 +63,17 @@ def test_prefill_path_against_oracle_and_decode_path(case, flags):
     x = torch.from_numpy(xb.view(np.int16)).cuda().view(torch.bfloat16)
     lin = td.linear(W)
     ids_d = torch.from_numpy(ids).cuda()
-    ws = torch.zeros(dc.dc_workspace_size(T, td.max_rank, max(d_in, d_out), 1, len(plans)), dtype=torch.uint8,
-                     device="cuda")
+    gw = Guarded(torch, (dc.dc_workspace_size(T, td.max_rank, max(d_in, d_out), 1, len(plans)),), torch.uint8, fill=0)
+    ws = gw.t
     outs = {}
     for extra in (0, dc.DC_DECODE_ONLY):
-        y = torch.full((T, d_out), float("nan"), dtype=torch.float32, device="cuda")
+        gy = Guarded(torch, (T, d_out), torch.float32, fill=float("nan"))
+        y = gy.t
         dc.dc_delta_linear_segmented(lin, x, y, ids_d, T, flags | extra, ws)
         torch.cuda.synchronize()
         assert dc.dc_read_device_status(ws) == 0
+        gy.check("prefill output")
+        gw.check("prefill workspace")
         outs[extra] = y.cpu().numpy().astype(np.float64)
     assert np.isfinite(outs[0]).all()
     want = oracle_y(wv.astype(np.float64), td, xv.astype(np.float64), ids, flags)
