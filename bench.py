@@ -607,9 +607,11 @@ def run_sweep(args):
     torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
     layers = args.layers or 32
     n_ten = args.tenants or 100
-    Ts = [1, 2, 4, 8, 16, 32, 64, 128, 256]
+    Ts = [int(t) for t in args.sweep_T.split(",")] if args.sweep_T else [1, 2, 4, 8, 16, 32, 64, 128, 256]
     budgets = [("1/16", 1 / 16, plans.MIXED_1_16), ("1/32", 1 / 32, plans.MIXED_1_32),
                ("all-3-bit", 1 / 16, plans.ALL_3BIT)]
+    if args.sweep_budgets:
+        budgets = [b for b in budgets if b[0] in args.sweep_budgets.split(",")]
     peak, peak_kind = _peaks()
     for name, ratio, widths in budgets:
         def plan_fn(l, p, d_out, d_in, t, ratio=ratio, widths=widths):
@@ -774,6 +776,9 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="smaller stack for profiling captures (default: 32)")
     ap.add_argument("--tenants", type=int, default=0, help="fewer resident tenants (default: 50)")
     ap.add_argument("--slots", type=int, default=0, help="paging workload: resident tenant slots (default: 32)")
+    ap.add_argument("--sweep-T", default="", help="sweep workload: comma-separated batch sizes (default: 1..256)")
+    ap.add_argument("--sweep-budgets", default="", help="sweep workload: comma-separated budgets among "
+                                                         "1/16,1/32,all-3-bit (default: all)")
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep", "paging"],
                     help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill "
                          "pass; sweep: 100 Zipf tenants, T = 1..256, three budgets (one line per point); paging: "

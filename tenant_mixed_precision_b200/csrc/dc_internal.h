@@ -96,8 +96,11 @@ struct DcWs {
 };
 
 // Segments of at least DC_PF_MIN tokens take the tensor-core (prefill) delta path when the batch
-// has at least that many tokens.
+// has at least twice that many tokens (a build may set another threshold with -DDC_PF_MIN=n; the
+// workspace size follows it).
+#ifndef DC_PF_MIN
 #define DC_PF_MIN 64
+#endif
 
 // Tensor-core backbone: CTAs of the persistent grid (at most; 148 SMs on B200) and the partial
 // tiles they may leave for split units (two per CTA: its first and its last unit).
