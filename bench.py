@@ -765,6 +765,95 @@ def run_paging(args):
     return 0
 
 
+# ------------------------------------------------------------------------------------------------
+# Device compressor (SVD + quantise/pack) for one tenant's 7B layer
+# ------------------------------------------------------------------------------------------------
+COMPRESS_METRIC = "seconds per tenant layer, device compression (top-r SVD + RTN pack) of 7B deltas at 1/16"
+
+
+def run_compress(args):
+    import numpy as np
+    import torch
+
+    import tenant_mixed_precision_b200 as dc
+    from tenant_mixed_precision_b200 import plans, synth
+
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    torch.cuda.set_device(int(os.environ.get("LOCAL_RANK", "0")))
+    shapes = synth.llama_proj_shapes(4096, 11008)
+    g = torch.Generator(device="cuda").manual_seed(4321)
+    jobs = []
+    for p, (d_out, d_in) in enumerate(shapes):
+        # a full-rank long-tail delta (sigma_i = 1.28 i^-0.8 over all min(d_out, d_in) ranks)
+        m = min(d_out, d_in)
+        Q1, _ = torch.linalg.qr(torch.randn((d_out, m), device="cuda", generator=g))
+        Q2, _ = torch.linalg.qr(torch.randn((d_in, m), device="cuda", generator=g))
+        sig = 1.28 * torch.arange(1, m + 1, device="cuda", dtype=torch.float32) ** -0.8
+        wb = (0.02 * torch.randn((d_out, d_in), device="cuda", generator=g)).to(torch.bfloat16)
+        wf = (wb.float() + (Q1 * sig) @ Q2.T).to(torch.bfloat16)
+        del Q1, Q2
+        plan = plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+        jobs.append((p, d_out, d_in, plan, wf, wb))
+    torch.cuda.synchronize()
+
+    def compress_layer(seed):
+        tot_sweeps = 0
+        errs = []
+        for p, d_out, d_in, plan, wf, wb in jobs:
+            r = sum(x for _, x in plan)
+            over = 16 + r // 10
+            U = torch.empty((r, d_out), dtype=torch.float32, device="cuda")
+            S = torch.empty(r, dtype=torch.float32, device="cuda")
+            Vt = torch.empty((r, d_in), dtype=torch.float32, device="cuda")
+            ws = torch.empty(dc.dc_svd_workspace_size(d_out, d_in, r, over), dtype=torch.uint8, device="cuda")
+            tot_sweeps += dc.dc_svd_device(wf, wb, r, over, 2, seed + p, U, S, Vt, ws)
+            desc = dc.make_desc(d_out, d_in, plan)
+            buf = torch.empty(dc.dc_packed_size(desc), dtype=torch.uint8, device="cuda")
+            scratch = torch.zeros(dc.dc_quantize_scratch_size(desc), dtype=torch.uint8, device="cuda")
+            dc.dc_quantize_pack_device(desc, U, Vt, S, buf, scratch)
+            if seed == 0:  # truncation error against the Eckart-Young optimum of the bf16 delta
+                D = wf.float() - wb.float()
+                e = torch.linalg.norm(D - (U.T * S) @ Vt).item()
+                sv = torch.linalg.svdvals(D)
+                errs.append(e / torch.sqrt(torch.sum(sv[r:] ** 2)).item())
+        torch.cuda.synchronize()
+        return tot_sweeps, errs
+
+    sweeps, ey = compress_layer(0)  # warm-up, and the accuracy check
+    times = []
+    for i in range(max(1, args.steps)):
+        t0 = time.perf_counter()
+        compress_layer(1000 + 17 * i)
+        times.append(time.perf_counter() - t0)
+    sec = statistics.median(times)
+    cpu = None
+    if not args.no_cpu_baseline:
+        import oracle
+        n = 2048  # a bounded sample: the leading 2048 x 2048 block of the q delta
+        D = (jobs[0][4].float() - jobs[0][5].float())[:n, :n].cpu().numpy().astype(np.float64)
+        t0 = time.perf_counter()
+        oracle.svd_factors(D)
+        t_svd = time.perf_counter() - t0
+        # a dense SVD costs ~ d_out * d_in * min(d_out, d_in): scale the sample to the layer's 7
+        work = sum(d_out * d_in * min(d_out, d_in) for _, d_out, d_in, _, _, _ in jobs)
+        scale = work / float(n) ** 3
+        cpu = {"value": t_svd * scale, "unit": "seconds per tenant layer", "cores": _cores(), "kind": "oracle",
+               "sample": f"fp64 LAPACK SVD (numpy) of a {n} x {n} block of the q delta, scaled by d_out*d_in*min(d) "
+                         f"to the layer's 7 projections (x{scale:.1f}); quantisation excluded"}
+    line = {"metric": COMPRESS_METRIC, "value": sec, "unit": "s", "n_gpus": 1, "steps": len(times), "warmup": 1,
+            "ms_per_step": sec * 1e3, "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32 GEMM and Jacobi rotations (f64 sums), u8 codes", "data": "synthetic",
+            "config": {"workload": "one tenant's Llama-2-7B layer (q, k, v, o 4096x4096; gate, up 11008x4096; down "
+                                   "4096x11008), full-rank deltas with sigma_i = 1.28 i^-0.8, 1/16 plan (r = 1002 / "
+                                   "1470), oversample r/10 + 16, 2 power iterations",
+                       "jacobi_sweeps_per_layer": sweeps},
+            "accuracy": {"truncation_error_over_eckart_young": ey},
+            "cpu_baseline": cpu}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -779,7 +868,7 @@ def main():
     ap.add_argument("--sweep-T", default="", help="sweep workload: comma-separated batch sizes (default: 1..256)")
     ap.add_argument("--sweep-budgets", default="", help="sweep workload: comma-separated budgets among "
                                                          "1/16,1/32,all-3-bit (default: all)")
-    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep", "paging"],
+    ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep", "paging", "compress"],
                     help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill "
                          "pass; sweep: 100 Zipf tenants, T = 1..256, three budgets (one line per point); paging: "
                          "100 Zipf tenants served from fewer device slots with on-demand host->device loads")
@@ -794,6 +883,8 @@ def main():
         return run_sweep(args)
     if args.workload == "paging":
         return run_paging(args)
+    if args.workload == "compress":
+        return run_compress(args)
     return run_gpu(args)
 
 

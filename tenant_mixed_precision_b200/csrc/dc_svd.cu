@@ -374,7 +374,9 @@ extern "C" dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t
   float* Ut = (float*)(b + W.ut);
   float* sig = (float*)(b + W.sig);
   int* off = (int*)(b + W.off);
-  const float tol = 1e-6f;
+  // the range finder's intermediate bases only have to span the right space: a looser tolerance
+  // there; the last basis Q and the final SVD of B are orthogonalised to 1e-6
+  const float tol = 1e-6f, tol_mid = 1e-4f;
   const int max_sweeps = 40;
   int sweeps = 0;
   const int64_t nd = (int64_t)d_out * d_in;
@@ -384,15 +386,16 @@ extern "C" dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t
   if (st) return st;
   // Y^T = Omega^T Delta^T, orth
   if ((st = gemm<true>(Zt, D, Qt, l, d_out, d_in, d_in, d_in, d_out, s))) return st;
-  if ((st = jacobi(Qt, l, d_out, nullptr, tol, max_sweeps, off, s, &sweeps))) return st;
+  if ((st = jacobi(Qt, l, d_out, nullptr, power_iters > 0 ? tol_mid : tol, max_sweeps, off, s, &sweeps))) return st;
   k_row_norms<<<l, 256, 0, s>>>(Qt, d_out, sig, 1);
   for (int it = 0; it < power_iters; ++it) {
     // Z^T = Q^T Delta (the columns of Delta^T Q), orth; Y^T = Z^T Delta^T, orth
     if ((st = gemm<false>(Qt, D, Zt, l, d_in, d_out, d_out, d_in, d_in, s))) return st;
-    if ((st = jacobi(Zt, l, d_in, nullptr, tol, max_sweeps, off, s, &sweeps))) return st;
+    if ((st = jacobi(Zt, l, d_in, nullptr, tol_mid, max_sweeps, off, s, &sweeps))) return st;
     k_row_norms<<<l, 256, 0, s>>>(Zt, d_in, sig, 1);
     if ((st = gemm<true>(Zt, D, Qt, l, d_out, d_in, d_in, d_in, d_out, s))) return st;
-    if ((st = jacobi(Qt, l, d_out, nullptr, tol, max_sweeps, off, s, &sweeps))) return st;
+    if ((st = jacobi(Qt, l, d_out, nullptr, it == power_iters - 1 ? tol : tol_mid, max_sweeps, off, s, &sweeps)))
+      return st;
     k_row_norms<<<l, 256, 0, s>>>(Qt, d_out, sig, 1);
   }
   // B^T = Delta^T Q (rows of Z^T), one-sided Jacobi with the rotations recorded in J
