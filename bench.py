@@ -771,6 +771,58 @@ def run_paging(args):
 COMPRESS_METRIC = "seconds per tenant layer, device compression (top-r SVD + RTN pack) of 7B deltas at 1/16"
 
 
+def _prinmix_vs_greedy(job, n_cal: int = 512, n_test: int = 256, r_cand: int = 1200):
+    """One projection: the device SVD's leading r_cand triplets, compressed at the 1/16 budget by
+    the greedy plan and by PrinMix (eq. 5 scores on calibration tokens, exact ILP, RTC); both
+    served by the kernels (delta only) on held-out tokens and compared with the exact delta product
+    (a plain fp32 GEMM of the bf16 delta).  Returns errors and the PrinMix host time."""
+    import ctypes
+
+    import numpy as np
+    import torch
+
+    import tenant_mixed_precision_b200 as dc
+    from tenant_mixed_precision_b200 import plans
+
+    p, d_out, d_in, plan, wf, wb = job
+    over = 16 + r_cand // 10
+    U = torch.empty((r_cand, d_out), dtype=torch.float32, device="cuda")
+    S = torch.empty(r_cand, dtype=torch.float32, device="cuda")
+    Vt = torch.empty((r_cand, d_in), dtype=torch.float32, device="cuda")
+    ws = torch.empty(dc.dc_svd_workspace_size(d_out, d_in, r_cand, over), dtype=torch.uint8, device="cuda")
+    dc.dc_svd_device(wf, wb, r_cand, over, 2, 77, U, S, Vt, ws)
+    g = torch.Generator(device="cuda").manual_seed(99)
+    Xc = torch.randn((n_cal, d_in), device="cuda", generator=g).to(torch.bfloat16).float()
+    Xt = torch.randn((n_test, d_in), device="cuda", generator=g).to(torch.bfloat16)
+    Uh, Sh, Vh, Xh = U.cpu().numpy().T.copy(), S.cpu().numpy(), Vt.cpu().numpy(), Xc.cpu().numpy()
+    t0 = time.perf_counter()
+    desc_p, _, Up, Sp, Vp, _ = dc.dc_prinmix_compress(Uh, Sh, Vh, Xh, 1 / 16, 3)
+    t_pm = time.perf_counter() - t0
+    greedy = plans.budget_plan(d_out, d_in, 1 / 16, plans.MIXED_1_16)
+    rg = sum(x for _, x in greedy)
+    cands = {"greedy": (dc.make_desc(d_out, d_in, greedy), Uh[:, :rg], Sh[:rg], Vh[:rg]),
+             "prinmix": (desc_p, Up, Sp, Vp)}
+    exact = Xt.float() @ (wf.float() - wb.float()).T
+    out = {"prinmix_host_s": t_pm, "prinmix_plan": [[desc_p.bits[i], desc_p.rank[i]] for i in range(desc_p.n_bands)],
+           "greedy_plan": [list(x) for x in greedy], "projection": int(p)}
+    for name, (desc, Uc, Sc, Vc) in cands.items():
+        cu, cv, su, sv = dc.dc_quantize_rtn(desc, Uc, Vc)
+        buf = torch.empty(dc.dc_packed_size(desc), dtype=torch.uint8, device="cuda")
+        h = dc.dc_pack_upload(desc, cu, cv, su, sv, Sc, buf)
+        table = torch.empty(ctypes.sizeof(dc.dc_delta_handle), dtype=torch.uint8, device="cuda")
+        keep = dc.dc_tenant_table_upload([h], table)
+        r = dc.desc_rank(desc)
+        lin = dc.make_linear(wb, d_out, d_in, 1, r, table)
+        y = torch.empty((n_test, d_out), dtype=torch.float32, device="cuda")
+        w2 = torch.zeros(dc.dc_workspace_size(n_test, r, max(d_in, d_out), 1, 1), dtype=torch.uint8, device="cuda")
+        ids = torch.zeros(n_test, dtype=torch.int32, device="cuda")
+        dc.dc_delta_linear_segmented(lin, Xt, y, ids, n_test, dc.DC_DELTA | dc.DC_DECODE_ONLY, w2)
+        torch.cuda.synchronize()
+        out[name + "_activation_error"] = (torch.linalg.norm(y - exact) / torch.linalg.norm(exact)).item()
+        del keep
+    return out
+
+
 def run_compress(args):
     import numpy as np
     import torch
@@ -827,6 +879,7 @@ def run_compress(args):
         compress_layer(1000 + 17 * i)
         times.append(time.perf_counter() - t0)
     sec = statistics.median(times)
+    pm = _prinmix_vs_greedy(jobs[0]) if args.prinmix else None
     cpu = None
     if not args.no_cpu_baseline:
         import oracle
@@ -849,6 +902,7 @@ def run_compress(args):
                                    "1470), oversample r/10 + 16, 2 power iterations",
                        "jacobi_sweeps_per_layer": sweeps},
             "accuracy": {"truncation_error_over_eckart_young": ey},
+            "prinmix": pm,
             "cpu_baseline": cpu}
     print(json.dumps(line), flush=True)
     return 0
@@ -865,6 +919,8 @@ def main():
     ap.add_argument("--layers", type=int, default=0, help="smaller stack for profiling captures (default: 32)")
     ap.add_argument("--tenants", type=int, default=0, help="fewer resident tenants (default: 50)")
     ap.add_argument("--slots", type=int, default=0, help="paging workload: resident tenant slots (default: 32)")
+    ap.add_argument("--prinmix", action="store_true", help="compress workload: also compare PrinMix with the greedy "
+                                                              "plan on one projection")
     ap.add_argument("--sweep-T", default="", help="sweep workload: comma-separated batch sizes (default: 1..256)")
     ap.add_argument("--sweep-budgets", default="", help="sweep workload: comma-separated budgets among "
                                                          "1/16,1/32,all-3-bit (default: all)")

@@ -269,15 +269,16 @@ dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* 
  *
  * Top-r singular triplets of Delta = W_ft - W_base on the GPU, for dc_quantize_pack_device: a
  * randomized range finder (Gaussian test matrix of r + oversample columns from `seed`, power_iters
- * power iterations, each basis made orthonormal by one-sided Jacobi) and a one-sided Jacobi SVD of
- * the projected matrix, in fp32 with fp64 Jacobi sums.  W_ft, W_base: device, row-major
+ * power iterations, each basis made orthonormal by CholeskyQR2 with fp64 Gram matrices) and a
+ * one-sided Jacobi SVD of the projected matrix, in fp32 with fp64 Jacobi sums.  W_ft, W_base: device, row-major
  * [d_out, d_in], dtype DC_DTYPE_F32 or DC_DTYPE_BF16.  Outputs (device, caller-owned):
  * U_out [r, d_out] (row i = u_i), S_out [r] (descending), Vt_out [r, d_in] (row i = v_i), each pair
  * signed so that the largest-magnitude entry of v_i is positive (the lowest index on ties).  The
  * truncation error approaches the Eckart-Young optimum sqrt(sum_{i>r} sigma_i^2) as oversample and
  * power_iters grow (e.g. oversample = r/10 + 16, power_iters = 2).  ws: caller device memory of
  * dc_svd_workspace_size bytes (256-byte aligned).  Synchronises the stream (once per Jacobi sweep,
- * to test convergence) and returns after the outputs are written; *sweeps_out (if not NULL)
+ * to test convergence, and once per basis, to check the Cholesky pivots: DC_ERR_INVALID_ARG if the
+ * basis lost rank) and returns after the outputs are written; *sweeps_out (if not NULL)
  * receives the number of Jacobi sweeps run. */
 size_t dc_svd_workspace_size(int32_t d_out, int32_t d_in, int32_t r, int32_t oversample);
 dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t dtype, int32_t d_out, int32_t d_in, int32_t r,

@@ -11,11 +11,12 @@
 //   B^T = Delta^T Q;  SVD of B by one-sided Jacobi (Hestenes): B^T J = W with orthogonal columns,
 //   sigma_j = |W_j|, v_j = W_j / sigma_j, u_j = Q J_j;  the r largest, signs fixed as the oracle
 //   does (the largest-magnitude entry of v_i positive, the lowest index on ties).
-// orth() is the same one-sided Jacobi without the rotation record: it makes the columns orthogonal
-// and then unit length.  Matrices whose columns the algorithm works on are stored transposed, one
-// column per contiguous row, so every Jacobi pair reads two contiguous rows.  Products run on an
-// fp32 tiled GEMM; Jacobi sums are accumulated in fp64.  The library allocates nothing: the caller
-// passes a workspace of dc_svd_workspace_size bytes.
+// orth() is CholeskyQR2: the Gram matrix in fp64, its Cholesky factor, the basis multiplied by the
+// factor's inverse, twice (bases of more than 4096 columns fall back to one-sided Jacobi).  Matrices
+// whose columns the algorithm works on are stored transposed, one column per contiguous row, so
+// every Jacobi pair reads two contiguous rows.  Products run on an fp32 tiled GEMM; Gram matrices,
+// Cholesky and Jacobi sums are fp64.  The library allocates nothing: the caller passes a workspace
+// of dc_svd_workspace_size bytes.
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -204,6 +205,111 @@ __global__ void __launch_bounds__(256) k_row_norms(float* __restrict__ M, int m,
   }
 }
 
+// ---- CholeskyQR2 for the range finder's bases (orthonormal rows of M, n x m):
+//   G = M M^T (fp64), G = L L^T, M <- L^-1 M, twice (the second pass repairs the first's
+//   rounding; Fukaya, Nakatsukasa, Yanagisawa, Yamamoto, "CholeskyQR2", ScalA 2014).
+// Its cost is two Gram products and two small triangular steps, against O(n^2 m) per sweep for
+// the one-sided Jacobi, which remains the method for the final SVD of B.
+
+// G = M M^T in fp64 (M rows of length m, fp32): 32 x 32 output tiles, upper tiles only, mirrored.
+__global__ void __launch_bounds__(256) k_gram64(const float* __restrict__ M, int n, int m, double* __restrict__ G) {
+  const int bi = blockIdx.y, bj = blockIdx.x;
+  if (bj < bi) return;
+  __shared__ float A[32][33], B[32][33];
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  double acc[2][2] = {};
+  for (int k0 = 0; k0 < m; k0 += 32) {
+    for (int e = threadIdx.x; e < 32 * 32; e += 256) {
+      const int r = e >> 5, c = e & 31;
+      const int ra = 32 * bi + r, rb = 32 * bj + r, k = k0 + c;
+      A[r][c] = (ra < n && k < m) ? M[(int64_t)ra * m + k] : 0.f;
+      B[r][c] = (rb < n && k < m) ? M[(int64_t)rb * m + k] : 0.f;
+    }
+    __syncthreads();
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+      const double a0 = A[ty][k], a1 = A[ty + 16][k], b0 = B[tx][k], b1 = B[tx + 16][k];
+      acc[0][0] = fma(a0, b0, acc[0][0]);
+      acc[0][1] = fma(a0, b1, acc[0][1]);
+      acc[1][0] = fma(a1, b0, acc[1][0]);
+      acc[1][1] = fma(a1, b1, acc[1][1]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int a = 0; a < 2; ++a)
+#pragma unroll
+    for (int b = 0; b < 2; ++b) {
+      const int i = 32 * bi + ty + 16 * a, j = 32 * bj + tx + 16 * b;
+      if (i < n && j < n) {
+        G[(int64_t)i * n + j] = acc[a][b];
+        G[(int64_t)j * n + i] = acc[a][b];
+      }
+    }
+}
+
+// Diagonal shift of G by eps * trace / n (keeps the factorisation defined when M's rows are nearly
+// dependent; those directions then get no weight in the range).  One block.
+__global__ void k_gram_shift(double* __restrict__ G, int n, double eps) {
+  __shared__ double red[8];
+  double t = 0.0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) t += G[(int64_t)i * n + i];
+  t = block_sum(t, red);
+  const double sh = eps * (t > 0.0 ? t / n : 1.0);
+  for (int i = threadIdx.x; i < n; i += blockDim.x) G[(int64_t)i * n + i] += sh;
+}
+
+// Step k of the right-looking Cholesky on the lower triangle: G[i][j] -= G[i][k] G[j][k] / G[k][k]
+// for k < j <= i (column k itself stays as it is; the factor is read off at the end).
+__global__ void k_chol_step(double* __restrict__ G, int n, int k) {
+  const int64_t w = n - k - 1;
+  const int64_t tot = w * (w + 1) / 2;
+  const double inv = 1.0 / G[(int64_t)k * n + k];
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < tot; e += (int64_t)gridDim.x * blockDim.x) {
+    // e -> (a, b), 0 <= b <= a < w, row-major over the triangle
+    int64_t a = (int64_t)((sqrt(8.0 * (double)e + 1.0) - 1.0) * 0.5);
+    while (a * (a + 1) / 2 > e) --a;
+    while ((a + 1) * (a + 2) / 2 <= e) ++a;
+    const int64_t b = e - a * (a + 1) / 2;
+    const int i = k + 1 + (int)a, j = k + 1 + (int)b;
+    G[(int64_t)i * n + j] -= G[(int64_t)i * n + k] * G[(int64_t)j * n + k] * inv;
+  }
+}
+
+// L[i][k] = G[i][k] / sqrt(G[k][k]) for i >= k (the Cholesky factor, in place, lower triangle);
+// a non-positive pivot is reported in *bad.
+__global__ void k_chol_finish(double* __restrict__ G, int n, int* __restrict__ bad) {
+  const int64_t tot = (int64_t)n * n;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < tot; e += (int64_t)gridDim.x * blockDim.x) {
+    const int i = (int)(e / n), k = (int)(e % n);
+    if (k > i) continue;
+    const double d = G[(int64_t)k * n + k];
+    if (!(d > 0.0)) {
+      if (i == k) atomicExch(bad, 1);
+      continue;
+    }
+    G[e] = G[e] / sqrt(d);  // the diagonal becomes sqrt(d) too
+  }
+}
+
+// X = L^-1 (lower triangular, fp32 out): block j solves L x = e_j by forward substitution.
+__global__ void __launch_bounds__(256) k_trinv(const double* __restrict__ L, int n, float* __restrict__ X) {
+  __shared__ double red[8];
+  __shared__ double xs[4096];
+  const int j = blockIdx.x;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) X[(int64_t)i * n + j] = 0.f;
+  if (threadIdx.x == 0) xs[j] = 1.0 / L[(int64_t)j * n + j];
+  __syncthreads();
+  for (int i = j + 1; i < n; ++i) {
+    double sacc = 0.0;
+    for (int t = j + threadIdx.x; t < i; t += blockDim.x) sacc += L[(int64_t)i * n + t] * xs[t];
+    sacc = block_sum(sacc, red);
+    if (threadIdx.x == 0) xs[i] = -sacc / L[(int64_t)i * n + i];
+    __syncthreads();
+  }
+  for (int i = j + threadIdx.x; i < n; i += blockDim.x) X[(int64_t)i * n + j] = (float)xs[i];
+}
+
 __global__ void k_identity(float* __restrict__ J, int n) {
   const int64_t total = (int64_t)n * n;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < total; i += (int64_t)gridDim.x * blockDim.x)
@@ -276,7 +382,7 @@ __global__ void __launch_bounds__(256) k_svd_emit(const float* __restrict__ sig,
 }
 
 struct SvdWs {
-  int64_t delta, qt, zt, jt, ut, sig, off, total;
+  int64_t delta, qt, zt, jt, ut, sig, gram, tinv, off, total;
 };
 
 SvdWs svd_ws(int d_out, int d_in, int l) {
@@ -291,8 +397,10 @@ SvdWs svd_ws(int d_out, int d_in, int l) {
   W.qt = take((int64_t)l * d_out * 4);
   W.zt = take((int64_t)l * d_in * 4);
   W.jt = take((int64_t)l * l * 4);
-  W.ut = take((int64_t)l * d_out * 4);
+  W.ut = take((int64_t)l * std::max(d_out, d_in) * 4);  // U^T at the end; scratch of the range finder
   W.sig = take((int64_t)l * 4);
+  W.gram = take((int64_t)l * l * 8);
+  W.tinv = take((int64_t)l * l * 4);
   W.off = take(256);
   W.total = o;
   return W;
@@ -338,6 +446,41 @@ dc_status jacobi(float* M, int n, int m, float* Jt, float tol, int max_sweeps, i
   return DC_OK;
 }
 
+// Orthonormal rows of M (n x m) spanning the same space, by CholeskyQR2; tmp: n x m fp32 scratch.
+// Synchronises the stream (to read the pivot flag).
+dc_status orth_cholqr2(float* M, int n, int m, float* tmp, double* G, float* X, int* bad, cudaStream_t s) {
+  if (n > 4096) {  // beyond k_trinv's shared vector: one-sided Jacobi, then unit rows
+    int sw = 0;
+    dc_status st = jacobi(M, n, m, nullptr, 1e-6f, 40, bad, s, &sw);
+    if (st) return st;
+    k_row_norms<<<n, 256, 0, s>>>(M, m, reinterpret_cast<float*>(G), 1);
+    return dc_cuda_check(cudaGetLastError(), "orth norms");
+  }
+  dc_status st = dc_cuda_check(cudaMemsetAsync(bad, 0, 4, s), "orth flag");
+  if (st) return st;
+  for (int pass = 0; pass < 2; ++pass) {
+    const dim3 gg((n + 31) / 32, (n + 31) / 32);
+    k_gram64<<<gg, 256, 0, s>>>(M, n, m, G);
+    k_gram_shift<<<1, 256, 0, s>>>(G, n, 1e-13);
+    for (int k = 0; k + 1 < n; ++k) {
+      const int64_t w = n - k - 1, tot = w * (w + 1) / 2;
+      k_chol_step<<<(unsigned)std::min<int64_t>((tot + 255) / 256, 148 * 8), 256, 0, s>>>(G, n, k);
+    }
+    k_chol_finish<<<(unsigned)std::min<int64_t>(((int64_t)n * n + 255) / 256, 148 * 8), 256, 0, s>>>(G, n, bad);
+    k_trinv<<<n, 256, 0, s>>>(G, n, X);
+    if ((st = gemm<false>(X, M, tmp, n, m, n, n, m, m, s))) return st;
+    st = dc_cuda_check(cudaMemcpyAsync(M, tmp, (size_t)n * m * 4, cudaMemcpyDeviceToDevice, s), "orth copy");
+    if (st) return st;
+  }
+  int hbad = 0;
+  st = dc_cuda_check(cudaMemcpyAsync(&hbad, bad, 4, cudaMemcpyDeviceToHost, s), "orth flag read");
+  if (st) return st;
+  st = dc_cuda_check(cudaStreamSynchronize(s), "orth sync");
+  if (st) return st;
+  if (hbad) return dc_fail(DC_ERR_INVALID_ARG, "svd: the range basis lost rank (Cholesky pivot <= 0)");
+  return DC_OK;
+}
+
 }  // namespace
 
 extern "C" size_t dc_svd_workspace_size(int32_t d_out, int32_t d_in, int32_t r, int32_t oversample) {
@@ -373,10 +516,10 @@ extern "C" dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t
   float* Jt = (float*)(b + W.jt);
   float* Ut = (float*)(b + W.ut);
   float* sig = (float*)(b + W.sig);
+  double* G64 = (double*)(b + W.gram);
+  float* Xinv = (float*)(b + W.tinv);
   int* off = (int*)(b + W.off);
-  // the range finder's intermediate bases only have to span the right space: a looser tolerance
-  // there; the last basis Q and the final SVD of B are orthogonalised to 1e-6
-  const float tol = 1e-6f, tol_mid = 1e-4f;
+  const float tol = 1e-6f;  // the final SVD's Jacobi tolerance
   const int max_sweeps = 40;
   int sweeps = 0;
   const int64_t nd = (int64_t)d_out * d_in;
@@ -386,17 +529,13 @@ extern "C" dc_status dc_svd_device(const void* W_ft, const void* W_base, int32_t
   if (st) return st;
   // Y^T = Omega^T Delta^T, orth
   if ((st = gemm<true>(Zt, D, Qt, l, d_out, d_in, d_in, d_in, d_out, s))) return st;
-  if ((st = jacobi(Qt, l, d_out, nullptr, power_iters > 0 ? tol_mid : tol, max_sweeps, off, s, &sweeps))) return st;
-  k_row_norms<<<l, 256, 0, s>>>(Qt, d_out, sig, 1);
+  if ((st = orth_cholqr2(Qt, l, d_out, Ut, G64, Xinv, off, s))) return st;
   for (int it = 0; it < power_iters; ++it) {
     // Z^T = Q^T Delta (the columns of Delta^T Q), orth; Y^T = Z^T Delta^T, orth
     if ((st = gemm<false>(Qt, D, Zt, l, d_in, d_out, d_out, d_in, d_in, s))) return st;
-    if ((st = jacobi(Zt, l, d_in, nullptr, tol_mid, max_sweeps, off, s, &sweeps))) return st;
-    k_row_norms<<<l, 256, 0, s>>>(Zt, d_in, sig, 1);
+    if ((st = orth_cholqr2(Zt, l, d_in, Ut, G64, Xinv, off, s))) return st;
     if ((st = gemm<true>(Zt, D, Qt, l, d_out, d_in, d_in, d_in, d_out, s))) return st;
-    if ((st = jacobi(Qt, l, d_out, nullptr, it == power_iters - 1 ? tol : tol_mid, max_sweeps, off, s, &sweeps)))
-      return st;
-    k_row_norms<<<l, 256, 0, s>>>(Qt, d_out, sig, 1);
+    if ((st = orth_cholqr2(Qt, l, d_out, Ut, G64, Xinv, off, s))) return st;
   }
   // B^T = Delta^T Q (rows of Z^T), one-sided Jacobi with the rotations recorded in J
   if ((st = gemm<false>(Qt, D, Zt, l, d_in, d_out, d_out, d_in, d_in, s))) return st;
