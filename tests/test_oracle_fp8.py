@@ -1,0 +1,69 @@
+"""Pins of the fp8 backbone oracle (oracle/fp8.py): the E4M3 format of the OCP 8-bit floating point
+specification, its round-to-nearest-even with saturation, and the per-row quantisation."""
+import numpy as np
+
+from oracle import fp8
+
+
+def test_e4m3_table_known_values():
+    v = fp8.E4M3_TABLE
+    assert v[0x00] == 0.0 and v[0x38] == 1.0 and v[0x3C] == 1.5 and v[0x7E] == 448.0
+    assert v[0x08] == 2.0 ** -6 and v[0x01] == 2.0 ** -9 and v[0x07] == 7 * 2.0 ** -9
+    assert np.isnan(v[0x7F]) and np.isnan(v[0xFF]) and v[0xFE] == -448.0 and v[0xB8] == -1.0
+    finite = v[~np.isnan(v)]
+    assert len(finite) == 254 and np.max(finite) == 448.0
+    pos = v[0x00:0x7F]
+    assert np.all(np.diff(pos) > 0)  # codes 0..126 increase in value
+
+
+def test_round_trip_of_every_finite_code():
+    for c in range(256):
+        if c in (0x7F, 0xFF, 0x80):
+            continue
+        assert int(fp8.e4m3_round(np.float32(fp8.E4M3_TABLE[c]))) == c
+    assert int(fp8.e4m3_round(np.float32(-0.0))) in (0x00, 0x80)
+
+
+def test_round_to_nearest_even_brute_force():
+    rng = np.random.default_rng(8)
+    x = np.concatenate([rng.standard_normal(4000) * 10 ** rng.uniform(-4, 2.5, 4000),
+                        rng.uniform(-500, 500, 500)]).astype(np.float32)
+    codes = fp8.e4m3_round(x)
+    cand = np.arange(256)
+    vals = fp8.E4M3_TABLE
+    ok = ~np.isnan(vals)
+    for xi, c in zip(x.astype(np.float64), codes):
+        t = np.clip(xi, -448.0, 448.0)
+        d = np.abs(vals[ok] - t)
+        best = cand[ok][d == d.min()]
+        best_vals = {vals[b] for b in best}
+        assert vals[c] in best_vals or (vals[c] == 0 and 0.0 in best_vals)
+        if len(best_vals) == 2:  # a tie: the even code
+            assert c % 2 == 0
+
+
+def test_midpoints_go_to_the_even_code_and_saturation():
+    v = fp8.E4M3_TABLE
+    for c in range(0, 0x7E):
+        mid = np.float32((v[c] + v[c + 1]) / 2)
+        if float(mid) != (v[c] + v[c + 1]) / 2:
+            continue  # not representable in fp32
+        got = int(fp8.e4m3_round(mid))
+        assert got == (c if c % 2 == 0 else c + 1), c
+    assert int(fp8.e4m3_round(np.float32(463.9))) == 0x7E
+    assert int(fp8.e4m3_round(np.float32(1e6))) == 0x7E and int(fp8.e4m3_round(np.float32(-1e6))) == 0xFE
+    assert int(fp8.e4m3_round(np.float32(2.0 ** -11))) == 0x00   # below half the smallest subnormal
+    assert int(fp8.e4m3_round(np.float32(2.0 ** -10 * 1.01))) == 0x01
+
+
+def test_quantize_rows_scale_and_error():
+    rng = np.random.default_rng(9)
+    w = (0.02 * rng.standard_normal((64, 512))).astype(np.float32)
+    w[3] = 0.0
+    codes, sc = fp8.quantize_rows(w)
+    assert sc[3] == 1.0 and np.all(codes[3] % 0x80 == 0)
+    wh = fp8.dequantize_rows(codes, sc)
+    # the row maximum lands on +-448; every element within half a step of the E4M3 grid scaled
+    assert np.all(np.abs(fp8.E4M3_TABLE[codes[np.arange(64) != 3].astype(np.int64)]).max(axis=1) == 448.0)
+    rel = np.abs(wh - w) / np.maximum(np.abs(w), 2.0 ** -6 * sc[:, None])
+    assert rel.max() <= 2.0 ** -4 + 1e-7
