@@ -54,7 +54,10 @@ enum {
   DC_ERR_UNSUPPORTED = 8   /* a valid request this build does not serve (see message)     */
 };
 
-enum { DC_DTYPE_F32 = 0, DC_DTYPE_BF16 = 1 };
+/* DC_DTYPE_FP8 is a backbone weight format only (dc_linear.w_dtype): W_base then points at the
+ * E4M3 codes row-major [d_out, d_in] followed directly by the fp32 row scales [d_out]
+ * (dc_quantize_fp8_rows); activations stay bf16 and are quantised per token inside the call. */
+enum { DC_DTYPE_F32 = 0, DC_DTYPE_BF16 = 1, DC_DTYPE_FP8 = 2 };
 
 /* flags of dc_delta_linear_segmented / dc_layer_forward */
 enum {
@@ -261,6 +264,18 @@ dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* 
                            void* const y[7], const int32_t* tenant_ids_dev, int32_t T,
                            int32_t dtype_in, int32_t dtype_out, int32_t flags, void* ws,
                            size_t ws_bytes, void* stream);
+
+/* ---- fp8 backbone weights.
+ * Passage: none (the pages fix no backbone precision; an optional serving precision of the shared
+ * backbone: E4M3 of the OCP 8-bit floating point specification, 1 sign, 4 exponent bits with bias 7,
+ * 3 mantissa bits, subnormals m 2^-9, largest finite 448).
+ * Per row r of W (host fp32 [rows, cols]): scales[r] = max|W[r]| / 448 in fp32 (1 for a zero row),
+ * codes[r][c] = E4M3 round-to-nearest-even of the fp32 quotient W[r][c] / scales[r], saturating at
+ * +-448.  Upload codes then scales contiguously (rows * cols bytes, then rows floats) as the W_base
+ * of a linear with w_dtype DC_DTYPE_FP8.  Its backbone product is then sum_j (code_w s_row)
+ * (code_x s_tok), the activations quantised per token by the same rule with the token's max|x|,
+ * accumulated in fp32 on the tensor cores (kind::f8f6f4). */
+dc_status dc_quantize_fp8_rows(const float* W, int32_t rows, int32_t cols, uint8_t* codes, float* scales);
 
 /* ---- Device compressor: the SVD step.
  * Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的技术原理"

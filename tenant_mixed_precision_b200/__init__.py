@@ -21,7 +21,7 @@ SYNTH_LIB_PATH = os.path.join(_HERE, "libdc_synth.so")
 
 DC_OK, DC_ERR_INVALID_ARG, DC_ERR_SHAPE, DC_ERR_BITS, DC_ERR_ALIGN = 0, 1, 2, 3, 4
 DC_ERR_WORKSPACE, DC_ERR_TENANT, DC_ERR_CUDA, DC_ERR_UNSUPPORTED = 5, 6, 7, 8
-DC_DTYPE_F32, DC_DTYPE_BF16 = 0, 1
+DC_DTYPE_F32, DC_DTYPE_BF16, DC_DTYPE_FP8 = 0, 1, 2
 DC_BASE, DC_DELTA, DC_REUSE_ROUTING, DC_DECODE_ONLY = 1, 2, 4, 8
 DC_MAX_BANDS = 4
 DC_GROUP = 128
@@ -92,6 +92,7 @@ def _load():
         "dc_read_device_status": (I32, [VP, VP, P(I32)]),
         "dc_profile_begin": (I32, [I32]),
         "dc_profile_end": (I32, [P(C.c_float), P(I32), I32]),
+        "dc_quantize_fp8_rows": (I32, [VP, I32, I32, VP, VP]),
         "dc_prinmix_scores": (I32, [VP, VP, I32, I32, VP, I32, VP, I32, VP]),
         "dc_prinmix_allocate": (I32, [VP, I32, VP, I32, I32, I32, C.c_double, I32, VP, P(C.c_double)]),
         "dc_prinmix_rtc": (I32, [VP, VP, VP, VP, I32, I32, I32, VP, I32, VP]),
@@ -127,7 +128,7 @@ def exported_symbols() -> list[str]:
             "dc_workspace_size", "dc_build_segments", "dc_read_segments", "dc_delta_linear_segmented",
             "dc_delta_linear_segmented_static",
             "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status", "dc_profile_begin",
-            "dc_profile_end", "dc_prinmix_scores", "dc_prinmix_allocate", "dc_prinmix_rtc", "dc_prinmix_compress",
+            "dc_profile_end", "dc_quantize_fp8_rows", "dc_prinmix_scores", "dc_prinmix_allocate", "dc_prinmix_rtc", "dc_prinmix_compress",
             "dc_svd_workspace_size", "dc_svd_device", "dc_pager_scratch_size", "dc_pager_create", "dc_pager_set_tenant", "dc_pager_prepare",
             "dc_pager_commit", "dc_pager_get_stats", "dc_pager_slot_of", "dc_pager_destroy"]
 
@@ -275,7 +276,10 @@ def make_linear(W_base, d_out: int, d_in: int, n_tenants: int, max_rank: int, te
                 w_dtype: int | None = None) -> dc_linear:
     lin = dc_linear()
     lin.W_base = _ptr(W_base)
-    lin.w_dtype = _dtype_code(W_base) if w_dtype is None and W_base is not None else (w_dtype or DC_DTYPE_BF16)
+    if w_dtype is not None:
+        lin.w_dtype = w_dtype
+    else:
+        lin.w_dtype = _dtype_code(W_base) if W_base is not None and not isinstance(W_base, int) else DC_DTYPE_BF16
     lin.d_out, lin.d_in, lin.n_tenants, lin.max_rank = d_out, d_in, n_tenants, max_rank
     lin.tenants_dev = _ptr(tenants_dev)
     return lin
@@ -336,6 +340,24 @@ def dc_profile_end(capacity: int):
     if n < 0:
         raise DcError(DC_ERR_CUDA, "profiling failed: " + dc_last_error())
     return [(KERNEL_KINDS[kinds[i]], float(ms[i])) for i in range(min(n, capacity))]
+
+
+# ------------------------------------------------------------------------------------------
+# fp8 backbone weights (host quantiser)
+# ------------------------------------------------------------------------------------------
+def dc_quantize_fp8_rows(W) -> tuple[np.ndarray, np.ndarray]:
+    """W: float32 [rows, cols] -> (E4M3 codes uint8 [rows, cols], fp32 row scales [rows])."""
+    W = np.ascontiguousarray(np.asarray(W, dtype=np.float32))
+    codes = np.zeros(W.shape, np.uint8)
+    scales = np.zeros(W.shape[0], np.float32)
+    _check(_load().dc_quantize_fp8_rows(_ptr(W), W.shape[0], W.shape[1], _ptr(codes), _ptr(scales)))
+    return codes, scales
+
+
+def fp8_weight_blob(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:
+    """The W_base buffer of a DC_DTYPE_FP8 linear: codes row-major, then the fp32 row scales."""
+    return np.concatenate([np.ascontiguousarray(codes, np.uint8).reshape(-1),
+                           np.ascontiguousarray(scales, np.float32).view(np.uint8)])
 
 
 # ------------------------------------------------------------------------------------------

@@ -250,3 +250,53 @@ extern "C" dc_status dc_tenant_table_upload(const dc_delta_handle* handles, int3
   return dc_cuda_check(cudaMemcpyAsync(dev_dst, handles, need, cudaMemcpyHostToDevice, (cudaStream_t)stream),
                        "tenant table upload");
 }
+
+// ---------------------------------------------------------------------------------------------
+// fp8 (E4M3) backbone weights: per-row scale max|w| / 448, codes rounded to nearest even with
+// saturation (OCP 8-bit floating point specification, E4M3: bias 7, 3 mantissa bits, subnormals
+// m * 2^-9, largest finite 448, no infinities).
+// ---------------------------------------------------------------------------------------------
+uint8_t dc_e4m3_rne(float x) {
+  const uint8_t sign = std::signbit(x) ? 0x80 : 0x00;
+  const double a = std::fabs((double)x);
+  if (a != a) return 0x7F;
+  if (a >= 448.0) return sign | 0x7E;
+  if (a == 0.0) return sign;
+  int e2 = 0;
+  std::frexp(a, &e2);  // a = f 2^e2, f in [0.5, 1)
+  const int E = e2 - 1;
+  uint32_t code;
+  if (E < -6) {  // subnormals: multiples of 2^-9 (8 * 2^-9 is the smallest normal, code 0x08)
+    code = (uint32_t)std::nearbyint(a * 512.0);
+  } else {
+    double q = std::nearbyint((a / std::ldexp(1.0, E) - 1.0) * 8.0);  // exact scaling, ties to even
+    int ee = E + 7;
+    if (q == 8.0) {
+      q = 0.0;
+      ++ee;
+    }
+    code = ((uint32_t)ee << 3) | (uint32_t)q;
+    if (code > 0x7E) code = 0x7E;
+  }
+  return sign | (uint8_t)code;
+}
+
+extern "C" dc_status dc_quantize_fp8_rows(const float* W, int32_t rows, int32_t cols, uint8_t* codes, float* scales) {
+  DC_NVTX("dc_quantize_fp8_rows");
+  dc_clear_error();
+  if (!W || !codes || !scales) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
+  if (rows <= 0 || cols <= 0) return dc_fail(DC_ERR_SHAPE, "rows and cols must be positive");
+  for (int32_t r = 0; r < rows; ++r) {
+    const float* w = W + (int64_t)r * cols;
+    float amax = 0.f;
+    for (int32_t c = 0; c < cols; ++c) {
+      if (!std::isfinite(w[c])) return dc_fail(DC_ERR_INVALID_ARG, "row %d: non-finite weight", r);
+      amax = std::max(amax, std::fabs(w[c]));
+    }
+    float s = amax / 448.0f;
+    if (s == 0.f) s = 1.f;
+    scales[r] = s;
+    for (int32_t c = 0; c < cols; ++c) codes[(int64_t)r * cols + c] = dc_e4m3_rne(w[c] / s);
+  }
+  return DC_OK;
+}

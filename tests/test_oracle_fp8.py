@@ -67,3 +67,19 @@ def test_quantize_rows_scale_and_error():
     assert np.all(np.abs(fp8.E4M3_TABLE[codes[np.arange(64) != 3].astype(np.int64)]).max(axis=1) == 448.0)
     rel = np.abs(wh - w) / np.maximum(np.abs(w), 2.0 ** -6 * sc[:, None])
     assert rel.max() <= 2.0 ** -4 + 1e-7
+
+
+def test_library_fp8_quantiser_matches_oracle():
+    import tenant_mixed_precision_b200 as dc
+    rng = np.random.default_rng(10)
+    w = np.concatenate([(0.02 * rng.standard_normal((40, 384))),
+                        rng.standard_normal((8, 384)) * 10 ** rng.uniform(-6, 3, size=(8, 1))]).astype(np.float32)
+    w[5] = 0.0
+    w[7, :] = 1e-30  # subnormal scale region
+    codes, sc = dc.dc_quantize_fp8_rows(w)
+    oc, osc = fp8.quantize_rows(w)
+    assert np.array_equal(sc, osc)
+    # the same values (a code 0x80, minus zero, equals 0x00)
+    assert np.array_equal(fp8.E4M3_TABLE[codes.astype(np.int64)], fp8.E4M3_TABLE[oc.astype(np.int64)])
+    blob = dc.fp8_weight_blob(codes, sc)
+    assert blob.nbytes == w.size + 4 * w.shape[0]
