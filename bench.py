@@ -325,6 +325,8 @@ def run_gpu(args):
     t_setup = time.time()
     stack = DeltaStack(W["hidden"], W["ffn"], W["layers"], W["n_tenants"], T, plan_fn, out_dtype=torch.bfloat16)
     populate(stack, W["seed"])
+    if args.fp8_backbone:
+        stack.to_fp8_backbone()
     ids = _ids(W["n_tenants"], T, W["ids_seed"] + 1000 * rank)
     ids_dev = torch.from_numpy(ids).cuda()
     setup_s = time.time() - t_setup
@@ -416,7 +418,8 @@ def run_gpu(args):
     step_gbs = ab["total"] / (ms_per_step * 1e-3) / 1e9
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and not args.layers and not args.tenants:
+    if (rank == 0 and world == 1 and not args.no_cpu_baseline and not args.layers and not args.tenants
+            and not args.fp8_backbone):
         s = OracleSample(ids)
         s.run_once()
         times = []
@@ -435,8 +438,12 @@ def run_gpu(args):
     line = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "u8xs8->s32 delta, bf16xbf16->f32 backbone", "data": "synthetic",
-        "config": {"workload": W["name"], "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
+        "vs_baseline": None,
+        "dtype": "u8xs8->s32 delta, " + ("e4m3xe4m3->f32 backbone (fp8 option)" if args.fp8_backbone
+                                         else "bf16xbf16->f32 backbone"),
+        "data": "synthetic",
+        "config": {"workload": W["name"] + (", fp8 (E4M3) backbone" if args.fp8_backbone else ""),
+                   "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
                    "tenants_resident": W["n_tenants"], "T": T, "distinct_tenants": ab["distinct_tenants"],
                    "budget": "1/16: 8-bit x2, 3-bit x32, 2-bit remainder", "output_dtype": "bf16",
                    "l2": f"inputs larger than L2 (~{ab['total'] / 1e9:.1f} GB read per step); no flush", "cuda_graph": True,
@@ -511,6 +518,8 @@ def run_prefill(args):
     t_setup = time.time()
     stack = DeltaStack(W["hidden"], W["ffn"], W["layers"], W["n_tenants"], T, plan_fn, out_dtype=torch.bfloat16)
     populate(stack, W["seed"], s0=0.02 * math.sqrt(W["hidden"]))
+    if args.fp8_backbone:
+        stack.to_fp8_backbone()
     ids = synth.prefill_segments(np.random.default_rng(W["ids_seed"]), T, W["n_tenants"])
     ids_dev = torch.from_numpy(ids).cuda()
     setup_s = time.time() - t_setup
@@ -561,6 +570,9 @@ def run_prefill(args):
                     r = sum(desc.rank[i] for i in range(desc.n_bands) if desc.bits[i])
                     delta_flops += 2.0 * r * (d_in + d_out)
     peak, peak_kind = _bf16_peak()
+    base_peak, base_peak_kind = peak, peak_kind
+    if args.fp8_backbone:  # the fp8 rate: the measured bf16 peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+        base_peak, base_peak_kind = 2.0 * peak, peak_kind + " x 2 (nominal fp8/bf16 ratio)"
     tf = (base_flops + delta_flops) / (ms_per_step * 1e-3) / 1e12
     base_ms = sum(per.get("backbone_output", [0])) / n_prof
     base_tf = base_flops / (base_ms * 1e-3) / 1e12 if base_ms else None
@@ -568,17 +580,20 @@ def run_prefill(args):
         "metric": PREFILL_METRIC, "value": T / (ms_per_step * 1e-3), "unit": "tokens/s", "n_gpus": 1,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16xbf16->f32 backbone, f16xf16->f32 delta (segments >= 64 tokens), u8xs8->s32 delta (shorter)",
+        "dtype": ("e4m3xe4m3->f32 backbone (fp8 option)" if args.fp8_backbone else "bf16xbf16->f32 backbone")
+                 + ", f16xf16->f32 delta (segments >= 64 tokens), u8xs8->s32 delta (shorter)",
         "data": "synthetic",
-        "config": {"workload": W["name"], "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
+        "config": {"workload": W["name"] + (", fp8 (E4M3) backbone" if args.fp8_backbone else ""),
+                   "hidden": W["hidden"], "ffn": W["ffn"], "layers": W["layers"],
                    "tenants_resident": W["n_tenants"], "T": T,
                    "segments": int(1 + np.count_nonzero(np.diff(ids))), "distinct_tenants": len(set(ids.tolist())),
                    "cuda_graph": True},
         "step_tensor": {"algorithmic_tflop": (base_flops + delta_flops) / 1e12, "base_tflop": base_flops / 1e12,
                         "delta_tflop": delta_flops / 1e12, "achieved_tflops": tf, "peak_tflops": peak,
                         "frac": tf / peak, "peak_source": peak_kind},
-        "roofline": {"bound": "tensor", "kernel": "k_base_tc", "achieved": base_tf, "peak": peak, "unit": "TFLOP/s",
-                     "frac": (base_tf / peak) if base_tf else None, "peak_source": peak_kind, "traffic": None},
+        "roofline": {"bound": "tensor", "kernel": "k_base_tc", "achieved": base_tf, "peak": base_peak,
+                     "unit": "TFLOP/s", "frac": (base_tf / base_peak) if base_tf else None,
+                     "peak_source": base_peak_kind, "traffic": None},
         "kernel_ms_per_step": {k: sum(v) / n_prof for k, v in per.items()},
         "gpu_launches": (1 + 6 * W["layers"]) * args.steps,
         "clocks": ck, "device_status": status, "setup_s": setup_s,
@@ -924,6 +939,8 @@ def main():
     ap.add_argument("--sweep-T", default="", help="sweep workload: comma-separated batch sizes (default: 1..256)")
     ap.add_argument("--sweep-budgets", default="", help="sweep workload: comma-separated budgets among "
                                                          "1/16,1/32,all-3-bit (default: all)")
+    ap.add_argument("--fp8-backbone", action="store_true", help="decode/prefill: serve the backbone in E4M3 "
+                    "(weights quantised per row on the device, activations per token inside the call)")
     ap.add_argument("--workload", default="decode", choices=["decode", "prefill", "sweep", "paging", "compress"],
                     help="decode: the 50-tenant 7B decode step (default); prefill: the 16-tenant 13B prefill "
                          "pass; sweep: 100 Zipf tenants, T = 1..256, three budgets (one line per point); paging: "

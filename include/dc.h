@@ -277,6 +277,16 @@ dc_status dc_layer_forward(const dc_linear lin[7], const void* x_h, const void* 
  * accumulated in fp32 on the tensor cores (kind::f8f6f4). */
 dc_status dc_quantize_fp8_rows(const float* W, int32_t rows, int32_t cols, uint8_t* codes, float* scales);
 
+/* The same rule on the device, with the rounding the call applies to the activations (an IEEE fp32
+ * division, then one conversion to E4M3 with round-to-nearest-even and saturation).  W: device,
+ * row-major [rows, cols], dtype DC_DTYPE_F32 or DC_DTYPE_BF16, 16-byte aligned, cols a multiple of
+ * 16; codes: device [rows, cols]; scales: device [rows] fp32 (both caller-owned, 16-byte aligned;
+ * codes then scales contiguously is a DC_DTYPE_FP8 W_base).  A value below half the smallest
+ * subnormal may come out as the negative zero code 0x80 (value 0).  Rows must be finite: a row
+ * holding an infinity or NaN gets a non-finite scale.  Asynchronous on `stream`. */
+dc_status dc_quantize_fp8_rows_device(const void* W, int32_t dtype, int32_t rows, int32_t cols, uint8_t* codes,
+                                      float* scales, void* stream);
+
 /* ---- Device compressor: the SVD step.
  * Passage: "Delta-CoMe – 清华联合 OpenBMB 等高校开源的新型增量压缩算法", section "Delta-CoMe的技术原理"
  * (SVD of the parameter delta); "Delta-CoMe: Training-Free Delta-Compression with Mixed-Precision for

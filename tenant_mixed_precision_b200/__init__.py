@@ -93,6 +93,7 @@ def _load():
         "dc_profile_begin": (I32, [I32]),
         "dc_profile_end": (I32, [P(C.c_float), P(I32), I32]),
         "dc_quantize_fp8_rows": (I32, [VP, I32, I32, VP, VP]),
+        "dc_quantize_fp8_rows_device": (I32, [VP, I32, I32, I32, VP, VP, VP]),
         "dc_prinmix_scores": (I32, [VP, VP, I32, I32, VP, I32, VP, I32, VP]),
         "dc_prinmix_allocate": (I32, [VP, I32, VP, I32, I32, I32, C.c_double, I32, VP, P(C.c_double)]),
         "dc_prinmix_rtc": (I32, [VP, VP, VP, VP, I32, I32, I32, VP, I32, VP]),
@@ -128,7 +129,7 @@ def exported_symbols() -> list[str]:
             "dc_workspace_size", "dc_build_segments", "dc_read_segments", "dc_delta_linear_segmented",
             "dc_delta_linear_segmented_static",
             "dc_layer_forward", "dc_unpack_codes_debug", "dc_read_device_status", "dc_profile_begin",
-            "dc_profile_end", "dc_quantize_fp8_rows", "dc_prinmix_scores", "dc_prinmix_allocate", "dc_prinmix_rtc", "dc_prinmix_compress",
+            "dc_profile_end", "dc_quantize_fp8_rows", "dc_quantize_fp8_rows_device", "dc_prinmix_scores", "dc_prinmix_allocate", "dc_prinmix_rtc", "dc_prinmix_compress",
             "dc_svd_workspace_size", "dc_svd_device", "dc_pager_scratch_size", "dc_pager_create", "dc_pager_set_tenant", "dc_pager_prepare",
             "dc_pager_commit", "dc_pager_get_stats", "dc_pager_slot_of", "dc_pager_destroy"]
 
@@ -278,8 +279,12 @@ def make_linear(W_base, d_out: int, d_in: int, n_tenants: int, max_rank: int, te
     lin.W_base = _ptr(W_base)
     if w_dtype is not None:
         lin.w_dtype = w_dtype
+    elif W_base is None or isinstance(W_base, int):
+        lin.w_dtype = DC_DTYPE_BF16
+    elif str(getattr(W_base, "dtype", "")) in ("torch.uint8", "uint8"):
+        lin.w_dtype = DC_DTYPE_FP8  # an fp8 weight blob (dc_quantize_fp8_rows_device / fp8_weight_blob)
     else:
-        lin.w_dtype = _dtype_code(W_base) if W_base is not None and not isinstance(W_base, int) else DC_DTYPE_BF16
+        lin.w_dtype = _dtype_code(W_base)
     lin.d_out, lin.d_in, lin.n_tenants, lin.max_rank = d_out, d_in, n_tenants, max_rank
     lin.tenants_dev = _ptr(tenants_dev)
     return lin
@@ -352,6 +357,18 @@ def dc_quantize_fp8_rows(W) -> tuple[np.ndarray, np.ndarray]:
     scales = np.zeros(W.shape[0], np.float32)
     _check(_load().dc_quantize_fp8_rows(_ptr(W), W.shape[0], W.shape[1], _ptr(codes), _ptr(scales)))
     return codes, scales
+
+
+def dc_quantize_fp8_rows_device(W, stream=None):
+    """W: device tensor [rows, cols] (fp32 or bf16) -> the DC_DTYPE_FP8 W_base blob as a device
+    uint8 tensor (codes row-major, then the fp32 row scales), quantised on the device."""
+    import torch
+    rows, cols = W.shape
+    W = W.contiguous()
+    blob = torch.empty(rows * cols + 4 * rows, dtype=torch.uint8, device=W.device)
+    _check(_load().dc_quantize_fp8_rows_device(_ptr(W), _dtype_code(W), rows, cols, _ptr(blob),
+                                               blob.data_ptr() + rows * cols, _stream(stream)))
+    return blob
 
 
 def fp8_weight_blob(codes: np.ndarray, scales: np.ndarray) -> np.ndarray:

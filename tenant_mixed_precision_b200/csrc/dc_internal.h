@@ -92,6 +92,8 @@ struct DcWs {
   int64_t tseg;      // per tenant-sorted token: its segment
   int64_t t16;       // fp16 t / 2^E(token): [n_lin][T][tcols] (prefill path)
   int64_t xs16;      // fp16 x * 2^(14 - E(token)), tenant-sorted: [n_in][T][max_d_in] (prefill path)
+  int64_t x8;        // E4M3 codes of x / s(token), tenant-sorted: [n_in][T][max_d_in] (fp8 backbone)
+  int64_t sx8;       // s(token) = max|x| / 448: [n_in][T] fp32 (fp8 backbone)
   int64_t total;
 };
 

@@ -83,6 +83,13 @@ __device__ __forceinline__ void mma_bf16(float (&c)[4], uint32_t a0, uint32_t a1
 
 __device__ __forceinline__ void set_status(int* st, int code) { atomicCAS(st + DC_WS_STATUS, 0, code); }
 
+// Two fp32 values to E4M3 (round to nearest even, saturating at +-448): lo in bits 0-7, hi in 8-15.
+__device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
+  unsigned short r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+
 // ---- register extraction from packed words (shared by the serving kernels and the debug unpacker)
 // V, 2-bit mask layout: word 2s+hh of the lane-row, group p -> 4 codes weighted by 4^p.
 __device__ __forceinline__ uint32_t v_reg_mask2(uint32_t w, int p) { return w & (0x03030303u << (2 * p)); }
@@ -146,6 +153,8 @@ DcWs dc_ws_layout(int32_t T, int32_t max_rank, int32_t max_d_in, int32_t n_lin, 
   W.tcols = (int32_t)dc_align(max_rank > 0 ? max_rank : 1, 64) + 64 * (DC_MAX_BANDS - 1);
   W.t16 = T >= DC_PF_MIN ? take((int64_t)n_lin * T * W.tcols * 2) : take(0);
   W.xs16 = T >= DC_PF_MIN ? take((int64_t)W.n_in * T * W.max_d_in * 2) : take(0);
+  W.x8 = take((int64_t)W.n_in * T * W.max_d_in);
+  W.sx8 = take((int64_t)W.n_in * T * 4);
   W.total = off;
   return W;
 }
@@ -179,6 +188,7 @@ struct DcFwd {
   int32_t bt_gtiles[8];        // per linear (same order): row tiles per group of the unit order
   CUtensorMap tmap;            // prefill path: fp16 t plane [n_lin T rows x tcols], box 64 x 256
   CUtensorMap xpf[3];          // prefill path: fp16 scaled tenant-sorted activations, box 64 x pf_box
+  int32_t fp8;                 // the backbone weights are E4M3 codes with fp32 row scales
   int32_t pf;                  // segments of >= DC_PF_MIN tokens take the prefill delta path
   int32_t pf_box;              // min(256, T)
   DcWs ws;
@@ -201,6 +211,8 @@ struct WsPtr {
   int* tseg;  // per sorted token: its segment
   __half* t16;    // prefill path: t / 2^E per token as fp16
   __half* xs16;   // prefill path: x * 2^(14 - E) per token as fp16
+  uint8_t* x8;    // fp8 backbone: E4M3 codes of x / s(token)
+  float* sx8;     // fp8 backbone: s(token)
 };
 __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   WsPtr p;
@@ -220,6 +232,8 @@ __device__ __forceinline__ WsPtr ws_ptr(const DcWs& W, uint8_t* ws) {
   p.tseg = (int*)(ws + W.tseg);
   p.t16 = (__half*)(ws + W.t16);
   p.xs16 = (__half*)(ws + W.xs16);
+  p.x8 = ws + W.x8;
+  p.sx8 = (float*)(ws + W.sx8);
   return p;
 }
 
@@ -446,12 +460,21 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
   // prefill operand: x * 2^(e - 8) = x * 2^(14 - E), below 2^14 in magnitude; a bf16 value
   // (8 significant bits) is exact in fp16 unless it is below 2^-31 max|x|
   const float sx16 = ldexpf(1.f, e - 8);
+  // fp8 backbone operand: E4M3 codes of x / s, s = max|x| / 448 (1 for a zero token), the quotient
+  // rounded once in fp32 (IEEE division) and then to nearest even E4M3, saturating
+  float s8 = __fdiv_rn(mx, 448.f);
+  if (s8 == 0.f) s8 = 1.f;
   for (int k = tid * 4; k < d; k += 1024) {
     float v[4];
     load4(k, v);
     if (F.dtype_in == DC_DTYPE_BF16)  // tenant-sorted copy for the backbone tiles
       *reinterpret_cast<uint2*>(P.xsort + ((int64_t)(m * T + j) * maxd + k) * 2) =
           *reinterpret_cast<const uint2*>((const __nv_bfloat16*)F.x[m] + (int64_t)i * d + k);
+    if (F.fp8) {
+      const uint32_t c01 = e4m3x2(__fdiv_rn(v[0], s8), __fdiv_rn(v[1], s8));
+      const uint32_t c23 = e4m3x2(__fdiv_rn(v[2], s8), __fdiv_rn(v[3], s8));
+      *reinterpret_cast<uint32_t*>(P.x8 + (int64_t)(m * T + j) * maxd + k) = c01 | (c23 << 16);
+    }
     if (F.pf) {
       const __half2 h01 = __floats2half2_rn(v[0] * sx16, v[1] * sx16);
       const __half2 h23 = __floats2half2_rn(v[2] * sx16, v[3] * sx16);
@@ -489,7 +512,10 @@ __global__ void __launch_bounds__(256) k_prep(const __grid_constant__ DcFwd F, u
       xs[0] = (float)s0, xs[1] = (float)s1, xs[2] = (float)s2, xs[3] = 0.f;
     }
   }
-  if (tid == 0) P.xe[m * T + j] = e;
+  if (tid == 0) {
+    P.xe[m * T + j] = e;
+    if (F.fp8) P.sx8[m * T + j] = s8;
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -1695,6 +1721,7 @@ struct BtTail {
   int last_flag;
   int perm[256];    // epilogue: original position of each token of the unit's block (-1: none)
   uint8_t dfl[256]; // epilogue: the token has a delta
+  float sxs[256];   // epilogue, fp8 backbone: the token's activation scale
   int nseg;         // segments of this CTA's chunk range (-1: more than BT_MAX_SEGS)
   int64_t sg[BT_MAX_SEGS];  // their first chunks, in processing order
 };
@@ -1720,7 +1747,7 @@ __device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1
   int slot = 0;
   while (slot + 1 < F.n_lin && g >= F.bt_chunk_prefix[slot + 1]) ++slot;
   S.slot = slot;
-  S.K = F.lin[F.order[slot]].d_in / 64;
+  S.K = F.lin[F.order[slot]].d_in / (F.fp8 ? 128 : 64);  // chunks of 128 bytes of a row
   const int64_t local = (g - F.bt_chunk_prefix[slot]) / S.K;
   // unit order inside a linear: groups of G row tiles (about one CTA's share of chunks), then the
   // token block, then the tile inside the group.  The CTAs working on one group for different
@@ -1805,6 +1832,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
     // ---------------- TMA producer
     uint32_t seq = 0;
     const int nseg = tail->nseg;
+    const int kc = F.fp8 ? 128 : 64;  // elements per 128-byte chunk
     int64_t g = g0;
     for (int si = 0; (nseg >= 0 ? si < nseg : g < g1) && !bt_aborted(tail); ++si) {
       const BtSeg S = bt_seg_at(F, nseg >= 0 ? tail->sg[si] : g, g1);
@@ -1816,8 +1844,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
         if (lane == 0) {
           uint8_t* st = sm + (size_t)s * stage_bytes;
           mbar_arrive_expect_tx(&tail->full[s], (uint32_t)stage_bytes);
-          tma_load_2d(st, &F.wmap[p], k * 64, S.ot * 128, &tail->full[s]);
-          tma_load_2d(st + BT_A_BYTES, &F.xmap[m], k * 64, S.tb * NB, &tail->full[s]);
+          tma_load_2d(st, &F.wmap[p], k * kc, S.ot * 128, &tail->full[s]);
+          tma_load_2d(st + BT_A_BYTES, &F.xmap[m], k * kc, S.tb * NB, &tail->full[s]);
         }
         __syncwarp();
       }
@@ -1825,7 +1853,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (one thread)
-    const uint32_t idesc = umma_idesc_bf16(128, NB);
+    const bool fp8 = F.fp8 != 0;
+    const uint32_t idesc = fp8 ? umma_idesc_e4m3(128, NB) : umma_idesc_bf16(128, NB);
     uint32_t seq = 0, segi = 0;
     const int nseg = tail->nseg;
     int64_t g = g0;
@@ -1846,9 +1875,16 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
         if (lane == 0) {
           const uint32_t a0 = smem_u32(sm + (size_t)s * stage_bytes);
           const uint64_t ad = umma_desc_sw128(a0), bd = umma_desc_sw128(a0 + BT_A_BYTES);
+          // 32 bytes of each row per MMA (K = 16 bf16 or K = 32 E4M3): 2 x 16 further inside the atom
+          if (fp8) {
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)  // K = 16 per MMA: 32 bytes further inside the swizzle atom
-            umma_f16(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (k > S.k0 || kk > 0) ? 1u : 0u);
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f8(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (k > S.k0 || kk > 0) ? 1u : 0u);
+          } else {
+#pragma unroll
+            for (int kk = 0; kk < 4; ++kk)
+              umma_f16(dt, ad + (uint64_t)(2 * kk), bd + (uint64_t)(2 * kk), idesc, (k > S.k0 || kk > 0) ? 1u : 0u);
+          }
           umma_commit(smem_u32(&tail->empty[s]));  // the stage is free once these MMAs have read it
         }
         __syncwarp();
@@ -1890,7 +1926,13 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
         const int ts = S.tb * NB + col;
         tail->perm[col] = ts < T ? P.perm[ts] : -1;
         tail->dfl[col] = (delta && ts < T) ? P.dflag[(int64_t)p * T + ts] : 0;
+        if (F.fp8) tail->sxs[col] = ts < T ? P.sx8[(int64_t)lin.input * T + ts] : 0.f;
       }
+      // fp8 backbone: the accumulator holds sum code_w code_x; the output row's weight scale and
+      // (per column) the token's activation scale turn it into W_hat x_hat
+      const float sw = F.fp8 ? reinterpret_cast<const float*>(static_cast<const uint8_t*>(lin.W) +
+                                                              (int64_t)lin.d_out * lin.d_in)[orow]
+                             : 1.f;
       named_bar(1, 256);
       const float* ydp = P.yd + (int64_t)p * T * F.ws.max_d_in + orow;
       for (int cb = 16 * wg; cb < NB; cb += 32) {
@@ -1903,6 +1945,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
           for (int j = 0; j < 16; ++j) {
             const int col = cb + j;
             yv[j] = __uint_as_float(r[j]);
+            if (F.fp8) yv[j] = yv[j] * sw * tail->sxs[col];
             if (tail->dfl[col]) yv[j] += ydp[(int64_t)(S.tb * NB + col) * F.ws.max_d_in];
           }
 #pragma unroll
@@ -1952,6 +1995,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
 #pragma unroll
             for (int j = 0; j < 16; ++j) {
               const int col = cb + j;
+              if (F.fp8) yv[j] = yv[j] * sw * tail->sxs[col];
               if (tail->dfl[col]) yv[j] += ydp[(int64_t)(S.tb * NB + col) * F.ws.max_d_in];
             }
 #pragma unroll
@@ -3116,6 +3160,61 @@ extern "C" int32_t dc_profile_end(float* ms_out, int32_t* kind_out, int32_t capa
   return rc;
 }
 
+// E4M3 rows: one block per row, 256 threads; the rounding is k_prep's (IEEE quotient, one conversion).
+__global__ void __launch_bounds__(256) k_quant_fp8_rows(const void* __restrict__ W, int bf16, int cols,
+                                                        uint8_t* __restrict__ codes, float* __restrict__ scales) {
+  const int64_t r = blockIdx.x;
+  const int tid = threadIdx.x;
+  auto load2 = [&](int k, float& a, float& b) {
+    if (bf16) {
+      const uint32_t q = *reinterpret_cast<const uint32_t*>((const __nv_bfloat16*)W + r * cols + k);
+      a = __uint_as_float(q << 16), b = __uint_as_float(q & 0xffff0000u);
+    } else {
+      const float2 q = *reinterpret_cast<const float2*>((const float*)W + r * cols + k);
+      a = q.x, b = q.y;
+    }
+  };
+  float mx = 0.f;
+  int bad = 0;
+  for (int k = 2 * tid; k < cols; k += 512) {
+    float a, b;
+    load2(k, a, b);
+    mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
+    bad |= (a - a != 0.f) | (b - b != 0.f);  // an infinity or a NaN
+  }
+  __shared__ float red[8];
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(FULLMASK, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  bad = __syncthreads_or(bad);
+  mx = red[0];
+#pragma unroll
+  for (int w = 1; w < 8; ++w) mx = fmaxf(mx, red[w]);
+  float s = __fdiv_rn(mx, 448.f);
+  if (s == 0.f) s = 1.f;
+  if (bad) s = __int_as_float(0x7fc00000);
+  for (int k = 2 * tid; k < cols; k += 512) {
+    float a, b;
+    load2(k, a, b);
+    *reinterpret_cast<uint16_t*>(codes + r * cols + k) = (uint16_t)e4m3x2(__fdiv_rn(a, s), __fdiv_rn(b, s));
+  }
+  if (tid == 0) scales[r] = s;
+}
+
+extern "C" dc_status dc_quantize_fp8_rows_device(const void* W, int32_t dtype, int32_t rows, int32_t cols,
+                                                 uint8_t* codes, float* scales, void* stream) {
+  DC_NVTX("dc_quantize_fp8_rows_device");
+  dc_clear_error();
+  if (rows < 0 || cols < 0) return dc_fail(DC_ERR_INVALID_ARG, "negative size");
+  if (cols % 16) return dc_fail(DC_ERR_SHAPE, "cols %d must be a multiple of 16", cols);
+  if (dtype != DC_DTYPE_F32 && dtype != DC_DTYPE_BF16) return dc_fail(DC_ERR_INVALID_ARG, "dtype");
+  if (rows == 0) return DC_OK;
+  if (!W || !codes || !scales) return dc_fail(DC_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(W) || !aligned16(codes) || !aligned16(scales)) return dc_fail(DC_ERR_ALIGN, "pointers must be 16-byte aligned");
+  k_quant_fp8_rows<<<rows, 256, 0, (cudaStream_t)stream>>>(W, dtype == DC_DTYPE_BF16, cols, codes, scales);
+  return dc_cuda_check(cudaGetLastError(), "fp8 quantise kernel");
+}
+
 extern "C" size_t dc_quantize_scratch_size(const dc_factor_desc* desc) {
   DC_NVTX("dc_quantize_scratch_size");
   DcLayout L;
@@ -3249,13 +3348,16 @@ static PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
 
 // 2-D tensor map of 16-bit elements (bf16 unless `dtype` says fp16): `rows` x `cols` (row pitch
 // `pitch` elements), box 64 columns x box_rows rows, 128-byte swizzle.
+// 2-D map of a row-major matrix (`pitch` elements between rows) whose box is one 128-byte row
+// segment (64 16-bit or 128 8-bit elements) by `box_rows` rows, 128-byte swizzle.
 static dc_status encode_map16(CUtensorMap* map, const void* base, int64_t cols, int64_t rows, int64_t pitch,
                                  int box_rows, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
   auto enc = tensor_map_encoder();
   if (!enc) return dc_fail(DC_ERR_CUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int esz = dtype == CU_TENSOR_MAP_DATA_TYPE_UINT8 ? 1 : 2;
   const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)pitch * 2};
-  const cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)pitch * esz};
+  const cuuint32_t box[2] = {(cuuint32_t)(128 / esz), (cuuint32_t)box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = enc(map, dtype, 2, const_cast<void*>(base), dims, strides, box, estr,
                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -3300,7 +3402,10 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
       return dc_fail(DC_ERR_SHAPE, "linear %d: d_out=%d d_in=%d must be multiples of 128", p, l.d_out, l.d_in);
     const int m = n_lin == 7 ? (p == 3 ? 1 : (p == 6 ? 2 : 0)) : 0;
     if (l.d_in != dxs[m]) return dc_fail(DC_ERR_SHAPE, "linear %d: d_in %d does not match its input (%d)", p, l.d_in, dxs[m]);
-    if (l.w_dtype != DC_DTYPE_BF16 && l.w_dtype != DC_DTYPE_F32) return dc_fail(DC_ERR_INVALID_ARG, "linear %d: w_dtype", p);
+    if (l.w_dtype != DC_DTYPE_BF16 && l.w_dtype != DC_DTYPE_F32 && l.w_dtype != DC_DTYPE_FP8)
+      return dc_fail(DC_ERR_INVALID_ARG, "linear %d: w_dtype", p);
+    if ((flags & DC_BASE) && (l.w_dtype == DC_DTYPE_FP8) != (lins[0].w_dtype == DC_DTYPE_FP8))
+      return dc_fail(DC_ERR_UNSUPPORTED, "linear %d: an fp8 backbone needs every linear of the call in fp8", p);
     if (l.w_dtype == DC_DTYPE_BF16 && dtype_in != DC_DTYPE_BF16 && (flags & DC_BASE))
       return dc_fail(DC_ERR_UNSUPPORTED, "linear %d: bf16 weights need bf16 activations", p);
     if (l.n_tenants < 0 || l.n_tenants > DC_MAX_TENANTS) return dc_fail(DC_ERR_INVALID_ARG, "linear %d: tenant count", p);
@@ -3321,10 +3426,24 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   F.ws = dc_ws_layout(T, max_rank, max_d_in, n_lin, max_ten);
   if (ws_bytes < (size_t)F.ws.total)
     return dc_fail(DC_ERR_WORKSPACE, "workspace holds %zu bytes, need %lld", ws_bytes, (long long)F.ws.total);
-  // bf16 backbones with bf16 activations run on the tcgen05 tensor cores
+  // bf16 backbones with bf16 activations, and fp8 backbones (activations quantised per token by
+  // k_prep), run on the tcgen05 tensor cores
+  F.fp8 = (flags & DC_BASE) && lins[0].w_dtype == DC_DTYPE_FP8;
   bool use_tc = (flags & DC_BASE) && dtype_in == DC_DTYPE_BF16;
   for (int p = 0; p < n_lin; ++p) use_tc = use_tc && lins[p].w_dtype == DC_DTYPE_BF16;
-  if (flags & DC_BASE) {
+  use_tc = use_tc || F.fp8;
+  if (F.fp8) {
+    for (int p = 0; p < n_lin; ++p) {
+      dc_status st0 = encode_map16(&F.wmap[p], lins[p].W_base, lins[p].d_in, lins[p].d_out, lins[p].d_in, 128,
+                                   CU_TENSOR_MAP_DATA_TYPE_UINT8);
+      if (st0) return st0;
+    }
+    for (int m = 0; m < n_in; ++m) {
+      const uint8_t* xb = (const uint8_t*)ws + F.ws.x8 + (int64_t)m * T * F.ws.max_d_in;
+      dc_status st0 = encode_map16(&F.xmap[m], xb, dxs[m], T, F.ws.max_d_in, F.ws.bt_nb, CU_TENSOR_MAP_DATA_TYPE_UINT8);
+      if (st0) return st0;
+    }
+  } else if (flags & DC_BASE) {
     for (int p = 0; p < n_lin; ++p)
       if (lins[p].w_dtype == DC_DTYPE_BF16) {
         dc_status st0 = encode_map16(&F.wmap[p], lins[p].W_base, lins[p].d_in, lins[p].d_out, lins[p].d_in, 128);
@@ -3435,9 +3554,10 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   if (use_tc) {
     F.bt_ntb = (T + F.ws.bt_nb - 1) / F.ws.bt_nb;
     F.bt_chunk_prefix[0] = 0;
+    const int kc = F.fp8 ? 128 : 64;  // elements per 128-byte chunk
     for (int i = 0; i < n_lin; ++i) {
       const dc_linear& l = lins[ord[i]];
-      F.bt_chunk_prefix[i + 1] = F.bt_chunk_prefix[i] + (int64_t)(l.d_out / 128) * F.bt_ntb * (l.d_in / 64);
+      F.bt_chunk_prefix[i + 1] = F.bt_chunk_prefix[i] + (int64_t)(l.d_out / 128) * F.bt_ntb * (l.d_in / kc);
     }
     F.bt_total = F.bt_chunk_prefix[n_lin];
     const int stage_bytes = BT_A_BYTES + F.ws.bt_nb * 128;
@@ -3446,7 +3566,7 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     for (int i = 0; i < n_lin; ++i) {  // tile groups of about one CTA's share of chunks
       const dc_linear& l = lins[ord[i]];
       const int64_t share = (F.bt_total + F.bt_grid - 1) / F.bt_grid;
-      F.bt_gtiles[i] = (int)std::max<int64_t>(1, std::min<int64_t>(l.d_out / 128, share / (l.d_in / 64)));
+      F.bt_gtiles[i] = (int)std::max<int64_t>(1, std::min<int64_t>(l.d_out / 128, share / (l.d_in / kc)));
     }
     const size_t tsmem = 1024 + (size_t)F.bt_ns * stage_bytes + sizeof(BtTail);
     st = allow_smem(dev, DC_K_BASE_TC, (const void*)k_base_tc, tsmem);

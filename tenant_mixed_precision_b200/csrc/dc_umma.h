@@ -3,7 +3,7 @@
 // completion tracking through mbarriers, and TMEM -> register loads.
 //
 // Conventions used here: both operands are K-major tiles in the 128-byte swizzle (rows of 64
-// 16-bit elements = 128 bytes, 8-row swizzle atoms of 1024 bytes, tile base
+// 16-bit or 128 8-bit elements = 128 bytes, 8-row swizzle atoms of 1024 bytes, tile base
 // 1024-byte aligned).  The accumulator is fp32 in TMEM: lane = row of A (M = 128), column =
 // row of B (N).  No instruction here uses cluster multicast.
 #pragma once
@@ -34,6 +34,11 @@ __host__ __device__ constexpr uint32_t umma_idesc_bf16(int M, int N) {
 __host__ __device__ constexpr uint32_t umma_idesc_f16(int M, int N) {
   return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// Instruction descriptor of kind::f8f6f4 with E4M3 A and B (format code 0 for both), fp32
+// accumulation, both K-major: the same bit fields as above, the kind being the instruction's.
+__host__ __device__ constexpr uint32_t umma_idesc_e4m3(int M, int N) {
+  return (1u << 4) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 
 // TMEM allocation of `ncols` columns (a power of two >= 32) by one whole warp; the base address
 // is written to shared memory at `dst_saddr`.
@@ -58,6 +63,17 @@ __device__ __forceinline__ void umma_f16(uint32_t d_tmem, uint64_t a_desc, uint6
   asm volatile(
       "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
       " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+
+// D[tmem] (+)= A * B^T for one K = 32 slice of kind::f8f6f4 (8-bit operands: 32 bytes of a K-major
+// row, the same byte step inside the swizzle atom as K = 16 of kind::f16); issued by one thread.
+__device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }

@@ -62,6 +62,17 @@ class DeltaStack:
                               device=device)
         self._lins = None
         self._keep = []
+        self.fp8 = False
+
+    def to_fp8_backbone(self, stream=None):
+        """Replace every bf16 backbone weight by its E4M3 blob (codes, then fp32 row scales),
+        quantised on the device, and rebuild the linear descriptors (DC_DTYPE_FP8)."""
+        from . import dc_quantize_fp8_rows_device
+        for l in range(self.layers):
+            for p in range(7):
+                self.W[l][p] = dc_quantize_fp8_rows_device(self.W[l][p], stream=stream)
+        self.fp8 = True
+        self.finalize()
 
     # -- loading -----------------------------------------------------------------------------
     def scratch_for(self, l: int, p: int, t: int) -> int:
@@ -121,7 +132,7 @@ class DeltaStack:
         v = u = w = act = 0
         for l in range(self.layers):
             for p, (d_out, d_in) in enumerate(self.shapes):
-                w += 2 * d_out * d_in
+                w += (d_out * d_in + 4 * d_out) if self.fp8 else 2 * d_out * d_in
                 act += T * (2 * d_in + out_es * d_out)
                 for t in distinct:
                     if (l, p, t) in self.descs:

@@ -103,3 +103,18 @@ def test_pager_and_svd():
     assert st == dc.DC_ERR_ALIGN
     st = _status("dc_svd_device", MIS, A, dc.DC_DTYPE_F32, 512, 512, 8, 8, 1, 0, A, A, A, A, BIG, None, C.byref(sw))
     assert st == dc.DC_ERR_ALIGN
+
+
+def test_fp8_quantiser_and_backbone_checks():
+    assert _status("dc_quantize_fp8_rows_device", MIS, dc.DC_DTYPE_F32, 4, 128, A, A, None) == dc.DC_ERR_ALIGN
+    assert _status("dc_quantize_fp8_rows_device", A, dc.DC_DTYPE_F32, 4, 128, A, MIS, None) == dc.DC_ERR_ALIGN
+    assert _status("dc_quantize_fp8_rows_device", A, dc.DC_DTYPE_F32, 4, 120, A, A, None) == dc.DC_ERR_SHAPE
+    assert _status("dc_quantize_fp8_rows_device", A, dc.DC_DTYPE_FP8, 4, 128, A, A, None) == dc.DC_ERR_INVALID_ARG
+    # an fp8 backbone is all or nothing within one call (one tensor-core kernel serves every linear)
+    lins = (dc.dc_linear * 7)(*[dc.make_linear(A, 512, 512 if p != 6 else 1024, 2, 64, A,
+                                               w_dtype=dc.DC_DTYPE_FP8 if p != 4 else dc.DC_DTYPE_BF16)
+                                for p in range(7)])
+    ys = (C.c_void_p * 7)(*[A] * 7)
+    st = _status("dc_layer_forward", lins, A, A, A, ys, A, 4, dc.DC_DTYPE_BF16, dc.DC_DTYPE_F32, dc.DC_BASE, A,
+                 BIG, None)
+    assert st == dc.DC_ERR_UNSUPPORTED
