@@ -182,9 +182,11 @@ struct DcFwd {
   int32_t n_lin, T, dtype_in, dtype_out, flags, pad;
   int32_t order[7];        // launch order of the linears in the U kernel (largest first)
   int32_t tile_prefix[8];  // cumulative 128-row output tiles in that order
-  int64_t bt_chunk_prefix[8];  // tensor-core backbone: cumulative 64-column chunks of all units, same order
+  int64_t bt_chunk_prefix[8];  // tensor-core backbone: cumulative 128-byte chunks of all units, same order
+                               // (with teams: of one token block's units)
   int64_t bt_total;            // total chunks
-  int32_t bt_ntb, bt_ns, bt_grid, bt_pad;  // token blocks, pipeline stages, CTAs
+  int64_t bt_ctb;              // with teams: chunks of one token block
+  int32_t bt_ntb, bt_ns, bt_grid, bt_team;  // token blocks, pipeline stages, CTAs, team size (0: no teams)
   int32_t bt_gtiles[8];        // per linear (same order): row tiles per group of the unit order
   CUtensorMap tmap;            // prefill path: fp16 t plane [n_lin T rows x tcols], box 64 x 256
   CUtensorMap xpf[3];          // prefill path: fp16 scaled tenant-sorted activations, box 64 x pf_box
@@ -1726,14 +1728,52 @@ struct BtTail {
   int64_t sg[BT_MAX_SEGS];  // their first chunks, in processing order
 };
 
-__device__ __forceinline__ int64_t bt_g0(const DcFwd& F, int c) { return (int64_t)c * F.bt_total / F.bt_grid; }
+// Two schedules share the chunk bookkeeping below.
+// Stream-K (one token block, or too many for teams): the chunks of all units in one sequence,
+// split into equal contiguous ranges, CTA c taking range c.
+// Teams (several token blocks): a team holds one CTA per token block; the chunks of one token
+// block's units (tile-major, k inner) are split into equal ranges, one per team, and CTA
+// (team, tb) takes its team's range for token block tb.  A team's CTAs walk the same weight
+// chunks in step, so each chunk comes from DRAM once and from L2 for the other token blocks.
+// Global chunk index with teams: tb * ctb + h, h the index inside the token block's sequence.
+__device__ __forceinline__ int64_t bt_share(const DcFwd& F, int64_t total, int parts, int i) {
+  return (int64_t)i * total / parts;
+}
+
+// [g0, g1): the chunk range of CTA c
+__device__ __forceinline__ void bt_range(const DcFwd& F, int c, int64_t& g0, int64_t& g1) {
+  if (F.bt_team) {
+    const int nt = F.bt_grid / F.bt_team, tau = c / F.bt_team, tb = c - tau * F.bt_team;
+    g0 = (int64_t)tb * F.bt_ctb + bt_share(F, F.bt_ctb, nt, tau);
+    g1 = (int64_t)tb * F.bt_ctb + bt_share(F, F.bt_ctb, nt, tau + 1);
+  } else {
+    g0 = bt_share(F, F.bt_total, F.bt_grid, c);
+    g1 = bt_share(F, F.bt_total, F.bt_grid, c + 1);
+  }
+}
+
+__device__ __forceinline__ int64_t bt_g0(const DcFwd& F, int c) {
+  int64_t g0, g1;
+  bt_range(F, c, g0, g1);
+  return g0;
+}
+
+// index of the equal share of `total` in `parts` that holds x
+__device__ __forceinline__ int bt_part_of(const DcFwd& F, int64_t x, int64_t total, int parts) {
+  int i = (int)(x * parts / total);
+  while (i + 1 < parts && bt_share(F, total, parts, i + 1) <= x) ++i;
+  while (i > 0 && bt_share(F, total, parts, i) > x) --i;
+  return i;
+}
 
 // CTA whose chunk range holds global chunk g
 __device__ __forceinline__ int bt_cta_of(const DcFwd& F, int64_t g) {
-  int c = (int)(g * F.bt_grid / F.bt_total);
-  while (c + 1 < F.bt_grid && bt_g0(F, c + 1) <= g) ++c;
-  while (c > 0 && bt_g0(F, c) > g) --c;
-  return c;
+  if (F.bt_team) {
+    const int nt = F.bt_grid / F.bt_team;
+    const int tb = (int)(g / F.bt_ctb);
+    return bt_part_of(F, g - (int64_t)tb * F.bt_ctb, F.bt_ctb, nt) * F.bt_team + tb;
+  }
+  return bt_part_of(F, g, F.bt_total, F.bt_grid);
 }
 
 struct BtSeg {
@@ -1744,6 +1784,22 @@ struct BtSeg {
 
 __device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1) {
   BtSeg S;
+  if (F.bt_team) {  // h: index inside token block tb's sequence; units tile-major
+    const int tb = (int)(g / F.bt_ctb);
+    const int64_t h = g - (int64_t)tb * F.bt_ctb;
+    int slot = 0;
+    while (slot + 1 < F.n_lin && h >= F.bt_chunk_prefix[slot + 1]) ++slot;
+    S.slot = slot;
+    S.K = F.lin[F.order[slot]].d_in / (F.fp8 ? 128 : 64);
+    const int tile = (int)((h - F.bt_chunk_prefix[slot]) / S.K);
+    S.u = (F.tile_prefix[slot] + tile) * F.bt_ntb + tb;
+    S.ot = tile;
+    S.tb = tb;
+    S.ustart = (int64_t)tb * F.bt_ctb + F.bt_chunk_prefix[slot] + (int64_t)tile * S.K;
+    S.k0 = (int)(g - S.ustart);
+    S.k1 = (int)min((int64_t)S.K, g1 - S.ustart);
+    return S;
+  }
   int slot = 0;
   while (slot + 1 < F.n_lin && g >= F.bt_chunk_prefix[slot + 1]) ++slot;
   S.slot = slot;
@@ -1786,7 +1842,8 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int T = F.ws.T;
   const int c = blockIdx.x;
-  const int64_t g0 = bt_g0(F, c), g1 = bt_g0(F, c + 1);
+  int64_t g0, g1;
+  bt_range(F, c, g0, g1);
   uint32_t ncols = 32;
   while (ncols < (uint32_t)(2 * NB)) ncols <<= 1;
   if (threadIdx.x == 0) {
@@ -1971,10 +2028,12 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
         // hand the partial over; the last contributor of the unit finishes it
         __threadfence();
         named_bar(1, 256);
+        // the unit's contributors: CTAs c0, c0 + cs, ..., c1 (cs = 1, or the team size)
         const int c0 = bt_cta_of(F, S.ustart), c1 = bt_cta_of(F, S.ustart + S.K - 1);
+        const int cs = F.bt_team ? F.bt_team : 1;
         if (et == 0) {
           const int old = atomicAdd(cnt + S.u, 1);
-          tail->last_flag = old == c1 - c0;
+          tail->last_flag = old == (c1 - c0) / cs;
           __threadfence();
         }
         named_bar(1, 256);
@@ -1983,7 +2042,7 @@ __global__ void __launch_bounds__(BT_THREADS, 1) k_base_tc(const __grid_constant
             float yv[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j) yv[j] = 0.f;
-            for (int cc = c0; cc <= c1; ++cc) {  // k order
+            for (int cc = c0; cc <= c1; cc += cs) {  // k order
               const int sl = S.ustart <= bt_g0(F, cc) ? 0 : 1;
               const float* pp = part_base + ((int64_t)(2 * cc + sl) * NB + cb) * 128 + row;
               float pv[16];
@@ -3553,16 +3612,25 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
   }
   if (use_tc) {
     F.bt_ntb = (T + F.ws.bt_nb - 1) / F.ws.bt_nb;
-    F.bt_chunk_prefix[0] = 0;
     const int kc = F.fp8 ? 128 : 64;  // elements per 128-byte chunk
+    const int max_ctas = std::min(n_sm, DC_BT_MAX_CTAS);
+    int64_t ctb = 0;  // chunks of one token block's units
+    for (int i = 0; i < n_lin; ++i) ctb += (int64_t)(lins[ord[i]].d_out / 128) * (lins[ord[i]].d_in / kc);
+    // teams of one CTA per token block when there are several blocks (prefill-sized batches)
+    F.bt_team = (F.bt_ntb >= 2 && F.bt_ntb <= max_ctas) ? F.bt_ntb : 0;
+    F.bt_ctb = ctb;
+    F.bt_chunk_prefix[0] = 0;
     for (int i = 0; i < n_lin; ++i) {
       const dc_linear& l = lins[ord[i]];
-      F.bt_chunk_prefix[i + 1] = F.bt_chunk_prefix[i] + (int64_t)(l.d_out / 128) * F.bt_ntb * (l.d_in / kc);
+      F.bt_chunk_prefix[i + 1] = F.bt_chunk_prefix[i] + (int64_t)(l.d_out / 128) * (F.bt_team ? 1 : F.bt_ntb) * (l.d_in / kc);
     }
-    F.bt_total = F.bt_chunk_prefix[n_lin];
+    F.bt_total = ctb * F.bt_ntb;
     const int stage_bytes = BT_A_BYTES + F.ws.bt_nb * 128;
     F.bt_ns = std::min(BT_MAX_STAGES, (int)((200 * 1024) / stage_bytes));
-    F.bt_grid = (int)std::min<int64_t>(std::min(n_sm, DC_BT_MAX_CTAS), F.bt_total);
+    if (F.bt_team)
+      F.bt_grid = (int)std::min<int64_t>(max_ctas / F.bt_team, ctb) * F.bt_team;
+    else
+      F.bt_grid = (int)std::min<int64_t>(max_ctas, F.bt_total);
     for (int i = 0; i < n_lin; ++i) {  // tile groups of about one CTA's share of chunks
       const dc_linear& l = lins[ord[i]];
       const int64_t share = (F.bt_total + F.bt_grid - 1) / F.bt_grid;
