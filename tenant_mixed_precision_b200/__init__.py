@@ -368,6 +368,9 @@ def dc_quantize_fp8_rows_device(W, stream=None):
     blob = torch.empty(rows * cols + 4 * rows, dtype=torch.uint8, device=W.device)
     _check(_load().dc_quantize_fp8_rows_device(_ptr(W), _dtype_code(W), rows, cols, _ptr(blob),
                                                blob.data_ptr() + rows * cols, _stream(stream)))
+    if isinstance(stream, torch.cuda.Stream):  # both buffers are in use on that stream
+        W.record_stream(stream)
+        blob.record_stream(stream)
     return blob
 
 

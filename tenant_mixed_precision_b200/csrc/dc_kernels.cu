@@ -1695,18 +1695,21 @@ __global__ void __launch_bounds__(KB_THREADS, 1) k_base(const __grid_constant__ 
 }
 
 // ---------------------------------------------------------------------------------------------
-// k_base_tc: y = W_base x (+ ydelta) on the tcgen05 tensor cores, for bf16 backbones.
-// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens), ordered inside
-// a linear by group of tiles, token block, tile; its K is cut into 64-column chunks.  The units'
-// chunks, largest-K linears first, form one sequence that is
-// split evenly over the persistent CTAs (stream-K), so every CTA moves the same number of bytes
-// whatever the tile count.  Per CTA: warp 0 loads each chunk's W slice (128 x 64) and activation
-// slice (NB x 64) with 2-D TMA into a ring of stages; warp 1 owns two NB-column fp32
-// accumulators in Tensor Memory and, from one thread, issues 4 MMAs (M 128, N NB, K 16) per
-// chunk, releasing the stage with a commit; warps 2-9 (two warpgroups, one TMEM lane quarter per
-// warp, lane = output row) drain a finished accumulator.  A unit shared by several CTAs leaves fp32 partial tiles;
-// the last contributor to arrive (a counter per unit) adds them in k order, so the result does
-// not depend on timing.  The epilogue adds the delta and writes y in the tokens' original order.
+// k_base_tc: y = W_base x (+ ydelta) on the tcgen05 tensor cores, for bf16 backbones (kind::f16)
+// and E4M3 backbones (kind::f8f6f4, activations quantised per token by k_prep).
+// A unit is (linear p, 128-row output tile ot, block of NB tenant-sorted tokens); its K is cut
+// into chunks of 128 bytes of a row (64 bf16 or 128 E4M3 columns).  With one token block the
+// units' chunks (ordered inside a linear by group of tiles, token block, tile), largest-K linears
+// first, form one sequence split evenly over the persistent CTAs (stream-K), so every CTA moves
+// the same number of bytes whatever the tile count; with several token blocks the CTAs form teams
+// of one CTA per block that split one block's sequence (see bt_range).  Per CTA: warp 0 loads each
+// chunk's W slice (128 rows) and activation slice (NB rows) with 2-D TMA into a ring of stages;
+// warp 1 owns two NB-column fp32 accumulators in Tensor Memory and, from one thread, issues 4 MMAs
+// (M 128, N NB, 32 bytes of K each) per chunk, releasing the stage with a commit; warps 2-9 (two
+// warpgroups, one TMEM lane quarter per warp, lane = output row) drain a finished accumulator.
+// A unit shared by several CTAs leaves fp32 partial tiles; the last contributor to arrive (a
+// counter per unit) adds them in k order, so the result does not depend on timing.  The epilogue
+// applies the E4M3 scales, adds the delta and writes y in the tokens' original order.
 // ---------------------------------------------------------------------------------------------
 #define BT_THREADS 320
 #define BT_MAX_STAGES 8
