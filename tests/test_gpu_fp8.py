@@ -111,11 +111,13 @@ def _run(lin, x, ids, T, d_out, flags, n_ten, max_rank, d_in):
 
 
 # (d_out, d_in, ids): ragged token counts (one partial 16-column block; more than one 256-token
-# block), several row tiles, d_in of 5 and 9 chunks of 128, long runs that take the prefill delta path
+# block, down to a last block of one token), several row tiles, d_in of 4, 5 and 9 chunks of 128,
+# long runs that take the prefill delta path
 LINEAR_CASES = [
     (384, 640, [1, 0, 2, 1, -1, 0, 0, 2, 1] * 4 + [2]),
     (256, 1152, [0] * 150 + [1] * 3 + [-1] * 7 + [2] * 140),
     (640, 256, [2, -1, 0]),
+    (384, 512, [0] * 100 + [2] * 90 + [1] * 67),  # 257 tokens: a last token block of one token
 ]
 
 

@@ -216,3 +216,23 @@ def test_t_zero_is_noop_and_errors_are_reported():
     with pytest.raises(dc.DcError) as e:
         dc.dc_delta_linear_segmented(bad, x, y, ids, 1, dc.DC_BASE, ws)
     assert e.value.status == dc.DC_ERR_SHAPE
+
+
+@pytest.mark.parametrize("T,d_out,d_in", [(257, 384, 640), (513, 640, 256), (1000, 128, 1152)])
+def test_backbone_team_schedule_edges(T, d_out, d_in):
+    """Batches of several 256-token blocks run the backbone in teams (one CTA per token block):
+    a last block of one token (257), an odd number of row tiles, a single row tile whose units
+    every team splits (128 rows x 9 chunks over many teams), against the oracle (full output and
+    the delta alone) and against the same batch forced onto the decode delta kernels."""
+    rng = np.random.default_rng(T)
+    n_ten = 3
+    plans = [[(8, 2), (3, 16), (2, 40)], [(2, 64)], [(3, 20)]]
+    ids = rng.integers(-1, n_ten, size=T).astype(np.int32)
+    td, W, x, wf, xf = _bf16_case(T + d_out, d_out, d_in, plans, n_ten, list(ids))
+    outs = {}
+    for flags in (dc.DC_BASE | dc.DC_DELTA, dc.DC_DELTA, dc.DC_BASE | dc.DC_DELTA | dc.DC_DECODE_ONLY):
+        outs[flags] = _run_linear(td, W, x, ids, flags).cpu().numpy()
+    assert_close(outs[dc.DC_BASE | dc.DC_DELTA], oracle_y(wf, td, xf, ids, dc.DC_BASE | dc.DC_DELTA), f"T={T} full")
+    assert_close(outs[dc.DC_DELTA], oracle_y(wf, td, xf, ids, dc.DC_DELTA), f"T={T} delta")
+    assert_close(outs[dc.DC_BASE | dc.DC_DELTA | dc.DC_DECODE_ONLY], oracle_y(wf, td, xf, ids, dc.DC_BASE | dc.DC_DELTA),
+                 f"T={T} decode kernels")
