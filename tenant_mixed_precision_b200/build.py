@@ -21,7 +21,7 @@ NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 LIBS = {
     "libdc.so": {
         "sources": ["dc_host.cpp", "dc_prinmix.cpp", "dc_kernels.cu", "dc_pager.cu", "dc_svd.cu"],
-        "headers": ["dc_layout.h", "dc_pack.h", "dc_internal.h", "dc_tma.h", "dc_umma.h", "dc_devstate.h", "dc_lru.h"],
+        "headers": ["dc_layout.h", "dc_pack.h", "dc_internal.h", "dc_tma.h", "dc_umma.h", "dc_devstate.h", "dc_lru.h", "dc_btsched.h"],
         "link": ["-lcudart"],
     },
     "libdc_synth.so": {

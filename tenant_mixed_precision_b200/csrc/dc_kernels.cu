@@ -28,6 +28,7 @@
 #include <mutex>
 
 #include "dc.h"
+#include "dc_btsched.h"
 #include "dc_devstate.h"
 #include "dc_internal.h"
 #include "dc_layout.h"
@@ -1731,99 +1732,7 @@ struct BtTail {
   int64_t sg[BT_MAX_SEGS];  // their first chunks, in processing order
 };
 
-// Two schedules share the chunk bookkeeping below.
-// Stream-K (one token block, or too many for teams): the chunks of all units in one sequence,
-// split into equal contiguous ranges, CTA c taking range c.
-// Teams (several token blocks): a team holds one CTA per token block; the chunks of one token
-// block's units (tile-major, k inner) are split into equal ranges, one per team, and CTA
-// (team, tb) takes its team's range for token block tb.  A team's CTAs walk the same weight
-// chunks in step, so each chunk comes from DRAM once and from L2 for the other token blocks.
-// Global chunk index with teams: tb * ctb + h, h the index inside the token block's sequence.
-__device__ __forceinline__ int64_t bt_share(const DcFwd& F, int64_t total, int parts, int i) {
-  return (int64_t)i * total / parts;
-}
-
-// [g0, g1): the chunk range of CTA c
-__device__ __forceinline__ void bt_range(const DcFwd& F, int c, int64_t& g0, int64_t& g1) {
-  if (F.bt_team) {
-    const int nt = F.bt_grid / F.bt_team, tau = c / F.bt_team, tb = c - tau * F.bt_team;
-    g0 = (int64_t)tb * F.bt_ctb + bt_share(F, F.bt_ctb, nt, tau);
-    g1 = (int64_t)tb * F.bt_ctb + bt_share(F, F.bt_ctb, nt, tau + 1);
-  } else {
-    g0 = bt_share(F, F.bt_total, F.bt_grid, c);
-    g1 = bt_share(F, F.bt_total, F.bt_grid, c + 1);
-  }
-}
-
-__device__ __forceinline__ int64_t bt_g0(const DcFwd& F, int c) {
-  int64_t g0, g1;
-  bt_range(F, c, g0, g1);
-  return g0;
-}
-
-// index of the equal share of `total` in `parts` that holds x
-__device__ __forceinline__ int bt_part_of(const DcFwd& F, int64_t x, int64_t total, int parts) {
-  int i = (int)(x * parts / total);
-  while (i + 1 < parts && bt_share(F, total, parts, i + 1) <= x) ++i;
-  while (i > 0 && bt_share(F, total, parts, i) > x) --i;
-  return i;
-}
-
-// CTA whose chunk range holds global chunk g
-__device__ __forceinline__ int bt_cta_of(const DcFwd& F, int64_t g) {
-  if (F.bt_team) {
-    const int nt = F.bt_grid / F.bt_team;
-    const int tb = (int)(g / F.bt_ctb);
-    return bt_part_of(F, g - (int64_t)tb * F.bt_ctb, F.bt_ctb, nt) * F.bt_team + tb;
-  }
-  return bt_part_of(F, g, F.bt_total, F.bt_grid);
-}
-
-struct BtSeg {
-  int u, slot, ot, tb, K;  // unit, linear order slot, tile, token block, chunks of the unit
-  int64_t ustart;          // global index of the unit's first chunk
-  int k0, k1;              // chunk range of this segment inside the unit
-};
-
-__device__ __forceinline__ BtSeg bt_seg_at(const DcFwd& F, int64_t g, int64_t g1) {
-  BtSeg S;
-  if (F.bt_team) {  // h: index inside token block tb's sequence; units tile-major
-    const int tb = (int)(g / F.bt_ctb);
-    const int64_t h = g - (int64_t)tb * F.bt_ctb;
-    int slot = 0;
-    while (slot + 1 < F.n_lin && h >= F.bt_chunk_prefix[slot + 1]) ++slot;
-    S.slot = slot;
-    S.K = F.lin[F.order[slot]].d_in / (F.fp8 ? 128 : 64);
-    const int tile = (int)((h - F.bt_chunk_prefix[slot]) / S.K);
-    S.u = (F.tile_prefix[slot] + tile) * F.bt_ntb + tb;
-    S.ot = tile;
-    S.tb = tb;
-    S.ustart = (int64_t)tb * F.bt_ctb + F.bt_chunk_prefix[slot] + (int64_t)tile * S.K;
-    S.k0 = (int)(g - S.ustart);
-    S.k1 = (int)min((int64_t)S.K, g1 - S.ustart);
-    return S;
-  }
-  int slot = 0;
-  while (slot + 1 < F.n_lin && g >= F.bt_chunk_prefix[slot + 1]) ++slot;
-  S.slot = slot;
-  S.K = F.lin[F.order[slot]].d_in / (F.fp8 ? 128 : 64);  // chunks of 128 bytes of a row
-  const int64_t local = (g - F.bt_chunk_prefix[slot]) / S.K;
-  // unit order inside a linear: groups of G row tiles (about one CTA's share of chunks), then the
-  // token block, then the tile inside the group.  The CTAs working on one group for different
-  // token blocks start within about one tile of each other and walk the same tiles in step, so a
-  // weight tile comes from DRAM once and from L2 for its other token blocks.
-  const int ntiles = F.lin[F.order[slot]].d_out / 128, ntb = F.bt_ntb, G = F.bt_gtiles[slot];
-  const int grp = (int)(local / ((int64_t)G * ntb));
-  const int gl = min(G, ntiles - grp * G);  // tiles of this group (the last may be short)
-  const int rem = (int)(local - (int64_t)grp * G * ntb);
-  S.u = (int)(F.tile_prefix[slot] * (int64_t)ntb + local);
-  S.ot = grp * G + rem % gl;
-  S.tb = rem / gl;
-  S.ustart = F.bt_chunk_prefix[slot] + local * S.K;
-  S.k0 = (int)(g - S.ustart);
-  S.k1 = (int)min((int64_t)S.K, g1 - S.ustart);
-  return S;
-}
+// The chunk bookkeeping of both schedules (stream-K, teams) is in dc_btsched.h.
 
 __device__ __forceinline__ bool bt_aborted(BtTail* tail) { return *reinterpret_cast<volatile int*>(&tail->abort) != 0; }
 
@@ -3518,15 +3427,8 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
         if (st0) return st0;
       }
   }
-  // U-kernel order: largest output tiles first (d_in decides the bytes per tile)
-  int ord[7];
-  for (int p = 0; p < n_lin; ++p) ord[p] = p;
-  std::stable_sort(ord, ord + n_lin, [&](int a, int b) { return lins[a].d_in > lins[b].d_in; });
-  F.tile_prefix[0] = 0;
-  for (int i = 0; i < n_lin; ++i) {
-    F.order[i] = ord[i];
-    F.tile_prefix[i + 1] = F.tile_prefix[i] + lins[ord[i]].d_out / 128;
-  }
+  // U-kernel and backbone order: largest output tiles first (d_in decides the bytes per tile)
+  bt_plan_order(F);
   // long segments take the tensor-core delta path when the batch is large enough
   F.pf = (flags & DC_DELTA) && !(flags & DC_DECODE_ONLY) && T >= 2 * DC_PF_MIN;
   if (F.pf) {
@@ -3614,31 +3516,9 @@ static dc_status run_forward(const dc_linear* lins, int n_lin, const void* const
     }
   }
   if (use_tc) {
-    F.bt_ntb = (T + F.ws.bt_nb - 1) / F.ws.bt_nb;
-    const int kc = F.fp8 ? 128 : 64;  // elements per 128-byte chunk
-    const int max_ctas = std::min(n_sm, DC_BT_MAX_CTAS);
-    int64_t ctb = 0;  // chunks of one token block's units
-    for (int i = 0; i < n_lin; ++i) ctb += (int64_t)(lins[ord[i]].d_out / 128) * (lins[ord[i]].d_in / kc);
-    // teams of one CTA per token block when there are several blocks (prefill-sized batches)
-    F.bt_team = (F.bt_ntb >= 2 && F.bt_ntb <= max_ctas) ? F.bt_ntb : 0;
-    F.bt_ctb = ctb;
-    F.bt_chunk_prefix[0] = 0;
-    for (int i = 0; i < n_lin; ++i) {
-      const dc_linear& l = lins[ord[i]];
-      F.bt_chunk_prefix[i + 1] = F.bt_chunk_prefix[i] + (int64_t)(l.d_out / 128) * (F.bt_team ? 1 : F.bt_ntb) * (l.d_in / kc);
-    }
-    F.bt_total = ctb * F.bt_ntb;
+    bt_plan(F, T, F.ws.bt_nb, std::min(n_sm, DC_BT_MAX_CTAS));
     const int stage_bytes = BT_A_BYTES + F.ws.bt_nb * 128;
     F.bt_ns = std::min(BT_MAX_STAGES, (int)((200 * 1024) / stage_bytes));
-    if (F.bt_team)
-      F.bt_grid = (int)std::min<int64_t>(max_ctas / F.bt_team, ctb) * F.bt_team;
-    else
-      F.bt_grid = (int)std::min<int64_t>(max_ctas, F.bt_total);
-    for (int i = 0; i < n_lin; ++i) {  // tile groups of about one CTA's share of chunks
-      const dc_linear& l = lins[ord[i]];
-      const int64_t share = (F.bt_total + F.bt_grid - 1) / F.bt_grid;
-      F.bt_gtiles[i] = (int)std::max<int64_t>(1, std::min<int64_t>(l.d_out / 128, share / (l.d_in / kc)));
-    }
     const size_t tsmem = 1024 + (size_t)F.bt_ns * stage_bytes + sizeof(BtTail);
     st = allow_smem(dev, DC_K_BASE_TC, (const void*)k_base_tc, tsmem);
     if (st) return st;
