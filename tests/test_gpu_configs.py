@@ -5,7 +5,8 @@
   output of three projections (q, gate, down: the three shapes) against the oracle;
 * the 13B-shaped prefill layer (2048 tokens in segments of 32-256, 16 tenants): sampled outputs
   of q, gate and down against the oracle, with sampled tokens taken both from tenants with 64+
-  tokens (the tensor-core prefill path) and from a tenant with fewer (the decode kernels);
+  tokens (the tensor-core prefill path) and from a tenant with fewer (the decode kernels); the
+  same layer with the fp8 (E4M3) backbone option against the oracle's fp8 backbone;
 * edge cases: a batch of backbone-only tokens, tenants without a delta, one token.
 """
 import numpy as np
@@ -139,3 +140,37 @@ def test_edge_cases(case):
             assert np.array_equal(got, want), case  # no delta anywhere: exactly zero
         else:
             assert_close(got, want, f"{case} flags={flags}")
+
+
+def test_13b_prefill_layer_fp8_backbone_sampled_against_oracle():
+    """The same 13B prefill layer with the fp8 (E4M3) backbone option: sampled outputs against the
+    oracle's fp8 backbone of the regenerated weights (within the fp32 accumulation bound of
+    tests/test_gpu_fp8.py) plus the delta oracle (at the serving path's parity bound)."""
+    from oracle import fp8 as ofp8
+
+    seed, s0, T = 20244, 0.02 * np.sqrt(5120.0), 2048
+    st = _stack(5120, 13824, 16, T, seed, s0)
+    st.to_fp8_backbone()
+    ids = synth.prefill_segments(np.random.default_rng(4), T, 16)
+    full = _run(st, ids, dc.DC_BASE | dc.DC_DELTA)
+    base = _run(st, ids, dc.DC_BASE)
+    rng = np.random.default_rng(9)
+    counts = np.bincount(ids, minlength=16)
+    long_t = [k for k in range(T) if counts[ids[k]] >= PF_MIN]
+    short_t = [k for k in range(T) if 0 < counts[ids[k]] < PF_MIN]
+    toks = np.array(sorted({long_t[0], long_t[-1], short_t[len(short_t) // 2], int(rng.integers(0, T))}))
+    for proj in (0, 4, 6):
+        d_out, d_in = st.shapes[proj]
+        rows = np.concatenate([np.arange(128) + 128 * int(rng.integers(0, d_out // 128)) for _ in range(2)])
+        _, xv = host_activations(seed, 0, synth.PROJ_INPUT[proj], T, d_in)
+        _, wv = synth.stream_base_weight(seed, 0, proj, d_out, d_in, rows=rows)
+        wc, ws = ofp8.quantize_rows(np.asarray(wv, np.float32))
+        x = np.asarray(xv, np.float32)[toks]
+        ref_b = ofp8.backbone(wc, ws, x)
+        xc, xs = ofp8.quantize_rows(x)
+        bound = 2.0 * (d_in + 2) * 2.0 ** -24 * (np.abs(ofp8.dequantize_rows(xc, xs)) @ np.abs(ofp8.dequantize_rows(wc, ws)).T)
+        got_b = base[proj][toks][:, rows]
+        assert np.all(np.abs(got_b - ref_b) <= bound + 1e-30), f"fp8 backbone, proj {proj}"
+        ref_d = _oracle(seed, s0, proj, d_out, d_in, T, ids, toks, rows, dc.DC_DELTA)
+        assert_close(full[proj][toks][:, rows] - got_b, ref_d, f"13B fp8 prefill proj {proj} delta")
+        assert_close(full[proj][toks][:, rows], ref_b + ref_d, f"13B fp8 prefill proj {proj}")
