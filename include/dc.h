@@ -56,7 +56,9 @@ enum {
 
 /* DC_DTYPE_FP8 is a backbone weight format only (dc_linear.w_dtype): W_base then points at the
  * E4M3 codes row-major [d_out, d_in] followed directly by the fp32 row scales [d_out]
- * (dc_quantize_fp8_rows); activations stay bf16 and are quantised per token inside the call. */
+ * (dc_quantize_fp8_rows, dc_quantize_fp8_rows_device); the activations (bf16 or fp32) are
+ * quantised per token inside the call.  With DC_BASE, either every linear of a call is fp8 or none
+ * is (DC_ERR_UNSUPPORTED otherwise). */
 enum { DC_DTYPE_F32 = 0, DC_DTYPE_BF16 = 1, DC_DTYPE_FP8 = 2 };
 
 /* flags of dc_delta_linear_segmented / dc_layer_forward */
@@ -95,8 +97,10 @@ typedef struct {
 
 /* One linear of the backbone plus the deltas of every tenant for it. */
 typedef struct {
-  const void* W_base;        /* device, row-major [d_out, d_in], dtype w_dtype                */
-  int32_t w_dtype;           /* DC_DTYPE_BF16 (tensor-core path) or DC_DTYPE_F32              */
+  const void* W_base;        /* device, row-major [d_out, d_in], dtype w_dtype (fp8: codes then
+                                row scales, see DC_DTYPE_FP8)                                  */
+  int32_t w_dtype;           /* DC_DTYPE_BF16 or DC_DTYPE_FP8 (tensor-core path), or
+                                DC_DTYPE_F32                                                   */
   int32_t d_out, d_in;
   int32_t n_tenants;         /* tenant ids run over 0..n_tenants-1                            */
   int32_t max_rank;          /* upper bound of rank_total over the tenants (workspace sizing) */
