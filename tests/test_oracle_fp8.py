@@ -83,3 +83,28 @@ def test_library_fp8_quantiser_matches_oracle():
     assert np.array_equal(fp8.E4M3_TABLE[codes.astype(np.int64)], fp8.E4M3_TABLE[oc.astype(np.int64)])
     blob = dc.fp8_weight_blob(codes, sc)
     assert blob.nbytes == w.size + 4 * w.shape[0]
+
+
+def test_backbone_is_the_plain_product_on_exact_inputs():
+    """F3 pinned: when every row's largest magnitude is 448 times a power of two and every element is
+    that power of two times an E4M3 value, the per-row/per-token scales are exact powers of two, the
+    quantisation loses nothing, and the oracle's fp8 backbone equals the plain product W x^T (for a
+    non-square W, so a transposed operand would show); `rows` selects output rows."""
+    rng = np.random.default_rng(21)
+    finite = fp8.E4M3_TABLE[np.arange(0x7F)]  # non-negative finite values, 0 .. 448
+
+    def exact_rows(n, m, expo):
+        v = rng.choice(finite, size=(n, m)) * rng.choice([-1.0, 1.0], size=(n, m))
+        v[:, 0] = 448.0  # the row maximum
+        return (v * (2.0 ** expo)[:, None]).astype(np.float32)
+
+    W = exact_rows(24, 40, rng.integers(-12, 3, size=24))
+    x = exact_rows(5, 40, rng.integers(-6, 6, size=5))
+    wc, ws = fp8.quantize_rows(W)
+    assert np.array_equal(fp8.dequantize_rows(wc, ws), W.astype(np.float64))
+    got = fp8.backbone(wc, ws, x)
+    want = x.astype(np.float64) @ W.astype(np.float64).T
+    assert got.shape == (5, 24)
+    assert np.array_equal(got, want)
+    rows = np.array([3, 17, 0])
+    assert np.array_equal(fp8.backbone(wc, ws, x, rows=rows), want[:, rows])
