@@ -20,7 +20,8 @@ F3  y = sum_j (code_w * s_row) (code_x * s_tok) + the token's delta, the backbon
     fp64 from the quantised values.
 
 Parity: the E4M3 rounding is pinned against a brute-force nearest search over the 254 finite
-values, ties, subnormals and saturation (tests/test_oracle_fp8.py).
+values, ties, subnormals and saturation, and the backbone against the plain product on inputs the
+quantisation represents exactly (tests/test_oracle_fp8.py).
 """
 from __future__ import annotations
 
